@@ -1,0 +1,490 @@
+#!/usr/bin/env python
+"""Throughput benchmark of the B200 retention library.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one call of the hot path on one batch of seeded synthetic input
+already resident in HBM:
+  retnet_1p3b       (default) ret_chunkwise, B=4 H=8 N=2048 dk=256 dv=512 chunk 64, bf16
+  retnet_6p7b_long  ret_chunkwise, B=1 H=16 N=8192 dk=256 dv=512 chunk 128, bf16
+  gated             gated_ret_chunkwise, B=2 H=8 N=16384 dk=dv=128 chunk 64, bf16
+  decode            ret_recurrent_step, B=64 H=16 dk=256 dv=512, fp32 state
+For N > 1 (torchrun, one rank per GPU) every rank runs its own batch of the
+same shape (batch sharding, no collective on the data path): weak scaling.
+Rank 0 prints one JSON line. `--impl reference` times the fp64 CPU oracle on a
+bounded sample of the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ----------------------------------------------------------------------------- workload arithmetic
+
+def workload(name: str):
+    """Shapes plus the algorithmic work of one step (one call)."""
+    from linear_attention_ret_b200 import inputs as I
+    cfg = I.CONFIGS[name]
+    B, H, N, dk, dv, C = cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk
+    if name == "decode":
+        state = B * H * dk * dv * 4
+        io = B * H * (2 * dk + 2 * dv) * 2
+        return dict(cfg=cfg, kind="decode", units=1, unit="steps/s", metric="decode steps/s",
+                    tokens=B, bytes=2 * state + io, flops=4 * B * H * dk * dv,
+                    h2d=B * H * (2 * dk + dv) * 2, d2h=B * H * dv * 2)
+    elt = 2
+    qkvo = B * H * N * (2 * dk + 2 * dv) * elt
+    gbytes = B * H * N * 4 if cfg.gamma_schedule == "gated" else 0
+    flops = B * H * N * (2 * C * (dk + dv) + 4 * dk * dv)
+    return dict(cfg=cfg, kind="gated" if gbytes else "chunkwise", units=B * N, unit="tokens/s",
+                metric="retention tokens/s (chunkwise fwd)", tokens=B * N, bytes=qkvo + gbytes, flops=flops,
+                h2d=B * H * N * (2 * dk + dv) * elt + gbytes, d2h=B * H * N * dv * elt)
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "linear_attention_ret_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(name: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary,
+    or None when no capture matches the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(name)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("source_sha") != kernel_source_sha():
+        return None
+    return rec.get("traffic_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def dist_init(world: int, backend: str):
+    import datetime
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank draws its own batch (batch sharding across GPUs)."""
+    return 1000 * rank
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if self.gpu_id:
+            cmd += ["-i", self.gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) == 8:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = max(float(r[1]) for r in rows if r[1].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+        loaded = [s for s in sm if s > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[2]) for r in rows
+                                                          if r[2].replace(".", "").isdigit())}
+
+
+def gpu_uuid(dev_index: int):
+    import torch
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(dev_index).uuid)
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def make_step(spec, dev, seed):
+    """Device-resident inputs and a closure that runs one step."""
+    import torch
+    from linear_attention_ret_b200 import inputs as I
+    from linear_attention_ret_b200 import ret
+    cfg = spec["cfg"]
+    if spec["kind"] == "decode":
+        gam = I.gammas(cfg.H, cfg.gamma_schedule).to(dev)
+        S = I.decode_state(cfg.B, cfg.H, cfg.dk, cfg.dv, seed=seed).to(dev)
+        steps = [tuple(t.to(dev) for t in I.decode_step_inputs(cfg.B, cfg.H, cfg.dk, cfg.dv, s, seed=seed))
+                 for s in range(8)]
+        o = torch.empty(cfg.B, cfg.H, cfg.dv, dtype=cfg.dtype, device=dev)
+        counter = [0]
+
+        def step():
+            q, k, v = steps[counter[0] % len(steps)]
+            counter[0] += 1
+            ret.ret_recurrent_step(q, k, v, gam, S, o=o)
+        return step, {"q": steps[0][0], "k": steps[0][1], "v": steps[0][2]}, o, 1
+
+    x = {key: val.to(dev) for key, val in I.config_inputs(cfg, seed=seed).items()}
+    o = torch.empty(cfg.B, cfg.H, cfg.N, cfg.dv, dtype=cfg.dtype, device=dev)
+    if spec["kind"] == "gated":
+        def step():
+            ret.gated_ret_chunkwise(x["q"], x["k"], x["v"], x["g"], cfg.chunk, o=o)
+    else:
+        def step():
+            ret.ret_chunkwise(x["q"], x["k"], x["v"], x["gamma"], cfg.chunk, o=o)
+    return step, x, o, launches_per_call(spec)
+
+
+def launches_per_call(spec) -> int:
+    """Kernels one call of the step launches (the library's own kernels only)."""
+    from linear_attention_ret_b200 import ret
+    cfg = spec["cfg"]
+    if spec["kind"] == "decode":
+        return 1
+    return ret.chunkwise_launches(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk, cfg.dtype)
+
+
+def run_ours(args, spec):
+    import torch
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_init(world, "nccl")
+    from linear_attention_ret_b200 import ret
+    ret.load()
+    stream = torch.cuda.current_stream(dev)
+
+    step, x, o, launches = make_step(spec, dev, rank_seed(rank))
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    err = ret.last_device_error()
+    if err != 0:
+        raise SystemExit(f"device error word set after warm-up: {err}")
+
+    clocks = ClockSampler(gpu_uuid(local))
+    clocks.start()
+    # timed region: K steps, barrier + synchronize on both sides, events per step on the launch stream
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    barrier(world, dev)
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for i in range(args.steps):
+        step()
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    clk = clocks.stop()
+    per_step = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms = ev[0].elapsed_time(ev[-1])
+    max_ms = max_over_ranks(total_ms, world, dev)
+    if ret.last_device_error() != 0:
+        raise SystemExit("device error word set in the timed region")
+
+    e2e = run_e2e(args, spec, dev, stream, world)
+
+    ms_per_step = max_ms / args.steps
+    value = spec["units"] * world / (ms_per_step / 1e3) if spec["kind"] != "decode" else world * 1e3 / ms_per_step
+    hbm, tf_burst, tf_sust, peak_src = measured_peaks()
+    # the dominant kernel's duration: a step is one launch of it (plus, for split
+    # sequences, two short launches whose share the ncu launch list records)
+    kern_ms = statistics.mean(per_step)
+    achieved = spec["bytes"] / (kern_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "traffic": ncu_traffic(args.workload),
+                "peak_source": peak_src + " (MEASURED_PEAKS.json hbm_gbs, copy)" if peak_src == "measured"
+                else "fallback 6.65 TB/s",
+                "kernel_ms": round(kern_ms, 5),
+                "tensor_tflops": round(spec["flops"] / (kern_ms / 1e3) / 1e12, 2),
+                "tensor_frac_of_bf16_burst": round(spec["flops"] / (kern_ms / 1e3) / 1e12 / tf_burst, 4)}
+    cfg = spec["cfg"]
+    line = {
+        "metric": spec["metric"], "value": round(value, 2), "unit": spec["unit"], "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1)/sqrt(dk); per-rank seeds)",
+        "config": {"workload": args.workload, "B": cfg.B, "H": cfg.H, "N": cfg.N, "dk": cfg.dk, "dv": cfg.dv,
+                   "chunk": cfg.chunk, "state": "fp32",
+                   "l2": f"working set {spec['bytes'] / 1e6:.0f} MB per step > 126 MB L2 (no flush)",
+                   "parallelism": f"batch-sharded x{world}" if world > 1 else "single GPU"},
+        "roofline": roofline,
+        "clocks": clk,
+        "e2e": e2e,
+        "gpu_launches": args.steps * launches,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(spec, budget_s=args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_e2e(args, spec, dev, stream, world):
+    """Same metric through the public API with host buffers: every step copies its
+    inputs host->device from pinned memory and the result device->host."""
+    import torch
+    from linear_attention_ret_b200 import inputs as I
+    from linear_attention_ret_b200 import ret
+    cfg = spec["cfg"]
+    rank = dist_env()[0]
+    if spec["kind"] == "decode":
+        host = [t.pin_memory() for t in I.decode_step_inputs(cfg.B, cfg.H, cfg.dk, cfg.dv, 0, seed=rank_seed(rank))]
+        dq, dk_, dv_ = (torch.empty_like(t, device=dev) for t in host)
+        gam = I.gammas(cfg.H, cfg.gamma_schedule).to(dev)
+        S = I.decode_state(cfg.B, cfg.H, cfg.dk, cfg.dv).to(dev)
+        o = torch.empty(cfg.B, cfg.H, cfg.dv, dtype=cfg.dtype, device=dev)
+        o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+
+        def step():
+            dq.copy_(host[0], non_blocking=True)
+            dk_.copy_(host[1], non_blocking=True)
+            dv_.copy_(host[2], non_blocking=True)
+            ret.ret_recurrent_step(dq, dk_, dv_, gam, S, o=o)
+            o_host.copy_(o, non_blocking=True)
+    else:
+        xh = {k: t.pin_memory() for k, t in I.config_inputs(cfg, seed=rank_seed(rank)).items()}
+        xd = {k: torch.empty_like(t, device=dev) for k, t in xh.items()}
+        o = torch.empty(cfg.B, cfg.H, cfg.N, cfg.dv, dtype=cfg.dtype, device=dev)
+        o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        gated = spec["kind"] == "gated"
+
+        def step():
+            for key in xh:
+                xd[key].copy_(xh[key], non_blocking=True)
+            if gated:
+                ret.gated_ret_chunkwise(xd["q"], xd["k"], xd["v"], xd["g"], cfg.chunk, o=o)
+            else:
+                ret.ret_chunkwise(xd["q"], xd["k"], xd["v"], xd["gamma"], cfg.chunk, o=o)
+            o_host.copy_(o, non_blocking=True)
+    steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, dev)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev) / steps
+    value = (spec["units"] if spec["kind"] != "decode" else 1) * world / (ms / 1e3)
+    return {"value": round(value, 2), "unit": spec["unit"], "ms_per_step": round(ms, 4),
+            "h2d_bytes_per_step": spec["h2d"], "d2h_bytes_per_step": spec["d2h"]}
+
+
+# ----------------------------------------------------------------------------- oracle timing
+
+def _oracle_sample_step(spec, heads, seed=0):
+    """Inputs for a bounded sample (the first `heads` (b, h) pairs) and a closure
+    that runs the oracle on it once. Returns (closure, units the sample covers)."""
+    import torch
+    from linear_attention_ret_b200 import inputs as I
+    from oracle import oracle as O
+    cfg = spec["cfg"]
+    if spec["kind"] == "decode":
+        gam = I.gammas(cfg.H, cfg.gamma_schedule)
+        q, k, v = I.decode_step_inputs(cfg.B, cfg.H, cfg.dk, cfg.dv, 0, seed=seed)
+        S = I.decode_state(cfg.B, cfg.H, cfg.dk, cfg.dv, seed=seed)
+        b_needed = max(1, -(-heads // cfg.H))
+        qs, ks, vs, Ss = (t[:b_needed] for t in (q, k, v, S))
+        state = [Ss.double().numpy()]
+
+        def run():
+            _, state[0] = O.ret_recurrent_step(qs, ks, vs, gam, state[0])
+        return run, b_needed * cfg.H / (cfg.B * cfg.H)  # fraction of one decode step
+    x = I.config_inputs(cfg, seed=seed, B=max(1, -(-heads // cfg.H)))
+    sl = {k: t.reshape(-1, *t.shape[2:])[:heads].unsqueeze(0) for k, t in x.items() if k != "gamma"}
+    if spec["kind"] == "gated":
+        def run():
+            O.gated_chunkwise(sl["q"], sl["k"], sl["v"], sl["g"], cfg.chunk)
+    else:
+        bh_idx = torch.arange(heads) % cfg.H
+        gam = x["gamma"][bh_idx]
+        # heads of the sample become the H axis of one batch element, each with its own gamma
+
+        def run():
+            O.ret_chunkwise(sl["q"], sl["k"], sl["v"], gam, cfg.chunk)
+    return run, heads * cfg.N / cfg.H  # tokens (all heads of a token count once)
+
+
+def cpu_baseline(spec, budget_s: float = 12.0):
+    from oracle import oracle as O
+    threads = O.max_threads()
+    cfg = spec["cfg"]
+    total_heads = cfg.B * cfg.H
+    heads = min(total_heads, threads)
+    run, units = _oracle_sample_step(spec, heads)
+    t0 = time.perf_counter()
+    run()
+    t = time.perf_counter() - t0
+    reps = 1
+    while time.perf_counter() - t0 + t <= budget_s and reps < 64:
+        run()
+        reps += 1
+    el = time.perf_counter() - t0
+    value = units * reps / el
+    what = "decode steps" if spec["kind"] == "decode" else f"{cfg.N} tokens"
+    return {"value": round(value, 3), "unit": spec["unit"], "cores": threads, "kind": "oracle",
+            "sample": f"{reps} run(s) of the fp64 oracle on {heads} of {total_heads} (b,h) heads x {what} "
+                      f"({el:.1f} s wall, OpenMP over heads)",
+            "cpu": _cpu_model()}
+
+
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def run_reference(args, spec):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return  # the oracle runs on rank 0's host cores only
+    from oracle import oracle as O
+    threads = O.max_threads()
+    cfg = spec["cfg"]
+    heads = min(cfg.B * cfg.H, threads)
+    run, units = _oracle_sample_step(spec, heads)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    el = time.perf_counter() - t0
+    value = units * args.steps / el
+    what = "decode steps" if spec["kind"] == "decode" else f"{cfg.N} tokens"
+    sample = (f"each step: fp64 oracle on {heads} of {cfg.B * cfg.H} (b,h) heads x {what}, "
+              f"OpenMP over heads")
+    line = {"impl": "reference", "metric": spec["metric"], "value": round(value, 4), "unit": spec["unit"],
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "B": cfg.B, "H": cfg.H, "N": cfg.N, "dk": cfg.dk,
+                       "dv": cfg.dv, "chunk": cfg.chunk},
+            "cpu_baseline": {"value": round(value, 4), "unit": spec["unit"], "cores": threads, "kind": "oracle",
+                             "sample": sample, "cpu": _cpu_model()},
+            "e2e": {"value": round(value, 4), "unit": spec["unit"], "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="retnet_1p3b",
+                    choices=["retnet_1p3b", "retnet_6p7b_long", "gated", "decode"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    spec = workload(args.workload)
+    if args.impl == "reference":
+        run_reference(args, spec)
+    else:
+        run_ours(args, spec)
+
+
+if __name__ == "__main__":
+    main()

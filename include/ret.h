@@ -1,0 +1,153 @@
+/*
+ * ret.h - C ABI of the B200 (sm_100a) retention library, libret.so.
+ *
+ * Retention is the sequence mixer of RetNet. Sources for the operations:
+ *   [RM] aiqz.cc, "RetNet retention mechanism" tutorial page: sections
+ *        保留机制初识 (first look, R_n = sum_{m<=n} gamma^(n-m) (Q_n K_m^T) V_m),
+ *        衰减矩阵 (decay matrix D_nm = gamma^(n-m) for n >= m, else 0),
+ *        并行训练 (parallel form R = (Q K^T (.) D) V),
+ *        递归推理 (recurrent form S_n = gamma S_{n-1} + K_n^T V_n, R_n = Q_n S_n),
+ *        块级循环 (chunkwise recurrent form: parallel inside a chunk, state
+ *        passed between chunks).
+ *   [RN] 171host.com, "Retentive Network (RetNet) 详解": section 3.1 (the three
+ *        equivalent forms) and 3.2 (multi-scale retention: one gamma per head).
+ *   [GR] pwwt.cn, "unilm RetNet 技术指南 ... Gated RetNet 的源码解析": the gated
+ *        form with a per-token, per-head log-decay g (parallel_gate_retention,
+ *        chunk_gate_retention = cross_chunk + inner_chunk,
+ *        recurrent_gate_retention).
+ *
+ * Conventions shared by every entry point
+ *   - Pointers are DEVICE pointers owned by the caller. The library never frees
+ *     caller memory and keeps no pointer after the call returns.
+ *   - Tensors are contiguous row-major, heads leading:
+ *       q, k [B, H, N, dk]   v, o [B, H, N, dv]   state [B, H, dk, dv] (fp32)
+ *       gamma [H] (fp32)     g [B, H, N] (fp32, natural-log decay, normally <= 0)
+ *   - dt selects the element type of q, k, v and o (RET_F32 or RET_BF16).
+ *     gamma, g and state are always fp32. Arithmetic accumulates in fp32.
+ *   - No 1/sqrt(dk) scale is applied: callers pass pre-scaled q or k.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t cast to void*;
+ *     NULL = the legacy default stream). Arguments are validated on the host
+ *     before anything is launched; a non-RET_OK status means nothing ran.
+ *   - Errors are returned, never raised: no exit(), no device trap.
+ *   - Calls keep no state between calls and are safe from several host threads.
+ *   - N == 0 is a valid empty problem: nothing is launched, state_out (if
+ *     given) receives state_in (or zeros).
+ */
+#ifndef RET_H_
+#define RET_H_
+
+#if defined(__GNUC__)
+#define RET_API __attribute__((visibility("default")))
+#else
+#define RET_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RET_OK = 0,
+    RET_ERR_NULL = 1,        /* a required pointer is NULL */
+    RET_ERR_SHAPE = 2,       /* a size is negative or zero where it must be positive */
+    RET_ERR_DTYPE = 3,       /* dt is not a ret_dtype value */
+    RET_ERR_UNSUPPORTED = 4, /* sizes outside what the kernels support (see each call) */
+    RET_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed */
+    RET_ERR_TIMEOUT = 6,     /* a kernel's bounded wait ran out (device error word set) */
+    RET_ERR_ALIGN = 7        /* a pointer is not 16-byte aligned */
+} ret_status;
+
+typedef enum { RET_F32 = 0, RET_BF16 = 1 } ret_dtype;
+
+/*
+ * Parallel form, [RM] 并行训练 / [RN] 3.1: O = (Q K^T (.) D) V with
+ * D_nm = gamma_h^(n-m) for n >= m and 0 above the diagonal ([RM] 衰减矩阵).
+ * O(N^2) work; meant for short sequences and as a cross-check of the other
+ * forms. Requires dk <= 1024, dv >= 1.
+ */
+RET_API ret_status ret_parallel(const void* q, const void* k, const void* v, const float* gamma,
+                        void* o, int B, int H, int N, int dk, int dv,
+                        ret_dtype dt, void* stream);
+
+/*
+ * Chunkwise recurrent form, [RM] 块级循环 / [RN] 3.1 and 4.3. The sequence is
+ * split into chunks of `chunk` tokens (the last may be shorter and behaves as
+ * zero padding). For chunk i of length L, local rows j, m = 0..L-1:
+ *   O_[i] = (Q_[i] K_[i]^T (.) D) V_[i] + diag(gamma^(j+1)) Q_[i] S_[i-1]
+ *   S_[i] = gamma^L S_[i-1] + sum_m gamma^(L-1-m) K_m^T V_m
+ * state_in : initial state [B, H, dk, dv] fp32, or NULL for zeros.
+ * state_out: final state [B, H, dk, dv] fp32, or NULL. May equal state_in.
+ * The result does not depend on `chunk` beyond rounding; chunks longer than 64
+ * tokens are evaluated as 64-token sub-chunks.
+ * Requires chunk >= 1, dk <= 256, dv >= 1. The tensor-core path (bf16,
+ * dk in {64, 128, 256}, dv a multiple of 128, chunk a multiple of 64) also
+ * needs 16-byte aligned q, k, v, o; other shapes use a CUDA-core path.
+ * May allocate stream-ordered scratch (cudaMallocAsync) for long sequences
+ * with few heads; it is freed on the same stream before the call returns.
+ */
+RET_API ret_status ret_chunkwise(const void* q, const void* k, const void* v, const float* gamma,
+                         void* o, const float* state_in, float* state_out,
+                         int B, int H, int N, int dk, int dv, int chunk,
+                         ret_dtype dt, void* stream);
+
+/*
+ * One recurrent (decode) step, [RM] 递归推理:
+ *   S <- gamma_h S + k^T v   (in place),   o = q S   (the updated state).
+ * q, k [B, H, dk]; v, o [B, H, dv] of type dt; state [B, H, dk, dv] fp32.
+ * The state is read and written once: the step is bound by HBM bandwidth.
+ * Requires dk <= 4096; state must be 16-byte aligned and dv a multiple of 4
+ * for the vectorised path (otherwise a scalar path runs).
+ */
+RET_API ret_status ret_recurrent_step(const void* q, const void* k, const void* v, const float* gamma,
+                              float* state, void* o, int B, int H, int dk, int dv,
+                              ret_dtype dt, void* stream);
+
+/*
+ * Gated chunkwise form, [GR] chunk_gate_retention: the per-token log-decay g
+ * replaces log(gamma). With Gl the inclusive cumulative sum of g restarted at
+ * each chunk:
+ *   inner: (Q K^T) * exp(Gl_j - Gl_m) for j >= m, times V
+ *   cross: exp(Gl_j) (Q_[i] S_[i-1])_j
+ *   state: S_[i] = exp(Gl_{L-1}) S_[i-1] + sum_m exp(Gl_{L-1} - Gl_m) K_m^T V_m
+ * Only in-chunk differences of the cumulative sum are exponentiated, so long
+ * sequences cannot underflow. Same shapes, state handling, limits and paths as
+ * ret_chunkwise.
+ */
+RET_API ret_status gated_ret_chunkwise(const void* q, const void* k, const void* v, const float* g,
+                               void* o, const float* state_in, float* state_out,
+                               int B, int H, int N, int dk, int dv, int chunk,
+                               ret_dtype dt, void* stream);
+
+/* Static description of a status code. Never NULL. */
+RET_API const char* ret_status_str(ret_status s);
+
+/*
+ * Synchronises `stream`, then reads and clears the library's device error
+ * word, which a kernel sets when one of its bounded waits runs out.
+ * Returns RET_ERR_TIMEOUT if it was set, RET_ERR_CUDA if the stream reports
+ * an error, RET_OK otherwise.
+ */
+RET_API ret_status ret_last_device_error(void* stream);
+
+/*
+ * Which kernel family ret_chunkwise / gated_ret_chunkwise would run for these
+ * arguments: 1 = tcgen05 tensor-core path, 0 = CUDA-core path, -1 = rejected.
+ * Pure host function; nothing is launched.
+ */
+RET_API int ret_chunkwise_path(int dk, int dv, int chunk, ret_dtype dt);
+
+/*
+ * Number of kernels one ret_chunkwise / gated_ret_chunkwise call with these
+ * arguments launches (0 for an empty sequence, -1 if the arguments would be
+ * rejected). Pure host function; nothing is launched.
+ */
+RET_API int ret_chunkwise_launches(int B, int H, int N, int dk, int dv, int chunk, ret_dtype dt);
+
+/* Library version, "major.minor.patch". */
+RET_API const char* ret_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RET_H_ */

@@ -1,0 +1,187 @@
+// C ABI of libret.so (declared in include/ret.h): host-side validation, kernel
+// selection and launch. One translation unit holds every kernel so that they
+// share the module-scope device error word.
+#include <cstdio>
+#include <cstring>
+
+#include "common.cuh"
+#include "simt.cuh"
+#include "decode.cuh"
+#include "tc_chunk.cuh"
+
+using namespace ret;
+
+namespace {
+
+constexpr int kMaxGridY = 65535;
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline ret_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? RET_OK : RET_ERR_CUDA;
+}
+
+ret_status check_common(int B, int H, int N, int dk, int dv, int dt) {
+    if (dt != RET_F32 && dt != RET_BF16) return RET_ERR_DTYPE;
+    if (B <= 0 || H <= 0 || N < 0 || dk <= 0 || dv <= 0) return RET_ERR_SHAPE;
+    if ((long long)B * H > kMaxGridY) return RET_ERR_UNSUPPORTED;
+    return RET_OK;
+}
+
+// state_out <- state_in (or zeros) for an empty sequence.
+ret_status empty_sequence_state(const float* state_in, float* state_out, int B, int H, int dk, int dv,
+                                cudaStream_t st) {
+    if (state_out == nullptr) return RET_OK;
+    const size_t bytes = sizeof(float) * (size_t)B * H * dk * dv;
+    cudaError_t e = state_in ? (state_in == state_out ? cudaSuccess
+                                                      : cudaMemcpyAsync(state_out, state_in, bytes,
+                                                                        cudaMemcpyDeviceToDevice, st))
+                             : cudaMemsetAsync(state_out, 0, bytes, st);
+    return e == cudaSuccess ? RET_OK : RET_ERR_CUDA;
+}
+
+template <typename T, bool GATED>
+ret_status launch_chunkwise_simt(const void* q, const void* k, const void* v, const float* decay,
+                                 void* o, const float* state_in, float* state_out,
+                                 int B, int H, int N, int dk, int dv, int chunk, cudaStream_t st) {
+    auto kern = chunkwise_simt_kernel<T, GATED>;
+    const size_t smem = chunkwise_simt_smem_bytes(dk);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return RET_ERR_CUDA;
+    dim3 grid((dv + kCwV - 1) / kCwV, B * H);
+    kern<<<grid, kCwThreads, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
+                                         static_cast<const T*>(v), decay, state_in, state_out,
+                                         static_cast<T*>(o), H, N, dk, dv, chunk);
+    return launch_status();
+}
+
+template <bool GATED>
+ret_status chunkwise_entry(const void* q, const void* k, const void* v, const float* decay,
+                           void* o, const float* state_in, float* state_out,
+                           int B, int H, int N, int dk, int dv, int chunk, ret_dtype dt, void* stream) {
+    ret_status s = check_common(B, H, N, dk, dv, dt);
+    if (s != RET_OK) return s;
+    if (chunk <= 0) return RET_ERR_SHAPE;
+    if (dk > 256) return RET_ERR_UNSUPPORTED;
+    cudaStream_t st = as_stream(stream);
+    if (N == 0) return empty_sequence_state(state_in, state_out, B, H, dk, dv, st);
+    if (!q || !k || !v || !decay || !o) return RET_ERR_NULL;
+    if (tc_chunk_supported(dk, dv, chunk, dt == RET_BF16)) {
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RET_ERR_ALIGN;
+        return tc_chunk_launch<GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dk, dv, st);
+    }
+    if (dt == RET_F32)
+        return launch_chunkwise_simt<float, GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dk, dv,
+                                                   chunk, st);
+    return launch_chunkwise_simt<__nv_bfloat16, GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dk,
+                                                       dv, chunk, st);
+}
+
+template <typename T>
+ret_status launch_parallel(const void* q, const void* k, const void* v, const float* gamma, void* o,
+                           int B, int H, int N, int dk, int dv, cudaStream_t st) {
+    dim3 grid((N + kParQ - 1) / kParQ, (dv + kParV - 1) / kParV, B * H);
+    if (grid.y > (unsigned)kMaxGridY) return RET_ERR_UNSUPPORTED;
+    parallel_simt_kernel<T><<<grid, kParThreads, 0, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
+                                                          static_cast<const T*>(v), gamma, static_cast<T*>(o),
+                                                          H, N, dk, dv);
+    return launch_status();
+}
+
+template <typename T>
+ret_status launch_step(const void* q, const void* k, const void* v, const float* gamma, float* state, void* o,
+                       int B, int H, int dk, int dv, cudaStream_t st) {
+    const size_t smem = sizeof(float) * 2 * (size_t)dk;
+    if ((dv & 3) == 0 && aligned16(state)) {
+        const int groups = dv / 4;
+        dim3 grid((groups + kDecThreads - 1) / kDecThreads, B * H);
+        recurrent_step_vec_kernel<T><<<grid, kDecThreads, smem, st>>>(
+            static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), gamma, state,
+            static_cast<T*>(o), H, dk, dv);
+    } else {
+        dim3 grid((dv + kDecThreads - 1) / kDecThreads, B * H);
+        recurrent_step_scalar_kernel<T><<<grid, kDecThreads, smem, st>>>(
+            static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), gamma, state,
+            static_cast<T*>(o), H, dk, dv);
+    }
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+ret_status ret_parallel(const void* q, const void* k, const void* v, const float* gamma, void* o,
+                        int B, int H, int N, int dk, int dv, ret_dtype dt, void* stream) {
+    ret_status s = check_common(B, H, N, dk, dv, dt);
+    if (s != RET_OK) return s;
+    if (dk > 1024) return RET_ERR_UNSUPPORTED;
+    if (N == 0) return RET_OK;
+    if (!q || !k || !v || !gamma || !o) return RET_ERR_NULL;
+    cudaStream_t st = as_stream(stream);
+    return dt == RET_F32 ? launch_parallel<float>(q, k, v, gamma, o, B, H, N, dk, dv, st)
+                         : launch_parallel<__nv_bfloat16>(q, k, v, gamma, o, B, H, N, dk, dv, st);
+}
+
+ret_status ret_chunkwise(const void* q, const void* k, const void* v, const float* gamma, void* o,
+                         const float* state_in, float* state_out, int B, int H, int N, int dk, int dv,
+                         int chunk, ret_dtype dt, void* stream) {
+    return chunkwise_entry<false>(q, k, v, gamma, o, state_in, state_out, B, H, N, dk, dv, chunk, dt, stream);
+}
+
+ret_status gated_ret_chunkwise(const void* q, const void* k, const void* v, const float* g, void* o,
+                               const float* state_in, float* state_out, int B, int H, int N, int dk, int dv,
+                               int chunk, ret_dtype dt, void* stream) {
+    return chunkwise_entry<true>(q, k, v, g, o, state_in, state_out, B, H, N, dk, dv, chunk, dt, stream);
+}
+
+ret_status ret_recurrent_step(const void* q, const void* k, const void* v, const float* gamma, float* state,
+                              void* o, int B, int H, int dk, int dv, ret_dtype dt, void* stream) {
+    ret_status s = check_common(B, H, 1, dk, dv, dt);
+    if (s != RET_OK) return s;
+    if (dk > 4096) return RET_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !gamma || !state || !o) return RET_ERR_NULL;
+    cudaStream_t st = as_stream(stream);
+    return dt == RET_F32 ? launch_step<float>(q, k, v, gamma, state, o, B, H, dk, dv, st)
+                         : launch_step<__nv_bfloat16>(q, k, v, gamma, state, o, B, H, dk, dv, st);
+}
+
+const char* ret_status_str(ret_status s) {
+    switch (s) {
+        case RET_OK: return "ok";
+        case RET_ERR_NULL: return "a required pointer is NULL";
+        case RET_ERR_SHAPE: return "invalid size";
+        case RET_ERR_DTYPE: return "invalid dtype";
+        case RET_ERR_UNSUPPORTED: return "sizes not supported by the kernels";
+        case RET_ERR_CUDA: return "CUDA error";
+        case RET_ERR_TIMEOUT: return "a kernel wait timed out (device error word set)";
+        case RET_ERR_ALIGN: return "pointer not 16-byte aligned";
+    }
+    return "unknown status";
+}
+
+ret_status ret_last_device_error(void* stream) {
+    if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return RET_ERR_CUDA;
+    unsigned int word = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return RET_ERR_CUDA;
+    if (word != 0 && cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return RET_ERR_CUDA;
+    return word ? RET_ERR_TIMEOUT : RET_OK;
+}
+
+int ret_chunkwise_path(int dk, int dv, int chunk, ret_dtype dt) {
+    if ((dt != RET_F32 && dt != RET_BF16) || dk <= 0 || dv <= 0 || chunk <= 0 || dk > 256) return -1;
+    return tc_chunk_supported(dk, dv, chunk, dt == RET_BF16) ? 1 : 0;
+}
+
+int ret_chunkwise_launches(int B, int H, int N, int dk, int dv, int chunk, ret_dtype dt) {
+    if (check_common(B, H, N, dk, dv, dt) != RET_OK || chunk <= 0 || dk > 256) return -1;
+    if (N == 0) return 0;
+    if (tc_chunk_supported(dk, dv, chunk, dt == RET_BF16)) return tc_chunk_launches(B, H, N, dk, dv);
+    return 1;
+}
+
+const char* ret_version(void) { return "0.1.0"; }
+
+}  // extern "C"

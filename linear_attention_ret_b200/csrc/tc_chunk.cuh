@@ -1,0 +1,659 @@
+// Tensor-core (tcgen05 + TMA + TMEM) chunkwise retention for sm_100a.
+//
+// Method: "RetNet retention mechanism" (aiqz.cc), section 块级循环 (chunkwise
+// recurrence), and the gated chunk_gate_retention (pwwt.cn page). For chunk i
+// (64 tokens, local rows j, m), with decays as in the CUDA-core kernel:
+//   O_[i] = (Q K^T (.) D) V + diag(r) Q S_[i-1]
+//   S_[i] = decay S_[i-1] + K^T diag(zeta) V
+//
+// Work split. One CTA owns one head and a 128-column slice of dv and walks the
+// chunks of its sequence range in order. The products run transposed so that
+// the large ones have M = 128 (one TMEM lane per dv column of the slice):
+//   A        = Q K^T                 M=64  N=64  K=dk  (SS)   -> TMEM, masked by the epilogue into P (bf16, smem)
+//   O_inter^T = S_op^T Q^T           M=128 N=64  K=dk  (TS: S_op = bf16 copy of the state, in TMEM)
+//   O_intra^T = V^T P^T              M=128 N=64  K=64  (SS, V read MN-major straight from the TMA tile)
+//   S^T      += (zeta V)^T K         M=128 N=dk  K=64  (SS, K read MN-major from the same TMA tile)
+// The fp32 state S^T lives in TMEM for the whole sequence. After each state
+// update the epilogue reads it once, writes its bf16 copy (the next chunk's
+// MMA operand) and writes back decay * S, so the next update accumulates onto
+// the decayed state. The decay mask is generated in registers.
+//
+// Roles (192 threads): warp 0 issues TMA loads (two stages of Q, K, V tiles),
+// warp 1 allocates TMEM and issues every tcgen05.mma from one thread, warps 2-5
+// are the epilogue (TMEM lane quarter = warp index % 4). All waits are bounded:
+// on timeout the kernel sets the device error word, the roles stop, in-flight
+// copies and MMAs are drained (bounded again) and TMEM is released.
+#pragma once
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+
+namespace ret {
+namespace tc {
+
+constexpr int kC = 64;          // chunk rows per tile
+constexpr int kDvS = 128;       // dv columns per CTA (TMEM lanes)
+constexpr int kThreads = 192;
+constexpr int kEpiThreads = 128;
+constexpr int kTile64 = kC * 128;  // one 64-row x 128-byte swizzled tile (8 KB)
+constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
+
+template <int DK>
+struct Layout {
+    static constexpr int kQBytes = DK / 64 * kTile64;
+    static constexpr int kKBytes = DK / 64 * kTile64;
+    static constexpr int kVBytes = 2 * kTile64;
+    static constexpr int kStageBytes = kQBytes + kKBytes + kVBytes;
+    static constexpr int kStage0 = 0;
+    static constexpr int kP = 2 * kStageBytes;              // P tile (64 x 64 bf16, SW128 K-major)
+    static constexpr int kZV = kP + kTile64;                // zeta-scaled V (same layout as the V tile)
+    static constexpr int kOst = kZV + kVBytes;              // O staging for the TMA store (no swizzle)
+    static constexpr int kBar = kOst + kVBytes;             // mbarriers
+    static constexpr int kNumBars = 12;
+    static constexpr int kDec = kBar + kNumBars * 8;        // decay tables, double-buffered by chunk parity
+    static constexpr int kDecFloats = 3 * kC + 4;           // cum | r | zeta | decay
+    static constexpr int kTmemSlot = kDec + 2 * kDecFloats * 4;
+    static constexpr int kAbort = kTmemSlot + 4;
+    static constexpr int kBytes = kAbort + 4;
+    static constexpr int kSmemAlloc = kBytes + 1024;        // slack to align the base to 1024 B
+    // TMEM columns
+    static constexpr int kColS = 0;                 // fp32 state S^T: DK columns
+    static constexpr int kColSop = DK;              // bf16 state copy: DK/2 columns
+    static constexpr int kColA = DK + DK / 2;       // Q K^T, then O_inter^T: 64 columns
+    static constexpr int kColO = kColA + kC;        // O_intra^T: 64 columns
+    static constexpr int kColsUsed = kColO + kC;
+    static constexpr int kTmemCols = kColsUsed <= 256 ? 256 : 512;
+    static_assert(kColsUsed <= 512, "TMEM overflow");
+    static_assert(kBytes + 1024 <= 227 * 1024, "shared memory overflow");
+};
+
+enum Bar { kFull0 = 0, kFull1, kEmpty0, kEmpty1, kAFull, kPReady, kOFull, kOFree, kSFull, kSReady, kDrain };
+
+// ------------------------------------------------------------------ PTX wrappers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait. Returns false (and sets the abort flag and the device error
+// word on the first timeout) if the phase did not complete within kWaitNs or
+// another role already gave up.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer() - t0 > kWaitNs) {
+            *abort_flag = 1;
+            raise_error(kErrWaitTimeout);
+            return false;
+        }
+    }
+}
+
+// Wait used while draining after an abort: bounded, never raises.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity) && globaltimer() - t0 < kWaitNs) {
+    }
+}
+
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, int x, int y, int z, uint32_t src) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3}], [%4];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_store_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void tma_store_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 format: start address,
+// leading and stride byte offsets in 16-byte units, version 1 at bit 46, layout 2 at bit 61).
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of kind::f16: bf16 A and B, fp32 D; majors 0 = K, 1 = MN.
+__host__ __device__ constexpr uint32_t idesc(int M, int N, int a_mn, int b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a), "l"(b), "r"(id), "r"(acc)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t id, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b), "r"(id), "r"(acc)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+// 32 lanes x 32 columns of 32-bit TMEM words: thread t of the warp gets lane (base+t), columns c..c+31.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+          "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+          "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
+    __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&u);
+    return __bfloat1622float2(h);
+}
+
+// ------------------------------------------------------------------ kernel
+
+struct Params {
+    const float* decay_in;   // gamma [H] or g [B, H, N]
+    const float* state_in;   // [B, H, dk, dv] or null
+    float* state_out;        // [B, H, dk, dv] or null
+    int H, N, dv;
+};
+
+template <int DK, bool GATED>
+__global__ void __launch_bounds__(kThreads, 1)
+chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, Params p) {
+    using Lay = Layout<DK>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    auto bar = [&](int b) { return sbase + Lay::kBar + 8 * b; };
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Lay::kAbort);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Lay::kTmemSlot);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int slice = blockIdx.x, bh = blockIdx.y;
+    const int dv0 = slice * kDvS;
+    const int nchunks = (p.N + kC - 1) / kC;
+
+    if (threadIdx.x == 0) {
+        for (int b = 0; b < Lay::kNumBars; ++b) mbar_init(bar(b), 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_q)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_k)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_v)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_o)) : "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(tmem_slot)), "r"(Lay::kTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int issued = -1;
+            for (int i = 0; i < nchunks; ++i) {
+                const int s = i & 1;
+                if (i >= 2 && !mbar_wait(bar(kEmpty0 + s), ((i >> 1) - 1) & 1, abort_flag)) break;
+                const uint32_t st = sbase + Lay::kStage0 + s * Lay::kStageBytes;
+                mbar_expect_tx(bar(kFull0 + s), Lay::kStageBytes);
+                const int t0 = i * kC;
+#pragma unroll
+                for (int kb = 0; kb < DK / 64; ++kb) {
+                    tma_load_3d(st + kb * kTile64, &tm_q, kb * 64, t0, bh, bar(kFull0 + s));
+                    tma_load_3d(st + Lay::kQBytes + kb * kTile64, &tm_k, kb * 64, t0, bh, bar(kFull0 + s));
+                }
+                tma_load_3d(st + Lay::kQBytes + Lay::kKBytes, &tm_v, dv0, t0, bh, bar(kFull0 + s));
+                tma_load_3d(st + Lay::kQBytes + Lay::kKBytes + kTile64, &tm_v, dv0 + 64, t0, bh, bar(kFull0 + s));
+                issued = i;
+            }
+            if (*abort_flag && issued >= 0) {
+                // drain the copies in flight before the CTA may exit
+                for (int i = (issued >= 1 ? issued - 1 : 0); i <= issued; ++i)
+                    mbar_drain(bar(kFull0 + (i & 1)), (i >> 1) & 1);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t id_qk = idesc(64, kC, 0, 0);
+            constexpr uint32_t id_oi = idesc(128, kC, 0, 0);
+            constexpr uint32_t id_ov = idesc(128, kC, 1, 0);
+            constexpr uint32_t id_up = idesc(128, DK, 1, 1);
+            const uint32_t tA = tmem + Lay::kColA, tO = tmem + Lay::kColO;
+            const uint32_t tS = tmem + Lay::kColS, tSop = tmem + Lay::kColSop;
+            const uint32_t sP = sbase + Lay::kP, sZV = sbase + Lay::kZV;
+            bool ok = true;
+            for (int i = 0; i < nchunks && ok; ++i) {
+                const int s = i & 1;
+                const uint32_t sQ = sbase + Lay::kStage0 + s * Lay::kStageBytes;
+                const uint32_t sK = sQ + Lay::kQBytes;
+                const uint32_t sV = sK + Lay::kKBytes;
+                ok = mbar_wait(bar(kFull0 + s), (i >> 1) & 1, abort_flag);
+                if (ok && i > 0) ok = mbar_wait(bar(kOFree), (i - 1) & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                // A = Q K^T (both K-major, 128-byte swizzle; 16-element K steps)
+#pragma unroll
+                for (int ks = 0; ks < DK / 16; ++ks) {
+                    const uint32_t off = (ks >> 2) * kTile64 + (ks & 3) * 32;
+                    mma_ss(tA, sdesc(sQ + off, 16, 1024), sdesc(sK + off, 16, 1024), id_qk, ks > 0);
+                }
+                mma_commit(bar(kAFull));
+                ok = mbar_wait(bar(kPReady), i & 1, abort_flag) && mbar_wait(bar(kSReady), i & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                // O_inter^T = S_op^T Q^T: A from TMEM (bf16 pairs per column), B = Q tile K-major
+#pragma unroll
+                for (int ks = 0; ks < DK / 16; ++ks) {
+                    const uint32_t off = (ks >> 2) * kTile64 + (ks & 3) * 32;
+                    mma_ts(tA, tSop + ks * 8, sdesc(sQ + off, 16, 1024), id_oi, ks > 0);
+                }
+                // O_intra^T = V^T P^T: A = V tile MN-major (dv blocks 8 KB apart), B = P K-major
+#pragma unroll
+                for (int ks = 0; ks < kC / 16; ++ks)
+                    mma_ss(tO, sdesc(sV + ks * 2048, kTile64, 1024), sdesc(sP + ks * 32, 16, 1024), id_ov, ks > 0);
+                mma_commit(bar(kOFull));
+                // S^T += (zeta V)^T K: A = ZV MN-major, B = K tile MN-major (dk blocks 8 KB apart)
+#pragma unroll
+                for (int ks = 0; ks < kC / 16; ++ks)
+                    mma_ss(tS, sdesc(sZV + ks * 2048, kTile64, 1024), sdesc(sK + ks * 2048, kTile64, 1024), id_up, 1);
+                mma_commit(bar(kSFull));
+                mma_commit(bar(kEmpty0 + s));
+            }
+            // make sure every issued MMA has completed before TMEM can be released
+            mma_commit(bar(kDrain));
+            mbar_drain(bar(kDrain), 0);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (warps 2..5)
+        const int te = threadIdx.x - 64;             // 0..127
+        const int quarter = warp & 3;                // TMEM lane quarter this warp may access
+        const int d = quarter * 32 + lane;           // dv column (within the slice) = TMEM lane
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        float* decf = reinterpret_cast<float*>(sm + Lay::kDec);
+        const float* G = GATED ? p.decay_in + (size_t)bh * p.N : nullptr;
+        const float lg = GATED ? 0.f : log2f(p.decay_in[bh % p.H]);
+
+        // decay tables of chunk c into buffer c & 1: cum (gated, log2 units), r, zeta, decay
+        auto prepare = [&](int c) {
+            float* tb = decf + (c & 1) * Lay::kDecFloats;
+            const int t0 = c * kC, L = min(kC, p.N - t0);
+            if (GATED) {
+                if (te < 32) {
+                    const int a = t0 + 2 * te;
+                    const float g0 = (a < p.N ? G[a] : 0.f) * kLog2e;
+                    const float g1 = (a + 1 < p.N ? G[a + 1] : 0.f) * kLog2e;
+                    const float pair = g0 + g1;
+                    float incl = pair;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const float y = __shfl_up_sync(0xffffffffu, incl, o);
+                        if (te >= o) incl += y;
+                    }
+                    tb[2 * te] = incl - pair + g0;
+                    tb[2 * te + 1] = incl;
+                }
+                epi_sync();
+                if (te < kC) {
+                    const float last = tb[L - 1];
+                    tb[kC + te] = exp2f(tb[te]);
+                    tb[2 * kC + te] = te < L ? exp2f(last - tb[te]) : 0.f;
+                    if (te == 0) tb[3 * kC] = exp2f(last);
+                }
+            } else {
+                if (te < kC) {
+                    tb[kC + te] = pow_int_log2(lg, te + 1);
+                    tb[2 * kC + te] = te < L ? pow_int_log2(lg, L - 1 - te) : 0.f;
+                    if (te == 0) tb[3 * kC] = pow_int_log2(lg, L);
+                }
+            }
+            epi_sync();
+        };
+
+        bool ok = true;
+        // initial state: S_op = bf16(S_in), S = decay_0 * S_in (S_in = 0 if absent)
+        prepare(0);
+        {
+            const float dec0 = decf[3 * kC];
+            const float* sin = p.state_in ? p.state_in + ((size_t)bh * DK) * p.dv + dv0 + d : nullptr;
+#pragma unroll 1
+            for (int cb = 0; cb < DK / 32; ++cb) {
+                uint32_t w[32], h[16];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const float x = sin ? sin[(size_t)(cb * 32 + c) * p.dv] : 0.f;
+                    w[c] = __float_as_uint(x * dec0);
+                    if (c & 1) h[c >> 1] = pack_bf16(__uint_as_float(w[c - 1]) / (dec0 != 0.f ? 1.f : 1.f), 0.f);
+                }
+                // bf16 copy from the undecayed values
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    const float x0 = sin ? sin[(size_t)(cb * 32 + 2 * c) * p.dv] : 0.f;
+                    const float x1 = sin ? sin[(size_t)(cb * 32 + 2 * c + 1) * p.dv] : 0.f;
+                    h[c] = pack_bf16(x0, x1);
+                }
+                tmem_st32(tmem + lane_off + Lay::kColS + cb * 32, w);
+                tmem_st16(tmem + lane_off + Lay::kColSop + cb * 16, h);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            epi_sync();
+            if (te == 0) mbar_arrive(bar(kSReady));
+        }
+
+        for (int i = 0; i < nchunks && ok; ++i) {
+            const int s = i & 1;
+            const int t0 = i * kC;
+            const float* tb = decf + s * Lay::kDecFloats;
+            // ---------------- P = mask(Q K^T) in bf16, and zeta-scaled V
+            if (!mbar_wait(bar(kAFull), i & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            {
+                uint32_t a0[32], a1[32];
+                tmem_ld32(tmem + lane_off + Lay::kColA, a0);
+                tmem_ld32(tmem + lane_off + Lay::kColA + 32, a1);
+                tmem_wait_ld();
+                if (lane < 16) {
+                    const int j = quarter * 16 + lane;  // M=64 accumulator: row j sits in lane 32*(j/16) + j%16
+                    const float cj = GATED ? tb[j] : 0.f;
+                    uint8_t* prow = sm + Lay::kP + j * 128;
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) {
+                        uint32_t u[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            float pv[2];
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                const int m = cc * 8 + e * 2 + h;
+                                const float a = __uint_as_float(m < 32 ? a0[m & 31] : a1[m & 31]);
+                                float w;
+                                if (m > j) w = 0.f;
+                                else if (m == j) w = 1.f;
+                                else w = GATED ? exp2f(cj - tb[m]) : exp2f(lg * (float)(j - m));
+                                pv[h] = a * w;
+                            }
+                            u[e] = pack_bf16(pv[0], pv[1]);
+                        }
+                        *reinterpret_cast<uint4*>(prow + ((cc ^ (j & 7)) << 4)) = make_uint4(u[0], u[1], u[2], u[3]);
+                    }
+                }
+                // zeta-scaled copy of the V tile (swizzle permutes 16-byte chunks inside a row only)
+                const uint8_t* vt = sm + Lay::kStage0 + s * Lay::kStageBytes + Lay::kQBytes + Lay::kKBytes;
+                uint8_t* zv = sm + Lay::kZV;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int ci = e * kEpiThreads + te;
+                    const int m = (ci & 511) >> 3;
+                    const float z = tb[2 * kC + m];
+                    uint4 x = *reinterpret_cast<const uint4*>(vt + ci * 16);
+                    float2 f;
+                    f = unpack_bf16(x.x); x.x = pack_bf16(f.x * z, f.y * z);
+                    f = unpack_bf16(x.y); x.y = pack_bf16(f.x * z, f.y * z);
+                    f = unpack_bf16(x.z); x.z = pack_bf16(f.x * z, f.y * z);
+                    f = unpack_bf16(x.w); x.w = pack_bf16(f.x * z, f.y * z);
+                    *reinterpret_cast<uint4*>(zv + ci * 16) = x;
+                }
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            epi_sync();
+            if (te == 0) mbar_arrive(bar(kPReady));
+
+            // ---------------- O = O_intra + r_j O_inter -> bf16 -> TMA store
+            if (!mbar_wait(bar(kOFull), i & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            if (te == 0) tma_store_wait_read();  // previous chunk's store has read the staging tile
+            epi_sync();
+            {
+                uint8_t* ost = sm + Lay::kOst + (d >> 6) * kTile64 + (d & 63) * 2;
+#pragma unroll
+                for (int jb = 0; jb < 2; ++jb) {
+                    uint32_t oi[32], oe[32];
+                    tmem_ld32(tmem + lane_off + Lay::kColO + jb * 32, oi);
+                    tmem_ld32(tmem + lane_off + Lay::kColA + jb * 32, oe);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) {
+                        const int j = jb * 32 + jj;
+                        const float o = fmaf(tb[kC + j], __uint_as_float(oe[jj]), __uint_as_float(oi[jj]));
+                        *reinterpret_cast<__nv_bfloat16*>(ost + j * 128) = __float2bfloat16_rn(o);
+                    }
+                }
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            epi_sync();
+            if (te == 0) {
+                mbar_arrive(bar(kOFree));
+                tma_store_3d(&tm_o, dv0, t0, bh, sbase + Lay::kOst);
+                tma_store_3d(&tm_o, dv0 + 64, t0, bh, sbase + Lay::kOst + kTile64);
+                tma_store_commit();
+            }
+
+            // ---------------- state: S_op = bf16(S_i); S = decay_{i+1} S_i (or write state_out)
+            const bool last = (i == nchunks - 1);
+            if (!last) prepare(i + 1);
+            if (!mbar_wait(bar(kSFull), i & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            if (last) {
+                if (p.state_out) {
+                    float* so = p.state_out + ((size_t)bh * DK) * p.dv + dv0 + d;
+#pragma unroll 1
+                    for (int cb = 0; cb < DK / 32; ++cb) {
+                        uint32_t w[32];
+                        tmem_ld32(tmem + lane_off + Lay::kColS + cb * 32, w);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) so[(size_t)(cb * 32 + c) * p.dv] = __uint_as_float(w[c]);
+                    }
+                }
+            } else {
+                const float dn = decf[((i + 1) & 1) * Lay::kDecFloats + 3 * kC];
+#pragma unroll 1
+                for (int cb = 0; cb < DK / 32; ++cb) {
+                    uint32_t w[32], h[16];
+                    tmem_ld32(tmem + lane_off + Lay::kColS + cb * 32, w);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 16; ++c)
+                        h[c] = pack_bf16(__uint_as_float(w[2 * c]), __uint_as_float(w[2 * c + 1]));
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(__uint_as_float(w[c]) * dn);
+                    tmem_st16(tmem + lane_off + Lay::kColSop + cb * 16, h);
+                    tmem_st32(tmem + lane_off + Lay::kColS + cb * 32, w);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                epi_sync();
+                if (te == 0) mbar_arrive(bar(kSReady));
+            }
+        }
+        if (te == 0) tma_store_wait_all();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(Lay::kTmemCols)
+                     : "memory");
+    }
+}
+
+// ------------------------------------------------------------------ host side
+
+inline bool tc_device_ok() {
+    static int cached = -1;
+    if (cached < 0) {
+        int dev = 0, major = 0, minor = 0;
+        cached = (cudaGetDevice(&dev) == cudaSuccess &&
+                  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess &&
+                  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) == cudaSuccess &&
+                  major == 10 && minor == 0) ? 1 : 0;
+    }
+    return cached == 1;
+}
+
+inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 3D bf16 map over [BH][N][inner] with a 64 x 64 box.
+inline bool make_map(CUtensorMap* m, const void* base, int inner, int N, int BH, bool swizzle) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)N, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)inner * 2 * N};
+    cuuint32_t box[3] = {64, 64, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace tc
+
+inline bool tc_chunk_supported(int dk, int dv, int chunk, bool bf16) {
+    return bf16 && (dk == 64 || dk == 128 || dk == 256) && dv % tc::kDvS == 0 && chunk % tc::kC == 0 &&
+           tc::tc_device_ok();
+}
+
+inline int tc_chunk_launches(int, int, int, int, int) { return 1; }
+
+template <int DK, bool GATED>
+ret_status tc_chunk_launch_dk(const void* q, const void* k, const void* v, const float* decay, void* o,
+                              const float* state_in, float* state_out, int B, int H, int N, int dv,
+                              cudaStream_t st) {
+    using Lay = tc::Layout<DK>;
+    const int BH = B * H;
+    CUtensorMap mq, mk, mv, mo;
+    if (!tc::make_map(&mq, q, DK, N, BH, true) || !tc::make_map(&mk, k, DK, N, BH, true) ||
+        !tc::make_map(&mv, v, dv, N, BH, true) || !tc::make_map(&mo, o, dv, N, BH, false))
+        return RET_ERR_CUDA;
+    auto kern = tc::chunk_tc_kernel<DK, GATED>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kSmemAlloc) != cudaSuccess)
+        return RET_ERR_CUDA;
+    tc::Params prm{decay, state_in, state_out, H, N, dv};
+    dim3 grid(dv / tc::kDvS, BH);
+    kern<<<grid, tc::kThreads, Lay::kSmemAlloc, st>>>(mq, mk, mv, mo, prm);
+    return cudaGetLastError() == cudaSuccess ? RET_OK : RET_ERR_CUDA;
+}
+
+template <bool GATED>
+ret_status tc_chunk_launch(const void* q, const void* k, const void* v, const float* decay, void* o,
+                           const float* state_in, float* state_out, int B, int H, int N, int dk, int dv,
+                           cudaStream_t st) {
+    switch (dk) {
+        case 64: return tc_chunk_launch_dk<64, GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dv, st);
+        case 128: return tc_chunk_launch_dk<128, GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dv, st);
+        case 256: return tc_chunk_launch_dk<256, GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dv, st);
+    }
+    return RET_ERR_UNSUPPORTED;
+}
+
+}  // namespace ret

@@ -1,0 +1,158 @@
+"""Thin Python binding of libret.so, the C ABI declared in include/ret.h.
+
+Argument marshalling only: shape and dtype checks, output allocation with
+torch (device memory is plumbing), and the call through ctypes. Every step of
+retention runs in the library's CUDA kernels; there is no fallback. If the
+library is missing, load() raises.
+
+Names match the C ABI: ret_parallel, ret_chunkwise, ret_recurrent_step,
+gated_ret_chunkwise. Tensors are CUDA, contiguous, heads leading:
+q, k [B, H, N, dk]; v [B, H, N, dv]; gamma [H] fp32; g [B, H, N] fp32;
+state [B, H, dk, dv] fp32. q, k, v share one dtype (float32 or bfloat16).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libret.so")
+
+RET_F32, RET_BF16 = 0, 1
+STATUS = {0: "RET_OK", 1: "RET_ERR_NULL", 2: "RET_ERR_SHAPE", 3: "RET_ERR_DTYPE", 4: "RET_ERR_UNSUPPORTED",
+          5: "RET_ERR_CUDA", 6: "RET_ERR_TIMEOUT", 7: "RET_ERR_ALIGN"}
+# every symbol include/ret.h declares
+SYMBOLS = ("ret_parallel", "ret_chunkwise", "ret_recurrent_step", "gated_ret_chunkwise", "ret_status_str",
+           "ret_last_device_error", "ret_chunkwise_path", "ret_chunkwise_launches", "ret_version")
+
+_lock = threading.Lock()
+_lib = None
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+
+
+class RetError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn}: {STATUS.get(code, code)} ({msg})")
+        self.code = code
+
+
+def load(path: str | None = None) -> ctypes.CDLL:
+    """Load libret.so (built in-tree by linear_attention_ret_b200.build)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise RuntimeError(f"libret.so not found at {p}: build it with "
+                               "`python -m linear_attention_ret_b200.build`")
+        lib = ctypes.CDLL(p)
+        lib.ret_parallel.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]
+        lib.ret_chunkwise.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
+        lib.gated_ret_chunkwise.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
+        lib.ret_recurrent_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
+        for fn in ("ret_parallel", "ret_chunkwise", "gated_ret_chunkwise", "ret_recurrent_step"):
+            getattr(lib, fn).restype = _i
+        lib.ret_status_str.argtypes = [_i]
+        lib.ret_status_str.restype = ctypes.c_char_p
+        lib.ret_last_device_error.argtypes = [_vp]
+        lib.ret_last_device_error.restype = _i
+        lib.ret_chunkwise_path.argtypes = [_i, _i, _i, _i]
+        lib.ret_chunkwise_path.restype = _i
+        lib.ret_chunkwise_launches.argtypes = [_i, _i, _i, _i, _i, _i, _i]
+        lib.ret_chunkwise_launches.restype = _i
+        lib.ret_version.argtypes = []
+        lib.ret_version.restype = ctypes.c_char_p
+        _lib = lib
+        return lib
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise RetError(fn, code, load().ret_status_str(code).decode())
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return RET_F32
+    if t.dtype == torch.bfloat16:
+        return RET_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def ret_parallel(q, k, v, gamma, o=None, stream=None):
+    """O = (Q K^T (.) D) V. Returns o [B, H, N, dv] (dtype of q)."""
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    o = torch.empty(B, H, N, dv, dtype=q.dtype, device=q.device) if o is None else o
+    _cuda(q, k, v, gamma, o)
+    _check("ret_parallel", load().ret_parallel(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(o),
+                                               B, H, N, dk, dv, _dt(q), _stream(stream)))
+    return o
+
+
+def ret_chunkwise(q, k, v, gamma, chunk, state_in=None, state_out=None, o=None, stream=None):
+    """Chunkwise retention. Returns o; writes the final state into state_out if given."""
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    o = torch.empty(B, H, N, dv, dtype=q.dtype, device=q.device) if o is None else o
+    _cuda(q, k, v, gamma, o, state_in, state_out)
+    _check("ret_chunkwise", load().ret_chunkwise(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(o),
+                                                 _ptr(state_in), _ptr(state_out), B, H, N, dk, dv, int(chunk),
+                                                 _dt(q), _stream(stream)))
+    return o
+
+
+def gated_ret_chunkwise(q, k, v, g, chunk, state_in=None, state_out=None, o=None, stream=None):
+    """Gated chunkwise retention (per-token log-decay g). Returns o."""
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    o = torch.empty(B, H, N, dv, dtype=q.dtype, device=q.device) if o is None else o
+    _cuda(q, k, v, g, o, state_in, state_out)
+    _check("gated_ret_chunkwise", load().gated_ret_chunkwise(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(o),
+                                                             _ptr(state_in), _ptr(state_out), B, H, N, dk, dv,
+                                                             int(chunk), _dt(q), _stream(stream)))
+    return o
+
+
+def ret_recurrent_step(q, k, v, gamma, state, o=None, stream=None):
+    """One decode step; updates state [B, H, dk, dv] in place and returns o [B, H, dv]."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    o = torch.empty(B, H, dv, dtype=q.dtype, device=q.device) if o is None else o
+    _cuda(q, k, v, gamma, state, o)
+    _check("ret_recurrent_step", load().ret_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(state),
+                                                           _ptr(o), B, H, dk, dv, _dt(q), _stream(stream)))
+    return o
+
+
+def last_device_error(stream=None) -> int:
+    return int(load().ret_last_device_error(_stream(stream)))
+
+
+def chunkwise_launches(B: int, H: int, N: int, dk: int, dv: int, chunk: int, dtype: torch.dtype) -> int:
+    return int(load().ret_chunkwise_launches(B, H, N, dk, dv, chunk, RET_BF16 if dtype == torch.bfloat16 else RET_F32))
+
+
+def chunkwise_path(dk: int, dv: int, chunk: int, dtype: torch.dtype) -> int:
+    return int(load().ret_chunkwise_path(dk, dv, chunk, RET_BF16 if dtype == torch.bfloat16 else RET_F32))

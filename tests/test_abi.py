@@ -1,0 +1,76 @@
+"""The C ABI library builds, loads without a GPU, exports every declared symbol,
+and rejects bad arguments on the host before anything is launched."""
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ret.h")
+
+
+def _declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"RET_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from linear_attention_ret_b200 import build, ret
+    build.build()
+    return ret.load()
+
+
+def test_header_declares_the_four_entry_points():
+    syms = _declared_symbols()
+    for name in ("ret_parallel", "ret_chunkwise", "ret_recurrent_step", "gated_ret_chunkwise"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from linear_attention_ret_b200 import ret
+    syms = _declared_symbols()
+    assert set(syms) == set(ret.SYMBOLS)
+    for name in syms:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code in range(8):
+        assert lib.ret_status_str(code)
+    assert lib.ret_status_str(99) == b"unknown status"
+    assert lib.ret_version() == b"0.1.0"
+
+
+def test_path_selection(lib):
+    from linear_attention_ret_b200.ret import RET_BF16, RET_F32
+    assert lib.ret_chunkwise_path(32, 32, 32, RET_F32) == 0
+    assert lib.ret_chunkwise_path(512, 64, 64, RET_BF16) == -1   # dk above 256
+    assert lib.ret_chunkwise_path(64, 64, 0, RET_BF16) == -1
+    assert lib.ret_chunkwise_path(64, 64, 64, 7) == -1
+
+
+def _call_chunkwise(lib, fn="ret_chunkwise", B=1, H=1, N=8, dk=64, dv=64, chunk=64, dt=1, ptr=None):
+    p = ptr
+    return getattr(lib, fn)(p, p, p, p, p, None, None, B, H, N, dk, dv, chunk, dt, None)
+
+
+@pytest.mark.parametrize("fn", ["ret_chunkwise", "gated_ret_chunkwise"])
+def test_chunkwise_validation(lib, fn):
+    # shape errors come first, then unsupported sizes, then null pointers: no launch in any case
+    assert _call_chunkwise(lib, fn, B=0) == 2
+    assert _call_chunkwise(lib, fn, N=-1) == 2
+    assert _call_chunkwise(lib, fn, chunk=0) == 2
+    assert _call_chunkwise(lib, fn, dt=5) == 3
+    assert _call_chunkwise(lib, fn, dk=300) == 4
+    assert _call_chunkwise(lib, fn, B=70000) == 4
+    assert _call_chunkwise(lib, fn) == 1  # NULL q, k, v
+
+
+def test_parallel_and_step_validation(lib):
+    assert lib.ret_parallel(None, None, None, None, None, 1, 1, 4, 2000, 8, 0, None) == 4
+    assert lib.ret_parallel(None, None, None, None, None, 1, 1, 4, 8, 8, 0, None) == 1
+    assert lib.ret_parallel(None, None, None, None, None, 1, 0, 4, 8, 8, 0, None) == 2
+    assert lib.ret_recurrent_step(None, None, None, None, None, None, 1, 1, 8, 8, 0, None) == 1
+    assert lib.ret_recurrent_step(None, None, None, None, None, None, 1, 1, 5000, 8, 0, None) == 4
+    assert lib.ret_recurrent_step(None, None, None, None, None, None, 1, 1, 8, 8, 2, None) == 3

@@ -1,0 +1,241 @@
+"""GPU parity: the CUDA library (through its C ABI) against the fp64 oracle.
+
+Small cases compare every output element; the full-size workloads run in the
+same launch configuration as bench.py and are compared on sampled heads, each
+of which the oracle computes independently (heads do not interact).
+"""
+import numpy as np
+import pytest
+import torch
+
+from linear_attention_ret_b200 import inputs as I
+from oracle import oracle as O
+from tests.parity import TOL_BF16, TOL_F32, assert_close, rel_l2, tol_for
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _dev(*ts):
+    return [None if t is None else t.to(DEV).contiguous() for t in ts]
+
+
+def _rand_inputs(B, H, N, dk, dv, dtype, seed):
+    return I.qkv(B, H, N, dk, dv, dtype, seed=seed)
+
+
+# ------------------------------------------------------------------ tiny fp32 config, all forms
+
+def test_tiny_config_all_forms(cuda_lib):
+    cfg = I.CONFIGS["tiny"]
+    x = I.config_inputs(cfg)
+    q, k, v, gam = _dev(x["q"], x["k"], x["v"], x["gamma"])
+    # parallel form
+    o_par = cuda_lib.ret_parallel(q, k, v, gam)
+    assert_close(o_par, O.ret_parallel(x["q"], x["k"], x["v"], x["gamma"]), torch.float32, "parallel")
+    # chunkwise form, chunk 32, with the final state
+    s_out = torch.empty(cfg.B, cfg.H, cfg.dk, cfg.dv, device=DEV)
+    o_chk = cuda_lib.ret_chunkwise(q, k, v, gam, cfg.chunk, state_out=s_out)
+    want_o, want_s = O.ret_chunkwise(x["q"], x["k"], x["v"], x["gamma"], cfg.chunk)
+    assert_close(o_chk, want_o, torch.float32, "chunkwise")
+    assert_close(s_out, want_s, torch.float32, "chunkwise state")
+    # recurrent form: N single-token steps from a zero state
+    S = torch.zeros(cfg.B, cfg.H, cfg.dk, cfg.dv, device=DEV)
+    outs = [cuda_lib.ret_recurrent_step(q[:, :, t].contiguous(), k[:, :, t].contiguous(),
+                                        v[:, :, t].contiguous(), gam, S) for t in range(cfg.N)]
+    o_rec = torch.stack(outs, dim=2)
+    want_rec, want_srec = O.ret_recurrent(x["q"], x["k"], x["v"], x["gamma"])
+    assert_close(o_rec, want_rec, torch.float32, "recurrent")
+    assert_close(S, want_srec, torch.float32, "recurrent state")
+    assert cuda_lib.last_device_error() == 0
+
+
+# ------------------------------------------------------------------ chunkwise, small shapes, all elements
+
+CHUNK_CASES = [
+    # B, H, N, dk, dv, chunk, dtype
+    (1, 4, 77, 48, 40, 16, torch.float32),    # ragged tail, odd dims
+    (2, 2, 130, 32, 96, 64, torch.float32),
+    (1, 2, 150, 64, 96, 32, torch.bfloat16),  # CUDA-core bf16
+    (2, 3, 200, 64, 128, 64, torch.bfloat16),
+    (1, 2, 257, 128, 256, 64, torch.bfloat16),
+    (1, 2, 320, 256, 128, 128, torch.bfloat16),
+    (1, 1, 64, 256, 512, 64, torch.bfloat16),
+    (1, 2, 1, 64, 128, 64, torch.bfloat16),    # single token
+]
+
+
+def _gammas_with_edges(H):
+    base = [0.0, 0.5, 0.96875, 1.0, 0.9, 0.999]
+    return torch.tensor([base[h % len(base)] for h in range(H)], dtype=torch.float32)
+
+
+@pytest.mark.parametrize("B,H,N,dk,dv,chunk,dtype", CHUNK_CASES)
+def test_chunkwise_matches_oracle(cuda_lib, B, H, N, dk, dv, chunk, dtype):
+    q, k, v = _rand_inputs(B, H, N, dk, dv, dtype, seed=N + dk)
+    gam = _gammas_with_edges(H)
+    S0 = torch.randn(B, H, dk, dv, generator=torch.Generator().manual_seed(3)) * 0.05
+    qd, kd, vd, gd, S0d = _dev(q, k, v, gam, S0)
+    s_out = torch.empty_like(S0d)
+    o = cuda_lib.ret_chunkwise(qd, kd, vd, gd, chunk, state_in=S0d, state_out=s_out)
+    want_o, want_s = O.ret_chunkwise(q, k, v, gam, chunk, state_in=S0)
+    assert_close(o, want_o, dtype, "o")
+    assert_close(s_out, want_s, dtype, "state")
+
+
+@pytest.mark.parametrize("B,H,N,dk,dv,chunk,dtype", CHUNK_CASES)
+def test_gated_chunkwise_matches_oracle(cuda_lib, B, H, N, dk, dv, chunk, dtype):
+    gen = torch.Generator().manual_seed(N * 7 + dv)
+    q, k, v = I.qkv(B, H, N, dk, dv, dtype, gen=gen)
+    g = I.gate(B, H, N, gen) * 4.0  # stronger decay than the workload, to exercise the weights
+    S0 = torch.randn(B, H, dk, dv, generator=gen) * 0.05
+    qd, kd, vd, gdv, S0d = _dev(q, k, v, g, S0)
+    s_out = torch.empty_like(S0d)
+    o = cuda_lib.gated_ret_chunkwise(qd, kd, vd, gdv, chunk, state_in=S0d, state_out=s_out)
+    want_o, want_s = O.gated_chunkwise(q, k, v, g, chunk, state_in=S0)
+    assert_close(o, want_o, dtype, "o")
+    assert_close(s_out, want_s, dtype, "state")
+
+
+def test_chunkwise_no_state_and_in_place_state(cuda_lib):
+    B, H, N, dk, dv = 2, 2, 96, 64, 128
+    q, k, v = _rand_inputs(B, H, N, dk, dv, torch.bfloat16, seed=11)
+    gam = I.gammas(H)
+    qd, kd, vd, gd = _dev(q, k, v, gam)
+    o = cuda_lib.ret_chunkwise(qd, kd, vd, gd, 64)
+    assert_close(o, O.ret_chunkwise(q, k, v, gam, 64)[0], torch.bfloat16, "no state")
+    # state_in == state_out (in place)
+    S0 = torch.randn(B, H, dk, dv, generator=torch.Generator().manual_seed(2)) * 0.05
+    S = S0.to(DEV)
+    o2 = cuda_lib.ret_chunkwise(qd, kd, vd, gd, 64, state_in=S, state_out=S)
+    want_o, want_s = O.ret_chunkwise(q, k, v, gam, 64, state_in=S0)
+    assert_close(o2, want_o, torch.bfloat16, "in-place o")
+    assert_close(S, want_s, torch.bfloat16, "in-place state")
+
+
+def test_chunkwise_split_sequence_matches_whole(cuda_lib):
+    """Prefill in two calls, passing the state, equals one call over the whole sequence."""
+    B, H, N, dk, dv, n1 = 1, 4, 300, 128, 128, 128
+    q, k, v = _rand_inputs(B, H, N, dk, dv, torch.bfloat16, seed=21)
+    gam = I.gammas(H)
+    qd, kd, vd, gd = _dev(q, k, v, gam)
+    S = torch.empty(B, H, dk, dv, device=DEV)
+    o1 = cuda_lib.ret_chunkwise(qd[:, :, :n1].contiguous(), kd[:, :, :n1].contiguous(),
+                                vd[:, :, :n1].contiguous(), gd, 64, state_out=S)
+    o2 = cuda_lib.ret_chunkwise(qd[:, :, n1:].contiguous(), kd[:, :, n1:].contiguous(),
+                                vd[:, :, n1:].contiguous(), gd, 64, state_in=S, state_out=S)
+    want_o, want_s = O.ret_chunkwise(q, k, v, gam, 64)
+    assert_close(torch.cat([o1, o2], dim=2), want_o, torch.bfloat16, "split o")
+    assert_close(S, want_s, torch.bfloat16, "split state")
+
+
+def test_empty_sequence_passes_state_through(cuda_lib):
+    B, H, dk, dv = 1, 2, 64, 128
+    q = torch.empty(B, H, 0, dk, dtype=torch.bfloat16, device=DEV)
+    v = torch.empty(B, H, 0, dv, dtype=torch.bfloat16, device=DEV)
+    gam = I.gammas(H).to(DEV)
+    S0 = torch.randn(B, H, dk, dv, device=DEV)
+    S1 = torch.full_like(S0, 7.0)
+    cuda_lib.ret_chunkwise(q, q, v, gam, 64, state_in=S0, state_out=S1)
+    torch.cuda.synchronize()
+    assert torch.equal(S0, S1)
+    cuda_lib.ret_chunkwise(q, q, v, gam, 64, state_out=S1)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(S1) == 0
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_parallel_matches_oracle(cuda_lib, dtype):
+    B, H, N, dk, dv = 2, 3, 100, 40, 72
+    q, k, v = _rand_inputs(B, H, N, dk, dv, dtype, seed=5)
+    gam = _gammas_with_edges(H)
+    o = cuda_lib.ret_parallel(*_dev(q, k, v, gam))
+    assert_close(o, O.ret_parallel(q, k, v, gam), dtype, "parallel")
+
+
+def test_gamma_special_cases_on_gpu(cuda_lib):
+    """gamma = 0 gives o_n = (q_n . k_n) v_n; gamma = 1 gives the undecayed prefix sum."""
+    B, H, N, dk, dv = 1, 2, 70, 64, 128
+    q, k, v = _rand_inputs(B, H, N, dk, dv, torch.float32, seed=9)
+    qn, kn, vn = (t.double().numpy() for t in (q, k, v))
+    gam = torch.tensor([0.0, 1.0])
+    o = cuda_lib.ret_chunkwise(*_dev(q, k, v, gam), 16).cpu().double().numpy()
+    want0 = np.einsum("nd,nd->n", qn[0, 0], kn[0, 0])[:, None] * vn[0, 0]
+    kv = np.cumsum(np.einsum("nd,ne->nde", kn[0, 1], vn[0, 1]), axis=0)
+    want1 = np.einsum("nd,nde->ne", qn[0, 1], kv)
+    assert rel_l2(o[0, 0], want0) < TOL_F32
+    assert rel_l2(o[0, 1], want1) < TOL_F32
+
+
+# ------------------------------------------------------------------ decode step
+
+@pytest.mark.parametrize("dtype,dv", [(torch.float32, 128), (torch.bfloat16, 512), (torch.float32, 30)])
+def test_recurrent_step_matches_oracle(cuda_lib, dtype, dv):
+    B, H, dk = 3, 4, 64
+    gam = I.gammas(H, "h/3")
+    S0 = I.decode_state(B, H, dk, dv, seed=1)
+    Sd = S0.to(DEV)
+    S_ref = S0.double().numpy()
+    for step in range(5):
+        q, k, v = I.decode_step_inputs(B, H, dk, dv, step, dtype=dtype)
+        o = cuda_lib.ret_recurrent_step(*_dev(q, k, v, gam), Sd)
+        want_o, S_ref = O.ret_recurrent_step(q, k, v, gam, S_ref)
+        assert_close(o, want_o, dtype, f"o step {step}")
+    assert_close(Sd, S_ref, dtype, "state")
+
+
+# ------------------------------------------------------------------ full-size workloads, sampled heads
+
+def _head(x, b, h):
+    return x[b:b + 1, h:h + 1].contiguous()
+
+
+@pytest.mark.parametrize("name", ["retnet_1p3b", "retnet_6p7b_long", "gated"])
+def test_full_size_workload_sampled_heads(cuda_lib, name):
+    cfg = I.CONFIGS[name]
+    x = I.config_inputs(cfg)
+    gated = "g" in x
+    dev = {key: val.to(DEV) for key, val in x.items()}
+    s_out = torch.empty(cfg.B, cfg.H, cfg.dk, cfg.dv, device=DEV)
+    if gated:
+        o = cuda_lib.gated_ret_chunkwise(dev["q"], dev["k"], dev["v"], dev["g"], cfg.chunk, state_out=s_out)
+    else:
+        o = cuda_lib.ret_chunkwise(dev["q"], dev["k"], dev["v"], dev["gamma"], cfg.chunk, state_out=s_out)
+    torch.cuda.synchronize()
+    assert cuda_lib.last_device_error() == 0
+    assert torch.isfinite(o).all()
+    samples = [(0, 0), (cfg.B - 1, cfg.H - 1), (cfg.B // 2, cfg.H // 2)]
+    for b, h in samples:
+        q, k, v = (_head(x[n], b, h) for n in ("q", "k", "v"))
+        if gated:
+            want_o, want_s = O.gated_chunkwise(q, k, v, _head(x["g"], b, h), cfg.chunk)
+        else:
+            want_o, want_s = O.ret_chunkwise(q, k, v, x["gamma"][h:h + 1], cfg.chunk)
+        assert_close(o[b:b + 1, h:h + 1], want_o, cfg.dtype, f"{name} head ({b},{h})")
+        assert_close(s_out[b:b + 1, h:h + 1], want_s, cfg.dtype, f"{name} state ({b},{h})")
+
+
+def test_full_size_decode_sampled_heads(cuda_lib):
+    cfg = I.CONFIGS["decode"]
+    B, H, dk, dv = cfg.B, cfg.H, cfg.dk, cfg.dv
+    gam = I.gammas(H, cfg.gamma_schedule)
+    S0 = I.decode_state(B, H, dk, dv)
+    Sd = S0.to(DEV)
+    gd = gam.to(DEV)
+    samples = [(0, 0), (B - 1, H - 1), (31, 7)]
+    S_ref = {s: S0[s[0]:s[0] + 1, s[1]:s[1] + 1].double().numpy() for s in samples}
+    got = {s: [] for s in samples}
+    want = {s: [] for s in samples}
+    for step in range(I.DECODE_STEPS):
+        q, k, v = I.decode_step_inputs(B, H, dk, dv, step)
+        o = cuda_lib.ret_recurrent_step(*_dev(q, k, v), gd, Sd)
+        for (b, h) in samples:
+            got[(b, h)].append(o[b, h].float().cpu())
+            sl = (slice(b, b + 1), slice(h, h + 1))
+            ow, S_ref[(b, h)] = O.ret_recurrent_step(q[sl], k[sl], v[sl], gam[h:h + 1], S_ref[(b, h)])
+            want[(b, h)].append(ow[0, 0])
+    assert cuda_lib.last_device_error() == 0
+    for s in samples:
+        assert rel_l2(torch.stack(got[s]), np.stack(want[s])) <= TOL_BF16, s
+        assert rel_l2(Sd[s[0], s[1]], S_ref[s][0, 0]) <= TOL_BF16, s
