@@ -404,6 +404,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             epi_sync();
         };
 
+        // Every epilogue thread reaches the named barrier whatever its wait returned;
+        // the abort decision after it is uniform, so no thread is left at a barrier.
+        auto epi_wait = [&](int b, uint32_t parity) {
+            mbar_wait(bar(b), parity, abort_flag);
+            epi_sync();
+            return *abort_flag == 0;
+        };
+
         bool ok = true;
         // initial state: S_op = bf16(S_in), S = decay_0 * S_in (S_in = 0 if absent)
         prepare(0);
@@ -414,18 +422,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int cb = 0; cb < DK / 32; ++cb) {
                 uint32_t w[32], h[16];
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const float x = sin ? sin[(size_t)(cb * 32 + c) * p.dv] : 0.f;
-                    w[c] = __float_as_uint(x * dec0);
-                    if (c & 1) h[c >> 1] = pack_bf16(__uint_as_float(w[c - 1]) / (dec0 != 0.f ? 1.f : 1.f), 0.f);
-                }
-                // bf16 copy from the undecayed values
+                for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(sin ? sin[(size_t)(cb * 32 + c) * p.dv] : 0.f);
+                // bf16 copy of the undecayed state (operand of the first cross term), then decay_0 * S_in
 #pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    const float x0 = sin ? sin[(size_t)(cb * 32 + 2 * c) * p.dv] : 0.f;
-                    const float x1 = sin ? sin[(size_t)(cb * 32 + 2 * c + 1) * p.dv] : 0.f;
-                    h[c] = pack_bf16(x0, x1);
-                }
+                for (int c = 0; c < 16; ++c)
+                    h[c] = pack_bf16(__uint_as_float(w[2 * c]), __uint_as_float(w[2 * c + 1]));
+#pragma unroll
+                for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(__uint_as_float(w[c]) * dec0);
                 tmem_st32(tmem + lane_off + Lay::kColS + cb * 32, w);
                 tmem_st16(tmem + lane_off + Lay::kColSop + cb * 16, h);
             }
@@ -440,7 +443,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const int t0 = i * kC;
             const float* tb = decf + s * Lay::kDecFloats;
             // ---------------- P = mask(Q K^T) in bf16, and zeta-scaled V
-            if (!mbar_wait(bar(kAFull), i & 1, abort_flag)) { ok = false; break; }
+            if (!epi_wait(kAFull, i & 1)) { ok = false; break; }
             tc_fence_after();
             {
                 uint32_t a0[32], a1[32];
@@ -495,10 +498,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (te == 0) mbar_arrive(bar(kPReady));
 
             // ---------------- O = O_intra + r_j O_inter -> bf16 -> TMA store
-            if (!mbar_wait(bar(kOFull), i & 1, abort_flag)) { ok = false; break; }
-            tc_fence_after();
             if (te == 0) tma_store_wait_read();  // previous chunk's store has read the staging tile
-            epi_sync();
+            if (!epi_wait(kOFull, i & 1)) { ok = false; break; }
+            tc_fence_after();
             {
                 uint8_t* ost = sm + Lay::kOst + (d >> 6) * kTile64 + (d & 63) * 2;
 #pragma unroll
@@ -528,7 +530,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // ---------------- state: S_op = bf16(S_i); S = decay_{i+1} S_i (or write state_out)
             const bool last = (i == nchunks - 1);
             if (!last) prepare(i + 1);
-            if (!mbar_wait(bar(kSFull), i & 1, abort_flag)) { ok = false; break; }
+            if (!epi_wait(kSFull, i & 1)) { ok = false; break; }
             tc_fence_after();
             if (last) {
                 if (p.state_out) {
