@@ -5,7 +5,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
-#include "../../include/ret.h"
+#include "ret.h"
 
 namespace ret {
 

@@ -13,15 +13,19 @@
 //   O_inter^T = S_op^T Q^T           M=128 N=64  K=dk  (TS: S_op = bf16 copy of the state, in TMEM)
 //   O_intra^T = V^T P^T              M=128 N=64  K=64  (SS, V read MN-major straight from the TMA tile)
 //   S^T      += (zeta V)^T K         M=128 N=dk  K=64  (SS, K read MN-major from the same TMA tile)
-// The fp32 state S^T lives in TMEM for the whole sequence. After each state
-// update the epilogue reads it once, writes its bf16 copy (the next chunk's
-// MMA operand) and writes back decay * S, so the next update accumulates onto
-// the decayed state. The decay mask is generated in registers.
+// The fp32 state lives in TMEM for the whole sequence as S = c T (c a scalar
+// kept in registers): each chunk the epilogue reads T once and writes the
+// bf16 copy of S (the next cross term's MMA operand); the update adds
+// (zeta V / c) onto T, and T is rescaled in place only when c would underflow.
+// The decay mask is generated in registers.
 //
-// Roles (192 threads): warp 0 issues TMA loads (two stages of Q, K, V tiles),
-// warp 1 allocates TMEM and issues every tcgen05.mma from one thread, warps 2-5
-// are the epilogue (TMEM lane quarter = warp index % 4). All waits are bounded:
-// on timeout the kernel sets the device error word, the roles stop, in-flight
+// Roles (320 threads): warp 0 issues TMA loads (two stages of Q, K, V tiles);
+// warp 1 allocates TMEM and issues every tcgen05.mma from one thread; warps 2-5
+// are the attention epilogue (mask P from Q K^T, combine and store O); warps
+// 6-9 are the state epilogue (zeta-scaled V into a double buffer, and the TMEM
+// round trip of the state). The two epilogue groups run concurrently; each
+// warp reads the TMEM lane quarter (warp index % 4). All waits are bounded: on
+// timeout the kernel sets the device error word, the roles stop, in-flight
 // copies and MMAs are drained (bounded again) and TMEM is released.
 #pragma once
 
@@ -35,8 +39,8 @@ namespace tc {
 
 constexpr int kC = 64;          // chunk rows per tile
 constexpr int kDvS = 128;       // dv columns per CTA (TMEM lanes)
-constexpr int kThreads = 192;
-constexpr int kEpiThreads = 128;
+constexpr int kThreads = 320;
+constexpr int kEpiThreads = 128;  // threads per epilogue group
 constexpr int kTile64 = kC * 128;  // one 64-row x 128-byte swizzled tile (8 KB)
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
 
@@ -48,13 +52,13 @@ struct Layout {
     static constexpr int kStageBytes = kQBytes + kKBytes + kVBytes;
     static constexpr int kStage0 = 0;
     static constexpr int kP = 2 * kStageBytes;              // P tile (64 x 64 bf16, SW128 K-major)
-    static constexpr int kZV = kP + kTile64;                // zeta-scaled V (same layout as the V tile)
-    static constexpr int kOst = kZV + kVBytes;              // O staging for the TMA store (no swizzle)
+    static constexpr int kZV = kP + kTile64;                // zeta-scaled V, two buffers (V tile layout)
+    static constexpr int kOst = kZV + 2 * kVBytes;          // O staging for the TMA store (128-byte swizzle)
     static constexpr int kBar = kOst + kVBytes;             // mbarriers
-    static constexpr int kNumBars = 12;
-    static constexpr int kDec = kBar + kNumBars * 8;        // decay tables, double-buffered by chunk parity
-    static constexpr int kDecFloats = 3 * kC + 4;           // cum | r | zeta | decay
-    static constexpr int kTmemSlot = kDec + 2 * kDecFloats * 4;
+    static constexpr int kNumBars = 14;
+    static constexpr int kAgTab = kBar + kNumBars * 8;      // attention group: cum[64] | r[64] | pw[68]
+    static constexpr int kSgTab = kAgTab + 196 * 4;         // state group: cum[64] | zeta[64] | decay
+    static constexpr int kTmemSlot = kSgTab + 132 * 4;
     static constexpr int kAbort = kTmemSlot + 4;
     static constexpr int kBytes = kAbort + 4;
     static constexpr int kSmemAlloc = kBytes + 1024;        // slack to align the base to 1024 B
@@ -66,10 +70,15 @@ struct Layout {
     static constexpr int kColsUsed = kColO + kC;
     static constexpr int kTmemCols = kColsUsed <= 256 ? 256 : 512;
     static_assert(kColsUsed <= 512, "TMEM overflow");
-    static_assert(kBytes + 1024 <= 227 * 1024, "shared memory overflow");
+    static_assert(kSmemAlloc <= 227 * 1024, "shared memory overflow");
 };
 
-enum Bar { kFull0 = 0, kFull1, kEmpty0, kEmpty1, kAFull, kPReady, kOFull, kOFree, kSFull, kSReady, kDrain };
+enum Bar {
+    kFull0 = 0, kFull1, kEmpty0, kEmpty1,  // TMA stages
+    kAFull, kPReady, kOFull, kOFree,       // attention epilogue <-> MMA
+    kSFull, kSReady, kZV0, kZV1,           // state epilogue <-> MMA
+    kDrain
+};
 
 // ------------------------------------------------------------------ PTX wrappers
 
@@ -132,18 +141,12 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
     }
 }
 
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Named barrier of one epilogue group (id 1: attention group, id 2: state group).
+__device__ __forceinline__ void group_sync(int id) { asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory"); }
 
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
-        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
-        : "memory");
-}
 
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, int x, int y, int z, uint32_t src) {
     asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3}], [%4];"
@@ -153,6 +156,14 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, int x, int 
 __device__ __forceinline__ void tma_store_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void tma_store_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
+
 
 // Shared-memory matrix descriptor, 128-byte swizzle (sm_100 format: start address,
 // leading and stride byte offsets in 16-byte units, version 1 at bit 46, layout 2 at bit 61).
@@ -194,6 +205,20 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
         "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
         "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+// 16 lanes x 2 halves: thread t gets lane (base + t % 16), columns c + 32 * (t / 16) .. +31.
+__device__ __forceinline__ void tmem_ld16x2(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], 32;"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
           "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
@@ -245,6 +270,20 @@ struct Params {
     int H, N, dv;
 };
 
+// In-chunk inclusive cumulative sum of the gate in log2 units, by one warp:
+// lane l holds g[2l], g[2l+1] (already scaled by log2(e)); writes cum[0..63].
+__device__ __forceinline__ void warp_cumsum64(float g0, float g1, int lane, float* cum) {
+    const float pair = g0 + g1;
+    float incl = pair;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    cum[2 * lane] = incl - pair + g0;
+    cum[2 * lane + 1] = incl;
+}
+
 template <int DK, bool GATED>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -280,6 +319,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const float* G = GATED ? p.decay_in + (size_t)bh * p.N : nullptr;
+    const float lg = GATED ? 0.f : log2f(p.decay_in[bh % p.H]);
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -315,16 +356,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             constexpr uint32_t id_up = idesc(128, DK, 1, 1);
             const uint32_t tA = tmem + Lay::kColA, tO = tmem + Lay::kColO;
             const uint32_t tS = tmem + Lay::kColS, tSop = tmem + Lay::kColSop;
-            const uint32_t sP = sbase + Lay::kP, sZV = sbase + Lay::kZV;
-            bool ok = true;
-            for (int i = 0; i < nchunks && ok; ++i) {
+            const uint32_t sP = sbase + Lay::kP;
+            for (int i = 0; i < nchunks; ++i) {
                 const int s = i & 1;
                 const uint32_t sQ = sbase + Lay::kStage0 + s * Lay::kStageBytes;
                 const uint32_t sK = sQ + Lay::kQBytes;
                 const uint32_t sV = sK + Lay::kKBytes;
-                ok = mbar_wait(bar(kFull0 + s), (i >> 1) & 1, abort_flag);
-                if (ok && i > 0) ok = mbar_wait(bar(kOFree), (i - 1) & 1, abort_flag);
-                if (!ok) break;
+                const uint32_t sZV = sbase + Lay::kZV + s * Lay::kVBytes;
+                if (!mbar_wait(bar(kFull0 + s), (i >> 1) & 1, abort_flag)) break;
+                if (i > 0 && !mbar_wait(bar(kOFree), (i - 1) & 1, abort_flag)) break;
                 tc_fence_after();
                 // A = Q K^T (both K-major, 128-byte swizzle; 16-element K steps)
 #pragma unroll
@@ -333,8 +373,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     mma_ss(tA, sdesc(sQ + off, 16, 1024), sdesc(sK + off, 16, 1024), id_qk, ks > 0);
                 }
                 mma_commit(bar(kAFull));
-                ok = mbar_wait(bar(kPReady), i & 1, abort_flag) && mbar_wait(bar(kSReady), i & 1, abort_flag);
-                if (!ok) break;
+                // The state update goes first: it needs only zeta V and the decayed state, so it
+                // runs while the epilogue builds P, and the O drain later has the pipe to itself.
+                if (!mbar_wait(bar(kZV0 + s), (i >> 1) & 1, abort_flag) || !mbar_wait(bar(kSReady), i & 1, abort_flag))
+                    break;
+                tc_fence_after();
+                // S^T += (zeta V)^T K: A = ZV MN-major, B = K tile MN-major (dk blocks 8 KB apart)
+#pragma unroll
+                for (int ks = 0; ks < kC / 16; ++ks)
+                    mma_ss(tS, sdesc(sZV + ks * 2048, kTile64, 1024), sdesc(sK + ks * 2048, kTile64, 1024), id_up, 1);
+                if (!mbar_wait(bar(kPReady), i & 1, abort_flag)) break;
                 tc_fence_after();
                 // O_inter^T = S_op^T Q^T: A from TMEM (bf16 pairs per column), B = Q tile K-major
 #pragma unroll
@@ -347,83 +395,231 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int ks = 0; ks < kC / 16; ++ks)
                     mma_ss(tO, sdesc(sV + ks * 2048, kTile64, 1024), sdesc(sP + ks * 32, 16, 1024), id_ov, ks > 0);
                 mma_commit(bar(kOFull));
-                // S^T += (zeta V)^T K: A = ZV MN-major, B = K tile MN-major (dk blocks 8 KB apart)
-#pragma unroll
-                for (int ks = 0; ks < kC / 16; ++ks)
-                    mma_ss(tS, sdesc(sZV + ks * 2048, kTile64, 1024), sdesc(sK + ks * 2048, kTile64, 1024), id_up, 1);
+                // S_i is final and the cross term has read S_op: the state epilogue may now
+                // overwrite S_op and decay S.
                 mma_commit(bar(kSFull));
                 mma_commit(bar(kEmpty0 + s));
             }
-            // make sure every issued MMA has completed before TMEM can be released
+            // every issued MMA must complete before TMEM can be released
             mma_commit(bar(kDrain));
             mbar_drain(bar(kDrain), 0);
         }
-    } else {
-        // ------------------------------------------------------------ epilogue (warps 2..5)
-        const int te = threadIdx.x - 64;             // 0..127
-        const int quarter = warp & 3;                // TMEM lane quarter this warp may access
-        const int d = quarter * 32 + lane;           // dv column (within the slice) = TMEM lane
+    } else if (warp < 6) {
+        // ------------------------------------------------------------ attention epilogue (warps 2..5)
+        const int te = threadIdx.x - 64;          // 0..127
+        const int quarter = warp & 3;             // TMEM lane quarter this warp may access
+        const int d = quarter * 32 + lane;        // dv column of the slice = TMEM lane
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        float* decf = reinterpret_cast<float*>(sm + Lay::kDec);
-        const float* G = GATED ? p.decay_in + (size_t)bh * p.N : nullptr;
-        const float lg = GATED ? 0.f : log2f(p.decay_in[bh % p.H]);
-
-        // decay tables of chunk c into buffer c & 1: cum (gated, log2 units), r, zeta, decay
-        auto prepare = [&](int c) {
-            float* tb = decf + (c & 1) * Lay::kDecFloats;
-            const int t0 = c * kC, L = min(kC, p.N - t0);
-            if (GATED) {
-                if (te < 32) {
-                    const int a = t0 + 2 * te;
-                    const float g0 = (a < p.N ? G[a] : 0.f) * kLog2e;
-                    const float g1 = (a + 1 < p.N ? G[a + 1] : 0.f) * kLog2e;
-                    const float pair = g0 + g1;
-                    float incl = pair;
-#pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) {
-                        const float y = __shfl_up_sync(0xffffffffu, incl, o);
-                        if (te >= o) incl += y;
-                    }
-                    tb[2 * te] = incl - pair + g0;
-                    tb[2 * te + 1] = incl;
-                }
-                epi_sync();
-                if (te < kC) {
-                    const float last = tb[L - 1];
-                    tb[kC + te] = exp2f(tb[te]);
-                    tb[2 * kC + te] = te < L ? exp2f(last - tb[te]) : 0.f;
-                    if (te == 0) tb[3 * kC] = exp2f(last);
-                }
-            } else {
-                if (te < kC) {
-                    tb[kC + te] = pow_int_log2(lg, te + 1);
-                    tb[2 * kC + te] = te < L ? pow_int_log2(lg, L - 1 - te) : 0.f;
-                    if (te == 0) tb[3 * kC] = pow_int_log2(lg, L);
-                }
-            }
-            epi_sync();
-        };
-
-        // Every epilogue thread reaches the named barrier whatever its wait returned;
-        // the abort decision after it is uniform, so no thread is left at a barrier.
-        auto epi_wait = [&](int b, uint32_t parity) {
+        float* cum = reinterpret_cast<float*>(sm + Lay::kAgTab);  // gated: in-chunk cumsum, log2 units
+        float* rr = cum + kC;                                     // cross-term row factor r_j
+        float* pw = rr + kC;                                      // fixed gamma: gamma^t, t = 0..64
+        auto wait_all = [&](int b, uint32_t parity) {  // every thread reaches the barrier; uniform result
             mbar_wait(bar(b), parity, abort_flag);
-            epi_sync();
+            group_sync(1);
             return *abort_flag == 0;
         };
+        if (!GATED) {
+            if (te <= kC) pw[te] = pow_int_log2(lg, te);
+            group_sync(1);
+            if (te < kC) rr[te] = pw[te + 1];
+        }
+        float g0 = 0.f, g1 = 0.f;  // gated: prefetched gate values of the next chunk (first warp)
+        if (GATED && te < 32) {
+            g0 = (2 * te < p.N ? G[2 * te] : 0.f) * kLog2e;
+            g1 = (2 * te + 1 < p.N ? G[2 * te + 1] : 0.f) * kLog2e;
+        }
+        for (int i = 0; i < nchunks; ++i) {
+            const int t0 = i * kC;
+            if (GATED) {
+                if (te < 32) {
+                    warp_cumsum64(g0, g1, lane, cum);
+                    const int a = t0 + kC + 2 * te;
+                    g0 = (a < p.N ? G[a] : 0.f) * kLog2e;
+                    g1 = (a + 1 < p.N ? G[a + 1] : 0.f) * kLog2e;
+                }
+                group_sync(1);
+                if (te < kC) rr[te] = exp2f(cum[te]);
+            }
+            // ---------------- P = mask(Q K^T) in bf16: row j, 32 columns per thread
+            if (!wait_all(kAFull, i & 1)) break;
+            tc_fence_after();
+            {
+                uint32_t a[32];
+                tmem_ld16x2(tmem + lane_off + Lay::kColA, a);
+                const int j = quarter * 16 + (lane & 15);  // M=64 accumulator: row j in lane 32*(j/16) + j%16
+                const int m0 = (lane >> 4) * 32;
+                // all table reads before any shared-memory store (the pointers may alias)
+                float w[32];
+                if (GATED) {
+                    const float cj = cum[j];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) w[c] = cj - cum[m0 + c];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const int m = m0 + c;
+                        w[c] = m > j ? 0.f : (m == j ? 1.f : exp2f(w[c]));
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const int m = m0 + c;
+                        w[c] = m > j ? 0.f : pw[j - m];
+                    }
+                }
+                tmem_wait_ld();
+                uint32_t u[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    u[c] = pack_bf16(__uint_as_float(a[2 * c]) * w[2 * c], __uint_as_float(a[2 * c + 1]) * w[2 * c + 1]);
+                uint8_t* prow = sm + Lay::kP + j * 128;
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    const int chunk16 = (m0 >> 3) + cc;
+                    *reinterpret_cast<uint4*>(prow + ((chunk16 ^ (j & 7)) << 4)) =
+                        make_uint4(u[4 * cc], u[4 * cc + 1], u[4 * cc + 2], u[4 * cc + 3]);
+                }
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            group_sync(1);
+            if (te == 0) {
+                mbar_arrive(bar(kPReady));
+                tma_store_wait_read();  // previous chunk's O store has read the staging tile
+            }
+            // ---------------- O = O_intra + r_j O_inter -> bf16 -> staging -> TMA store
+            if (!wait_all(kOFull, i & 1)) break;
+            tc_fence_after();
+            {
+                // Each thread owns dv column d for all 64 tokens. A lane-pair shuffle packs two
+                // adjacent dv columns into one 4-byte store: even lanes store token j, odd lanes
+                // token j + 4. With the 128-byte swizzle those two rows hit disjoint banks.
+                const bool odd = lane & 1;
+                const int cb = ((d & 63) & ~1) * 2;  // byte offset of the dv pair inside a 128-byte row
+                uint8_t* ost = sm + Lay::kOst + (d >> 6) * kTile64;
+#pragma unroll
+                for (int jb = 0; jb < 2; ++jb) {
+                    uint32_t oi[32], oe[32];
+                    tmem_ld32(tmem + lane_off + Lay::kColO + jb * 32, oi);
+                    tmem_ld32(tmem + lane_off + Lay::kColA + jb * 32, oe);
+                    float rv[32];
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) rv[jj] = rr[jb * 32 + jj];
+                    tmem_wait_ld();
+                    float o[32];
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) o[jj] = fmaf(rv[jj], __uint_as_float(oe[jj]), __uint_as_float(oi[jj]));
+                    uint32_t w[16];
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) {
+                        const int ja = 8 * (u >> 2) + (u & 3);  // token pair (ja, ja + 4) inside the block
+                        const float send = odd ? o[ja] : o[ja + 4];
+                        const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+                        w[u] = odd ? pack_bf16(recv, o[ja + 4]) : pack_bf16(o[ja], recv);
+                    }
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) {
+                        const int j = jb * 32 + 8 * (u >> 2) + (u & 3) + (odd ? 4 : 0);
+                        *reinterpret_cast<uint32_t*>(ost + j * 128 + ((((cb >> 4) ^ (j & 7)) << 4) | (cb & 15))) = w[u];
+                    }
+                }
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            group_sync(1);
+            if (te == 0) {
+                mbar_arrive(bar(kOFree));
+                tma_store_3d(&tm_o, dv0, t0, bh, sbase + Lay::kOst);
+                tma_store_3d(&tm_o, dv0 + 64, t0, bh, sbase + Lay::kOst + kTile64);
+                tma_store_commit();
+            }
+        }
+        if (te == 0) tma_store_wait_all();
+    } else {
+        // ------------------------------------------------------------ state epilogue (warps 6..9)
+        const int ts = threadIdx.x - 192;         // 0..127
+        const int quarter = warp & 3;
+        const int d = quarter * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        float* cum = reinterpret_cast<float*>(sm + Lay::kSgTab);
+        float* zeta = cum + kC;
+        float* dec = zeta + kC;
+        auto wait_all = [&](int b, uint32_t parity) {
+            mbar_wait(bar(b), parity, abort_flag);
+            group_sync(2);
+            return *abort_flag == 0;
+        };
+        float g0 = 0.f, g1 = 0.f;
+        if (GATED && ts < 32) {
+            g0 = (2 * ts < p.N ? G[2 * ts] : 0.f) * kLog2e;
+            g1 = (2 * ts + 1 < p.N ? G[2 * ts + 1] : 0.f) * kLog2e;
+        }
+        // Lazy decay. The state is held as S_i = c_i * T_i with T in TMEM and the scalar c_i in
+        // a register: the update adds (zeta V / c_{i+1}) onto T, and T is rewritten only when
+        // c would drop below kRenorm (then T <- c_i d_{i+1} T_i and c_{i+1} = 1). This keeps the
+        // per-chunk round trip to one read of T and one write of the bf16 copy.
+        constexpr float kRenorm = 9.094947e-13f;  // 2^-40
+        // zeta-scaled V of chunk c into ZV buffer c & 1, divided by the scale c_{next} that
+        // make_zv picks from c_prev (the current scale) and the chunk's decay.
+        auto make_zv = [&](int c, float c_prev, bool force_renorm, float& decay, bool& renorm, float& c_next) {
+            const int t0 = c * kC, L = min(kC, p.N - t0);
+            if (GATED) {
+                if (ts < 32) {
+                    warp_cumsum64(g0, g1, lane, cum);
+                    const int a = t0 + kC + 2 * ts;
+                    g0 = (a < p.N ? G[a] : 0.f) * kLog2e;
+                    g1 = (a + 1 < p.N ? G[a + 1] : 0.f) * kLog2e;
+                }
+                group_sync(2);
+                if (ts < kC) zeta[ts] = ts < L ? exp2f(cum[L - 1] - cum[ts]) : 0.f;
+                if (ts == 0) dec[0] = exp2f(cum[L - 1]);
+            } else {
+                if (ts < kC) zeta[ts] = ts < L ? pow_int_log2(lg, L - 1 - ts) : 0.f;
+                if (ts == 0) dec[0] = pow_int_log2(lg, L);
+            }
+            if (!wait_all(kFull0 + (c & 1), (c >> 1) & 1)) return false;  // V tile of chunk c has landed
+            decay = dec[0];
+            renorm = force_renorm || !(c_prev * decay >= kRenorm);
+            c_next = renorm ? 1.f : c_prev * decay;
+            const float inv = 1.f / c_next;
+            const uint8_t* vt = sm + Lay::kStage0 + (c & 1) * Lay::kStageBytes + Lay::kQBytes + Lay::kKBytes;
+            uint8_t* zv = sm + Lay::kZV + (c & 1) * Lay::kVBytes;
+            // 16-byte chunks ci = e * 128 + ts; the swizzle stays inside a 128-byte row, so the
+            // row (token) of a chunk is (ci mod 512) / 8. All loads before any store (aliasing).
+            uint4 x[8];
+            float z[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int ci = e * kEpiThreads + ts;
+                z[e] = zeta[(ci & 511) >> 3] * inv;
+                x[e] = *reinterpret_cast<const uint4*>(vt + ci * 16);
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                float2 f;
+                f = unpack_bf16(x[e].x); x[e].x = pack_bf16(f.x * z[e], f.y * z[e]);
+                f = unpack_bf16(x[e].y); x[e].y = pack_bf16(f.x * z[e], f.y * z[e]);
+                f = unpack_bf16(x[e].z); x[e].z = pack_bf16(f.x * z[e], f.y * z[e]);
+                f = unpack_bf16(x[e].w); x[e].w = pack_bf16(f.x * z[e], f.y * z[e]);
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) *reinterpret_cast<uint4*>(zv + (e * kEpiThreads + ts) * 16) = x[e];
+            fence_proxy_async();
+            group_sync(2);
+            if (ts == 0) mbar_arrive(bar(kZV0 + (c & 1)));
+            return true;
+        };
 
-        bool ok = true;
-        // initial state: S_op = bf16(S_in), S = decay_0 * S_in (S_in = 0 if absent)
-        prepare(0);
-        {
-            const float dec0 = decf[3 * kC];
+        float dec0 = 0.f, c_cur = 1.f;
+        bool renorm = true;
+        bool ok = make_zv(0, 1.f, true, dec0, renorm, c_cur);
+        if (ok) {
+            // initial state: S_op = bf16(S_in), T = decay_0 * S_in, c = 1 (S_in = 0 if absent)
             const float* sin = p.state_in ? p.state_in + ((size_t)bh * DK) * p.dv + dv0 + d : nullptr;
 #pragma unroll 1
             for (int cb = 0; cb < DK / 32; ++cb) {
                 uint32_t w[32], h[16];
 #pragma unroll
                 for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(sin ? sin[(size_t)(cb * 32 + c) * p.dv] : 0.f);
-                // bf16 copy of the undecayed state (operand of the first cross term), then decay_0 * S_in
 #pragma unroll
                 for (int c = 0; c < 16; ++c)
                     h[c] = pack_bf16(__uint_as_float(w[2 * c]), __uint_as_float(w[2 * c + 1]));
@@ -434,103 +630,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             tmem_wait_st();
             tc_fence_before();
-            epi_sync();
-            if (te == 0) mbar_arrive(bar(kSReady));
+            group_sync(2);
+            if (ts == 0) mbar_arrive(bar(kSReady));
         }
-
         for (int i = 0; i < nchunks && ok; ++i) {
-            const int s = i & 1;
-            const int t0 = i * kC;
-            const float* tb = decf + s * Lay::kDecFloats;
-            // ---------------- P = mask(Q K^T) in bf16, and zeta-scaled V
-            if (!epi_wait(kAFull, i & 1)) { ok = false; break; }
-            tc_fence_after();
-            {
-                uint32_t a0[32], a1[32];
-                tmem_ld32(tmem + lane_off + Lay::kColA, a0);
-                tmem_ld32(tmem + lane_off + Lay::kColA + 32, a1);
-                tmem_wait_ld();
-                if (lane < 16) {
-                    const int j = quarter * 16 + lane;  // M=64 accumulator: row j sits in lane 32*(j/16) + j%16
-                    const float cj = GATED ? tb[j] : 0.f;
-                    uint8_t* prow = sm + Lay::kP + j * 128;
-#pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) {
-                        uint32_t u[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            float pv[2];
-#pragma unroll
-                            for (int h = 0; h < 2; ++h) {
-                                const int m = cc * 8 + e * 2 + h;
-                                const float a = __uint_as_float(m < 32 ? a0[m & 31] : a1[m & 31]);
-                                float w;
-                                if (m > j) w = 0.f;
-                                else if (m == j) w = 1.f;
-                                else w = GATED ? exp2f(cj - tb[m]) : exp2f(lg * (float)(j - m));
-                                pv[h] = a * w;
-                            }
-                            u[e] = pack_bf16(pv[0], pv[1]);
-                        }
-                        *reinterpret_cast<uint4*>(prow + ((cc ^ (j & 7)) << 4)) = make_uint4(u[0], u[1], u[2], u[3]);
-                    }
-                }
-                // zeta-scaled copy of the V tile (swizzle permutes 16-byte chunks inside a row only)
-                const uint8_t* vt = sm + Lay::kStage0 + s * Lay::kStageBytes + Lay::kQBytes + Lay::kKBytes;
-                uint8_t* zv = sm + Lay::kZV;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int ci = e * kEpiThreads + te;
-                    const int m = (ci & 511) >> 3;
-                    const float z = tb[2 * kC + m];
-                    uint4 x = *reinterpret_cast<const uint4*>(vt + ci * 16);
-                    float2 f;
-                    f = unpack_bf16(x.x); x.x = pack_bf16(f.x * z, f.y * z);
-                    f = unpack_bf16(x.y); x.y = pack_bf16(f.x * z, f.y * z);
-                    f = unpack_bf16(x.z); x.z = pack_bf16(f.x * z, f.y * z);
-                    f = unpack_bf16(x.w); x.w = pack_bf16(f.x * z, f.y * z);
-                    *reinterpret_cast<uint4*>(zv + ci * 16) = x;
-                }
-            }
-            fence_proxy_async();
-            tc_fence_before();
-            epi_sync();
-            if (te == 0) mbar_arrive(bar(kPReady));
-
-            // ---------------- O = O_intra + r_j O_inter -> bf16 -> TMA store
-            if (te == 0) tma_store_wait_read();  // previous chunk's store has read the staging tile
-            if (!epi_wait(kOFull, i & 1)) { ok = false; break; }
-            tc_fence_after();
-            {
-                uint8_t* ost = sm + Lay::kOst + (d >> 6) * kTile64 + (d & 63) * 2;
-#pragma unroll
-                for (int jb = 0; jb < 2; ++jb) {
-                    uint32_t oi[32], oe[32];
-                    tmem_ld32(tmem + lane_off + Lay::kColO + jb * 32, oi);
-                    tmem_ld32(tmem + lane_off + Lay::kColA + jb * 32, oe);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
-                        const int j = jb * 32 + jj;
-                        const float o = fmaf(tb[kC + j], __uint_as_float(oe[jj]), __uint_as_float(oi[jj]));
-                        *reinterpret_cast<__nv_bfloat16*>(ost + j * 128) = __float2bfloat16_rn(o);
-                    }
-                }
-            }
-            fence_proxy_async();
-            tc_fence_before();
-            epi_sync();
-            if (te == 0) {
-                mbar_arrive(bar(kOFree));
-                tma_store_3d(&tm_o, dv0, t0, bh, sbase + Lay::kOst);
-                tma_store_3d(&tm_o, dv0 + 64, t0, bh, sbase + Lay::kOst + kTile64);
-                tma_store_commit();
-            }
-
-            // ---------------- state: S_op = bf16(S_i); S = decay_{i+1} S_i (or write state_out)
             const bool last = (i == nchunks - 1);
-            if (!last) prepare(i + 1);
-            if (!epi_wait(kSFull, i & 1)) { ok = false; break; }
+            float dec_next = 0.f, c_next = 1.f;
+            // the next chunk's zeta V is ready before this chunk's state update completes
+            if (!last && !make_zv(i + 1, c_cur, false, dec_next, renorm, c_next)) break;
+            if (!wait_all(kSFull, i & 1)) break;
             tc_fence_after();
             if (last) {
                 if (p.state_out) {
@@ -541,31 +649,44 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         tmem_ld32(tmem + lane_off + Lay::kColS + cb * 32, w);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) so[(size_t)(cb * 32 + c) * p.dv] = __uint_as_float(w[c]);
+                        for (int c = 0; c < 32; ++c) so[(size_t)(cb * 32 + c) * p.dv] = __uint_as_float(w[c]) * c_cur;
                     }
                 }
             } else {
-                const float dn = decf[((i + 1) & 1) * Lay::kDecFloats + 3 * kC];
+                // S_op = bf16(c_i T_i) for the next cross term; on renormalisation also
+                // T <- c_i d_{i+1} T_i so that the next update (scaled by 1/c_{i+1} = 1) adds onto it.
+                const float tscale = c_cur * dec_next;
 #pragma unroll 1
-                for (int cb = 0; cb < DK / 32; ++cb) {
-                    uint32_t w[32], h[16];
-                    tmem_ld32(tmem + lane_off + Lay::kColS + cb * 32, w);
+                for (int cb = 0; cb < DK / 64; ++cb) {
+                    uint32_t w0[32], w1[32], h[16];
+                    tmem_ld32(tmem + lane_off + Lay::kColS + cb * 64, w0);
+                    tmem_ld32(tmem + lane_off + Lay::kColS + cb * 64 + 32, w1);
                     tmem_wait_ld();
 #pragma unroll
                     for (int c = 0; c < 16; ++c)
-                        h[c] = pack_bf16(__uint_as_float(w[2 * c]), __uint_as_float(w[2 * c + 1]));
+                        h[c] = pack_bf16(__uint_as_float(w0[2 * c]) * c_cur, __uint_as_float(w0[2 * c + 1]) * c_cur);
+                    tmem_st16(tmem + lane_off + Lay::kColSop + cb * 32, h);
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(__uint_as_float(w[c]) * dn);
-                    tmem_st16(tmem + lane_off + Lay::kColSop + cb * 16, h);
-                    tmem_st32(tmem + lane_off + Lay::kColS + cb * 32, w);
+                    for (int c = 0; c < 16; ++c)
+                        h[c] = pack_bf16(__uint_as_float(w1[2 * c]) * c_cur, __uint_as_float(w1[2 * c + 1]) * c_cur);
+                    tmem_st16(tmem + lane_off + Lay::kColSop + cb * 32 + 16, h);
+                    if (renorm) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            w0[c] = __float_as_uint(__uint_as_float(w0[c]) * tscale);
+                            w1[c] = __float_as_uint(__uint_as_float(w1[c]) * tscale);
+                        }
+                        tmem_st32(tmem + lane_off + Lay::kColS + cb * 64, w0);
+                        tmem_st32(tmem + lane_off + Lay::kColS + cb * 64 + 32, w1);
+                    }
                 }
                 tmem_wait_st();
                 tc_fence_before();
-                epi_sync();
-                if (te == 0) mbar_arrive(bar(kSReady));
+                group_sync(2);
+                if (ts == 0) mbar_arrive(bar(kSReady));
+                c_cur = c_next;
             }
         }
-        if (te == 0) tma_store_wait_all();
     }
 
     tc_fence_before();
@@ -603,8 +724,8 @@ inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 3D bf16 map over [BH][N][inner] with a 64 x 64 box.
-inline bool make_map(CUtensorMap* m, const void* base, int inner, int N, int BH, bool swizzle) {
+// 3D bf16 map over [BH][N][inner] with a 64 x 64 box and 128-byte swizzle.
+inline bool make_map(CUtensorMap* m, const void* base, int inner, int N, int BH) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)N, (cuuint64_t)BH};
@@ -613,7 +734,7 @@ inline bool make_map(CUtensorMap* m, const void* base, int inner, int N, int BH,
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -634,8 +755,8 @@ ret_status tc_chunk_launch_dk(const void* q, const void* k, const void* v, const
     using Lay = tc::Layout<DK>;
     const int BH = B * H;
     CUtensorMap mq, mk, mv, mo;
-    if (!tc::make_map(&mq, q, DK, N, BH, true) || !tc::make_map(&mk, k, DK, N, BH, true) ||
-        !tc::make_map(&mv, v, dv, N, BH, true) || !tc::make_map(&mo, o, dv, N, BH, false))
+    if (!tc::make_map(&mq, q, DK, N, BH) || !tc::make_map(&mk, k, DK, N, BH) || !tc::make_map(&mv, v, dv, N, BH) ||
+        !tc::make_map(&mo, o, dv, N, BH))
         return RET_ERR_CUDA;
     auto kern = tc::chunk_tc_kernel<DK, GATED>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kSmemAlloc) != cudaSuccess)
