@@ -29,6 +29,7 @@
 // copies and MMAs are drained (bounded again) and TMEM is released.
 #pragma once
 
+#include <algorithm>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -267,7 +268,10 @@ struct Params {
     const float* decay_in;   // gamma [H] or g [B, H, N]
     const float* state_in;   // [B, H, dk, dv] or null
     float* state_out;        // [B, H, dk, dv] or null
+    float* seg_state;        // [G-1, B*H, dk, dv]: local end state of segments 0..G-2 (scratch)
+    float* seg_ldec;         // [G-1, B*H]: log2 of each of those segments' total decay (scratch)
     int H, N, dv;
+    int seg_chunks;          // chunks per sequence segment (blockIdx.z = segment)
 };
 
 // In-chunk inclusive cumulative sum of the gate in log2 units, by one warp:
@@ -284,7 +288,13 @@ __device__ __forceinline__ void warp_cumsum64(float g0, float g1, int lane, floa
     cum[2 * lane + 1] = incl;
 }
 
-template <int DK, bool GATED>
+// STATE_ONLY: the first pass of a split sequence. Each CTA runs the state
+// recurrence of one segment from a zero state (update products only; Q is not
+// loaded and no output is formed) and writes the segment's end state and total
+// decay to the scratch buffers. The full pass then starts segment g from
+// S_in(g) = decay_{g-1} S_in(g-1) + U_{g-1}, S_in(0) = state_in, which its state
+// epilogue evaluates in its prologue.
+template <int DK, bool GATED, bool STATE_ONLY>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, Params p) {
@@ -299,7 +309,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int slice = blockIdx.x, bh = blockIdx.y;
     const int dv0 = slice * kDvS;
-    const int nchunks = (p.N + kC - 1) / kC;
+    const int seg = blockIdx.z;
+    const int cbase = seg * p.seg_chunks;                          // first chunk of this segment
+    const int nchunks = min(p.seg_chunks, (p.N + kC - 1) / kC - cbase);
+    const bool last_seg = (cbase + nchunks) * kC >= p.N;
 
     if (threadIdx.x == 0) {
         for (int b = 0; b < Lay::kNumBars; ++b) mbar_init(bar(b), 1);
@@ -330,11 +343,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const int s = i & 1;
                 if (i >= 2 && !mbar_wait(bar(kEmpty0 + s), ((i >> 1) - 1) & 1, abort_flag)) break;
                 const uint32_t st = sbase + Lay::kStage0 + s * Lay::kStageBytes;
-                mbar_expect_tx(bar(kFull0 + s), Lay::kStageBytes);
-                const int t0 = i * kC;
+                mbar_expect_tx(bar(kFull0 + s), STATE_ONLY ? Lay::kKBytes + Lay::kVBytes : Lay::kStageBytes);
+                const int t0 = (cbase + i) * kC;
 #pragma unroll
                 for (int kb = 0; kb < DK / 64; ++kb) {
-                    tma_load_3d(st + kb * kTile64, &tm_q, kb * 64, t0, bh, bar(kFull0 + s));
+                    if (!STATE_ONLY) tma_load_3d(st + kb * kTile64, &tm_q, kb * 64, t0, bh, bar(kFull0 + s));
                     tma_load_3d(st + Lay::kQBytes + kb * kTile64, &tm_k, kb * 64, t0, bh, bar(kFull0 + s));
                 }
                 tma_load_3d(st + Lay::kQBytes + Lay::kKBytes, &tm_v, dv0, t0, bh, bar(kFull0 + s));
@@ -364,6 +377,18 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const uint32_t sV = sK + Lay::kKBytes;
                 const uint32_t sZV = sbase + Lay::kZV + s * Lay::kVBytes;
                 if (!mbar_wait(bar(kFull0 + s), (i >> 1) & 1, abort_flag)) break;
+                if (STATE_ONLY) {
+                    if (!mbar_wait(bar(kZV0 + s), (i >> 1) & 1, abort_flag) ||
+                        !mbar_wait(bar(kSReady), i & 1, abort_flag))
+                        break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < kC / 16; ++ks)
+                        mma_ss(tS, sdesc(sZV + ks * 2048, kTile64, 1024), sdesc(sK + ks * 2048, kTile64, 1024), id_up, 1);
+                    mma_commit(bar(kSFull));
+                    mma_commit(bar(kEmpty0 + s));
+                    continue;
+                }
                 if (i > 0 && !mbar_wait(bar(kOFree), (i - 1) & 1, abort_flag)) break;
                 tc_fence_after();
                 // A = Q K^T (both K-major, 128-byte swizzle; 16-element K steps)
@@ -406,6 +431,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
     } else if (warp < 6) {
         // ------------------------------------------------------------ attention epilogue (warps 2..5)
+      if (!STATE_ONLY) {
         const int te = threadIdx.x - 64;          // 0..127
         const int quarter = warp & 3;             // TMEM lane quarter this warp may access
         const int d = quarter * 32 + lane;        // dv column of the slice = TMEM lane
@@ -425,11 +451,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         float g0 = 0.f, g1 = 0.f;  // gated: prefetched gate values of the next chunk (first warp)
         if (GATED && te < 32) {
-            g0 = (2 * te < p.N ? G[2 * te] : 0.f) * kLog2e;
-            g1 = (2 * te + 1 < p.N ? G[2 * te + 1] : 0.f) * kLog2e;
+            const int a = cbase * kC + 2 * te;
+            g0 = (a < p.N ? G[a] : 0.f) * kLog2e;
+            g1 = (a + 1 < p.N ? G[a + 1] : 0.f) * kLog2e;
         }
         for (int i = 0; i < nchunks; ++i) {
-            const int t0 = i * kC;
+            const int t0 = (cbase + i) * kC;
             if (GATED) {
                 if (te < 32) {
                     warp_cumsum64(g0, g1, lane, cum);
@@ -534,6 +561,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         }
         if (te == 0) tma_store_wait_all();
+      }
     } else {
         // ------------------------------------------------------------ state epilogue (warps 6..9)
         const int ts = threadIdx.x - 192;         // 0..127
@@ -550,9 +578,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         };
         float g0 = 0.f, g1 = 0.f;
         if (GATED && ts < 32) {
-            g0 = (2 * ts < p.N ? G[2 * ts] : 0.f) * kLog2e;
-            g1 = (2 * ts + 1 < p.N ? G[2 * ts + 1] : 0.f) * kLog2e;
+            const int a = cbase * kC + 2 * ts;
+            g0 = (a < p.N ? G[a] : 0.f) * kLog2e;
+            g1 = (a + 1 < p.N ? G[a + 1] : 0.f) * kLog2e;
         }
+        float ldec_sum = 0.f;  // log2 of the decay accumulated over this segment
         // Lazy decay. The state is held as S_i = c_i * T_i with T in TMEM and the scalar c_i in
         // a register: the update adds (zeta V / c_{i+1}) onto T, and T is rewritten only when
         // c would drop below kRenorm (then T <- c_i d_{i+1} T_i and c_{i+1} = 1). This keeps the
@@ -561,7 +591,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // zeta-scaled V of chunk c into ZV buffer c & 1, divided by the scale c_{next} that
         // make_zv picks from c_prev (the current scale) and the chunk's decay.
         auto make_zv = [&](int c, float c_prev, bool force_renorm, float& decay, bool& renorm, float& c_next) {
-            const int t0 = c * kC, L = min(kC, p.N - t0);
+            const int t0 = (cbase + c) * kC, L = min(kC, p.N - t0);
             if (GATED) {
                 if (ts < 32) {
                     warp_cumsum64(g0, g1, lane, cum);
@@ -571,13 +601,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 group_sync(2);
                 if (ts < kC) zeta[ts] = ts < L ? exp2f(cum[L - 1] - cum[ts]) : 0.f;
-                if (ts == 0) dec[0] = exp2f(cum[L - 1]);
+                if (ts == 0) {
+                    dec[0] = exp2f(cum[L - 1]);
+                    dec[1] = cum[L - 1];
+                }
             } else {
                 if (ts < kC) zeta[ts] = ts < L ? pow_int_log2(lg, L - 1 - ts) : 0.f;
-                if (ts == 0) dec[0] = pow_int_log2(lg, L);
+                if (ts == 0) {
+                    dec[0] = pow_int_log2(lg, L);
+                    dec[1] = lg * (float)L;
+                }
             }
             if (!wait_all(kFull0 + (c & 1), (c >> 1) & 1)) return false;  // V tile of chunk c has landed
             decay = dec[0];
+            ldec_sum += dec[1];
             renorm = force_renorm || !(c_prev * decay >= kRenorm);
             c_next = renorm ? 1.f : c_prev * decay;
             const float inv = 1.f / c_next;
@@ -613,13 +650,25 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         bool renorm = true;
         bool ok = make_zv(0, 1.f, true, dec0, renorm, c_cur);
         if (ok) {
-            // initial state: S_op = bf16(S_in), T = decay_0 * S_in, c = 1 (S_in = 0 if absent)
-            const float* sin = p.state_in ? p.state_in + ((size_t)bh * DK) * p.dv + dv0 + d : nullptr;
+            // initial state: S_op = bf16(S_in), T = decay_0 * S_in, c = 1. S_in is state_in (or
+            // zero) for the first segment; segment g > 0 folds in the earlier segments' end states:
+            // S_in(g) = decay_{g-1} S_in(g-1) + U_{g-1}. The state-only pass starts from zero.
+            const float* sin = (!STATE_ONLY && p.state_in) ? p.state_in + ((size_t)bh * DK) * p.dv + dv0 + d : nullptr;
+            const size_t seg_stride = (size_t)gridDim.y * DK * p.dv;
+            const float* useg = STATE_ONLY ? nullptr : p.seg_state + ((size_t)bh * DK) * p.dv + dv0 + d;
+            const int nprev = STATE_ONLY ? 0 : seg;
 #pragma unroll 1
             for (int cb = 0; cb < DK / 32; ++cb) {
                 uint32_t w[32], h[16];
 #pragma unroll
                 for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(sin ? sin[(size_t)(cb * 32 + c) * p.dv] : 0.f);
+#pragma unroll 1
+                for (int hs = 0; hs < nprev; ++hs) {
+                    const float gam = exp2f(p.seg_ldec[(size_t)hs * gridDim.y + bh]);
+                    const float* u = useg + hs * seg_stride + (size_t)(cb * 32) * p.dv;
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(fmaf(gam, __uint_as_float(w[c]), u[(size_t)c * p.dv]));
+                }
 #pragma unroll
                 for (int c = 0; c < 16; ++c)
                     h[c] = pack_bf16(__uint_as_float(w[2 * c]), __uint_as_float(w[2 * c + 1]));
@@ -641,8 +690,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (!wait_all(kSFull, i & 1)) break;
             tc_fence_after();
             if (last) {
-                if (p.state_out) {
-                    float* so = p.state_out + ((size_t)bh * DK) * p.dv + dv0 + d;
+                float* so = nullptr;
+                if (STATE_ONLY) {
+                    so = p.seg_state + ((size_t)seg * gridDim.y + bh) * DK * p.dv + dv0 + d;
+                    if (slice == 0 && ts == 0) p.seg_ldec[(size_t)seg * gridDim.y + bh] = ldec_sum;
+                } else if (last_seg) {
+                    so = p.state_out;
+                    if (so) so += ((size_t)bh * DK) * p.dv + dv0 + d;
+                }
+                if (so) {
 #pragma unroll 1
                     for (int cb = 0; cb < DK / 32; ++cb) {
                         uint32_t w[32];
@@ -652,9 +708,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         for (int c = 0; c < 32; ++c) so[(size_t)(cb * 32 + c) * p.dv] = __uint_as_float(w[c]) * c_cur;
                     }
                 }
-            } else {
+            } else if (!STATE_ONLY || renorm) {
                 // S_op = bf16(c_i T_i) for the next cross term; on renormalisation also
                 // T <- c_i d_{i+1} T_i so that the next update (scaled by 1/c_{i+1} = 1) adds onto it.
+                // The state-only pass needs no S_op and touches T only to renormalise.
                 const float tscale = c_cur * dec_next;
 #pragma unroll 1
                 for (int cb = 0; cb < DK / 64; ++cb) {
@@ -662,14 +719,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     tmem_ld32(tmem + lane_off + Lay::kColS + cb * 64, w0);
                     tmem_ld32(tmem + lane_off + Lay::kColS + cb * 64 + 32, w1);
                     tmem_wait_ld();
+                    if (!STATE_ONLY) {
 #pragma unroll
-                    for (int c = 0; c < 16; ++c)
-                        h[c] = pack_bf16(__uint_as_float(w0[2 * c]) * c_cur, __uint_as_float(w0[2 * c + 1]) * c_cur);
-                    tmem_st16(tmem + lane_off + Lay::kColSop + cb * 32, h);
+                        for (int c = 0; c < 16; ++c)
+                            h[c] = pack_bf16(__uint_as_float(w0[2 * c]) * c_cur, __uint_as_float(w0[2 * c + 1]) * c_cur);
+                        tmem_st16(tmem + lane_off + Lay::kColSop + cb * 32, h);
 #pragma unroll
-                    for (int c = 0; c < 16; ++c)
-                        h[c] = pack_bf16(__uint_as_float(w1[2 * c]) * c_cur, __uint_as_float(w1[2 * c + 1]) * c_cur);
-                    tmem_st16(tmem + lane_off + Lay::kColSop + cb * 32 + 16, h);
+                        for (int c = 0; c < 16; ++c)
+                            h[c] = pack_bf16(__uint_as_float(w1[2 * c]) * c_cur, __uint_as_float(w1[2 * c + 1]) * c_cur);
+                        tmem_st16(tmem + lane_off + Lay::kColSop + cb * 32 + 16, h);
+                    }
                     if (renorm) {
 #pragma unroll
                         for (int c = 0; c < 32; ++c) {
@@ -681,6 +740,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                 }
                 tmem_wait_st();
+            }
+            if (!last) {
                 tc_fence_before();
                 group_sync(2);
                 if (ts == 0) mbar_arrive(bar(kSReady));
@@ -746,37 +807,139 @@ inline bool tc_chunk_supported(int dk, int dv, int chunk, bool bf16) {
            tc::tc_device_ok();
 }
 
-inline int tc_chunk_launches(int, int, int, int, int) { return 1; }
+namespace tc {
+
+constexpr int kMaxSegments = 16;
+
+inline int sm_count() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            n = 148;
+    }
+    return n;
+}
+
+// Sequence split: with few (head, dv-slice) CTAs the sequence is cut into G
+// segments so that about one CTA per SM runs. Segments are whole chunks.
+struct Plan {
+    int G;           // segments
+    int seg_chunks;  // chunks per segment
+};
+
+inline Plan plan(int B, int H, int N, int dv) {
+    const int ctas = B * H * (dv / kDvS);
+    const int nchunks = (N + kC - 1) / kC;
+    int G = 1;
+    if (2 * ctas <= sm_count()) G = std::min(std::min(sm_count() / ctas, kMaxSegments), nchunks / 4);
+    if (G < 2) return {1, nchunks};
+    const int seg_chunks = (nchunks + G - 1) / G;
+    return {(nchunks + seg_chunks - 1) / seg_chunks, seg_chunks};
+}
+
+// Scratch of a split sequence: end states [G-1, BH, dk, dv] fp32, log2 decays [G-1, BH], and,
+// when state_in and state_out are the same buffer, a copy of state_in (every segment reads
+// state_in while the last one writes state_out, so they must not share memory).
+inline size_t scratch_states_bytes(const Plan& pl, int BH, int dk, int dv) {
+    return sizeof(float) * (size_t)(pl.G - 1) * BH * dk * dv;
+}
+inline size_t scratch_ldec_bytes(const Plan& pl, int BH) {
+    return (sizeof(float) * (size_t)(pl.G - 1) * BH + 255) & ~size_t(255);
+}
+inline size_t scratch_bytes(const Plan& pl, int BH, int dk, int dv, bool alias) {
+    if (pl.G < 2) return 0;
+    return scratch_states_bytes(pl, BH, dk, dv) + scratch_ldec_bytes(pl, BH) +
+           (alias ? sizeof(float) * (size_t)BH * dk * dv : 0);
+}
 
 template <int DK, bool GATED>
-ret_status tc_chunk_launch_dk(const void* q, const void* k, const void* v, const float* decay, void* o,
-                              const float* state_in, float* state_out, int B, int H, int N, int dv,
-                              cudaStream_t st) {
-    using Lay = tc::Layout<DK>;
+ret_status launch_dk(const void* q, const void* k, const void* v, const float* decay, void* o,
+                     const float* state_in, float* state_out, int B, int H, int N, int dv, const Plan& pl,
+                     void* scratch, cudaStream_t st) {
+    using Lay = Layout<DK>;
     const int BH = B * H;
     CUtensorMap mq, mk, mv, mo;
-    if (!tc::make_map(&mq, q, DK, N, BH) || !tc::make_map(&mk, k, DK, N, BH) || !tc::make_map(&mv, v, dv, N, BH) ||
-        !tc::make_map(&mo, o, dv, N, BH))
+    if (!make_map(&mq, q, DK, N, BH) || !make_map(&mk, k, DK, N, BH) || !make_map(&mv, v, dv, N, BH) ||
+        !make_map(&mo, o, dv, N, BH))
         return RET_ERR_CUDA;
-    auto kern = tc::chunk_tc_kernel<DK, GATED>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kSmemAlloc) != cudaSuccess)
+    Params prm{decay, state_in, state_out, nullptr, nullptr, H, N, dv, pl.seg_chunks};
+    if (pl.G > 1) {
+        uint8_t* sc = static_cast<uint8_t*>(scratch);
+        prm.seg_state = reinterpret_cast<float*>(sc);
+        prm.seg_ldec = reinterpret_cast<float*>(sc + scratch_states_bytes(pl, BH, DK, dv));
+        if (state_in && state_in == state_out) {
+            float* copy = reinterpret_cast<float*>(sc + scratch_states_bytes(pl, BH, DK, dv) + scratch_ldec_bytes(pl, BH));
+            if (cudaMemcpyAsync(copy, state_in, sizeof(float) * (size_t)BH * DK * dv, cudaMemcpyDeviceToDevice, st) !=
+                cudaSuccess)
+                return RET_ERR_CUDA;
+            prm.state_in = copy;
+        }
+        auto k1 = chunk_tc_kernel<DK, GATED, true>;
+        if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kSmemAlloc) != cudaSuccess)
+            return RET_ERR_CUDA;
+        k1<<<dim3(dv / kDvS, BH, pl.G - 1), kThreads, Lay::kSmemAlloc, st>>>(mq, mk, mv, mo, prm);
+        if (cudaGetLastError() != cudaSuccess) return RET_ERR_CUDA;
+    }
+    auto k2 = chunk_tc_kernel<DK, GATED, false>;
+    if (cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kSmemAlloc) != cudaSuccess)
         return RET_ERR_CUDA;
-    tc::Params prm{decay, state_in, state_out, H, N, dv};
-    dim3 grid(dv / tc::kDvS, BH);
-    kern<<<grid, tc::kThreads, Lay::kSmemAlloc, st>>>(mq, mk, mv, mo, prm);
+    k2<<<dim3(dv / kDvS, BH, pl.G), kThreads, Lay::kSmemAlloc, st>>>(mq, mk, mv, mo, prm);
     return cudaGetLastError() == cudaSuccess ? RET_OK : RET_ERR_CUDA;
 }
 
+// Runs the tensor-core path with caller-provided scratch (at least scratch_bytes()).
+template <bool GATED>
+ret_status launch_with_scratch(const void* q, const void* k, const void* v, const float* decay, void* o,
+                               const float* state_in, float* state_out, int B, int H, int N, int dk, int dv,
+                               const Plan& pl, void* scratch, cudaStream_t st) {
+    switch (dk) {
+        case 64: return launch_dk<64, GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dv, pl, scratch, st);
+        case 128: return launch_dk<128, GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dv, pl, scratch, st);
+        case 256: return launch_dk<256, GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dv, pl, scratch, st);
+    }
+    return RET_ERR_UNSUPPORTED;
+}
+
+}  // namespace tc
+
+inline int tc_chunk_launches(int B, int H, int N, int, int dv) { return tc::plan(B, H, N, dv).G > 1 ? 2 : 1; }
+
+namespace tc {
+
+// The default stream-ordered pool of a device returns its memory to the system
+// at every synchronisation unless its release threshold is raised; then each
+// call would map fresh memory. Raise it once per device so that repeated calls
+// reuse the pool's memory.
+inline void keep_pool_memory() {
+    static bool done[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || done[dev]) return;
+    done[dev] = true;
+    cudaMemPool_t pool;
+    if (cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
+        uint64_t threshold = UINT64_MAX;
+        cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &threshold);
+    }
+}
+
+}  // namespace tc
+
+// Tensor-core path; a split sequence takes its scratch from the stream-ordered
+// allocator and returns it on the same stream after the two launches.
 template <bool GATED>
 ret_status tc_chunk_launch(const void* q, const void* k, const void* v, const float* decay, void* o,
                            const float* state_in, float* state_out, int B, int H, int N, int dk, int dv,
                            cudaStream_t st) {
-    switch (dk) {
-        case 64: return tc_chunk_launch_dk<64, GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dv, st);
-        case 128: return tc_chunk_launch_dk<128, GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dv, st);
-        case 256: return tc_chunk_launch_dk<256, GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dv, st);
-    }
-    return RET_ERR_UNSUPPORTED;
+    const tc::Plan pl = tc::plan(B, H, N, dv);
+    void* scratch = nullptr;
+    const size_t bytes = tc::scratch_bytes(pl, B * H, dk, dv, state_in != nullptr && state_in == state_out);
+    if (bytes) tc::keep_pool_memory();
+    if (bytes && cudaMallocAsync(&scratch, bytes, st) != cudaSuccess) return RET_ERR_CUDA;
+    const ret_status r = tc::launch_with_scratch<GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dk, dv,
+                                                        pl, scratch, st);
+    if (scratch && cudaFreeAsync(scratch, st) != cudaSuccess) return RET_ERR_CUDA;
+    return r;
 }
 
 }  // namespace ret

@@ -239,3 +239,50 @@ def test_full_size_decode_sampled_heads(cuda_lib):
     for s in samples:
         assert rel_l2(torch.stack(got[s]), np.stack(want[s])) <= TOL_BF16, s
         assert rel_l2(Sd[s[0], s[1]], S_ref[s][0, 0]) <= TOL_BF16, s
+
+
+# ------------------------------------------------------------------ split sequences (few heads, long N)
+
+SPLIT_CASES = [
+    # B, H, N, dk, dv
+    (1, 2, 1000, 64, 128),
+    (1, 1, 2053, 128, 128),
+    (2, 1, 777, 256, 256),
+]
+
+
+@pytest.mark.parametrize("gated", [False, True])
+@pytest.mark.parametrize("inplace", [False, True])
+@pytest.mark.parametrize("B,H,N,dk,dv", SPLIT_CASES)
+def test_split_sequence_matches_oracle(cuda_lib, B, H, N, dk, dv, gated, inplace):
+    """The tensor-core path cuts long sequences of few heads into segments (a
+    state-only pass, then the full pass seeded per segment); the result must not
+    change, including the final state and an in-place state buffer."""
+    assert cuda_lib.chunkwise_launches(B, H, N, dk, dv, 64, torch.bfloat16) == 2
+    gen = torch.Generator().manual_seed(N + dk + int(gated))
+    q, k, v = I.qkv(B, H, N, dk, dv, torch.bfloat16, gen=gen)
+    S0 = torch.randn(B, H, dk, dv, generator=gen) * 0.05
+    qd, kd, vd, S0d = _dev(q, k, v, S0)
+    s_out = S0d if inplace else torch.empty_like(S0d)
+    if gated:
+        g = I.gate(B, H, N, gen) * 4.0
+        o = cuda_lib.gated_ret_chunkwise(qd, kd, vd, g.to(DEV), 64, state_in=S0d, state_out=s_out)
+        want_o, want_s = O.gated_chunkwise(q, k, v, g, 64, state_in=S0)
+    else:
+        gam = _gammas_with_edges(H + 2)[-H:]  # includes 1.0 and 0.9 style heads
+        o = cuda_lib.ret_chunkwise(qd, kd, vd, gam.to(DEV), 64, state_in=S0d, state_out=s_out)
+        want_o, want_s = O.ret_chunkwise(q, k, v, gam, 64, state_in=S0)
+    assert cuda_lib.last_device_error() == 0
+    assert_close(o, want_o, torch.bfloat16, "o")
+    assert_close(s_out, want_s, torch.bfloat16, "state")
+
+
+def test_split_sequence_gamma_zero(cuda_lib):
+    """gamma = 0 makes every segment's decay exactly zero; the split must still give (q.k) v."""
+    B, H, N, dk, dv = 1, 1, 900, 64, 128
+    q, k, v = _rand_inputs(B, H, N, dk, dv, torch.bfloat16, seed=31)
+    gam = torch.zeros(1)
+    o = cuda_lib.ret_chunkwise(*_dev(q, k, v, gam), 64)
+    qn, kn, vn = (t.double().numpy()[0, 0] for t in (q, k, v))
+    want = np.einsum("nd,nd->n", qn, kn)[:, None] * vn
+    assert rel_l2(o[0, 0], want) <= TOL_BF16
