@@ -54,7 +54,8 @@ typedef enum {
     RET_ERR_UNSUPPORTED = 4, /* sizes outside what the kernels support (see each call) */
     RET_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed */
     RET_ERR_TIMEOUT = 6,     /* a kernel's bounded wait ran out (device error word set) */
-    RET_ERR_ALIGN = 7        /* a pointer is not 16-byte aligned */
+    RET_ERR_ALIGN = 7,       /* a pointer is not 16-byte aligned */
+    RET_ERR_SCRATCH = 8      /* ret_chunkwise_noalloc: the problem needs more scratch than its fixed buffer */
 } ret_status;
 
 typedef enum { RET_F32 = 0, RET_BF16 = 1 } ret_dtype;
@@ -142,6 +143,39 @@ RET_API int ret_chunkwise_path(int dk, int dv, int chunk, ret_dtype dt);
  * rejected). Pure host function; nothing is launched.
  */
 RET_API int ret_chunkwise_launches(int B, int H, int N, int dk, int dv, int chunk, ret_dtype dt);
+
+/*
+ * ret_chunkwise without any device allocation. The paper has no counterpart for
+ * this entry point: it is an interface for callers, not part of the method.
+ *
+ * ret_chunkwise may take stream-ordered scratch from the device's default
+ * memory pool when it splits a long sequence of few heads into segments. Some
+ * callers cannot let a library allocate: a framework whose own allocator has
+ * reserved the device memory up front, a serving loop that forbids allocations
+ * after start-up, or code that must not touch the default pool. This entry
+ * point computes exactly what ret_chunkwise computes, with the same arguments
+ * and the same kernels, but takes its scratch from a fixed buffer compiled into
+ * the library: a file-scope device array of RET_NOALLOC_SCRATCH_BYTES (16 MiB)
+ * that every GPU which loads the library holds until the process exits.
+ *
+ *  - The first call on a device, with that device current, looks up the
+ *    buffer's device address (cudaGetSymbolAddress) and caches it. Make that
+ *    first call before any stream capture.
+ *  - A problem whose scratch would exceed the buffer is rejected on the host
+ *    with RET_ERR_SCRATCH before anything is launched. Passing state_in and
+ *    state_out as the same buffer needs an extra copy of the state in scratch.
+ *  - All calls share the one buffer, which keeps the previous call's contents;
+ *    every scratch byte a call reads is written earlier in that same call, so
+ *    nothing has to be cleared. Calls that overlap on the GPU (for example on
+ *    two streams) race on the buffer: serialise them.
+ *  - Neither cudaMalloc, cudaMallocAsync, cudaFree nor any other allocating
+ *    routine is called.
+ */
+#define RET_NOALLOC_SCRATCH_BYTES (16u << 20)
+RET_API ret_status ret_chunkwise_noalloc(const void* q, const void* k, const void* v, const float* gamma,
+                                 void* o, const float* state_in, float* state_out,
+                                 int B, int H, int N, int dk, int dv, int chunk,
+                                 ret_dtype dt, void* stream);
 
 /* Library version, "major.minor.patch". */
 RET_API const char* ret_version(void);

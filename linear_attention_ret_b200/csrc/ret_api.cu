@@ -3,6 +3,7 @@
 // share the module-scope device error word.
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "simt.cuh"
@@ -158,6 +159,7 @@ const char* ret_status_str(ret_status s) {
         case RET_ERR_CUDA: return "CUDA error";
         case RET_ERR_TIMEOUT: return "a kernel wait timed out (device error word set)";
         case RET_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case RET_ERR_SCRATCH: return "problem needs more scratch than the fixed no-allocation buffer holds";
     }
     return "unknown status";
 }
@@ -185,3 +187,63 @@ int ret_chunkwise_launches(int B, int H, int N, int dk, int dv, int chunk, ret_d
 const char* ret_version(void) { return "0.1.0"; }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ no-allocation entry point
+//
+// For callers that must not let the library allocate device memory (their own
+// allocator owns the memory, or allocation is forbidden after start-up): the
+// scratch of a split sequence comes from this fixed buffer instead of the
+// stream-ordered pool. Each device that loads the library holds the buffer
+// until exit. Host code must not use its name as a pointer (that is a
+// host-side stand-in); the device address is looked up once per device below.
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[RET_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up on the
+// first call per device (with that device current) and cached; null on error.
+void* noalloc_scratch() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+        g_noalloc_ptr[dev] = p;
+    }
+    return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" ret_status ret_chunkwise_noalloc(const void* q, const void* k, const void* v, const float* gamma,
+                                            void* o, const float* state_in, float* state_out, int B, int H, int N,
+                                            int dk, int dv, int chunk, ret_dtype dt, void* stream) {
+    ret_status s = check_common(B, H, N, dk, dv, dt);
+    if (s != RET_OK) return s;
+    if (chunk <= 0) return RET_ERR_SHAPE;
+    if (dk > 256) return RET_ERR_UNSUPPORTED;
+    cudaStream_t st = as_stream(stream);
+    if (N == 0) return empty_sequence_state(state_in, state_out, B, H, dk, dv, st);  // copy or memset only
+    if (!q || !k || !v || !gamma || !o) return RET_ERR_NULL;
+    if (!tc_chunk_supported(dk, dv, chunk, dt == RET_BF16)) {
+        // the CUDA-core kernel keeps its state in shared memory and needs no scratch
+        return dt == RET_F32 ? launch_chunkwise_simt<float, false>(q, k, v, gamma, o, state_in, state_out, B, H, N,
+                                                                   dk, dv, chunk, st)
+                             : launch_chunkwise_simt<__nv_bfloat16, false>(q, k, v, gamma, o, state_in, state_out,
+                                                                           B, H, N, dk, dv, chunk, st);
+    }
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RET_ERR_ALIGN;
+    const tc::Plan pl = tc::plan(B, H, N, dv);
+    const size_t bytes = tc::scratch_bytes(pl, B * H, dk, dv, state_in != nullptr && state_in == state_out);
+    if (bytes > RET_NOALLOC_SCRATCH_BYTES) return RET_ERR_SCRATCH;
+    void* scratch = nullptr;
+    if (bytes) {
+        scratch = noalloc_scratch();
+        if (scratch == nullptr) return RET_ERR_CUDA;
+    }
+    return tc::launch_with_scratch<false>(q, k, v, gamma, o, state_in, state_out, B, H, N, dk, dv, pl, scratch, st);
+}

@@ -23,10 +23,11 @@ LIB_PATH = os.path.join(_PKG, "libret.so")
 
 RET_F32, RET_BF16 = 0, 1
 STATUS = {0: "RET_OK", 1: "RET_ERR_NULL", 2: "RET_ERR_SHAPE", 3: "RET_ERR_DTYPE", 4: "RET_ERR_UNSUPPORTED",
-          5: "RET_ERR_CUDA", 6: "RET_ERR_TIMEOUT", 7: "RET_ERR_ALIGN"}
+          5: "RET_ERR_CUDA", 6: "RET_ERR_TIMEOUT", 7: "RET_ERR_ALIGN", 8: "RET_ERR_SCRATCH"}
 # every symbol include/ret.h declares
 SYMBOLS = ("ret_parallel", "ret_chunkwise", "ret_recurrent_step", "gated_ret_chunkwise", "ret_status_str",
-           "ret_last_device_error", "ret_chunkwise_path", "ret_chunkwise_launches", "ret_version")
+           "ret_last_device_error", "ret_chunkwise_path", "ret_chunkwise_launches", "ret_version",
+           "ret_chunkwise_noalloc")
 
 _lock = threading.Lock()
 _lib = None
@@ -55,8 +56,10 @@ def load(path: str | None = None) -> ctypes.CDLL:
         lib.ret_parallel.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]
         lib.ret_chunkwise.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
         lib.gated_ret_chunkwise.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
+        lib.ret_chunkwise_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
         lib.ret_recurrent_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
-        for fn in ("ret_parallel", "ret_chunkwise", "gated_ret_chunkwise", "ret_recurrent_step"):
+        for fn in ("ret_parallel", "ret_chunkwise", "gated_ret_chunkwise", "ret_recurrent_step",
+                   "ret_chunkwise_noalloc"):
             getattr(lib, fn).restype = _i
         lib.ret_status_str.argtypes = [_i]
         lib.ret_status_str.restype = ctypes.c_char_p
@@ -120,6 +123,19 @@ def ret_chunkwise(q, k, v, gamma, chunk, state_in=None, state_out=None, o=None, 
     _check("ret_chunkwise", load().ret_chunkwise(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(o),
                                                  _ptr(state_in), _ptr(state_out), B, H, N, dk, dv, int(chunk),
                                                  _dt(q), _stream(stream)))
+    return o
+
+
+def ret_chunkwise_noalloc(q, k, v, gamma, chunk, state_in=None, state_out=None, o=None, stream=None):
+    """ret_chunkwise without device allocation by the library: scratch comes from a
+    fixed 16 MiB buffer inside libret.so (see include/ret.h). Returns o."""
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    o = torch.empty(B, H, N, dv, dtype=q.dtype, device=q.device) if o is None else o
+    _cuda(q, k, v, gamma, o, state_in, state_out)
+    _check("ret_chunkwise_noalloc", load().ret_chunkwise_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(o),
+                                                                 _ptr(state_in), _ptr(state_out), B, H, N, dk, dv,
+                                                                 int(chunk), _dt(q), _stream(stream)))
     return o
 
 

@@ -36,7 +36,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(8):
+    for code in range(9):
         assert lib.ret_status_str(code)
     assert lib.ret_status_str(99) == b"unknown status"
     assert lib.ret_version() == b"0.1.0"
