@@ -244,15 +244,23 @@ def run_ours(args, spec):
     stream = torch.cuda.current_stream(dev)
 
     step, x, o, launches = make_step(spec, dev, rank_seed(rank))
+    # nvidia-smi samples every 100 ms while a timed region lasts milliseconds, so sampling
+    # starts before the warm-up and an untimed burn-in keeps the same load for about a
+    # second; the samples then describe the clocks the timed region runs at.
+    clocks = ClockSampler(gpu_uuid(local))
+    clocks.start()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     err = ret.last_device_error()
     if err != 0:
         raise SystemExit(f"device error word set after warm-up: {err}")
+    t_burn = time.perf_counter()
+    while time.perf_counter() - t_burn < args.burn_in:
+        for _ in range(10):
+            step()
+        torch.cuda.synchronize()
 
-    clocks = ClockSampler(gpu_uuid(local))
-    clocks.start()
     # timed region: K steps, barrier + synchronize on both sides, events per step on the launch stream
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     barrier(world, dev)
@@ -297,9 +305,10 @@ def run_ours(args, spec):
                    "l2": f"working set {spec['bytes'] / 1e6:.0f} MB per step > 126 MB L2 (no flush)",
                    "parallelism": f"batch-sharded x{world}" if world > 1 else "single GPU"},
         "roofline": roofline,
-        "clocks": clk,
+        "clocks": dict(clk, window="warm-up, ~1 s untimed burn-in and the timed region") if clk else None,
         "e2e": e2e,
         "gpu_launches": args.steps * launches,
+        "launches_per_step": launches,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(spec, budget_s=args.cpu_seconds)
@@ -476,6 +485,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--burn-in", type=float, default=1.0,
+                    help="seconds of untimed steps after warm-up while clocks are sampled")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
