@@ -52,13 +52,21 @@ struct Layout {
     static constexpr int kVBytes = 2 * kTile64;
     static constexpr int kStageBytes = kQBytes + kKBytes + kVBytes;
     static constexpr int kStage0 = 0;
-    static constexpr int kP = 2 * kStageBytes;              // P tile (64 x 64 bf16, SW128 K-major)
-    static constexpr int kZV = kP + kTile64;                // zeta-scaled V, two buffers (V tile layout)
+    // Attention buffers: with dk <= 128 there is TMEM for two sets of {Q K^T / O_inter,
+    // O_intra} accumulators and shared memory for two P tiles, so chunk i+1's Q K^T and mask
+    // overlap chunk i's output products and drain. With dk = 256 the state fills TMEM and
+    // one set is used in turn.
+    static constexpr int kNBuf = DK <= 128 ? 2 : 1;
+    // TMA stages of Q, K, V tiles: three where shared memory allows, so that loads run two
+    // chunks ahead of the products that read them.
+    static constexpr int kStages = DK <= 128 ? 3 : 2;
+    static constexpr int kP = kStages * kStageBytes;        // P tiles (64 x 64 bf16, SW128 K-major), kNBuf of them
+    static constexpr int kZV = kP + kNBuf * kTile64;        // zeta-scaled V, two buffers (V tile layout)
     static constexpr int kOst = kZV + 2 * kVBytes;          // O staging for the TMA store (128-byte swizzle)
     static constexpr int kBar = kOst + kVBytes;             // mbarriers
-    static constexpr int kNumBars = 14;
-    static constexpr int kAgTab = kBar + kNumBars * 8;      // attention group: cum[64] | r[64] | pw[68]
-    static constexpr int kSgTab = kAgTab + 196 * 4;         // state group: cum[64] | zeta[64] | decay
+    static constexpr int kNumBars = 22;
+    static constexpr int kAgTab = kBar + kNumBars * 8;      // attention group: cum[2][64] | r[2][64] | pw[68]
+    static constexpr int kSgTab = kAgTab + 324 * 4;         // state group: cum[64] | zeta[64] | decay
     static constexpr int kTmemSlot = kSgTab + 132 * 4;
     static constexpr int kAbort = kTmemSlot + 4;
     static constexpr int kBytes = kAbort + 4;
@@ -66,18 +74,19 @@ struct Layout {
     // TMEM columns
     static constexpr int kColS = 0;                 // fp32 state S^T: DK columns
     static constexpr int kColSop = DK;              // bf16 state copy: DK/2 columns
-    static constexpr int kColA = DK + DK / 2;       // Q K^T, then O_inter^T: 64 columns
-    static constexpr int kColO = kColA + kC;        // O_intra^T: 64 columns
-    static constexpr int kColsUsed = kColO + kC;
+    static constexpr int kColA = DK + DK / 2;       // buffer b: Q K^T then O_inter^T at kColA + 2*kC*b (64 columns)
+    static constexpr int kColO = kColA + kC;        // buffer b: O_intra^T at kColO + 2*kC*b (64 columns)
+    static constexpr int kColsUsed = kColA + 2 * kC * kNBuf;
     static constexpr int kTmemCols = kColsUsed <= 256 ? 256 : 512;
     static_assert(kColsUsed <= 512, "TMEM overflow");
     static_assert(kSmemAlloc <= 227 * 1024, "shared memory overflow");
 };
 
 enum Bar {
-    kFull0 = 0, kFull1, kEmpty0, kEmpty1,  // TMA stages
-    kAFull, kPReady, kOFull, kOFree,       // attention epilogue <-> MMA
-    kSFull, kSReady, kZV0, kZV1,           // state epilogue <-> MMA
+    kFull0 = 0, kFull1, kFull2, kEmpty0, kEmpty1, kEmpty2,  // TMA stages
+    kAFull0, kAFull1, kARead0, kARead1,          // attention epilogue <-> MMA, per attention buffer
+    kPReady0, kPReady1, kOFull0, kOFull1, kOFree0, kOFree1,
+    kSFull, kSReady, kZV0, kZV1,                 // state epilogue <-> MMA
     kDrain
 };
 
@@ -339,9 +348,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             int issued = -1;
+            constexpr int NS = Lay::kStages;
             for (int i = 0; i < nchunks; ++i) {
-                const int s = i & 1;
-                if (i >= 2 && !mbar_wait(bar(kEmpty0 + s), ((i >> 1) - 1) & 1, abort_flag)) break;
+                const int s = i % NS;
+                if (i >= NS && !mbar_wait(bar(kEmpty0 + s), ((i / NS) - 1) & 1, abort_flag)) break;
                 const uint32_t st = sbase + Lay::kStage0 + s * Lay::kStageBytes;
                 mbar_expect_tx(bar(kFull0 + s), STATE_ONLY ? Lay::kKBytes + Lay::kVBytes : Lay::kStageBytes);
                 const int t0 = (cbase + i) * kC;
@@ -356,8 +366,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             if (*abort_flag && issued >= 0) {
                 // drain the copies in flight before the CTA may exit
-                for (int i = (issued >= 1 ? issued - 1 : 0); i <= issued; ++i)
-                    mbar_drain(bar(kFull0 + (i & 1)), (i >> 1) & 1);
+                for (int i = std::max(issued - NS + 1, 0); i <= issued; ++i)
+                    mbar_drain(bar(kFull0 + i % NS), (i / NS) & 1);
             }
         }
     } else if (warp == 1) {
@@ -367,18 +377,38 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             constexpr uint32_t id_oi = idesc(128, kC, 0, 0);
             constexpr uint32_t id_ov = idesc(128, kC, 1, 0);
             constexpr uint32_t id_up = idesc(128, DK, 1, 1);
-            const uint32_t tA = tmem + Lay::kColA, tO = tmem + Lay::kColO;
+            constexpr int NB = Lay::kNBuf;
             const uint32_t tS = tmem + Lay::kColS, tSop = tmem + Lay::kColSop;
-            const uint32_t sP = sbase + Lay::kP;
-            for (int i = 0; i < nchunks; ++i) {
-                const int s = i & 1;
+            // A = Q K^T of chunk c into attention buffer c % NB (both K-major, 128-byte swizzle,
+            // 16-element K steps); the buffer is free once chunk c - NB has been drained.
+            auto issue_qk = [&](int c) {
+                const int s = c % Lay::kStages, b = c % NB;
+                const uint32_t sQ = sbase + Lay::kStage0 + s * Lay::kStageBytes;
+                const uint32_t sK = sQ + Lay::kQBytes;
+                if (!mbar_wait(bar(kFull0 + s), (c / Lay::kStages) & 1, abort_flag)) return false;
+                if (c >= NB && !mbar_wait(bar(kOFree0 + b), ((c / NB) - 1) & 1, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t tA = tmem + Lay::kColA + 2 * kC * b;
+#pragma unroll
+                for (int ks = 0; ks < DK / 16; ++ks) {
+                    const uint32_t off = (ks >> 2) * kTile64 + (ks & 3) * 32;
+                    mma_ss(tA, sdesc(sQ + off, 16, 1024), sdesc(sK + off, 16, 1024), id_qk, ks > 0);
+                }
+                mma_commit(bar(kAFull0 + b));
+                return true;
+            };
+            const bool primed = STATE_ONLY || NB == 1 || nchunks == 0 || issue_qk(0);
+            for (int i = 0; primed && i < nchunks; ++i) {
+                const int s = i % Lay::kStages, z = i & 1, b = i % NB;  // TMA stage, ZV buffer, attention buffer
                 const uint32_t sQ = sbase + Lay::kStage0 + s * Lay::kStageBytes;
                 const uint32_t sK = sQ + Lay::kQBytes;
                 const uint32_t sV = sK + Lay::kKBytes;
-                const uint32_t sZV = sbase + Lay::kZV + s * Lay::kVBytes;
-                if (!mbar_wait(bar(kFull0 + s), (i >> 1) & 1, abort_flag)) break;
+                const uint32_t sZV = sbase + Lay::kZV + z * Lay::kVBytes;
+                const uint32_t tA = tmem + Lay::kColA + 2 * kC * b, tO = tmem + Lay::kColO + 2 * kC * b;
+                const uint32_t sP = sbase + Lay::kP + b * kTile64;
                 if (STATE_ONLY) {
-                    if (!mbar_wait(bar(kZV0 + s), (i >> 1) & 1, abort_flag) ||
+                    if (!mbar_wait(bar(kFull0 + s), (i / Lay::kStages) & 1, abort_flag)) break;
+                    if (!mbar_wait(bar(kZV0 + z), (i >> 1) & 1, abort_flag) ||
                         !mbar_wait(bar(kSReady), i & 1, abort_flag))
                         break;
                     tc_fence_after();
@@ -389,37 +419,39 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     mma_commit(bar(kEmpty0 + s));
                     continue;
                 }
-                if (i > 0 && !mbar_wait(bar(kOFree), (i - 1) & 1, abort_flag)) break;
-                tc_fence_after();
-                // A = Q K^T (both K-major, 128-byte swizzle; 16-element K steps)
-#pragma unroll
-                for (int ks = 0; ks < DK / 16; ++ks) {
-                    const uint32_t off = (ks >> 2) * kTile64 + (ks & 3) * 32;
-                    mma_ss(tA, sdesc(sQ + off, 16, 1024), sdesc(sK + off, 16, 1024), id_qk, ks > 0);
+                // With two buffers the next chunk's Q K^T is issued ahead, so the tensor pipe has
+                // it while the epilogue masks this chunk; with one buffer it is this chunk's.
+                if (NB == 1) {
+                    if (!issue_qk(i)) break;
+                } else if (i + 1 < nchunks) {
+                    if (!issue_qk(i + 1)) break;
                 }
-                mma_commit(bar(kAFull));
-                // The state update goes first: it needs only zeta V and the decayed state, so it
+                // The state update goes next: it needs only zeta V and the decayed state, so it
                 // runs while the epilogue builds P, and the O drain later has the pipe to itself.
-                if (!mbar_wait(bar(kZV0 + s), (i >> 1) & 1, abort_flag) || !mbar_wait(bar(kSReady), i & 1, abort_flag))
+                if (!mbar_wait(bar(kZV0 + z), (i >> 1) & 1, abort_flag) || !mbar_wait(bar(kSReady), i & 1, abort_flag))
                     break;
                 tc_fence_after();
                 // S^T += (zeta V)^T K: A = ZV MN-major, B = K tile MN-major (dk blocks 8 KB apart)
 #pragma unroll
                 for (int ks = 0; ks < kC / 16; ++ks)
                     mma_ss(tS, sdesc(sZV + ks * 2048, kTile64, 1024), sdesc(sK + ks * 2048, kTile64, 1024), id_up, 1);
-                if (!mbar_wait(bar(kPReady), i & 1, abort_flag)) break;
+                // O_inter^T = S_op^T Q^T into the same TMEM columns as Q K^T: only needs the
+                // epilogue to have read Q K^T, not to have finished P.
+                if (!mbar_wait(bar(kARead0 + b), (i / NB) & 1, abort_flag)) break;
                 tc_fence_after();
-                // O_inter^T = S_op^T Q^T: A from TMEM (bf16 pairs per column), B = Q tile K-major
+                // A from TMEM (bf16 pairs per column), B = Q tile K-major
 #pragma unroll
                 for (int ks = 0; ks < DK / 16; ++ks) {
                     const uint32_t off = (ks >> 2) * kTile64 + (ks & 3) * 32;
                     mma_ts(tA, tSop + ks * 8, sdesc(sQ + off, 16, 1024), id_oi, ks > 0);
                 }
+                if (!mbar_wait(bar(kPReady0 + b), (i / NB) & 1, abort_flag)) break;
+                tc_fence_after();
                 // O_intra^T = V^T P^T: A = V tile MN-major (dv blocks 8 KB apart), B = P K-major
 #pragma unroll
                 for (int ks = 0; ks < kC / 16; ++ks)
                     mma_ss(tO, sdesc(sV + ks * 2048, kTile64, 1024), sdesc(sP + ks * 32, 16, 1024), id_ov, ks > 0);
-                mma_commit(bar(kOFull));
+                mma_commit(bar(kOFull0 + b));
                 // S_i is final and the cross term has read S_op: the state epilogue may now
                 // overwrite S_op and decay S.
                 mma_commit(bar(kSFull));
@@ -436,9 +468,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int quarter = warp & 3;             // TMEM lane quarter this warp may access
         const int d = quarter * 32 + lane;        // dv column of the slice = TMEM lane
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        float* cum = reinterpret_cast<float*>(sm + Lay::kAgTab);  // gated: in-chunk cumsum, log2 units
-        float* rr = cum + kC;                                     // cross-term row factor r_j
-        float* pw = rr + kC;                                      // fixed gamma: gamma^t, t = 0..64
+        constexpr int NB = Lay::kNBuf;
+        float* cum = reinterpret_cast<float*>(sm + Lay::kAgTab);  // gated: in-chunk cumsum (log2 units), per buffer
+        float* rr = cum + 2 * kC;                                 // cross-term row factor r_j, per buffer
+        float* pw = rr + 2 * kC;                                  // fixed gamma: gamma^t, t = 0..64
         auto wait_all = [&](int b, uint32_t parity) {  // every thread reaches the barrier; uniform result
             mbar_wait(bar(b), parity, abort_flag);
             group_sync(1);
@@ -455,32 +488,34 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             g0 = (a < p.N ? G[a] : 0.f) * kLog2e;
             g1 = (a + 1 < p.N ? G[a + 1] : 0.f) * kLog2e;
         }
-        for (int i = 0; i < nchunks; ++i) {
-            const int t0 = (cbase + i) * kC;
+        // ---------------- P = mask(Q K^T) of chunk c in bf16 (buffer c % NB): row j, 32 columns per thread
+        auto do_p = [&](int ci) {
+            const int b = ci % NB;
+            const int t0 = (cbase + ci) * kC;
+            float* cumb = cum + b * kC;
             if (GATED) {
                 if (te < 32) {
-                    warp_cumsum64(g0, g1, lane, cum);
+                    warp_cumsum64(g0, g1, lane, cumb);
                     const int a = t0 + kC + 2 * te;
                     g0 = (a < p.N ? G[a] : 0.f) * kLog2e;
                     g1 = (a + 1 < p.N ? G[a + 1] : 0.f) * kLog2e;
                 }
                 group_sync(1);
-                if (te < kC) rr[te] = exp2f(cum[te]);
+                if (te < kC) rr[b * kC + te] = exp2f(cumb[te]);
             }
-            // ---------------- P = mask(Q K^T) in bf16: row j, 32 columns per thread
-            if (!wait_all(kAFull, i & 1)) break;
+            if (!wait_all(kAFull0 + b, (ci / NB) & 1)) return false;
             tc_fence_after();
             {
                 uint32_t a[32];
-                tmem_ld16x2(tmem + lane_off + Lay::kColA, a);
+                tmem_ld16x2(tmem + lane_off + Lay::kColA + 2 * kC * b, a);
                 const int j = quarter * 16 + (lane & 15);  // M=64 accumulator: row j in lane 32*(j/16) + j%16
                 const int m0 = (lane >> 4) * 32;
                 // all table reads before any shared-memory store (the pointers may alias)
                 float w[32];
                 if (GATED) {
-                    const float cj = cum[j];
+                    const float cj = cumb[j];
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) w[c] = cj - cum[m0 + c];
+                    for (int c = 0; c < 32; ++c) w[c] = cj - cumb[m0 + c];
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
                         const int m = m0 + c;
@@ -494,11 +529,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                 }
                 tmem_wait_ld();
+                // Q K^T is in registers: the cross-term product may overwrite those columns now
+                tc_fence_before();
+                group_sync(1);
+                if (te == 0) mbar_arrive(bar(kARead0 + b));
                 uint32_t u[16];
 #pragma unroll
                 for (int c = 0; c < 16; ++c)
                     u[c] = pack_bf16(__uint_as_float(a[2 * c]) * w[2 * c], __uint_as_float(a[2 * c + 1]) * w[2 * c + 1]);
-                uint8_t* prow = sm + Lay::kP + j * 128;
+                uint8_t* prow = sm + Lay::kP + b * kTile64 + j * 128;
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
                     const int chunk16 = (m0 >> 3) + cc;
@@ -509,12 +548,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             fence_proxy_async();
             tc_fence_before();
             group_sync(1);
-            if (te == 0) {
-                mbar_arrive(bar(kPReady));
-                tma_store_wait_read();  // previous chunk's O store has read the staging tile
-            }
-            // ---------------- O = O_intra + r_j O_inter -> bf16 -> staging -> TMA store
-            if (!wait_all(kOFull, i & 1)) break;
+            if (te == 0) mbar_arrive(bar(kPReady0 + b));
+            return true;
+        };
+        // ---------------- O = O_intra + r_j O_inter of chunk c -> bf16 -> staging -> TMA store
+        auto do_drain = [&](int ci) {
+            const int b = ci % NB;
+            const int t0 = (cbase + ci) * kC;
+            const float* rrb = GATED ? rr + b * kC : rr;
+            if (te == 0) tma_store_wait_read();  // the previous chunk's O store has read the staging tile
+            if (!wait_all(kOFull0 + b, (ci / NB) & 1)) return false;
             tc_fence_after();
             {
                 // Each thread owns dv column d for all 64 tokens. A lane-pair shuffle packs two
@@ -523,18 +566,28 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const bool odd = lane & 1;
                 const int cb = ((d & 63) & ~1) * 2;  // byte offset of the dv pair inside a 128-byte row
                 uint8_t* ost = sm + Lay::kOst + (d >> 6) * kTile64;
+                // Both accumulators of all 64 tokens into registers first, then release the TMEM
+                // columns so the next chunk's Q K^T can start while this drain finishes.
+                uint32_t oi[2][32], oe[2][32];
 #pragma unroll
                 for (int jb = 0; jb < 2; ++jb) {
-                    uint32_t oi[32], oe[32];
-                    tmem_ld32(tmem + lane_off + Lay::kColO + jb * 32, oi);
-                    tmem_ld32(tmem + lane_off + Lay::kColA + jb * 32, oe);
-                    float rv[32];
+                    tmem_ld32(tmem + lane_off + Lay::kColO + 2 * kC * b + jb * 32, oi[jb]);
+                    tmem_ld32(tmem + lane_off + Lay::kColA + 2 * kC * b + jb * 32, oe[jb]);
+                }
+                tmem_wait_ld();
+                tc_fence_before();
+                group_sync(1);
+                if (te == 0) mbar_arrive(bar(kOFree0 + b));
+                // combine in place, every table read before the first shared store (aliasing)
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) rv[jj] = rr[jb * 32 + jj];
-                    tmem_wait_ld();
-                    float o[32];
+                for (int jb = 0; jb < 2; ++jb)
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) o[jj] = fmaf(rv[jj], __uint_as_float(oe[jj]), __uint_as_float(oi[jj]));
+                    for (int jj = 0; jj < 32; ++jj)
+                        oi[jb][jj] = __float_as_uint(
+                            fmaf(rrb[jb * 32 + jj], __uint_as_float(oe[jb][jj]), __uint_as_float(oi[jb][jj])));
+#pragma unroll
+                for (int jb = 0; jb < 2; ++jb) {
+                    const float* o = reinterpret_cast<const float*>(oi[jb]);
                     uint32_t w[16];
 #pragma unroll
                     for (int u = 0; u < 16; ++u) {
@@ -551,14 +604,25 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
             }
             fence_proxy_async();
-            tc_fence_before();
             group_sync(1);
             if (te == 0) {
-                mbar_arrive(bar(kOFree));
                 tma_store_3d(&tm_o, dv0, t0, bh, sbase + Lay::kOst);
                 tma_store_3d(&tm_o, dv0 + 64, t0, bh, sbase + Lay::kOst + kTile64);
                 tma_store_commit();
             }
+            return true;
+        };
+        // With two buffers the mask of chunk i+1 is built while chunk i's output products run,
+        // then chunk i is drained; with one buffer the chunks go mask, drain, mask, drain.
+        if (NB == 2) {
+            bool ok = nchunks == 0 || do_p(0);
+            for (int i = 0; ok && i < nchunks; ++i) {
+                if (i + 1 < nchunks) ok = do_p(i + 1);
+                ok = ok && do_drain(i);
+            }
+        } else {
+            for (int i = 0; i < nchunks; ++i)
+                if (!do_p(i) || !do_drain(i)) break;
         }
         if (te == 0) tma_store_wait_all();
       }
@@ -612,13 +676,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     dec[1] = lg * (float)L;
                 }
             }
-            if (!wait_all(kFull0 + (c & 1), (c >> 1) & 1)) return false;  // V tile of chunk c has landed
+            if (!wait_all(kFull0 + c % Lay::kStages, (c / Lay::kStages) & 1)) return false;  // V tile of chunk c landed
             decay = dec[0];
             ldec_sum += dec[1];
             renorm = force_renorm || !(c_prev * decay >= kRenorm);
             c_next = renorm ? 1.f : c_prev * decay;
             const float inv = 1.f / c_next;
-            const uint8_t* vt = sm + Lay::kStage0 + (c & 1) * Lay::kStageBytes + Lay::kQBytes + Lay::kKBytes;
+            const uint8_t* vt = sm + Lay::kStage0 + (c % Lay::kStages) * Lay::kStageBytes + Lay::kQBytes + Lay::kKBytes;
             uint8_t* zv = sm + Lay::kZV + (c & 1) * Lay::kVBytes;
             // 16-byte chunks ci = e * 128 + ts; the swizzle stays inside a 128-byte row, so the
             // row (token) of a chunk is (ci mod 512) / 8. All loads before any store (aliasing).
