@@ -17,7 +17,10 @@
 // kept in registers): each chunk the epilogue reads T once and writes the
 // bf16 copy of S (the next cross term's MMA operand); the update adds
 // (zeta V / c) onto T, and T is rescaled in place only when c would underflow.
-// The decay mask is generated in registers.
+// The decay mask is generated in registers. For a fixed gamma in [1/2, 1] the two
+// output products add into one accumulator (decay factors moved onto the state copy,
+// P and the drain; derivation at the kernel), which frees TMEM to double-buffer the
+// attention products even at dk = 256.
 //
 // Roles (320 threads): warp 0 issues TMA loads (two stages of Q, K, V tiles);
 // warp 1 allocates TMEM and issues every tcgen05.mma from one thread; warps 2-5
@@ -52,16 +55,18 @@ struct Layout {
     static constexpr int kVBytes = 2 * kTile64;
     static constexpr int kStageBytes = kQBytes + kKBytes + kVBytes;
     static constexpr int kStage0 = 0;
-    // Attention buffers: with dk <= 128 there is TMEM for two sets of {Q K^T / O_inter,
-    // O_intra} accumulators and shared memory for two P tiles, so chunk i+1's Q K^T and mask
-    // overlap chunk i's output products and drain. With dk = 256 the state fills TMEM and
-    // one set is used in turn.
-    static constexpr int kNBuf = DK <= 128 ? 2 : 1;
+    // Attention buffers. Two of them let chunk i+1's Q K^T and mask overlap chunk i's output
+    // products and drain. A buffer holds Q K^T, then O_inter^T in the same columns, plus a
+    // separate O_intra^T region (128 columns) -- or, with the merged output accumulator
+    // (fixed gamma, see the kernel), one region of 64 columns that both products add into.
+    // With dk <= 128 TMEM has room for two split buffers; with dk = 256 the state takes 384
+    // columns and the remaining 128 hold two merged buffers or one split buffer.
+    static constexpr int kPTiles = 2;
     // TMA stages of Q, K, V tiles: three where shared memory allows, so that loads run two
     // chunks ahead of the products that read them.
     static constexpr int kStages = DK <= 128 ? 3 : 2;
-    static constexpr int kP = kStages * kStageBytes;        // P tiles (64 x 64 bf16, SW128 K-major), kNBuf of them
-    static constexpr int kZV = kP + kNBuf * kTile64;        // zeta-scaled V, two buffers (V tile layout)
+    static constexpr int kP = kStages * kStageBytes;        // P tiles (64 x 64 bf16, SW128 K-major), one per buffer
+    static constexpr int kZV = kP + kPTiles * kTile64;      // zeta-scaled V, two buffers (V tile layout)
     static constexpr int kOst = kZV + 2 * kVBytes;          // O staging for the TMA store (128-byte swizzle)
     static constexpr int kBar = kOst + kVBytes;             // mbarriers
     static constexpr int kNumBars = 22;
@@ -74,9 +79,8 @@ struct Layout {
     // TMEM columns
     static constexpr int kColS = 0;                 // fp32 state S^T: DK columns
     static constexpr int kColSop = DK;              // bf16 state copy: DK/2 columns
-    static constexpr int kColA = DK + DK / 2;       // buffer b: Q K^T then O_inter^T at kColA + 2*kC*b (64 columns)
-    static constexpr int kColO = kColA + kC;        // buffer b: O_intra^T at kColO + 2*kC*b (64 columns)
-    static constexpr int kColsUsed = kColA + 2 * kC * kNBuf;
+    static constexpr int kColA = DK + DK / 2;       // attention buffers from here (Q K^T, O_inter^T, O_intra^T)
+    static constexpr int kColsUsed = kColA + (DK <= 128 ? 4 : 2) * kC;
     static constexpr int kTmemCols = kColsUsed <= 256 ? 256 : 512;
     static_assert(kColsUsed <= 512, "TMEM overflow");
     static_assert(kSmemAlloc <= 227 * 1024, "shared memory overflow");
@@ -343,6 +347,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t tmem = *tmem_slot;
     const float* G = GATED ? p.decay_in + (size_t)bh * p.N : nullptr;
     const float lg = GATED ? 0.f : log2f(p.decay_in[bh % p.H]);
+    // Merged output accumulator (fixed gamma). With zeta'_j = gamma^(63-j), the decay mask
+    // factors as gamma^(j-m) = zeta'_m / zeta'_j and the cross factor as gamma^(j+1) =
+    // gamma^64 / zeta'_j, so
+    //   O_j = (1 / zeta'_j) [ q_j (gamma^64 S) + sum_{m<=j} zeta'_m A_jm v_m ]
+    // and both products accumulate into one TMEM region: the bf16 state copy holds
+    // gamma^64 S, P holds zeta'_m A_jm, and the drain scales row j by 1 / zeta'_j. All
+    // factors stay within [2^-64, 2^63] when gamma is in [1/2, 1], so nothing leaves the
+    // normal range of bf16 or fp32 that the split form would keep; other gammas (and the
+    // gated form) use the split accumulators. The choice is per CTA (one head).
+    const bool merged = !GATED && !STATE_ONLY && lg >= -1.f && lg <= 0.f;
+    const int nb = (DK <= 128 || merged) ? 2 : 1;  // attention buffers in use
+    const int bcols = merged ? kC : 2 * kC;        // TMEM columns per attention buffer
+    auto abuf = [&](int c) { return nb == 2 ? (c & 1) : 0; };   // attention buffer of chunk c
+    auto ause = [&](int c) { return nb == 2 ? (c >> 1) : c; };  // how many chunks used that buffer before
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -377,18 +395,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             constexpr uint32_t id_oi = idesc(128, kC, 0, 0);
             constexpr uint32_t id_ov = idesc(128, kC, 1, 0);
             constexpr uint32_t id_up = idesc(128, DK, 1, 1);
-            constexpr int NB = Lay::kNBuf;
             const uint32_t tS = tmem + Lay::kColS, tSop = tmem + Lay::kColSop;
-            // A = Q K^T of chunk c into attention buffer c % NB (both K-major, 128-byte swizzle,
-            // 16-element K steps); the buffer is free once chunk c - NB has been drained.
+            // A = Q K^T of chunk c into its attention buffer (both K-major, 128-byte swizzle,
+            // 16-element K steps); the buffer is free once its previous chunk has been drained.
             auto issue_qk = [&](int c) {
-                const int s = c % Lay::kStages, b = c % NB;
+                const int s = c % Lay::kStages, b = abuf(c);
                 const uint32_t sQ = sbase + Lay::kStage0 + s * Lay::kStageBytes;
                 const uint32_t sK = sQ + Lay::kQBytes;
                 if (!mbar_wait(bar(kFull0 + s), (c / Lay::kStages) & 1, abort_flag)) return false;
-                if (c >= NB && !mbar_wait(bar(kOFree0 + b), ((c / NB) - 1) & 1, abort_flag)) return false;
+                if (c >= nb && !mbar_wait(bar(kOFree0 + b), (ause(c) - 1) & 1, abort_flag)) return false;
                 tc_fence_after();
-                const uint32_t tA = tmem + Lay::kColA + 2 * kC * b;
+                const uint32_t tA = tmem + Lay::kColA + bcols * b;
 #pragma unroll
                 for (int ks = 0; ks < DK / 16; ++ks) {
                     const uint32_t off = (ks >> 2) * kTile64 + (ks & 3) * 32;
@@ -397,14 +414,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 mma_commit(bar(kAFull0 + b));
                 return true;
             };
-            const bool primed = STATE_ONLY || NB == 1 || nchunks == 0 || issue_qk(0);
+            const bool primed = STATE_ONLY || nb == 1 || nchunks == 0 || issue_qk(0);
             for (int i = 0; primed && i < nchunks; ++i) {
-                const int s = i % Lay::kStages, z = i & 1, b = i % NB;  // TMA stage, ZV buffer, attention buffer
+                const int s = i % Lay::kStages, z = i & 1, b = abuf(i);  // TMA stage, ZV buffer, attention buffer
                 const uint32_t sQ = sbase + Lay::kStage0 + s * Lay::kStageBytes;
                 const uint32_t sK = sQ + Lay::kQBytes;
                 const uint32_t sV = sK + Lay::kKBytes;
                 const uint32_t sZV = sbase + Lay::kZV + z * Lay::kVBytes;
-                const uint32_t tA = tmem + Lay::kColA + 2 * kC * b, tO = tmem + Lay::kColO + 2 * kC * b;
+                // merged: both output products add into the Q K^T columns; split: O_intra has its own
+                const uint32_t tA = tmem + Lay::kColA + bcols * b, tO = merged ? tA : tA + kC;
                 const uint32_t sP = sbase + Lay::kP + b * kTile64;
                 if (STATE_ONLY) {
                     if (!mbar_wait(bar(kFull0 + s), (i / Lay::kStages) & 1, abort_flag)) break;
@@ -419,15 +437,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     mma_commit(bar(kEmpty0 + s));
                     continue;
                 }
-                // With two buffers the next chunk's Q K^T is issued ahead, so the tensor pipe has
-                // it while the epilogue masks this chunk; with one buffer it is this chunk's.
-                if (NB == 1) {
-                    if (!issue_qk(i)) break;
-                } else if (i + 1 < nchunks) {
-                    if (!issue_qk(i + 1)) break;
-                }
-                // The state update goes next: it needs only zeta V and the decayed state, so it
-                // runs while the epilogue builds P, and the O drain later has the pipe to itself.
+                // Issue order. The state round trip (the state epilogue reads S_i and writes the
+                // next bf16 copy) is the loop-carried chain, so the products it waits for go first
+                // and are committed on their own: update(i), O_inter(i) -> kSFull. The rest of the
+                // chunk's tensor work -- the next chunk's Q K^T (two buffers) and O_intra(i) --
+                // then runs in the pipe while the round trip is under way.
+                if (nb == 1 && !issue_qk(i)) break;
                 if (!mbar_wait(bar(kZV0 + z), (i >> 1) & 1, abort_flag) || !mbar_wait(bar(kSReady), i & 1, abort_flag))
                     break;
                 tc_fence_after();
@@ -437,7 +452,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     mma_ss(tS, sdesc(sZV + ks * 2048, kTile64, 1024), sdesc(sK + ks * 2048, kTile64, 1024), id_up, 1);
                 // O_inter^T = S_op^T Q^T into the same TMEM columns as Q K^T: only needs the
                 // epilogue to have read Q K^T, not to have finished P.
-                if (!mbar_wait(bar(kARead0 + b), (i / NB) & 1, abort_flag)) break;
+                if (!mbar_wait(bar(kARead0 + b), ause(i) & 1, abort_flag)) break;
                 tc_fence_after();
                 // A from TMEM (bf16 pairs per column), B = Q tile K-major
 #pragma unroll
@@ -445,16 +460,18 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     const uint32_t off = (ks >> 2) * kTile64 + (ks & 3) * 32;
                     mma_ts(tA, tSop + ks * 8, sdesc(sQ + off, 16, 1024), id_oi, ks > 0);
                 }
-                if (!mbar_wait(bar(kPReady0 + b), (i / NB) & 1, abort_flag)) break;
+                // S_i is final and the cross term has read S_op: the state epilogue may now
+                // overwrite S_op and decay S.
+                mma_commit(bar(kSFull));
+                if (nb == 2 && i + 1 < nchunks && !issue_qk(i + 1)) break;
+                if (!mbar_wait(bar(kPReady0 + b), ause(i) & 1, abort_flag)) break;
                 tc_fence_after();
                 // O_intra^T = V^T P^T: A = V tile MN-major (dv blocks 8 KB apart), B = P K-major
 #pragma unroll
                 for (int ks = 0; ks < kC / 16; ++ks)
-                    mma_ss(tO, sdesc(sV + ks * 2048, kTile64, 1024), sdesc(sP + ks * 32, 16, 1024), id_ov, ks > 0);
+                    mma_ss(tO, sdesc(sV + ks * 2048, kTile64, 1024), sdesc(sP + ks * 32, 16, 1024), id_ov,
+                           merged || ks > 0);
                 mma_commit(bar(kOFull0 + b));
-                // S_i is final and the cross term has read S_op: the state epilogue may now
-                // overwrite S_op and decay S.
-                mma_commit(bar(kSFull));
                 mma_commit(bar(kEmpty0 + s));
             }
             // every issued MMA must complete before TMEM can be released
@@ -468,9 +485,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int quarter = warp & 3;             // TMEM lane quarter this warp may access
         const int d = quarter * 32 + lane;        // dv column of the slice = TMEM lane
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        constexpr int NB = Lay::kNBuf;
         float* cum = reinterpret_cast<float*>(sm + Lay::kAgTab);  // gated: in-chunk cumsum (log2 units), per buffer
-        float* rr = cum + 2 * kC;                                 // cross-term row factor r_j, per buffer
+        float* rr = cum + 2 * kC;  // row factor of the drain, per buffer: r_j (split), 1 / zeta'_j (merged)
         float* pw = rr + 2 * kC;                                  // fixed gamma: gamma^t, t = 0..64
         auto wait_all = [&](int b, uint32_t parity) {  // every thread reaches the barrier; uniform result
             mbar_wait(bar(b), parity, abort_flag);
@@ -480,7 +496,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (!GATED) {
             if (te <= kC) pw[te] = pow_int_log2(lg, te);
             group_sync(1);
-            if (te < kC) rr[te] = pw[te + 1];
+            if (te < kC) rr[te] = merged ? pow_int_log2(-lg, kC - 1 - te) : pw[te + 1];
         }
         float g0 = 0.f, g1 = 0.f;  // gated: prefetched gate values of the next chunk (first warp)
         if (GATED && te < 32) {
@@ -488,9 +504,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             g0 = (a < p.N ? G[a] : 0.f) * kLog2e;
             g1 = (a + 1 < p.N ? G[a + 1] : 0.f) * kLog2e;
         }
-        // ---------------- P = mask(Q K^T) of chunk c in bf16 (buffer c % NB): row j, 32 columns per thread
+        // ---------------- P = mask(Q K^T) of chunk c in bf16 (its attention buffer): row j, 32 columns per thread
         auto do_p = [&](int ci) {
-            const int b = ci % NB;
+            const int b = abuf(ci);
             const int t0 = (cbase + ci) * kC;
             float* cumb = cum + b * kC;
             if (GATED) {
@@ -503,11 +519,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 group_sync(1);
                 if (te < kC) rr[b * kC + te] = exp2f(cumb[te]);
             }
-            if (!wait_all(kAFull0 + b, (ci / NB) & 1)) return false;
+            if (!wait_all(kAFull0 + b, ause(ci) & 1)) return false;
             tc_fence_after();
             {
                 uint32_t a[32];
-                tmem_ld16x2(tmem + lane_off + Lay::kColA + 2 * kC * b, a);
+                tmem_ld16x2(tmem + lane_off + Lay::kColA + bcols * b, a);
                 const int j = quarter * 16 + (lane & 15);  // M=64 accumulator: row j in lane 32*(j/16) + j%16
                 const int m0 = (lane >> 4) * 32;
                 // all table reads before any shared-memory store (the pointers may alias)
@@ -522,10 +538,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         w[c] = m > j ? 0.f : (m == j ? 1.f : exp2f(w[c]));
                     }
                 } else {
+                    // split: gamma^(j-m); merged: zeta'_m = gamma^(63-m)
+                    const int base = merged ? kC - 1 : j;
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
                         const int m = m0 + c;
-                        w[c] = m > j ? 0.f : pw[j - m];
+                        w[c] = m > j ? 0.f : pw[base - m];
                     }
                 }
                 tmem_wait_ld();
@@ -553,11 +571,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         };
         // ---------------- O = O_intra + r_j O_inter of chunk c -> bf16 -> staging -> TMA store
         auto do_drain = [&](int ci) {
-            const int b = ci % NB;
+            const int b = abuf(ci);
             const int t0 = (cbase + ci) * kC;
             const float* rrb = GATED ? rr + b * kC : rr;
+            const uint32_t tA = tmem + lane_off + Lay::kColA + bcols * b;
             if (te == 0) tma_store_wait_read();  // the previous chunk's O store has read the staging tile
-            if (!wait_all(kOFull0 + b, (ci / NB) & 1)) return false;
+            if (!wait_all(kOFull0 + b, ause(ci) & 1)) return false;
             tc_fence_after();
             {
                 // Each thread owns dv column d for all 64 tokens. A lane-pair shuffle packs two
@@ -566,25 +585,41 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const bool odd = lane & 1;
                 const int cb = ((d & 63) & ~1) * 2;  // byte offset of the dv pair inside a 128-byte row
                 uint8_t* ost = sm + Lay::kOst + (d >> 6) * kTile64;
-                // Both accumulators of all 64 tokens into registers first, then release the TMEM
+                // The accumulators of all 64 tokens into registers first, then release the TMEM
                 // columns so the next chunk's Q K^T can start while this drain finishes.
-                uint32_t oi[2][32], oe[2][32];
+                uint32_t oi[2][32];
+                if (merged) {
 #pragma unroll
-                for (int jb = 0; jb < 2; ++jb) {
-                    tmem_ld32(tmem + lane_off + Lay::kColO + 2 * kC * b + jb * 32, oi[jb]);
-                    tmem_ld32(tmem + lane_off + Lay::kColA + 2 * kC * b + jb * 32, oe[jb]);
+                    for (int jb = 0; jb < 2; ++jb) tmem_ld32(tA + jb * 32, oi[jb]);
+                    tmem_wait_ld();
+                    tc_fence_before();
+                    group_sync(1);
+                    if (te == 0) mbar_arrive(bar(kOFree0 + b));
+                    // O_j = Z_j / zeta'_j, every table read before the first shared store (aliasing)
+#pragma unroll
+                    for (int jb = 0; jb < 2; ++jb)
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj)
+                            oi[jb][jj] = __float_as_uint(rrb[jb * 32 + jj] * __uint_as_float(oi[jb][jj]));
+                } else {
+                    uint32_t oe[2][32];
+#pragma unroll
+                    for (int jb = 0; jb < 2; ++jb) {
+                        tmem_ld32(tA + kC + jb * 32, oi[jb]);
+                        tmem_ld32(tA + jb * 32, oe[jb]);
+                    }
+                    tmem_wait_ld();
+                    tc_fence_before();
+                    group_sync(1);
+                    if (te == 0) mbar_arrive(bar(kOFree0 + b));
+                    // O = O_intra + r_j O_inter in place, every table read before the first shared store
+#pragma unroll
+                    for (int jb = 0; jb < 2; ++jb)
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj)
+                            oi[jb][jj] = __float_as_uint(
+                                fmaf(rrb[jb * 32 + jj], __uint_as_float(oe[jb][jj]), __uint_as_float(oi[jb][jj])));
                 }
-                tmem_wait_ld();
-                tc_fence_before();
-                group_sync(1);
-                if (te == 0) mbar_arrive(bar(kOFree0 + b));
-                // combine in place, every table read before the first shared store (aliasing)
-#pragma unroll
-                for (int jb = 0; jb < 2; ++jb)
-#pragma unroll
-                    for (int jj = 0; jj < 32; ++jj)
-                        oi[jb][jj] = __float_as_uint(
-                            fmaf(rrb[jb * 32 + jj], __uint_as_float(oe[jb][jj]), __uint_as_float(oi[jb][jj])));
 #pragma unroll
                 for (int jb = 0; jb < 2; ++jb) {
                     const float* o = reinterpret_cast<const float*>(oi[jb]);
@@ -614,7 +649,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         };
         // With two buffers the mask of chunk i+1 is built while chunk i's output products run,
         // then chunk i is drained; with one buffer the chunks go mask, drain, mask, drain.
-        if (NB == 2) {
+        if (nb == 2) {
             bool ok = nchunks == 0 || do_p(0);
             for (int i = 0; ok && i < nchunks; ++i) {
                 if (i + 1 < nchunks) ok = do_p(i + 1);
@@ -710,11 +745,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             return true;
         };
 
+        // The bf16 state copy is S (split output accumulators) or gamma^64 S (merged).
+        const float sop = merged ? pow_int_log2(lg, kC) : 1.f;
         float dec0 = 0.f, c_cur = 1.f;
         bool renorm = true;
         bool ok = make_zv(0, 1.f, true, dec0, renorm, c_cur);
         if (ok) {
-            // initial state: S_op = bf16(S_in), T = decay_0 * S_in, c = 1. S_in is state_in (or
+            // initial state: S_op = bf16(sop S_in), T = decay_0 * S_in, c = 1. S_in is state_in (or
             // zero) for the first segment; segment g > 0 folds in the earlier segments' end states:
             // S_in(g) = decay_{g-1} S_in(g-1) + U_{g-1}. The state-only pass starts from zero.
             const float* sin = (!STATE_ONLY && p.state_in) ? p.state_in + ((size_t)bh * DK) * p.dv + dv0 + d : nullptr;
@@ -735,7 +772,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
 #pragma unroll
                 for (int c = 0; c < 16; ++c)
-                    h[c] = pack_bf16(__uint_as_float(w[2 * c]), __uint_as_float(w[2 * c + 1]));
+                    h[c] = pack_bf16(__uint_as_float(w[2 * c]) * sop, __uint_as_float(w[2 * c + 1]) * sop);
 #pragma unroll
                 for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(__uint_as_float(w[c]) * dec0);
                 tmem_st32(tmem + lane_off + Lay::kColS + cb * 32, w);
@@ -773,10 +810,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                 }
             } else if (!STATE_ONLY || renorm) {
-                // S_op = bf16(c_i T_i) for the next cross term; on renormalisation also
+                // S_op = bf16(sop c_i T_i) for the next cross term; on renormalisation also
                 // T <- c_i d_{i+1} T_i so that the next update (scaled by 1/c_{i+1} = 1) adds onto it.
                 // The state-only pass needs no S_op and touches T only to renormalise.
-                const float tscale = c_cur * dec_next;
+                const float tscale = c_cur * dec_next, hscale = c_cur * sop;
 #pragma unroll 1
                 for (int cb = 0; cb < DK / 64; ++cb) {
                     uint32_t w0[32], w1[32], h[16];
@@ -786,11 +823,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     if (!STATE_ONLY) {
 #pragma unroll
                         for (int c = 0; c < 16; ++c)
-                            h[c] = pack_bf16(__uint_as_float(w0[2 * c]) * c_cur, __uint_as_float(w0[2 * c + 1]) * c_cur);
+                            h[c] = pack_bf16(__uint_as_float(w0[2 * c]) * hscale, __uint_as_float(w0[2 * c + 1]) * hscale);
                         tmem_st16(tmem + lane_off + Lay::kColSop + cb * 32, h);
 #pragma unroll
                         for (int c = 0; c < 16; ++c)
-                            h[c] = pack_bf16(__uint_as_float(w1[2 * c]) * c_cur, __uint_as_float(w1[2 * c + 1]) * c_cur);
+                            h[c] = pack_bf16(__uint_as_float(w1[2 * c]) * hscale, __uint_as_float(w1[2 * c + 1]) * hscale);
                         tmem_st16(tmem + lane_off + Lay::kColSop + cb * 32 + 16, h);
                     }
                     if (renorm) {

@@ -168,6 +168,30 @@ def test_gamma_special_cases_on_gpu(cuda_lib):
     assert rel_l2(o[0, 1], want1) < TOL_F32
 
 
+MODE_GAMMAS = [0.0, 0.3, 0.49, 0.5, 0.75, 0.96875, 0.999, 1.0]
+
+
+@pytest.mark.parametrize("dk", [64, 128, 256])
+def test_tensor_core_output_modes_per_head(cuda_lib, dk):
+    """On the tensor-core path a head with gamma in [1/2, 1] adds both output
+    products into one accumulator (its decay factors moved onto the state copy,
+    P and the drain); other heads keep two. One launch mixes both kinds, with a
+    ragged last chunk and an initial state; every head must match the oracle."""
+    B, H, N, dv = 1, len(MODE_GAMMAS), 300, 128
+    assert cuda_lib.chunkwise_path(dk, dv, 64, torch.bfloat16) == 1
+    gam = torch.tensor(MODE_GAMMAS, dtype=torch.float32)
+    q, k, v = _rand_inputs(B, H, N, dk, dv, torch.bfloat16, seed=41 + dk)
+    S0 = torch.randn(B, H, dk, dv, generator=torch.Generator().manual_seed(dk)) * 0.05
+    qd, kd, vd, gd, S0d = _dev(q, k, v, gam, S0)
+    s_out = torch.empty_like(S0d)
+    o = cuda_lib.ret_chunkwise(qd, kd, vd, gd, 64, state_in=S0d, state_out=s_out).cpu()
+    assert cuda_lib.last_device_error() == 0
+    want_o, want_s = O.ret_chunkwise(q, k, v, gam, 64, state_in=S0)
+    for h, g in enumerate(MODE_GAMMAS):
+        assert rel_l2(o[0, h], want_o[0, h]) <= TOL_BF16, ("o", g)
+        assert rel_l2(s_out[0, h].cpu(), want_s[0, h]) <= TOL_BF16, ("state", g)
+
+
 # ------------------------------------------------------------------ decode step
 
 @pytest.mark.parametrize("dtype,dv", [(torch.float32, 128), (torch.bfloat16, 512), (torch.float32, 30)])
