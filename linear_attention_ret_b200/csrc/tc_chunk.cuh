@@ -301,6 +301,14 @@ __device__ __forceinline__ void warp_cumsum64(float g0, float g1, int lane, floa
     cum[2 * lane + 1] = incl;
 }
 
+}  // namespace tc
+}  // namespace ret
+
+#include "tc_wide.cuh"
+
+namespace ret {
+namespace tc {
+
 // STATE_ONLY: the first pass of a split sequence. Each CTA runs the state
 // recurrence of one segment from a zero state (update products only; Q is not
 // loaded and no output is formed) and writes the segment's end state and total
@@ -311,6 +319,15 @@ template <int DK, bool GATED, bool STATE_ONLY>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, Params p) {
+    // Heads with gamma close to 1 take the 128-token body (tc_wide.cuh); the choice is per
+    // CTA, so one launch serves a mix of heads.
+    if constexpr (!GATED && !STATE_ONLY && DK >= 128) {
+        const float lgw = log2f(p.decay_in[blockIdx.y % p.H]);
+        if (lgw >= kWideMinLog2 && lgw <= 0.f) {
+            wide_body<DK>(tm_q, tm_k, tm_v, tm_o, p, lgw);
+            return;
+        }
+    }
     using Lay = Layout<DK>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -935,7 +952,8 @@ inline Plan plan(int B, int H, int N, int dv) {
     int G = 1;
     if (2 * ctas <= sm_count()) G = std::min(std::min(sm_count() / ctas, kMaxSegments), nchunks / 4);
     if (G < 2) return {1, nchunks};
-    const int seg_chunks = (nchunks + G - 1) / G;
+    // an even number of 64-token chunks, so that 128-token tiles do not straddle segments
+    const int seg_chunks = ((nchunks + G - 1) / G + 1) & ~1;
     return {(nchunks + seg_chunks - 1) / seg_chunks, seg_chunks};
 }
 
@@ -954,11 +972,18 @@ inline size_t scratch_bytes(const Plan& pl, int BH, int dk, int dv, bool alias) 
            (alias ? sizeof(float) * (size_t)BH * dk * dv : 0);
 }
 
+// Dynamic shared memory of one instantiation: the 64-token layout, or the 128-token one
+// where the kernel may run that body.
+template <int DK, bool GATED, bool STATE_ONLY>
+constexpr int kernel_smem() {
+    return (!GATED && !STATE_ONLY && DK >= 128) ? std::max(Layout<DK>::kSmemAlloc, WideLayout<DK>::kSmemAlloc)
+                                                : Layout<DK>::kSmemAlloc;
+}
+
 template <int DK, bool GATED>
 ret_status launch_dk(const void* q, const void* k, const void* v, const float* decay, void* o,
                      const float* state_in, float* state_out, int B, int H, int N, int dv, const Plan& pl,
                      void* scratch, cudaStream_t st) {
-    using Lay = Layout<DK>;
     const int BH = B * H;
     CUtensorMap mq, mk, mv, mo;
     if (!make_map(&mq, q, DK, N, BH) || !make_map(&mk, k, DK, N, BH) || !make_map(&mv, v, dv, N, BH) ||
@@ -977,15 +1002,17 @@ ret_status launch_dk(const void* q, const void* k, const void* v, const float* d
             prm.state_in = copy;
         }
         auto k1 = chunk_tc_kernel<DK, GATED, true>;
-        if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kSmemAlloc) != cudaSuccess)
+        constexpr int smem1 = kernel_smem<DK, GATED, true>();
+        if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1) != cudaSuccess)
             return RET_ERR_CUDA;
-        k1<<<dim3(dv / kDvS, BH, pl.G - 1), kThreads, Lay::kSmemAlloc, st>>>(mq, mk, mv, mo, prm);
+        k1<<<dim3(dv / kDvS, BH, pl.G - 1), kThreads, smem1, st>>>(mq, mk, mv, mo, prm);
         if (cudaGetLastError() != cudaSuccess) return RET_ERR_CUDA;
     }
     auto k2 = chunk_tc_kernel<DK, GATED, false>;
-    if (cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kSmemAlloc) != cudaSuccess)
+    constexpr int smem2 = kernel_smem<DK, GATED, false>();
+    if (cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2) != cudaSuccess)
         return RET_ERR_CUDA;
-    k2<<<dim3(dv / kDvS, BH, pl.G), kThreads, Lay::kSmemAlloc, st>>>(mq, mk, mv, mo, prm);
+    k2<<<dim3(dv / kDvS, BH, pl.G), kThreads, smem2, st>>>(mq, mk, mv, mo, prm);
     return cudaGetLastError() == cudaSuccess ? RET_OK : RET_ERR_CUDA;
 }
 

@@ -1,0 +1,483 @@
+// Tensor-core chunkwise retention with 128-token tiles, for a fixed decay gamma close
+// to 1 (sm_100a). Included by tc_chunk.cuh, whose kernel runs this body for the CTAs
+// of heads with log2(gamma) in [kWideMinLog2, 0] and dk in {128, 256}.
+//
+// Method: "RetNet retention mechanism" (aiqz.cc), section 块级循环 (chunkwise
+// recurrence). Two changes against the 64-token body:
+//
+// 1. Tiles of 128 tokens. One tcgen05.mma takes about the same time for N = 64 and
+//    N = 128 (on B200, 16 products of M64 N64 K16 take ~1160 cycles and of M128 N128
+//    K16 ~1200), so Q K^T and the cross term cost half as much per token as with
+//    64-token tiles.
+//
+// 2. One output accumulator, fed by zeta V in place of V. For a tile of L tokens let
+//    zeta_m = gamma^(L-1-m) (the key weights of the state update) and hold the state as
+//    S = kappa T (kappa a scalar, T in TMEM). With T the state before this tile's update,
+//      O_j = (kappa / zeta_j) [ q_j T + sum_{m<=j} A_jm (zeta_m v_m / kappa) ],  A = Q K^T,
+//    since gamma^(j-m) = zeta_m / zeta_j and gamma^(j+1) S_prev = gamma^L S_prev / zeta_j
+//    = kappa T / zeta_j. So O_inter (from the bf16 copy of T) and O_intra (from the plain
+//    causal mask of A and the same zeta V / kappa tile that the state update reads) add
+//    into one TMEM region, and the drain scales token j by kappa / zeta_j. The state
+//    epilogue turns the V tile into zeta V / kappa in place, so no V copy is kept.
+//    With log2(gamma) >= kWideMinLog2 every factor stays within [2^-96, 2^96] (times
+//    kappa in [2^-40, 1]), inside the normal range of bf16 and fp32.
+//
+// Products per tile (transposed so that M = 128 is the dv slice where it can be):
+//   A   = Q K^T             M=128 (j) N=128 (m) K=dk   SS             -> TMEM region R
+//   S^T += (zeta V / kappa)^T K   M=128 N=dk K=128     SS, both MN-major
+//   Z^T  = T_op^T Q^T       M=128 N=128 K=dk           TS (bf16 T copy in TMEM) -> R
+//   Z^T += (zeta V / kappa)^T P^T  M=128 N=128 K=128   SS, P = causal mask of A (bf16)
+// TMEM: S^T (dk columns), its bf16 copy (dk/2), R (128 columns) -- 512 at dk = 256.
+// Shared memory: one Q, K and V tile, each with its own full/empty barriers so that it
+// reloads as soon as its last reader is done (K after the update, Q after the cross
+// term, V after O_intra), and one P tile that is also the staging tile of the O store.
+#pragma once
+
+namespace ret {
+namespace tc {
+
+constexpr int kW = 128;                 // tokens per tile
+constexpr int kBlk = kW * 128;          // one 128-row x 128-byte swizzled block (16 KB)
+constexpr float kWideMinLog2 = -0.75f;  // gamma >= 2^-0.75 ~= 0.595
+
+template <int DK>
+struct WideLayout {
+    static constexpr int kQ = 0;                        // Q tile: DK/64 blocks (rows = tokens)
+    static constexpr int kK = kQ + DK / 64 * kBlk;      // K tile
+    static constexpr int kV = kK + DK / 64 * kBlk;      // V tile, then zeta V / kappa (2 blocks of 64 dv columns)
+    static constexpr int kP = kV + 2 * kBlk;            // P (2 blocks of 64 m columns); O staging (4 x 64 x 64)
+    static constexpr int kBar = kP + 2 * kBlk;
+    static constexpr int kNumBars = 16;
+    static constexpr int kAgTab = kBar + kNumBars * 8;  // attention group: drain row factors [128]
+    static constexpr int kSgTab = kAgTab + kW * 4;      // state group: zeta / kappa [128]
+    static constexpr int kTmemSlot = kSgTab + kW * 4;
+    static constexpr int kAbort = kTmemSlot + 4;
+    static constexpr int kBytes = kAbort + 4;
+    static constexpr int kSmemAlloc = kBytes + 1024;    // slack to align the base to 1024 B
+    static constexpr int kColS = 0;
+    static constexpr int kColSop = DK;
+    static constexpr int kColR = DK + DK / 2;
+    static constexpr int kTmemCols = kColR + kW <= 256 ? 256 : 512;
+    static_assert(kColR + kW <= 512, "TMEM overflow");
+    static_assert(kSmemAlloc <= 227 * 1024, "shared memory overflow");
+};
+
+enum WideBar {
+    wQFull = 0, wKFull, wVFull, wQEmpty, wKEmpty, wVEmpty,
+    wAFull, wARead, wPReady, wOFull, wOFree,
+    wSFull, wSReady, wZV, wDrain
+};
+
+// Lazy decay normalisation (S = kappa T). Given the current kappa and the next tile's
+// decay gamma^L, returns the next kappa: kappa gamma^L, or 1 when that would fall below
+// 2^-40 (then T itself is rescaled by kappa gamma^L). Both epilogue groups evaluate it,
+// with the same operations, so they agree on kappa bit for bit.
+__device__ __forceinline__ float lazy_next_scale(float kappa, float decay, bool force, bool& renorm) {
+    renorm = force || !(kappa * decay >= 9.094947e-13f);  // 2^-40
+    return renorm ? 1.f : kappa * decay;
+}
+
+template <int DK>
+__device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                                          const CUtensorMap& tm_o, const Params& p, float lg) {
+    using Lay = WideLayout<DK>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    auto bar = [&](int b) { return sbase + Lay::kBar + 8 * b; };
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Lay::kAbort);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Lay::kTmemSlot);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int slice = blockIdx.x, bh = blockIdx.y, seg = blockIdx.z;
+    const int dv0 = slice * kDvS;
+    const int tbeg = seg * p.seg_chunks * kC;                 // first token of this segment
+    const int tend = min(tbeg + p.seg_chunks * kC, p.N);      // one past its last token
+    const int ntiles = (tend - tbeg + kW - 1) / kW;
+    const bool last_seg = tend >= p.N;
+    auto tile_len = [&](int c) { return min(kW, tend - (tbeg + c * kW)); };
+
+    if (threadIdx.x == 0) {
+        for (int b = 0; b < Lay::kNumBars; ++b) mbar_init(bar(b), 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_q)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_k)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_v)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_o)) : "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(tmem_slot)), "r"(Lay::kTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            // 64 x 64 boxes; two of them (tokens t0 and t0 + 64) fill one 128-row block.
+            // Rows past the segment end are loaded too and masked by the epilogues; rows
+            // past N read as zero.
+            int issued[3] = {-1, -1, -1};  // K, Q, V: last tile whose copies were issued
+            for (int c = 0; c < ntiles; ++c) {
+                const int t0 = tbeg + c * kW;
+                const uint32_t ph = (c - 1) & 1;
+                if (c > 0 && !mbar_wait(bar(wKEmpty), ph, abort_flag)) break;
+                mbar_expect_tx(bar(wKFull), DK / 64 * kBlk);
+#pragma unroll
+                for (int kb = 0; kb < DK / 64; ++kb)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        tma_load_3d(sbase + Lay::kK + kb * kBlk + h * kTile64, &tm_k, kb * 64, t0 + 64 * h, bh, bar(wKFull));
+                issued[0] = c;
+                if (c > 0 && !mbar_wait(bar(wQEmpty), ph, abort_flag)) break;
+                mbar_expect_tx(bar(wQFull), DK / 64 * kBlk);
+#pragma unroll
+                for (int kb = 0; kb < DK / 64; ++kb)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        tma_load_3d(sbase + Lay::kQ + kb * kBlk + h * kTile64, &tm_q, kb * 64, t0 + 64 * h, bh, bar(wQFull));
+                issued[1] = c;
+                if (c > 0 && !mbar_wait(bar(wVEmpty), ph, abort_flag)) break;
+                mbar_expect_tx(bar(wVFull), 2 * kBlk);
+#pragma unroll
+                for (int db = 0; db < 2; ++db)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        tma_load_3d(sbase + Lay::kV + db * kBlk + h * kTile64, &tm_v, dv0 + 64 * db, t0 + 64 * h, bh,
+                                    bar(wVFull));
+                issued[2] = c;
+            }
+            if (*abort_flag) {
+                // drain the copies in flight before the CTA may exit
+                if (issued[0] >= 0) mbar_drain(bar(wKFull), issued[0] & 1);
+                if (issued[1] >= 0) mbar_drain(bar(wQFull), issued[1] & 1);
+                if (issued[2] >= 0) mbar_drain(bar(wVFull), issued[2] & 1);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t id_qk = idesc(128, kW, 0, 0);
+            constexpr uint32_t id_oi = idesc(128, kW, 0, 0);
+            constexpr uint32_t id_ov = idesc(128, kW, 1, 0);
+            constexpr uint32_t id_up = idesc(128, DK, 1, 1);
+            const uint32_t tS = tmem + Lay::kColS, tSop = tmem + Lay::kColSop, tR = tmem + Lay::kColR;
+            const uint32_t sQ = sbase + Lay::kQ, sK = sbase + Lay::kK, sZ = sbase + Lay::kV, sP = sbase + Lay::kP;
+            for (int c = 0; c < ntiles; ++c) {
+                const uint32_t ph = c & 1;
+                // A = Q K^T (both K-major; 16-element K steps, 64-column blocks 16 KB apart);
+                // region R is free once the previous tile's output has been read out.
+                if (!mbar_wait(bar(wQFull), ph, abort_flag) || !mbar_wait(bar(wKFull), ph, abort_flag)) break;
+                if (c > 0 && !mbar_wait(bar(wOFree), (c - 1) & 1, abort_flag)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < DK / 16; ++ks) {
+                    const uint32_t off = (ks >> 2) * kBlk + (ks & 3) * 32;
+                    mma_ss(tR, sdesc(sQ + off, 16, 1024), sdesc(sK + off, 16, 1024), id_qk, ks > 0);
+                }
+                mma_commit(bar(wAFull));
+                // S^T += (zeta V / kappa)^T K while the epilogue reads A: A operand = the
+                // scaled V tile MN-major (dv blocks 16 KB apart), B = K tile MN-major.
+                if (!mbar_wait(bar(wZV), ph, abort_flag) || !mbar_wait(bar(wSReady), ph, abort_flag)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < kW / 16; ++ks)
+                    mma_ss(tS, sdesc(sZ + ks * 2048, kBlk, 1024), sdesc(sK + ks * 2048, kBlk, 1024), id_up, 1);
+                mma_commit(bar(wKEmpty));
+                // Z^T = T_op^T Q^T into R once A has been read (A from TMEM, B = Q tile K-major)
+                if (!mbar_wait(bar(wARead), ph, abort_flag)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < DK / 16; ++ks) {
+                    const uint32_t off = (ks >> 2) * kBlk + (ks & 3) * 32;
+                    mma_ts(tR, tSop + ks * 8, sdesc(sQ + off, 16, 1024), id_oi, ks > 0);
+                }
+                // the update and the cross term are done: the state epilogue may read S and
+                // overwrite its bf16 copy; the Q tile may reload
+                mma_commit(bar(wSFull));
+                mma_commit(bar(wQEmpty));
+                // Z^T += (zeta V / kappa)^T P^T (B = P K-major, m blocks 16 KB apart)
+                if (!mbar_wait(bar(wPReady), ph, abort_flag)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < kW / 16; ++ks)
+                    mma_ss(tR, sdesc(sZ + ks * 2048, kBlk, 1024), sdesc(sP + (ks >> 2) * kBlk + (ks & 3) * 32, 16, 1024),
+                           id_ov, 1);
+                mma_commit(bar(wOFull));
+                mma_commit(bar(wVEmpty));
+            }
+            // every issued MMA must complete before TMEM can be released
+            mma_commit(bar(wDrain));
+            mbar_drain(bar(wDrain), 0);
+        }
+    } else if (warp < 6) {
+        // ------------------------------------------------------------ attention epilogue (warps 2..5)
+        const int te = threadIdx.x - 64;   // 0..127
+        const int quarter = warp & 3;      // TMEM lane quarter this warp may access
+        const int r = quarter * 32 + lane;  // TMEM lane: token row j of A, dv column d of Z^T
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const uint32_t tR = tmem + lane_off + Lay::kColR;
+        float* rowf = reinterpret_cast<float*>(sm + Lay::kAgTab);
+        auto wait_all = [&](int b, uint32_t parity) {  // every thread reaches the barrier; uniform result
+            mbar_wait(bar(b), parity, abort_flag);
+            group_sync(1);
+            return *abort_flag == 0;
+        };
+        float kappa = 1.f;
+        for (int c = 0; c < ntiles; ++c) {
+            const int t0 = tbeg + c * kW, L = tile_len(c);
+            if (c > 0) {
+                bool rn;
+                kappa = lazy_next_scale(kappa, pow_int_log2(lg, L), false, rn);
+            }
+            // ---------------- P = causal mask of A in bf16, row j = r (K-major, 128-byte swizzle)
+            if (!wait_all(wAFull, c & 1)) break;
+            tc_fence_after();
+            uint32_t pk[64];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t a0[32], a1[32];
+                tmem_ld32(tR + hh * 64, a0);
+                tmem_ld32(tR + hh * 64 + 32, a1);
+                tmem_wait_ld();
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int m = hh * 64 + 2 * u;
+                    pk[hh * 32 + u] = pack_bf16(m <= r ? __uint_as_float(a0[2 * u]) : 0.f,
+                                                m + 1 <= r ? __uint_as_float(a0[2 * u + 1]) : 0.f);
+                    pk[hh * 32 + 16 + u] = pack_bf16(m + 32 <= r ? __uint_as_float(a1[2 * u]) : 0.f,
+                                                     m + 33 <= r ? __uint_as_float(a1[2 * u + 1]) : 0.f);
+                }
+            }
+            // A is in registers: the cross term may overwrite R. The previous tile's O store
+            // must have read the staging tile (the P region) before P is written.
+            tc_fence_before();
+            if (te == 0) tma_store_wait_read();
+            group_sync(1);
+            if (te == 0) mbar_arrive(bar(wARead));
+            {
+                uint8_t* prow = sm + Lay::kP + r * 128;
+#pragma unroll
+                for (int q = 0; q < 16; ++q)
+                    *reinterpret_cast<uint4*>(prow + (q >> 3) * kBlk + (((q & 7) ^ (r & 7)) << 4)) =
+                        make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+            }
+            fence_proxy_async();
+            group_sync(1);
+            if (te == 0) mbar_arrive(bar(wPReady));
+            // ---------------- O_j = (kappa / zeta_j) Z_j -> bf16 -> staging -> TMA store
+            rowf[te] = te < L ? kappa * pow_int_log2(-lg, L - 1 - te) : 0.f;
+            if (!wait_all(wOFull, c & 1)) break;
+            tc_fence_after();
+            {
+                uint32_t z[4][32];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) tmem_ld32(tR + h * 32, z[h]);
+                tmem_wait_ld();
+                tc_fence_before();
+                group_sync(1);
+                if (te == 0) mbar_arrive(bar(wOFree));
+                // row factors into registers before the first shared store (aliasing)
+#pragma unroll
+                for (int h = 0; h < 4; ++h)
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj)
+                        z[h][jj] = __float_as_uint(rowf[h * 32 + jj] * __uint_as_float(z[h][jj]));
+                // Thread r owns dv column d = r for all 128 tokens. A lane-pair shuffle packs two
+                // adjacent dv columns into one 4-byte store: even lanes store token j, odd lanes
+                // token j + 4 (disjoint banks under the 128-byte swizzle). Staging block
+                // (token half th, dv half db) is the 64 x 64 box at kP + (2 th + db) * 8 KB.
+                const bool odd = lane & 1;
+                const int cb = ((r & 63) & ~1) * 2;  // byte offset of the dv pair inside a 128-byte row
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    uint8_t* ost = sm + Lay::kP + ((h >> 1) * 2 + (r >> 6)) * kTile64;
+                    const float* o = reinterpret_cast<const float*>(z[h]);
+                    uint32_t w[16];
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) {
+                        const int ja = 8 * (u >> 2) + (u & 3);  // token pair (ja, ja + 4) inside the 32-token block
+                        const float send = odd ? o[ja] : o[ja + 4];
+                        const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+                        w[u] = odd ? pack_bf16(recv, o[ja + 4]) : pack_bf16(o[ja], recv);
+                    }
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) {
+                        const int jr = (h & 1) * 32 + 8 * (u >> 2) + (u & 3) + (odd ? 4 : 0);  // row in the box
+                        *reinterpret_cast<uint32_t*>(ost + jr * 128 + ((((cb >> 4) ^ (jr & 7)) << 4) | (cb & 15))) = w[u];
+                    }
+                }
+            }
+            fence_proxy_async();
+            group_sync(1);
+            if (te == 0) {
+                // tokens past the segment end belong to the next segment: store only the
+                // 64-token halves that start inside this tile (rows past N are clipped)
+#pragma unroll
+                for (int th = 0; th < 2; ++th) {
+                    if (th * 64 >= L) break;
+                    tma_store_3d(&tm_o, dv0, t0 + 64 * th, bh, sbase + Lay::kP + (2 * th) * kTile64);
+                    tma_store_3d(&tm_o, dv0 + 64, t0 + 64 * th, bh, sbase + Lay::kP + (2 * th + 1) * kTile64);
+                }
+                tma_store_commit();
+            }
+        }
+        if (te == 0) tma_store_wait_all();
+    } else {
+        // ------------------------------------------------------------ state epilogue (warps 6..9)
+        const int ts = threadIdx.x - 192;  // 0..127
+        const int quarter = warp & 3;
+        const int d = quarter * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        float* zk = reinterpret_cast<float*>(sm + Lay::kSgTab);  // zeta_m / kappa
+        auto wait_all = [&](int b, uint32_t parity) {
+            mbar_wait(bar(b), parity, abort_flag);
+            group_sync(2);
+            return *abort_flag == 0;
+        };
+        // The V tile of tile c becomes zeta V / kappa in place: 16-byte chunks ci = e * 128 + ts,
+        // two 16 KB blocks of 128 token rows, so the token of a chunk is (ci mod 1024) / 8.
+        auto build_zv = [&](int c, float kappa) {
+            const int L = tile_len(c);
+            zk[ts] = ts < L ? pow_int_log2(lg, L - 1 - ts) * (1.f / kappa) : 0.f;
+            if (!wait_all(wVFull, c & 1)) return false;
+            uint8_t* vt = sm + Lay::kV;
+#pragma unroll
+            for (int pass = 0; pass < 2; ++pass) {
+                uint4 x[8];
+                float z[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {  // all loads before any store (aliasing)
+                    const int ci = (pass * 8 + e) * kEpiThreads + ts;
+                    z[e] = zk[(ci & 1023) >> 3];
+                    x[e] = *reinterpret_cast<const uint4*>(vt + ci * 16);
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    float2 f;
+                    f = unpack_bf16(x[e].x); x[e].x = pack_bf16(f.x * z[e], f.y * z[e]);
+                    f = unpack_bf16(x[e].y); x[e].y = pack_bf16(f.x * z[e], f.y * z[e]);
+                    f = unpack_bf16(x[e].z); x[e].z = pack_bf16(f.x * z[e], f.y * z[e]);
+                    f = unpack_bf16(x[e].w); x[e].w = pack_bf16(f.x * z[e], f.y * z[e]);
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    *reinterpret_cast<uint4*>(vt + ((pass * 8 + e) * kEpiThreads + ts) * 16) = x[e];
+            }
+            fence_proxy_async();
+            group_sync(2);
+            if (ts == 0) mbar_arrive(bar(wZV));
+            return true;
+        };
+
+        // Initial state: kappa = 1, T = gamma^L0 S_in, bf16 copy = bf16(T). S_in is state_in (or
+        // zero) for the first segment; segment g > 0 folds in the earlier segments' end states:
+        // S_in(g) = decay_{g-1} S_in(g-1) + U_{g-1}.
+        float kappa;
+        {
+            bool rn;
+            const float dec0 = pow_int_log2(lg, tile_len(0));
+            kappa = lazy_next_scale(1.f, dec0, true, rn);
+            const float* sin = p.state_in ? p.state_in + ((size_t)bh * DK) * p.dv + dv0 + d : nullptr;
+            const size_t seg_stride = (size_t)gridDim.y * DK * p.dv;
+            const float* useg = p.seg_state + ((size_t)bh * DK) * p.dv + dv0 + d;
+#pragma unroll 1
+            for (int cb = 0; cb < DK / 32; ++cb) {
+                uint32_t w[32], h[16];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(sin ? sin[(size_t)(cb * 32 + c) * p.dv] : 0.f);
+#pragma unroll 1
+                for (int hs = 0; hs < seg; ++hs) {
+                    const float gam = exp2f(p.seg_ldec[(size_t)hs * gridDim.y + bh]);
+                    const float* u = useg + hs * seg_stride + (size_t)(cb * 32) * p.dv;
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(fmaf(gam, __uint_as_float(w[c]), u[(size_t)c * p.dv]));
+                }
+#pragma unroll
+                for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(__uint_as_float(w[c]) * dec0);
+#pragma unroll
+                for (int c = 0; c < 16; ++c) h[c] = pack_bf16(__uint_as_float(w[2 * c]), __uint_as_float(w[2 * c + 1]));
+                tmem_st32(tmem + lane_off + Lay::kColS + cb * 32, w);
+                tmem_st16(tmem + lane_off + Lay::kColSop + cb * 16, h);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            group_sync(2);
+            if (ts == 0) mbar_arrive(bar(wSReady));
+        }
+        bool ok = build_zv(0, kappa);
+        for (int c = 0; c < ntiles && ok; ++c) {
+            const bool last = c == ntiles - 1;
+            bool rn = false;
+            float dec_next = 0.f, k_next = 1.f;
+            if (!last) {
+                dec_next = pow_int_log2(lg, tile_len(c + 1));
+                k_next = lazy_next_scale(kappa, dec_next, false, rn);
+            }
+            if (!wait_all(wSFull, c & 1)) break;
+            tc_fence_after();
+            if (last) {
+                float* so = last_seg ? p.state_out : nullptr;
+                if (so) {
+                    so += ((size_t)bh * DK) * p.dv + dv0 + d;
+#pragma unroll 1
+                    for (int cb = 0; cb < DK / 32; ++cb) {
+                        uint32_t w[32];
+                        tmem_ld32(tmem + lane_off + Lay::kColS + cb * 32, w);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int cc = 0; cc < 32; ++cc) so[(size_t)(cb * 32 + cc) * p.dv] = __uint_as_float(w[cc]) * kappa;
+                    }
+                }
+                break;
+            }
+            // Next bf16 copy = bf16(T'), T' = T, or kappa gamma^L T when kappa renormalises
+            // (then T' is also written back).
+            const float tscale = kappa * dec_next;
+#pragma unroll 1
+            for (int cb = 0; cb < DK / 64; ++cb) {
+                uint32_t w0[32], w1[32], h[16];
+                tmem_ld32(tmem + lane_off + Lay::kColS + cb * 64, w0);
+                tmem_ld32(tmem + lane_off + Lay::kColS + cb * 64 + 32, w1);
+                tmem_wait_ld();
+                if (rn) {
+#pragma unroll
+                    for (int cc = 0; cc < 32; ++cc) {
+                        w0[cc] = __float_as_uint(__uint_as_float(w0[cc]) * tscale);
+                        w1[cc] = __float_as_uint(__uint_as_float(w1[cc]) * tscale);
+                    }
+                    tmem_st32(tmem + lane_off + Lay::kColS + cb * 64, w0);
+                    tmem_st32(tmem + lane_off + Lay::kColS + cb * 64 + 32, w1);
+                }
+#pragma unroll
+                for (int cc = 0; cc < 16; ++cc) h[cc] = pack_bf16(__uint_as_float(w0[2 * cc]), __uint_as_float(w0[2 * cc + 1]));
+                tmem_st16(tmem + lane_off + Lay::kColSop + cb * 32, h);
+#pragma unroll
+                for (int cc = 0; cc < 16; ++cc) h[cc] = pack_bf16(__uint_as_float(w1[2 * cc]), __uint_as_float(w1[2 * cc + 1]));
+                tmem_st16(tmem + lane_off + Lay::kColSop + cb * 32 + 16, h);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            group_sync(2);
+            if (ts == 0) mbar_arrive(bar(wSReady));
+            kappa = k_next;
+            ok = build_zv(c + 1, kappa);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(Lay::kTmemCols)
+                     : "memory");
+    }
+}
+
+}  // namespace tc
+}  // namespace ret
