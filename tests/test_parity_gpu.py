@@ -171,13 +171,14 @@ def test_gamma_special_cases_on_gpu(cuda_lib):
 MODE_GAMMAS = [0.0, 0.3, 0.49, 0.5, 0.75, 0.96875, 0.999, 1.0]
 
 
+@pytest.mark.parametrize("dv", [128, 256])
 @pytest.mark.parametrize("dk", [64, 128, 256])
-def test_tensor_core_output_modes_per_head(cuda_lib, dk):
-    """On the tensor-core path a head with gamma in [1/2, 1] adds both output
-    products into one accumulator (its decay factors moved onto the state copy,
-    P and the drain); other heads keep two. One launch mixes both kinds, with a
-    ragged last chunk and an initial state; every head must match the oracle."""
-    B, H, N, dv = 1, len(MODE_GAMMAS), 300, 128
+def test_tensor_core_output_modes_per_head(cuda_lib, dk, dv):
+    """The tensor-core path picks a kernel body per head from its gamma: the
+    64-token body with split or merged output accumulators, or the 128-token
+    body. One call mixes all of them, with a ragged last tile and an initial
+    state, over one and two dv slices; every head must match the oracle."""
+    B, H, N = 1, len(MODE_GAMMAS), 300
     assert cuda_lib.chunkwise_path(dk, dv, 64, torch.bfloat16) == 1
     gam = torch.tensor(MODE_GAMMAS, dtype=torch.float32)
     q, k, v = _rand_inputs(B, H, N, dk, dv, torch.bfloat16, seed=41 + dk)
