@@ -164,6 +164,9 @@ RET_API int ret_chunkwise_launches(int B, int H, int N, int dk, int dv, int chun
  *  - A problem whose scratch would exceed the buffer is rejected on the host
  *    with RET_ERR_SCRATCH before anything is launched. Passing state_in and
  *    state_out as the same buffer needs an extra copy of the state in scratch.
+ *    Where ret_chunkwise would cut its state-only pass finer than its segments
+ *    and that does not fit, this entry point keeps one piece per segment (the
+ *    same result up to rounding order).
  *  - All calls share the one buffer, which keeps the previous call's contents;
  *    every scratch byte a call reads is written earlier in that same call, so
  *    nothing has to be cleared. Calls that overlap on the GPU (for example on

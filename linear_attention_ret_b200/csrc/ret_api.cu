@@ -237,8 +237,10 @@ extern "C" ret_status ret_chunkwise_noalloc(const void* q, const void* k, const 
                                                                            B, H, N, dk, dv, chunk, st);
     }
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RET_ERR_ALIGN;
-    const tc::Plan pl = tc::plan(B, H, N, dv);
-    const size_t bytes = tc::scratch_bytes(pl, B * H, dk, dv, state_in != nullptr && state_in == state_out);
+    const bool alias = state_in != nullptr && state_in == state_out;
+    tc::Plan pl = tc::plan(B, H, N, dv);
+    if (tc::scratch_bytes(pl, B * H, dk, dv, alias) > RET_NOALLOC_SCRATCH_BYTES) pl = tc::plan(B, H, N, dv, false);
+    const size_t bytes = tc::scratch_bytes(pl, B * H, dk, dv, alias);
     if (bytes > RET_NOALLOC_SCRATCH_BYTES) return RET_ERR_SCRATCH;
     void* scratch = nullptr;
     if (bytes) {

@@ -285,6 +285,7 @@ struct Params {
     float* seg_ldec;         // [G-1, B*H]: log2 of each of those segments' total decay (scratch)
     int H, N, dv;
     int seg_chunks;          // chunks per sequence segment (blockIdx.z = segment)
+    int sub_per_seg;         // state-only sub-segments per full-pass segment (their start states are in seg_state)
 };
 
 // In-chunk inclusive cumulative sum of the gate in log2 units, by one warp:
@@ -309,19 +310,32 @@ __device__ __forceinline__ void warp_cumsum64(float g0, float g1, int lane, floa
 namespace ret {
 namespace tc {
 
+// Start state of segment seg of a split sequence, column `col` of head bh: state_in (or
+// none: zero) for the first segment; for segment g > 0 the prefix pass has left it in
+// seg_state[g F - 1] (F = sub_per_seg: the state-only pass may cut segments finer). Rows
+// are dv apart.
+__device__ __forceinline__ const float* segment_start_state(const Params& p, int seg, int bh, int dk, int col) {
+    if (seg > 0) return p.seg_state + ((size_t)(seg * p.sub_per_seg - 1) * gridDim.y + bh) * dk * p.dv + col;
+    return p.state_in ? p.state_in + ((size_t)bh * dk) * p.dv + col : nullptr;
+}
+
+constexpr bool wide_capable(int dk, bool gated, bool state_only) {
+    return !state_only && !gated && dk >= 128;
+}
+
 // STATE_ONLY: the first pass of a split sequence. Each CTA runs the state
 // recurrence of one segment from a zero state (update products only; Q is not
-// loaded and no output is formed) and writes the segment's end state and total
-// decay to the scratch buffers. The full pass then starts segment g from
-// S_in(g) = decay_{g-1} S_in(g-1) + U_{g-1}, S_in(0) = state_in, which its state
-// epilogue evaluates in its prologue.
+// loaded and no output is formed) and writes the segment's end state U and total
+// decay to the scratch buffers. seg_prefix_kernel then turns them into the
+// segment start states S_in(g) = decay_{g-1} S_in(g-1) + U_{g-1}, S_in(0) =
+// state_in, and the full pass starts each segment from its S_in.
 template <int DK, bool GATED, bool STATE_ONLY>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, Params p) {
     // Heads with gamma close to 1 take the 128-token body (tc_wide.cuh); the choice is per
     // CTA, so one launch serves a mix of heads.
-    if constexpr (!GATED && !STATE_ONLY && DK >= 128) {
+    if constexpr (wide_capable(DK, GATED, STATE_ONLY)) {
         const float lgw = log2f(p.decay_in[blockIdx.y % p.H]);
         if (lgw >= kWideMinLog2 && lgw <= 0.f) {
             wide_body<DK>(tm_q, tm_k, tm_v, tm_o, p, lgw);
@@ -768,25 +782,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         bool renorm = true;
         bool ok = make_zv(0, 1.f, true, dec0, renorm, c_cur);
         if (ok) {
-            // initial state: S_op = bf16(sop S_in), T = decay_0 * S_in, c = 1. S_in is state_in (or
-            // zero) for the first segment; segment g > 0 folds in the earlier segments' end states:
-            // S_in(g) = decay_{g-1} S_in(g-1) + U_{g-1}. The state-only pass starts from zero.
-            const float* sin = (!STATE_ONLY && p.state_in) ? p.state_in + ((size_t)bh * DK) * p.dv + dv0 + d : nullptr;
-            const size_t seg_stride = (size_t)gridDim.y * DK * p.dv;
-            const float* useg = STATE_ONLY ? nullptr : p.seg_state + ((size_t)bh * DK) * p.dv + dv0 + d;
-            const int nprev = STATE_ONLY ? 0 : seg;
+            // initial state: S_op = bf16(sop S_in), T = decay_0 * S_in, c = 1. The state-only pass
+            // starts from zero; the full pass from segment_start_state().
+            const float* sin = STATE_ONLY ? nullptr : segment_start_state(p, seg, bh, DK, dv0 + d);
 #pragma unroll 1
             for (int cb = 0; cb < DK / 32; ++cb) {
                 uint32_t w[32], h[16];
 #pragma unroll
                 for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(sin ? sin[(size_t)(cb * 32 + c) * p.dv] : 0.f);
-#pragma unroll 1
-                for (int hs = 0; hs < nprev; ++hs) {
-                    const float gam = exp2f(p.seg_ldec[(size_t)hs * gridDim.y + bh]);
-                    const float* u = useg + hs * seg_stride + (size_t)(cb * 32) * p.dv;
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(fmaf(gam, __uint_as_float(w[c]), u[(size_t)c * p.dv]));
-                }
 #pragma unroll
                 for (int c = 0; c < 16; ++c)
                     h[c] = pack_bf16(__uint_as_float(w[2 * c]) * sop, __uint_as_float(w[2 * c + 1]) * sop);
@@ -877,6 +880,39 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
 }
 
+constexpr int kMaxSegments = 16;  // segments of a split sequence, at most
+
+// Segment start states of a split sequence, between the two passes: seg_state[g] holds
+// U_g (segment g's end state from a zero start) on entry and S_in(g + 1) = Gamma_g S_in(g)
+// + U_g on exit, with S_in(0) = state_in (or zero) and Gamma_g = 2^seg_ldec[g]. One thread
+// per 4 consecutive state elements; all of a thread's G - 1 loads are issued before the
+// sequential recurrence, so every full-pass CTA then reads one state instead of folding
+// all earlier segments itself. seg_state is the library's scratch (16-byte aligned);
+// state_in is read element by element (only 4-byte alignment is required of it).
+__global__ void __launch_bounds__(256)
+seg_prefix_kernel(const float* __restrict__ state_in, float* __restrict__ seg_state, const float* __restrict__ seg_ldec,
+                  int G, int BH, int per_bh) {
+    const size_t n4 = (size_t)BH * per_bh / 4;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
+        const int bh = (int)(i * 4 / per_bh);
+        float4 u[kMaxSegments - 1];
+#pragma unroll
+        for (int g = 0; g < kMaxSegments - 1; ++g)
+            if (g < G - 1) u[g] = reinterpret_cast<const float4*>(seg_state + (size_t)g * BH * per_bh)[i];
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (state_in) x = make_float4(state_in[4 * i], state_in[4 * i + 1], state_in[4 * i + 2], state_in[4 * i + 3]);
+#pragma unroll
+        for (int g = 0; g < kMaxSegments - 1; ++g) {
+            if (g < G - 1) {
+                const float gam = exp2f(seg_ldec[(size_t)g * BH + bh]);
+                x = make_float4(fmaf(gam, x.x, u[g].x), fmaf(gam, x.y, u[g].y), fmaf(gam, x.z, u[g].z),
+                                fmaf(gam, x.w, u[g].w));
+                reinterpret_cast<float4*>(seg_state + (size_t)g * BH * per_bh)[i] = x;
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------------------ host side
 
 inline bool tc_device_ok() {
@@ -927,8 +963,6 @@ inline bool tc_chunk_supported(int dk, int dv, int chunk, bool bf16) {
 
 namespace tc {
 
-constexpr int kMaxSegments = 16;
-
 inline int sm_count() {
     static int n = 0;
     if (n == 0) {
@@ -944,27 +978,36 @@ inline int sm_count() {
 struct Plan {
     int G;           // segments
     int seg_chunks;  // chunks per segment
+    int F;           // state-only sub-segments per segment (seg_chunks / F chunks each)
+    int subs() const { return F * (G - 1); }  // sub-segments whose end states the state-only pass writes
 };
 
-inline Plan plan(int B, int H, int N, int dv) {
+// sub_segments = false keeps one state-only CTA per segment (less scratch).
+inline Plan plan(int B, int H, int N, int dv, bool sub_segments = true) {
     const int ctas = B * H * (dv / kDvS);
     const int nchunks = (N + kC - 1) / kC;
     int G = 1;
     if (2 * ctas <= sm_count()) G = std::min(std::min(sm_count() / ctas, kMaxSegments), nchunks / 4);
-    if (G < 2) return {1, nchunks};
+    if (G < 2) return {1, nchunks, 1};
     // an even number of 64-token chunks, so that 128-token tiles do not straddle segments
     const int seg_chunks = ((nchunks + G - 1) / G + 1) & ~1;
-    return {(nchunks + seg_chunks - 1) / seg_chunks, seg_chunks};
+    G = (nchunks + seg_chunks - 1) / seg_chunks;
+    // Only segments 0..G-2 need end states, so the state-only pass would leave SMs idle: cut
+    // each of those segments into F sub-segments while that still fits the SMs.
+    int F = 1;
+    if (sub_segments)
+        while (2 * F * ctas * (G - 1) <= sm_count() && seg_chunks % (2 * F) == 0 && 2 * F * (G - 1) < kMaxSegments) F *= 2;
+    return {G, seg_chunks, F};
 }
 
-// Scratch of a split sequence: end states [G-1, BH, dk, dv] fp32, log2 decays [G-1, BH], and,
-// when state_in and state_out are the same buffer, a copy of state_in (every segment reads
-// state_in while the last one writes state_out, so they must not share memory).
+// Scratch of a split sequence: end states [F(G-1), BH, dk, dv] fp32, log2 decays [F(G-1), BH],
+// and, when state_in and state_out are the same buffer, a copy of state_in (every segment
+// reads state_in while the last one writes state_out, so they must not share memory).
 inline size_t scratch_states_bytes(const Plan& pl, int BH, int dk, int dv) {
-    return sizeof(float) * (size_t)(pl.G - 1) * BH * dk * dv;
+    return sizeof(float) * (size_t)pl.subs() * BH * dk * dv;
 }
 inline size_t scratch_ldec_bytes(const Plan& pl, int BH) {
-    return (sizeof(float) * (size_t)(pl.G - 1) * BH + 255) & ~size_t(255);
+    return (sizeof(float) * (size_t)pl.subs() * BH + 255) & ~size_t(255);
 }
 inline size_t scratch_bytes(const Plan& pl, int BH, int dk, int dv, bool alias) {
     if (pl.G < 2) return 0;
@@ -976,8 +1019,10 @@ inline size_t scratch_bytes(const Plan& pl, int BH, int dk, int dv, bool alias) 
 // where the kernel may run that body.
 template <int DK, bool GATED, bool STATE_ONLY>
 constexpr int kernel_smem() {
-    return (!GATED && !STATE_ONLY && DK >= 128) ? std::max(Layout<DK>::kSmemAlloc, WideLayout<DK>::kSmemAlloc)
-                                                : Layout<DK>::kSmemAlloc;
+    if constexpr (wide_capable(DK, GATED, STATE_ONLY))
+        return std::max(Layout<DK>::kSmemAlloc, WideLayout<DK>::kSmemAlloc);
+    else
+        return Layout<DK>::kSmemAlloc;
 }
 
 template <int DK, bool GATED>
@@ -989,7 +1034,7 @@ ret_status launch_dk(const void* q, const void* k, const void* v, const float* d
     if (!make_map(&mq, q, DK, N, BH) || !make_map(&mk, k, DK, N, BH) || !make_map(&mv, v, dv, N, BH) ||
         !make_map(&mo, o, dv, N, BH))
         return RET_ERR_CUDA;
-    Params prm{decay, state_in, state_out, nullptr, nullptr, H, N, dv, pl.seg_chunks};
+    Params prm{decay, state_in, state_out, nullptr, nullptr, H, N, dv, pl.seg_chunks, pl.F};
     if (pl.G > 1) {
         uint8_t* sc = static_cast<uint8_t*>(scratch);
         prm.seg_state = reinterpret_cast<float*>(sc);
@@ -1005,7 +1050,13 @@ ret_status launch_dk(const void* q, const void* k, const void* v, const float* d
         constexpr int smem1 = kernel_smem<DK, GATED, true>();
         if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1) != cudaSuccess)
             return RET_ERR_CUDA;
-        k1<<<dim3(dv / kDvS, BH, pl.G - 1), kThreads, smem1, st>>>(mq, mk, mv, mo, prm);
+        Params prm1 = prm;  // the state-only pass runs over the sub-segments
+        prm1.seg_chunks = pl.seg_chunks / pl.F;
+        k1<<<dim3(dv / kDvS, BH, pl.subs()), kThreads, smem1, st>>>(mq, mk, mv, mo, prm1);
+        if (cudaGetLastError() != cudaSuccess) return RET_ERR_CUDA;
+        const int n4 = BH * DK * dv / 4;
+        seg_prefix_kernel<<<std::min((n4 + 255) / 256, 4 * sm_count()), 256, 0, st>>>(
+            prm.state_in, prm.seg_state, prm.seg_ldec, pl.subs() + 1, BH, DK * dv);
         if (cudaGetLastError() != cudaSuccess) return RET_ERR_CUDA;
     }
     auto k2 = chunk_tc_kernel<DK, GATED, false>;
@@ -1031,7 +1082,7 @@ ret_status launch_with_scratch(const void* q, const void* k, const void* v, cons
 
 }  // namespace tc
 
-inline int tc_chunk_launches(int B, int H, int N, int, int dv) { return tc::plan(B, H, N, dv).G > 1 ? 2 : 1; }
+inline int tc_chunk_launches(int B, int H, int N, int, int dv) { return tc::plan(B, H, N, dv).G > 1 ? 3 : 1; }
 
 namespace tc {
 

@@ -375,29 +375,19 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
             return true;
         };
 
-        // Initial state: kappa = 1, T = gamma^L0 S_in, bf16 copy = bf16(T). S_in is state_in (or
-        // zero) for the first segment; segment g > 0 folds in the earlier segments' end states:
-        // S_in(g) = decay_{g-1} S_in(g-1) + U_{g-1}.
+        // Initial state: kappa = 1, T = gamma^L0 S_in, bf16 copy = bf16(T), S_in from
+        // segment_start_state().
         float kappa;
         {
             bool rn;
             const float dec0 = pow_int_log2(lg, tile_len(0));
             kappa = lazy_next_scale(1.f, dec0, true, rn);
-            const float* sin = p.state_in ? p.state_in + ((size_t)bh * DK) * p.dv + dv0 + d : nullptr;
-            const size_t seg_stride = (size_t)gridDim.y * DK * p.dv;
-            const float* useg = p.seg_state + ((size_t)bh * DK) * p.dv + dv0 + d;
+            const float* sin = segment_start_state(p, seg, bh, DK, dv0 + d);
 #pragma unroll 1
             for (int cb = 0; cb < DK / 32; ++cb) {
                 uint32_t w[32], h[16];
 #pragma unroll
                 for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(sin ? sin[(size_t)(cb * 32 + c) * p.dv] : 0.f);
-#pragma unroll 1
-                for (int hs = 0; hs < seg; ++hs) {
-                    const float gam = exp2f(p.seg_ldec[(size_t)hs * gridDim.y + bh]);
-                    const float* u = useg + hs * seg_stride + (size_t)(cb * 32) * p.dv;
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(fmaf(gam, __uint_as_float(w[c]), u[(size_t)c * p.dv]));
-                }
 #pragma unroll
                 for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(__uint_as_float(w[c]) * dec0);
 #pragma unroll

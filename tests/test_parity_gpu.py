@@ -283,7 +283,7 @@ def test_split_sequence_matches_oracle(cuda_lib, B, H, N, dk, dv, gated, inplace
     """The tensor-core path cuts long sequences of few heads into segments (a
     state-only pass, then the full pass seeded per segment); the result must not
     change, including the final state and an in-place state buffer."""
-    assert cuda_lib.chunkwise_launches(B, H, N, dk, dv, 64, torch.bfloat16) == 2
+    assert cuda_lib.chunkwise_launches(B, H, N, dk, dv, 64, torch.bfloat16) == 3  # state-only pass, segment prefix, full pass
     gen = torch.Generator().manual_seed(N + dk + int(gated))
     q, k, v = I.qkv(B, H, N, dk, dv, torch.bfloat16, gen=gen)
     S0 = torch.randn(B, H, dk, dv, generator=gen) * 0.05
