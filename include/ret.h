@@ -131,6 +131,19 @@ RET_API const char* ret_status_str(ret_status s);
 RET_API ret_status ret_last_device_error(void* stream);
 
 /*
+ * Self-test of the failure path (the paper has no counterpart; a diagnostic).
+ * Launches one CTA on `stream` that takes tensor memory as the tensor-core
+ * kernels do, waits on an mbarrier that nothing completes with the kernels'
+ * bounded wait limited to limit_us microseconds (1 .. 1,000,000), sets the
+ * device error word when the wait runs out, releases the tensor memory and
+ * returns. Nothing faults or hangs; afterwards ret_last_device_error reports
+ * RET_ERR_TIMEOUT once and the device stays usable. Returns RET_ERR_SHAPE for
+ * a limit out of range, RET_ERR_UNSUPPORTED without an sm_100 device,
+ * RET_ERR_CUDA if the launch fails, RET_OK otherwise.
+ */
+RET_API ret_status ret_selftest_wait_timeout(unsigned int limit_us, void* stream);
+
+/*
  * Which kernel family ret_chunkwise / gated_ret_chunkwise would run for these
  * arguments: 1 = tcgen05 tensor-core path, 0 = CUDA-core path, -1 = rejected.
  * Pure host function; nothing is launched.

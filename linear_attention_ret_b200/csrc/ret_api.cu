@@ -184,6 +184,13 @@ int ret_chunkwise_launches(int B, int H, int N, int dk, int dv, int chunk, ret_d
     return 1;
 }
 
+ret_status ret_selftest_wait_timeout(unsigned int limit_us, void* stream) {
+    if (limit_us == 0 || limit_us > 1000000u) return RET_ERR_SHAPE;
+    if (!tc::tc_device_ok()) return RET_ERR_UNSUPPORTED;
+    tc::selftest_wait_kernel<<<1, 64, 0, as_stream(stream)>>>((unsigned long long)limit_us * 1000ull);
+    return cudaGetLastError() == cudaSuccess ? RET_OK : RET_ERR_CUDA;
+}
+
 const char* ret_version(void) { return "0.1.0"; }
 
 }  // extern "C"

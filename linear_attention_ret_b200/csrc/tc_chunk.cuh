@@ -132,15 +132,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Bounded wait. Returns false (and sets the abort flag and the device error
-// word on the first timeout) if the phase did not complete within kWaitNs or
+// word on the first timeout) if the phase did not complete within limit_ns or
 // another role already gave up.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_ns = kWaitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (globaltimer() - t0 > kWaitNs) {
+        if (globaltimer() - t0 > limit_ns) {
             *abort_flag = 1;
             raise_error(kErrWaitTimeout);
             return false;
@@ -910,6 +911,39 @@ seg_prefix_kernel(const float* __restrict__ state_in, float* __restrict__ seg_st
                 reinterpret_cast<float4*>(seg_state + (size_t)g * BH * per_bh)[i] = x;
             }
         }
+    }
+}
+
+// Self-test of the failure path: one CTA takes TMEM like the chunk kernels, waits with
+// their bounded wait on an mbarrier that nothing completes, takes the timeout path (device
+// error word, abort flag), releases TMEM and returns. Nothing faults or hangs.
+__global__ void __launch_bounds__(64, 1) selftest_wait_kernel(unsigned long long limit_ns) {
+    __shared__ __align__(8) uint64_t bar_storage;
+    __shared__ uint32_t slot;
+    __shared__ int abort_storage;
+    const uint32_t b = smem_u32(&bar_storage);
+    volatile int* abort_flag = &abort_storage;
+    const int warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) {
+        mbar_init(b, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&slot)), "r"(32)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = slot;
+    if (threadIdx.x == 0) mbar_wait(b, 0, abort_flag, limit_ns);  // nothing arrives: runs out
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(32) : "memory");
     }
 }
 

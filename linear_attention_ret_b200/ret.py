@@ -27,7 +27,7 @@ STATUS = {0: "RET_OK", 1: "RET_ERR_NULL", 2: "RET_ERR_SHAPE", 3: "RET_ERR_DTYPE"
 # every symbol include/ret.h declares
 SYMBOLS = ("ret_parallel", "ret_chunkwise", "ret_recurrent_step", "gated_ret_chunkwise", "ret_status_str",
            "ret_last_device_error", "ret_chunkwise_path", "ret_chunkwise_launches", "ret_version",
-           "ret_chunkwise_noalloc")
+           "ret_chunkwise_noalloc", "ret_selftest_wait_timeout")
 
 _lock = threading.Lock()
 _lib = None
@@ -65,6 +65,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
         lib.ret_status_str.restype = ctypes.c_char_p
         lib.ret_last_device_error.argtypes = [_vp]
         lib.ret_last_device_error.restype = _i
+        lib.ret_selftest_wait_timeout.argtypes = [ctypes.c_uint, _vp]
+        lib.ret_selftest_wait_timeout.restype = _i
         lib.ret_chunkwise_path.argtypes = [_i, _i, _i, _i]
         lib.ret_chunkwise_path.restype = _i
         lib.ret_chunkwise_launches.argtypes = [_i, _i, _i, _i, _i, _i, _i]
@@ -164,6 +166,11 @@ def ret_recurrent_step(q, k, v, gamma, state, o=None, stream=None):
 
 def last_device_error(stream=None) -> int:
     return int(load().ret_last_device_error(_stream(stream)))
+
+
+def selftest_wait_timeout(limit_us: int, stream=None) -> int:
+    """Launch the failure-path self-test (a bounded wait that runs out); returns the launch status."""
+    return int(load().ret_selftest_wait_timeout(limit_us, _stream(stream)))
 
 
 def chunkwise_launches(B: int, H: int, N: int, dk: int, dv: int, chunk: int, dtype: torch.dtype) -> int:
