@@ -9,6 +9,7 @@ already resident in HBM:
   retnet_6p7b_long  ret_chunkwise, B=1 H=16 N=8192 dk=256 dv=512 chunk 128, bf16
   gated             gated_ret_chunkwise, B=2 H=8 N=16384 dk=dv=128 chunk 64, bf16
   decode            ret_recurrent_step, B=64 H=16 dk=256 dv=512, fp32 state
+  gated_decode      gated_ret_recurrent_step, same shapes, a fresh log-decay g [B, H] per step
 For N > 1 (torchrun, one rank per GPU) every rank runs its own batch of the
 same shape (batch sharding, no collective on the data path): weak scaling.
 Rank 0 prints one JSON line. `--impl reference` times the fp64 CPU oracle on a
@@ -42,12 +43,14 @@ def workload(name: str):
     from linear_attention_ret_b200 import inputs as I
     cfg = I.CONFIGS[name]
     B, H, N, dk, dv, C = cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk
-    if name == "decode":
+    if name in ("decode", "gated_decode"):
+        gated = name == "gated_decode"
         state = B * H * dk * dv * 4
-        io = B * H * (2 * dk + 2 * dv) * 2
-        return dict(cfg=cfg, kind="decode", units=1, unit="steps/s", metric="decode steps/s",
+        io = B * H * (2 * dk + 2 * dv) * 2 + (B * H * 4 if gated else 0)  # + the step's g [B, H] fp32
+        return dict(cfg=cfg, kind="decode", gated=gated, units=1, unit="steps/s",
+                    metric="gated decode steps/s" if gated else "decode steps/s",
                     tokens=B, bytes=2 * state + io, flops=4 * B * H * dk * dv,
-                    h2d=B * H * (2 * dk + dv) * 2, d2h=B * H * dv * 2)
+                    h2d=B * H * (2 * dk + dv) * 2 + (B * H * 4 if gated else 0), d2h=B * H * dv * 2)
     elt = 2
     qkvo = B * H * N * (2 * dk + 2 * dv) * elt
     gbytes = B * H * N * 4 if cfg.gamma_schedule == "gated" else 0
@@ -198,17 +201,22 @@ def make_step(spec, dev, seed):
     from linear_attention_ret_b200 import ret
     cfg = spec["cfg"]
     if spec["kind"] == "decode":
-        gam = I.gammas(cfg.H, cfg.gamma_schedule).to(dev)
+        gated = spec["gated"]
+        gam = None if gated else I.gammas(cfg.H, cfg.gamma_schedule).to(dev)
         S = I.decode_state(cfg.B, cfg.H, cfg.dk, cfg.dv, seed=seed).to(dev)
         steps = [tuple(t.to(dev) for t in I.decode_step_inputs(cfg.B, cfg.H, cfg.dk, cfg.dv, s, seed=seed))
+                 + ((I.decode_gate(cfg.B, cfg.H, s, seed=seed).to(dev),) if gated else ())
                  for s in range(8)]
         o = torch.empty(cfg.B, cfg.H, cfg.dv, dtype=cfg.dtype, device=dev)
         counter = [0]
 
         def step():
-            q, k, v = steps[counter[0] % len(steps)]
+            x = steps[counter[0] % len(steps)]
             counter[0] += 1
-            ret.ret_recurrent_step(q, k, v, gam, S, o=o)
+            if gated:
+                ret.gated_ret_recurrent_step(x[0], x[1], x[2], x[3], S, o=o)
+            else:
+                ret.ret_recurrent_step(x[0], x[1], x[2], gam, S, o=o)
         return step, {"q": steps[0][0], "k": steps[0][1], "v": steps[0][2]}, o, 1
 
     x = {key: val.to(dev) for key, val in I.config_inputs(cfg, seed=seed).items()}
@@ -328,18 +336,23 @@ def run_e2e(args, spec, dev, stream, world):
     cfg = spec["cfg"]
     rank = dist_env()[0]
     if spec["kind"] == "decode":
+        gated = spec["gated"]
         host = [t.pin_memory() for t in I.decode_step_inputs(cfg.B, cfg.H, cfg.dk, cfg.dv, 0, seed=rank_seed(rank))]
-        dq, dk_, dv_ = (torch.empty_like(t, device=dev) for t in host)
-        gam = I.gammas(cfg.H, cfg.gamma_schedule).to(dev)
+        if gated:
+            host.append(I.decode_gate(cfg.B, cfg.H, 0, seed=rank_seed(rank)).pin_memory())
+        dev_in = [torch.empty_like(t, device=dev) for t in host]
+        gam = None if gated else I.gammas(cfg.H, cfg.gamma_schedule).to(dev)
         S = I.decode_state(cfg.B, cfg.H, cfg.dk, cfg.dv).to(dev)
         o = torch.empty(cfg.B, cfg.H, cfg.dv, dtype=cfg.dtype, device=dev)
         o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
 
         def step():
-            dq.copy_(host[0], non_blocking=True)
-            dk_.copy_(host[1], non_blocking=True)
-            dv_.copy_(host[2], non_blocking=True)
-            ret.ret_recurrent_step(dq, dk_, dv_, gam, S, o=o)
+            for d, h in zip(dev_in, host):
+                d.copy_(h, non_blocking=True)
+            if gated:
+                ret.gated_ret_recurrent_step(dev_in[0], dev_in[1], dev_in[2], dev_in[3], S, o=o)
+            else:
+                ret.ret_recurrent_step(dev_in[0], dev_in[1], dev_in[2], gam, S, o=o)
             o_host.copy_(o, non_blocking=True)
     else:
         xh = {k: t.pin_memory() for k, t in I.config_inputs(cfg, seed=rank_seed(rank)).items()}
@@ -383,12 +396,18 @@ def _oracle_sample_step(spec, heads, seed=0):
     from oracle import oracle as O
     cfg = spec["cfg"]
     if spec["kind"] == "decode":
-        gam = I.gammas(cfg.H, cfg.gamma_schedule)
         q, k, v = I.decode_step_inputs(cfg.B, cfg.H, cfg.dk, cfg.dv, 0, seed=seed)
         S = I.decode_state(cfg.B, cfg.H, cfg.dk, cfg.dv, seed=seed)
         b_needed = max(1, -(-heads // cfg.H))
         qs, ks, vs, Ss = (t[:b_needed] for t in (q, k, v, S))
         state = [Ss.double().numpy()]
+        if spec["gated"]:
+            gs = I.decode_gate(cfg.B, cfg.H, 0, seed=seed)[:b_needed]
+
+            def run():
+                _, state[0] = O.gated_recurrent_step(qs, ks, vs, gs, state[0])
+            return run, b_needed * cfg.H / (cfg.B * cfg.H)
+        gam = I.gammas(cfg.H, cfg.gamma_schedule)
 
         def run():
             _, state[0] = O.ret_recurrent_step(qs, ks, vs, gam, state[0])
@@ -481,7 +500,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="retnet_1p3b",
-                    choices=["retnet_1p3b", "retnet_6p7b_long", "gated", "decode"])
+                    choices=["retnet_1p3b", "retnet_6p7b_long", "gated", "decode", "gated_decode"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

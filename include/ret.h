@@ -78,8 +78,8 @@ RET_API ret_status ret_parallel(const void* q, const void* k, const void* v, con
  *   S_[i] = gamma^L S_[i-1] + sum_m gamma^(L-1-m) K_m^T V_m
  * state_in : initial state [B, H, dk, dv] fp32, or NULL for zeros.
  * state_out: final state [B, H, dk, dv] fp32, or NULL. May equal state_in.
- * The result does not depend on `chunk` beyond rounding; chunks longer than 64
- * tokens are evaluated as 64-token sub-chunks.
+ * The result does not depend on `chunk` beyond rounding: the tensor-core path
+ * computes on tiles of 64 or (gamma_h >= 2^-0.75, dk >= 128) 128 tokens.
  * Requires chunk >= 1, dk <= 256, dv >= 1. The tensor-core path (bf16,
  * dk in {64, 128, 256}, dv a multiple of 128, chunk a multiple of 64) also
  * needs 16-byte aligned q, k, v, o; other shapes use a CUDA-core path.
@@ -102,6 +102,17 @@ RET_API ret_status ret_chunkwise(const void* q, const void* k, const void* v, co
 RET_API ret_status ret_recurrent_step(const void* q, const void* k, const void* v, const float* gamma,
                               float* state, void* o, int B, int H, int dk, int dv,
                               ret_dtype dt, void* stream);
+
+/*
+ * One gated recurrent (decode) step, [GR] recurrent_gate_retention:
+ *   S <- exp(g_bh) S + k^T v   (in place),   o = q S   (the updated state).
+ * g [B, H] fp32: this step's natural-log decay per (batch, head), normally <= 0
+ * (the decode counterpart of gated_ret_chunkwise's g[:, :, n]). Other tensors,
+ * layouts and requirements as ret_recurrent_step.
+ */
+RET_API ret_status gated_ret_recurrent_step(const void* q, const void* k, const void* v, const float* g,
+                                    float* state, void* o, int B, int H, int dk, int dv,
+                                    ret_dtype dt, void* stream);
 
 /*
  * Gated chunkwise form, [GR] chunk_gate_retention: the per-token log-decay g

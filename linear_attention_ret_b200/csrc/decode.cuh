@@ -1,5 +1,7 @@
 // Recurrent (decode) step: "RetNet retention mechanism" (aiqz.cc), section
 // 递归推理 (recurrent inference): S_n = gamma S_{n-1} + K_n^T V_n, R_n = Q_n S_n.
+// Gated form (GATED, the chunk_gate_retention page's recurrent form): the decay of
+// step n is exp(g_n) with g the step's log-decay per (b, h), S_n = e^{g_n} S_{n-1} + K_n^T V_n.
 //
 // The fp32 state [B, H, dk, dv] is read once and written once per step, so the
 // kernel is bound by HBM bandwidth (0.5 flop per byte). Each thread owns four
@@ -17,7 +19,13 @@ namespace ret {
 constexpr int kDecThreads = 128;
 constexpr int kDecUnroll = 8;
 
-template <typename T>
+// decay: gamma [H] (fixed), or g [B, H] natural-log step decays (GATED)
+template <typename T, bool GATED>
+__device__ __forceinline__ float step_decay(const float* decay, int bh, int H) {
+    return GATED ? expf(decay[bh]) : decay[bh % H];
+}
+
+template <typename T, bool GATED>
 __global__ void __launch_bounds__(kDecThreads)
 recurrent_step_vec_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                           const float* __restrict__ gamma, float* __restrict__ state, T* __restrict__ o,
@@ -34,7 +42,7 @@ recurrent_step_vec_kernel(const T* __restrict__ q, const T* __restrict__ k, cons
     const int cg = blockIdx.x * blockDim.x + threadIdx.x;  // column group: columns 4cg .. 4cg+3
     const int ngroups = dv >> 2;
     if (cg >= ngroups) return;
-    const float gm = gamma[bh % H];
+    const float gm = step_decay<T, GATED>(gamma, bh, H);
     const T* vp = v + (size_t)bh * dv + 4 * cg;
     const float v0 = ld_elem(vp), v1 = ld_elem(vp + 1), v2 = ld_elem(vp + 2), v3 = ld_elem(vp + 3);
     float4* S = reinterpret_cast<float4*>(state + (size_t)bh * dk * dv) + cg;
@@ -79,7 +87,7 @@ recurrent_step_vec_kernel(const T* __restrict__ q, const T* __restrict__ k, cons
 }
 
 // Scalar variant for dv not a multiple of 4 or a state that is not 16-byte aligned.
-template <typename T>
+template <typename T, bool GATED>
 __global__ void __launch_bounds__(kDecThreads)
 recurrent_step_scalar_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                              const float* __restrict__ gamma, float* __restrict__ state, T* __restrict__ o,
@@ -95,7 +103,7 @@ recurrent_step_scalar_kernel(const T* __restrict__ q, const T* __restrict__ k, c
     __syncthreads();
     const int c = blockIdx.x * blockDim.x + threadIdx.x;
     if (c >= dv) return;
-    const float gm = gamma[bh % H];
+    const float gm = step_decay<T, GATED>(gamma, bh, H);
     const float vc = ld_elem(v + (size_t)bh * dv + c);
     float* S = state + (size_t)bh * dk * dv + c;
     float acc = 0.f;

@@ -91,19 +91,19 @@ ret_status launch_parallel(const void* q, const void* k, const void* v, const fl
     return launch_status();
 }
 
-template <typename T>
+template <typename T, bool GATED>
 ret_status launch_step(const void* q, const void* k, const void* v, const float* gamma, float* state, void* o,
                        int B, int H, int dk, int dv, cudaStream_t st) {
     const size_t smem = sizeof(float) * 2 * (size_t)dk;
     if ((dv & 3) == 0 && aligned16(state)) {
         const int groups = dv / 4;
         dim3 grid((groups + kDecThreads - 1) / kDecThreads, B * H);
-        recurrent_step_vec_kernel<T><<<grid, kDecThreads, smem, st>>>(
+        recurrent_step_vec_kernel<T, GATED><<<grid, kDecThreads, smem, st>>>(
             static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), gamma, state,
             static_cast<T*>(o), H, dk, dv);
     } else {
         dim3 grid((dv + kDecThreads - 1) / kDecThreads, B * H);
-        recurrent_step_scalar_kernel<T><<<grid, kDecThreads, smem, st>>>(
+        recurrent_step_scalar_kernel<T, GATED><<<grid, kDecThreads, smem, st>>>(
             static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), gamma, state,
             static_cast<T*>(o), H, dk, dv);
     }
@@ -145,8 +145,19 @@ ret_status ret_recurrent_step(const void* q, const void* k, const void* v, const
     if (dk > 4096) return RET_ERR_UNSUPPORTED;
     if (!q || !k || !v || !gamma || !state || !o) return RET_ERR_NULL;
     cudaStream_t st = as_stream(stream);
-    return dt == RET_F32 ? launch_step<float>(q, k, v, gamma, state, o, B, H, dk, dv, st)
-                         : launch_step<__nv_bfloat16>(q, k, v, gamma, state, o, B, H, dk, dv, st);
+    return dt == RET_F32 ? launch_step<float, false>(q, k, v, gamma, state, o, B, H, dk, dv, st)
+                         : launch_step<__nv_bfloat16, false>(q, k, v, gamma, state, o, B, H, dk, dv, st);
+}
+
+ret_status gated_ret_recurrent_step(const void* q, const void* k, const void* v, const float* g, float* state,
+                                    void* o, int B, int H, int dk, int dv, ret_dtype dt, void* stream) {
+    ret_status s = check_common(B, H, 1, dk, dv, dt);
+    if (s != RET_OK) return s;
+    if (dk > 4096) return RET_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !g || !state || !o) return RET_ERR_NULL;
+    cudaStream_t st = as_stream(stream);
+    return dt == RET_F32 ? launch_step<float, true>(q, k, v, g, state, o, B, H, dk, dv, st)
+                         : launch_step<__nv_bfloat16, true>(q, k, v, g, state, o, B, H, dk, dv, st);
 }
 
 const char* ret_status_str(ret_status s) {

@@ -46,6 +46,7 @@ CONFIGS = {
     "retnet_6p7b_long": RetConfig("retnet_6p7b_long", 1, 16, 8192, 256, 512, 128, torch.bfloat16, "h/3"),
     "decode": RetConfig("decode", 64, 16, 1, 256, 512, 1, torch.bfloat16, "h/3"),
     "gated": RetConfig("gated", 2, 8, 16384, 128, 128, 64, torch.bfloat16, "gated"),
+    "gated_decode": RetConfig("gated_decode", 64, 16, 1, 256, 512, 1, torch.bfloat16, "gated"),
 }
 DECODE_STEPS = 1024
 
@@ -103,6 +104,12 @@ def decode_state(B: int, H: int, dk: int, dv: int, seed: int = 0) -> torch.Tenso
     """Initial decode state S_0 ~ N(0, 0.01^2), fp32 [B, H, dk, dv]."""
     g = _gen(seed + 7919)
     return torch.randn(B, H, dk, dv, generator=g) * 0.01
+
+
+def decode_gate(B: int, H: int, step: int, seed: int = 0) -> torch.Tensor:
+    """Log-decay g [B, H] of gated decode step `step`: logsigmoid(x)/16, x ~ N(0,1) (seed + 50021 + step)."""
+    g = _gen(seed + 50021 + step)
+    return torch.nn.functional.logsigmoid(torch.randn(B, H, generator=g)) / 16.0
 
 
 def decode_step_inputs(B: int, H: int, dk: int, dv: int, step: int, seed: int = 0,

@@ -27,7 +27,7 @@ STATUS = {0: "RET_OK", 1: "RET_ERR_NULL", 2: "RET_ERR_SHAPE", 3: "RET_ERR_DTYPE"
 # every symbol include/ret.h declares
 SYMBOLS = ("ret_parallel", "ret_chunkwise", "ret_recurrent_step", "gated_ret_chunkwise", "ret_status_str",
            "ret_last_device_error", "ret_chunkwise_path", "ret_chunkwise_launches", "ret_version",
-           "ret_chunkwise_noalloc", "ret_selftest_wait_timeout")
+           "ret_chunkwise_noalloc", "ret_selftest_wait_timeout", "gated_ret_recurrent_step")
 
 _lock = threading.Lock()
 _lib = None
@@ -58,8 +58,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
         lib.gated_ret_chunkwise.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
         lib.ret_chunkwise_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
         lib.ret_recurrent_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
+        lib.gated_ret_recurrent_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
         for fn in ("ret_parallel", "ret_chunkwise", "gated_ret_chunkwise", "ret_recurrent_step",
-                   "ret_chunkwise_noalloc"):
+                   "ret_chunkwise_noalloc", "gated_ret_recurrent_step"):
             getattr(lib, fn).restype = _i
         lib.ret_status_str.argtypes = [_i]
         lib.ret_status_str.restype = ctypes.c_char_p
@@ -161,6 +162,18 @@ def ret_recurrent_step(q, k, v, gamma, state, o=None, stream=None):
     _cuda(q, k, v, gamma, state, o)
     _check("ret_recurrent_step", load().ret_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(state),
                                                            _ptr(o), B, H, dk, dv, _dt(q), _stream(stream)))
+    return o
+
+
+def gated_ret_recurrent_step(q, k, v, g, state, o=None, stream=None):
+    """One gated decode step with log-decay g [B, H] (fp32); updates state in place, returns o [B, H, dv]."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    o = torch.empty(B, H, dv, dtype=q.dtype, device=q.device) if o is None else o
+    _cuda(q, k, v, g, state, o)
+    _check("gated_ret_recurrent_step", load().gated_ret_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                                                       _ptr(state), _ptr(o), B, H, dk, dv, _dt(q),
+                                                                       _stream(stream)))
     return o
 
 

@@ -194,6 +194,14 @@ def gated_recurrent(q, k, v, g, state_in=None):
     return o, s_out
 
 
+def gated_recurrent_step(q, k, v, g, state):
+    """One gated decode step (Gated RetNet page, recurrent_gate_retention): the gated
+    recurrent form over a single token, S = exp(g) S + k^T v, o = q S (updated state).
+    q, k [B, H, dk]; v [B, H, dv]; g [B, H]; returns (o [B, H, dv], new_state)."""
+    o, s = gated_recurrent(_f64(q)[:, :, None], _f64(k)[:, :, None], _f64(v)[:, :, None], _f64(g)[:, :, None], state)
+    return o[:, :, 0], s
+
+
 def gated_chunkwise(q, k, v, g, chunk, state_in=None):
     q, k, v, g, s_in = map(_f64, (q, k, v, g, state_in))
     B, H, N, dk, dv = _dims(q, v)

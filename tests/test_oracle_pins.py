@@ -244,6 +244,39 @@ def test_gated_forms_agree(chunk):
     np.testing.assert_allclose(s_chk, s_rec, rtol=1e-11, atol=1e-12)
 
 
+def test_gated_step_constant_gate_equals_fixed_step():
+    """A gated decode step with g = ln(gamma_h) is the fixed-gamma decode step."""
+    rng = np.random.default_rng(21)
+    q, k, v = rng.standard_normal((2, 2, 5)), rng.standard_normal((2, 2, 5)), rng.standard_normal((2, 2, 3))
+    S = rng.standard_normal((2, 2, 5, 3))
+    g = np.broadcast_to(np.log(GAMMAS)[None, :], (2, 2)).copy()
+    o_g, S_g = O.gated_recurrent_step(q, k, v, g, S)
+    o_f, S_f = O.ret_recurrent_step(q, k, v, GAMMAS, S)
+    np.testing.assert_allclose(o_g, o_f, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(S_g, S_f, rtol=1e-12, atol=1e-13)
+
+
+def test_gated_steps_equal_gated_chunkwise():
+    """Twelve gated decode steps from a state equal the gated chunkwise form over the
+    same twelve tokens (in-chunk cumulative sums, a different computation), per token
+    and in the final state; one step by hand: S' = e^g S + k^T v, o = q S'."""
+    q, k, v = _inputs(B=1, H=2, N=12, seed=22)
+    g = _gate(1, 2, 12, seed=3, scale=8.0)
+    S0 = np.random.default_rng(23).standard_normal((1, 2, 5, 3))
+    S = S0
+    outs = []
+    for t in range(12):
+        o, S = O.gated_recurrent_step(q[:, :, t], k[:, :, t], v[:, :, t], g[:, :, t], S)
+        outs.append(o)
+    o_chk, s_chk = O.gated_chunkwise(q, k, v, g, 5, state_in=S0)
+    np.testing.assert_allclose(np.stack(outs, axis=2), o_chk, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(S, s_chk, rtol=1e-11, atol=1e-12)
+    S1 = np.exp(g[:, :, 0])[..., None, None] * S0 + np.einsum("bhd,bhe->bhde", k[:, :, 0], v[:, :, 0])
+    o1, S1_or = O.gated_recurrent_step(q[:, :, 0], k[:, :, 0], v[:, :, 0], g[:, :, 0], S0)
+    np.testing.assert_allclose(S1_or, S1, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(o1, np.einsum("bhd,bhde->bhe", q[:, :, 0], S1), rtol=1e-13, atol=1e-13)
+
+
 def test_gated_long_sequence_stays_finite():
     """A long strongly decaying gate drives the global cumulative sum far below
     exp's range; the chunkwise form uses in-chunk sums only and stays finite."""

@@ -210,6 +210,23 @@ def test_recurrent_step_matches_oracle(cuda_lib, dtype, dv):
     assert_close(Sd, S_ref, dtype, "state")
 
 
+@pytest.mark.parametrize("dtype,dv", [(torch.float32, 128), (torch.bfloat16, 512), (torch.float32, 30)])
+def test_gated_recurrent_step_matches_oracle(cuda_lib, dtype, dv):
+    """Gated decode step (vector path, and the scalar path for dv = 30), five steps
+    with a fresh log-decay per step and (b, h), from a nonzero state."""
+    B, H, dk = 3, 4, 64
+    S0 = I.decode_state(B, H, dk, dv, seed=2)
+    Sd = S0.to(DEV)
+    S_ref = S0.double().numpy()
+    for step in range(5):
+        q, k, v = I.decode_step_inputs(B, H, dk, dv, step, dtype=dtype)
+        g = I.decode_gate(B, H, step) * 8.0  # stronger decay than the workload
+        o = cuda_lib.gated_ret_recurrent_step(*_dev(q, k, v, g), Sd)
+        want_o, S_ref = O.gated_recurrent_step(q, k, v, g, S_ref)
+        assert_close(o, want_o, dtype, f"o step {step}")
+    assert_close(Sd, S_ref, dtype, "state")
+
+
 # ------------------------------------------------------------------ full-size workloads, sampled heads
 
 def _head(x, b, h):
@@ -259,6 +276,32 @@ def test_full_size_decode_sampled_heads(cuda_lib):
             got[(b, h)].append(o[b, h].float().cpu())
             sl = (slice(b, b + 1), slice(h, h + 1))
             ow, S_ref[(b, h)] = O.ret_recurrent_step(q[sl], k[sl], v[sl], gam[h:h + 1], S_ref[(b, h)])
+            want[(b, h)].append(ow[0, 0])
+    assert cuda_lib.last_device_error() == 0
+    for s in samples:
+        assert rel_l2(torch.stack(got[s]), np.stack(want[s])) <= TOL_BF16, s
+        assert rel_l2(Sd[s[0], s[1]], S_ref[s][0, 0]) <= TOL_BF16, s
+
+
+def test_full_size_gated_decode_sampled_heads(cuda_lib):
+    """The gated decode workload at full size (1 GiB state) for 256 steps, sampled heads
+    checked against the oracle every step and in the final state."""
+    cfg = I.CONFIGS["gated_decode"]
+    B, H, dk, dv = cfg.B, cfg.H, cfg.dk, cfg.dv
+    S0 = I.decode_state(B, H, dk, dv)
+    Sd = S0.to(DEV)
+    samples = [(0, 0), (B - 1, H - 1), (17, 9)]
+    S_ref = {s: S0[s[0]:s[0] + 1, s[1]:s[1] + 1].double().numpy() for s in samples}
+    got = {s: [] for s in samples}
+    want = {s: [] for s in samples}
+    for step in range(256):
+        q, k, v = I.decode_step_inputs(B, H, dk, dv, step)
+        g = I.decode_gate(B, H, step)
+        o = cuda_lib.gated_ret_recurrent_step(*_dev(q, k, v, g), Sd)
+        for (b, h) in samples:
+            got[(b, h)].append(o[b, h].float().cpu())
+            sl = (slice(b, b + 1), slice(h, h + 1))
+            ow, S_ref[(b, h)] = O.gated_recurrent_step(q[sl], k[sl], v[sl], g[sl], S_ref[(b, h)])
             want[(b, h)].append(ow[0, 0])
     assert cuda_lib.last_device_error() == 0
     for s in samples:
