@@ -10,6 +10,8 @@ already resident in HBM:
   gated             gated_ret_chunkwise, B=2 H=8 N=16384 dk=dv=128 chunk 64, bf16
   decode            ret_recurrent_step, B=64 H=16 dk=256 dv=512, fp32 state
   gated_decode      gated_ret_recurrent_step, same shapes, a fresh log-decay g [B, H] per step
+  seqpar_6p7b       the retnet_6p7b_long sequence split across the ranks (strong scaling):
+                    segment end states, one all-gather, start states, ret_chunkwise per segment
 For N > 1 (torchrun, one rank per GPU) every rank runs its own batch of the
 same shape (batch sharding, no collective on the data path): weak scaling.
 Rank 0 prints one JSON line. `--impl reference` times the fp64 CPU oracle on a
@@ -41,6 +43,12 @@ L2_BYTES = 126 * 1024 * 1024
 def workload(name: str):
     """Shapes plus the algorithmic work of one step (one call)."""
     from linear_attention_ret_b200 import inputs as I
+    if name == "seqpar_6p7b":
+        # the 6.7B-shaped sequence split across the ranks (strong scaling): per step the
+        # whole sequence once, each rank its segment; work counted as for ret_chunkwise
+        spec = workload("retnet_6p7b_long")
+        spec.update(kind="seqpar", metric="retention tokens/s (sequence-parallel chunkwise fwd)")
+        return spec
     cfg = I.CONFIGS[name]
     B, H, N, dk, dv, C = cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk
     if name in ("decode", "gated_decode"):
@@ -219,6 +227,14 @@ def make_step(spec, dev, seed):
                 ret.ret_recurrent_step(x[0], x[1], x[2], gam, S, o=o)
         return step, {"q": steps[0][0], "k": steps[0][1], "v": steps[0][2]}, o, 1
 
+    if spec["kind"] == "seqpar":
+        from linear_attention_ret_b200 import seqpar
+        rank, world, _ = dist_env()
+        x = {key: val.to(dev) for key, val in seqpar_segment(cfg, rank, world).items()}
+
+        def step():
+            seqpar.sequence_parallel_chunkwise(x["q"], x["k"], x["v"], x["gamma"], cfg.chunk)
+        return step, x, None, launches_per_call(spec)
     x = {key: val.to(dev) for key, val in I.config_inputs(cfg, seed=seed).items()}
     o = torch.empty(cfg.B, cfg.H, cfg.N, cfg.dv, dtype=cfg.dtype, device=dev)
     if spec["kind"] == "gated":
@@ -230,12 +246,25 @@ def make_step(spec, dev, seed):
     return step, x, o, launches_per_call(spec)
 
 
+def seqpar_segment(cfg, rank, world):
+    """Rank `rank`'s consecutive slice of one seeded sequence (the same seed on every rank)."""
+    from linear_attention_ret_b200 import inputs as I
+    x = I.config_inputs(cfg, seed=0)
+    t0, t1 = cfg.N * rank // world, cfg.N * (rank + 1) // world
+    return {k: (t[:, :, t0:t1].contiguous() if t.dim() == 4 else t) for k, t in x.items()}
+
+
 def launches_per_call(spec) -> int:
     """Kernels one call of the step launches (the library's own kernels only)."""
     from linear_attention_ret_b200 import ret
     cfg = spec["cfg"]
     if spec["kind"] == "decode":
         return 1
+    if spec["kind"] == "seqpar":
+        _, world, _ = dist_env()
+        n = cfg.N // world + (1 if cfg.N % world else 0)
+        return (ret.chunkwise_state_launches(cfg.B, cfg.H, n, cfg.dk, cfg.dv, cfg.chunk, cfg.dtype) + 1
+                + ret.chunkwise_launches(cfg.B, cfg.H, n, cfg.dk, cfg.dv, cfg.chunk, cfg.dtype))
     return ret.chunkwise_launches(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk, cfg.dtype)
 
 
@@ -289,7 +318,11 @@ def run_ours(args, spec):
     e2e = run_e2e(args, spec, dev, stream, world)
 
     ms_per_step = max_ms / args.steps
-    value = spec["units"] * world / (ms_per_step / 1e3) if spec["kind"] != "decode" else world * 1e3 / ms_per_step
+    strong = spec["kind"] == "seqpar"  # one sequence split across the ranks
+    if spec["kind"] == "decode":
+        value = world * 1e3 / ms_per_step
+    else:
+        value = spec["units"] * (1 if strong else world) / (ms_per_step / 1e3)
     hbm, tf_burst, tf_sust, peak_src = measured_peaks()
     # the dominant kernel's duration: a step is one launch of it (plus, for split
     # sequences, two short launches whose share the ncu launch list records)
@@ -306,12 +339,14 @@ def run_ours(args, spec):
     line = {
         "metric": spec["metric"], "value": round(value, 2), "unit": spec["unit"], "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1)/sqrt(dk); per-rank seeds)",
+        "higher_is_better": True, "scaling": "strong" if strong else "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1)/sqrt(dk); " + ("one sequence split across ranks)" if strong
+                                                        else "per-rank seeds)"),
         "config": {"workload": args.workload, "B": cfg.B, "H": cfg.H, "N": cfg.N, "dk": cfg.dk, "dv": cfg.dv,
                    "chunk": cfg.chunk, "state": "fp32",
                    "l2": f"working set {spec['bytes'] / 1e6:.0f} MB per step > 126 MB L2 (no flush)",
-                   "parallelism": f"batch-sharded x{world}" if world > 1 else "single GPU"},
+                   "parallelism": (f"sequence-parallel x{world} (one all-gather of segment states)" if strong
+                                   else f"batch-sharded x{world}") if world > 1 else "single GPU"},
         "roofline": roofline,
         "clocks": dict(clk, window="warm-up, ~1 s untimed burn-in and the timed region") if clk else None,
         "e2e": e2e,
@@ -354,6 +389,17 @@ def run_e2e(args, spec, dev, stream, world):
             else:
                 ret.ret_recurrent_step(dev_in[0], dev_in[1], dev_in[2], gam, S, o=o)
             o_host.copy_(o, non_blocking=True)
+    elif spec["kind"] == "seqpar":
+        from linear_attention_ret_b200 import seqpar
+        xh = {k: t.pin_memory() for k, t in seqpar_segment(cfg, rank, world).items()}
+        xd = {k: torch.empty_like(t, device=dev) for k, t in xh.items()}
+        o_host = torch.empty(xh["v"].shape, dtype=cfg.dtype).pin_memory()
+
+        def step():
+            for key in xh:
+                xd[key].copy_(xh[key], non_blocking=True)
+            o, _ = seqpar.sequence_parallel_chunkwise(xd["q"], xd["k"], xd["v"], xd["gamma"], cfg.chunk)
+            o_host.copy_(o, non_blocking=True)
     else:
         xh = {k: t.pin_memory() for k, t in I.config_inputs(cfg, seed=rank_seed(rank)).items()}
         xd = {k: torch.empty_like(t, device=dev) for k, t in xh.items()}
@@ -381,7 +427,7 @@ def run_e2e(args, spec, dev, stream, world):
     t1.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(t0.elapsed_time(t1), world, dev) / steps
-    value = (spec["units"] if spec["kind"] != "decode" else 1) * world / (ms / 1e3)
+    value = (spec["units"] if spec["kind"] != "decode" else 1) * (1 if spec["kind"] == "seqpar" else world) / (ms / 1e3)
     return {"value": round(value, 2), "unit": spec["unit"], "ms_per_step": round(ms, 4),
             "h2d_bytes_per_step": spec["h2d"], "d2h_bytes_per_step": spec["d2h"]}
 
@@ -500,7 +546,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="retnet_1p3b",
-                    choices=["retnet_1p3b", "retnet_6p7b_long", "gated", "decode", "gated_decode"])
+                    choices=["retnet_1p3b", "retnet_6p7b_long", "gated", "decode", "gated_decode", "seqpar_6p7b"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

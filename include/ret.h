@@ -142,6 +142,47 @@ RET_API const char* ret_status_str(ret_status s);
 RET_API ret_status ret_last_device_error(void* stream);
 
 /*
+ * Sequence split into consecutive segments computed separately (for example
+ * one per GPU, then one exchange of states), [RM] 块级循环 / [GR] cross_chunk:
+ * the chunkwise recurrence composes over segments as
+ *   S_in(0) = state_in,   S_in(r + 1) = D_r S_in(r) + U_r,
+ * where U_r is segment r's end state from a zero start and D_r its total decay
+ * (gamma_h^{N_r}, or exp of the sum of its gates). Running ret_chunkwise (or
+ * gated_ret_chunkwise) on segment r from S_in(r) then gives exactly that
+ * segment's outputs of the whole sequence, and S_in(R) is the final state.
+ *
+ * ret_chunkwise_state / gated_ret_chunkwise_state: U and log2 D of one segment
+ * (k, v, gamma or g as in the chunkwise calls; no q, no outputs).
+ *   state_out  [B, H, dk, dv] fp32: U (from a zero start).
+ *   log2_decay [B, H] fp32: log2 D per (b, h) (-inf where gamma_h = 0).
+ * Same size rules and tensor-core path conditions as ret_chunkwise; may take
+ * stream-ordered scratch (freed on the same stream before returning).
+ */
+RET_API ret_status ret_chunkwise_state(const void* k, const void* v, const float* gamma, float* state_out,
+                               float* log2_decay, int B, int H, int N, int dk, int dv, int chunk,
+                               ret_dtype dt, void* stream);
+RET_API ret_status gated_ret_chunkwise_state(const void* k, const void* v, const float* g, float* state_out,
+                                     float* log2_decay, int B, int H, int N, int dk, int dv, int chunk,
+                                     ret_dtype dt, void* stream);
+
+/* Kernels one ret_chunkwise_state / gated_ret_chunkwise_state call launches (0 for
+ * an empty segment, -1 if the arguments would be rejected). Host function. */
+RET_API int ret_chunkwise_state_launches(int B, int H, int N, int dk, int dv, int chunk, ret_dtype dt);
+
+/*
+ * Start states of R consecutive segments from their end states and decays:
+ *   seg_states [R, B, H, dk, dv] fp32 (U_0 .. U_{R-1}), seg_log2_decay [R, B, H],
+ *   state_in [B, H, dk, dv] or NULL (zeros),
+ *   start_states [R, B, H, dk, dv] receives S_in(0 .. R-1),
+ *   end_state [B, H, dk, dv] or NULL receives S_in(R) (the state after all R).
+ * start_states and end_state must not overlap the inputs. Errors: RET_ERR_SHAPE
+ * for non-positive sizes, RET_ERR_NULL for a missing required pointer.
+ */
+RET_API ret_status ret_state_prefix(const float* seg_states, const float* seg_log2_decay,
+                            const float* state_in, float* start_states, float* end_state,
+                            int R, int B, int H, int dk, int dv, void* stream);
+
+/*
  * Self-test of the failure path (the paper has no counterpart; a diagnostic).
  * Launches one CTA on `stream` that takes tensor memory as the tensor-core
  * kernels do, waits on an mbarrier that nothing completes with the kernels'

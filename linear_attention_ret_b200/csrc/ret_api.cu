@@ -9,6 +9,7 @@
 #include "simt.cuh"
 #include "decode.cuh"
 #include "tc_chunk.cuh"
+#include "seqpar.cuh"
 
 using namespace ret;
 
@@ -78,6 +79,38 @@ ret_status chunkwise_entry(const void* q, const void* k, const void* v, const fl
                                                    chunk, st);
     return launch_chunkwise_simt<__nv_bfloat16, GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dk,
                                                        dv, chunk, st);
+}
+
+// End state of a sequence from a zero start and log2 of its total decay, without outputs.
+template <bool GATED>
+ret_status chunkwise_state_entry(const void* k, const void* v, const float* decay, float* state_out, float* log2_decay,
+                                 int B, int H, int N, int dk, int dv, int chunk, ret_dtype dt, void* stream) {
+    ret_status s = check_common(B, H, N, dk, dv, dt);
+    if (s != RET_OK) return s;
+    if (chunk <= 0) return RET_ERR_SHAPE;
+    if (dk > 256) return RET_ERR_UNSUPPORTED;
+    if (!state_out || !log2_decay) return RET_ERR_NULL;
+    cudaStream_t st = as_stream(stream);
+    if (N == 0) {
+        if (cudaMemsetAsync(log2_decay, 0, sizeof(float) * (size_t)B * H, st) != cudaSuccess) return RET_ERR_CUDA;
+        return empty_sequence_state(nullptr, state_out, B, H, dk, dv, st);
+    }
+    if (!k || !v || !decay) return RET_ERR_NULL;
+    const bool tc = tc_chunk_supported(dk, dv, chunk, dt == RET_BF16);
+    if (tc && (!aligned16(k) || !aligned16(v))) return RET_ERR_ALIGN;
+    segment_log2_decay_kernel<GATED><<<B * H, 256, 0, st>>>(decay, log2_decay, H, N);
+    if (cudaGetLastError() != cudaSuccess) return RET_ERR_CUDA;
+    if (tc) return tc_state_launch<GATED>(k, v, decay, state_out, B, H, N, dk, dv, st);
+    // CUDA-core path: the chunkwise kernel with its outputs sent to scratch (K stands in for Q)
+    void* o = nullptr;
+    if (cudaMallocAsync(&o, (size_t)B * H * N * dv * (dt == RET_F32 ? 4 : 2), st) != cudaSuccess) return RET_ERR_CUDA;
+    const ret_status r =
+        dt == RET_F32
+            ? launch_chunkwise_simt<float, GATED>(k, k, v, decay, o, nullptr, state_out, B, H, N, dk, dv, chunk, st)
+            : launch_chunkwise_simt<__nv_bfloat16, GATED>(k, k, v, decay, o, nullptr, state_out, B, H, N, dk, dv,
+                                                          chunk, st);
+    if (cudaFreeAsync(o, st) != cudaSuccess) return RET_ERR_CUDA;
+    return r;
 }
 
 template <typename T>
@@ -195,11 +228,41 @@ int ret_chunkwise_launches(int B, int H, int N, int dk, int dv, int chunk, ret_d
     return 1;
 }
 
+ret_status ret_chunkwise_state(const void* k, const void* v, const float* gamma, float* state_out, float* log2_decay,
+                               int B, int H, int N, int dk, int dv, int chunk, ret_dtype dt, void* stream) {
+    return chunkwise_state_entry<false>(k, v, gamma, state_out, log2_decay, B, H, N, dk, dv, chunk, dt, stream);
+}
+
+ret_status gated_ret_chunkwise_state(const void* k, const void* v, const float* g, float* state_out,
+                                     float* log2_decay, int B, int H, int N, int dk, int dv, int chunk, ret_dtype dt,
+                                     void* stream) {
+    return chunkwise_state_entry<true>(k, v, g, state_out, log2_decay, B, H, N, dk, dv, chunk, dt, stream);
+}
+
+ret_status ret_state_prefix(const float* seg_states, const float* seg_log2_decay, const float* state_in,
+                            float* start_states, float* end_state, int R, int B, int H, int dk, int dv, void* stream) {
+    if (R <= 0 || B <= 0 || H <= 0 || dk <= 0 || dv <= 0) return RET_ERR_SHAPE;
+    if (!seg_states || !seg_log2_decay || !start_states) return RET_ERR_NULL;
+    const long long n = (long long)B * H * dk * dv;
+    if ((long long)dk * dv > 0x7fffffffLL) return RET_ERR_UNSUPPORTED;
+    const int blocks = (int)std::min<long long>((n + 255) / 256, 4LL * tc::sm_count());
+    state_prefix_kernel<<<blocks, 256, 0, as_stream(stream)>>>(seg_states, seg_log2_decay, state_in, start_states,
+                                                                end_state, R, B * H, dk * dv);
+    return launch_status();
+}
+
 ret_status ret_selftest_wait_timeout(unsigned int limit_us, void* stream) {
     if (limit_us == 0 || limit_us > 1000000u) return RET_ERR_SHAPE;
     if (!tc::tc_device_ok()) return RET_ERR_UNSUPPORTED;
     tc::selftest_wait_kernel<<<1, 64, 0, as_stream(stream)>>>((unsigned long long)limit_us * 1000ull);
     return cudaGetLastError() == cudaSuccess ? RET_OK : RET_ERR_CUDA;
+}
+
+int ret_chunkwise_state_launches(int B, int H, int N, int dk, int dv, int chunk, ret_dtype dt) {
+    if (check_common(B, H, N, dk, dv, dt) != RET_OK || chunk <= 0 || dk > 256) return -1;
+    if (N == 0) return 0;
+    // the decay kernel, then the state-only pass (+ prefix) or the CUDA-core chunkwise kernel
+    return 1 + (tc_chunk_supported(dk, dv, chunk, dt == RET_BF16) ? tc_state_launches(B, H, N, dv) : 1);
 }
 
 const char* ret_version(void) { return "0.1.0"; }

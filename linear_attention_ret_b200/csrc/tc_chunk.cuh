@@ -1136,7 +1136,77 @@ inline void keep_pool_memory() {
     }
 }
 
+// End state of a whole sequence from a zero start, without outputs: the state-only kernel
+// over `subs` sub-segments of sub_chunks chunks (enough CTAs to fill the SMs), combined by
+// seg_prefix_kernel; with one sub-segment it writes state_out directly. Scratch: the
+// sub-segments' states (only when subs > 1) and their log2 decays.
+inline void state_plan(int B, int H, int N, int dv, int& subs, int& sub_chunks) {
+    const int ctas = B * H * (dv / kDvS);
+    const int nchunks = (N + kC - 1) / kC;
+    subs = std::max(1, std::min(std::min(sm_count() / ctas, kMaxSegments - 1), nchunks));
+    sub_chunks = (nchunks + subs - 1) / subs;
+    subs = (nchunks + sub_chunks - 1) / sub_chunks;
+}
+inline size_t state_scratch_bytes(int subs, int BH, int dk, int dv) {
+    return (subs > 1 ? sizeof(float) * (size_t)subs * BH * dk * dv : 0) +
+           ((sizeof(float) * (size_t)subs * BH + 255) & ~size_t(255));
+}
+
+template <int DK, bool GATED>
+ret_status launch_state_dk(const void* k, const void* v, const float* decay, float* state_out, int B, int H, int N,
+                           int dv, int subs, int sub_chunks, void* scratch, cudaStream_t st) {
+    const int BH = B * H;
+    // the state-only pass reads only K and V: the Q and O maps are placeholders over K and V
+    CUtensorMap mk, mv;
+    if (!make_map(&mk, k, DK, N, BH) || !make_map(&mv, v, dv, N, BH)) return RET_ERR_CUDA;
+    uint8_t* sc = static_cast<uint8_t*>(scratch);
+    float* states = subs > 1 ? reinterpret_cast<float*>(sc) : state_out;
+    float* ldec = reinterpret_cast<float*>(sc + (subs > 1 ? sizeof(float) * (size_t)subs * BH * DK * dv : 0));
+    Params prm{decay, nullptr, nullptr, states, ldec, H, N, dv, sub_chunks, 1};
+    auto k1 = chunk_tc_kernel<DK, GATED, true>;
+    constexpr int smem1 = kernel_smem<DK, GATED, true>();
+    if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1) != cudaSuccess)
+        return RET_ERR_CUDA;
+    k1<<<dim3(dv / kDvS, BH, subs), kThreads, smem1, st>>>(mk, mk, mv, mv, prm);
+    if (cudaGetLastError() != cudaSuccess) return RET_ERR_CUDA;
+    if (subs > 1) {
+        const int n4 = BH * DK * dv / 4;
+        seg_prefix_kernel<<<std::min((n4 + 255) / 256, 4 * sm_count()), 256, 0, st>>>(nullptr, states, ldec, subs + 1,
+                                                                                       BH, DK * dv);
+        if (cudaGetLastError() != cudaSuccess) return RET_ERR_CUDA;
+        if (cudaMemcpyAsync(state_out, states + (size_t)(subs - 1) * BH * DK * dv, sizeof(float) * (size_t)BH * DK * dv,
+                            cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+            return RET_ERR_CUDA;
+    }
+    return RET_OK;
+}
+
 }  // namespace tc
+
+// State-only tensor-core pass over a whole sequence; scratch from the stream-ordered allocator.
+template <bool GATED>
+ret_status tc_state_launch(const void* k, const void* v, const float* decay, float* state_out, int B, int H, int N,
+                           int dk, int dv, cudaStream_t st) {
+    int subs = 1, sub_chunks = 1;
+    tc::state_plan(B, H, N, dv, subs, sub_chunks);
+    void* scratch = nullptr;
+    tc::keep_pool_memory();
+    if (cudaMallocAsync(&scratch, tc::state_scratch_bytes(subs, B * H, dk, dv), st) != cudaSuccess) return RET_ERR_CUDA;
+    ret_status r = RET_ERR_UNSUPPORTED;
+    switch (dk) {
+        case 64: r = tc::launch_state_dk<64, GATED>(k, v, decay, state_out, B, H, N, dv, subs, sub_chunks, scratch, st); break;
+        case 128: r = tc::launch_state_dk<128, GATED>(k, v, decay, state_out, B, H, N, dv, subs, sub_chunks, scratch, st); break;
+        case 256: r = tc::launch_state_dk<256, GATED>(k, v, decay, state_out, B, H, N, dv, subs, sub_chunks, scratch, st); break;
+    }
+    if (cudaFreeAsync(scratch, st) != cudaSuccess) return RET_ERR_CUDA;
+    return r;
+}
+
+inline int tc_state_launches(int B, int H, int N, int dv) {
+    int subs = 1, sub_chunks = 1;
+    tc::state_plan(B, H, N, dv, subs, sub_chunks);
+    return subs > 1 ? 2 : 1;  // state-only pass (+ prefix); the final copy is not a kernel
+}
 
 // Tensor-core path; a split sequence takes its scratch from the stream-ordered
 // allocator and returns it on the same stream after the two launches.

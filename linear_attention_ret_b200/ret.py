@@ -27,7 +27,8 @@ STATUS = {0: "RET_OK", 1: "RET_ERR_NULL", 2: "RET_ERR_SHAPE", 3: "RET_ERR_DTYPE"
 # every symbol include/ret.h declares
 SYMBOLS = ("ret_parallel", "ret_chunkwise", "ret_recurrent_step", "gated_ret_chunkwise", "ret_status_str",
            "ret_last_device_error", "ret_chunkwise_path", "ret_chunkwise_launches", "ret_version",
-           "ret_chunkwise_noalloc", "ret_selftest_wait_timeout", "gated_ret_recurrent_step")
+           "ret_chunkwise_noalloc", "ret_selftest_wait_timeout", "gated_ret_recurrent_step",
+           "ret_chunkwise_state", "gated_ret_chunkwise_state", "ret_state_prefix", "ret_chunkwise_state_launches")
 
 _lock = threading.Lock()
 _lib = None
@@ -59,8 +60,14 @@ def load(path: str | None = None) -> ctypes.CDLL:
         lib.ret_chunkwise_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
         lib.ret_recurrent_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
         lib.gated_ret_recurrent_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
+        lib.ret_chunkwise_state.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
+        lib.gated_ret_chunkwise_state.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
+        lib.ret_state_prefix.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
+        lib.ret_chunkwise_state_launches.argtypes = [_i, _i, _i, _i, _i, _i, _i]
+        lib.ret_chunkwise_state_launches.restype = _i
         for fn in ("ret_parallel", "ret_chunkwise", "gated_ret_chunkwise", "ret_recurrent_step",
-                   "ret_chunkwise_noalloc", "gated_ret_recurrent_step"):
+                   "ret_chunkwise_noalloc", "gated_ret_recurrent_step", "ret_chunkwise_state",
+                   "gated_ret_chunkwise_state", "ret_state_prefix"):
             getattr(lib, fn).restype = _i
         lib.ret_status_str.argtypes = [_i]
         lib.ret_status_str.restype = ctypes.c_char_p
@@ -177,6 +184,32 @@ def gated_ret_recurrent_step(q, k, v, g, state, o=None, stream=None):
     return o
 
 
+def chunkwise_state(k, v, decay, chunk, gated=False, state_out=None, log2_decay=None, stream=None):
+    """End state U [B, H, dk, dv] of a segment from a zero start and log2 of its total decay
+    [B, H] (decay: gamma [H], or g [B, H, N] with gated=True). Returns (U, log2_decay)."""
+    B, H, N, dk = k.shape
+    dv = v.shape[-1]
+    state_out = torch.empty(B, H, dk, dv, dtype=torch.float32, device=k.device) if state_out is None else state_out
+    log2_decay = torch.empty(B, H, dtype=torch.float32, device=k.device) if log2_decay is None else log2_decay
+    _cuda(k, v, decay, state_out, log2_decay)
+    name = "gated_ret_chunkwise_state" if gated else "ret_chunkwise_state"
+    _check(name, getattr(load(), name)(_ptr(k), _ptr(v), _ptr(decay), _ptr(state_out), _ptr(log2_decay),
+                                       B, H, N, dk, dv, int(chunk), _dt(k), _stream(stream)))
+    return state_out, log2_decay
+
+
+def state_prefix(seg_states, seg_log2_decay, state_in=None, stream=None):
+    """Start states [R, B, H, dk, dv] of R consecutive segments and the state after all of
+    them, from their end states U [R, B, H, dk, dv] and log2 decays [R, B, H]."""
+    R, B, H, dk, dv = seg_states.shape
+    starts = torch.empty_like(seg_states)
+    end = torch.empty(B, H, dk, dv, dtype=torch.float32, device=seg_states.device)
+    _cuda(seg_states, seg_log2_decay, state_in, starts, end)
+    _check("ret_state_prefix", load().ret_state_prefix(_ptr(seg_states), _ptr(seg_log2_decay), _ptr(state_in),
+                                                       _ptr(starts), _ptr(end), R, B, H, dk, dv, _stream(stream)))
+    return starts, end
+
+
 def last_device_error(stream=None) -> int:
     return int(load().ret_last_device_error(_stream(stream)))
 
@@ -188,6 +221,11 @@ def selftest_wait_timeout(limit_us: int, stream=None) -> int:
 
 def chunkwise_launches(B: int, H: int, N: int, dk: int, dv: int, chunk: int, dtype: torch.dtype) -> int:
     return int(load().ret_chunkwise_launches(B, H, N, dk, dv, chunk, RET_BF16 if dtype == torch.bfloat16 else RET_F32))
+
+
+def chunkwise_state_launches(B: int, H: int, N: int, dk: int, dv: int, chunk: int, dtype: torch.dtype) -> int:
+    return int(load().ret_chunkwise_state_launches(B, H, N, dk, dv, chunk,
+                                                   RET_BF16 if dtype == torch.bfloat16 else RET_F32))
 
 
 def chunkwise_path(dk: int, dv: int, chunk: int, dtype: torch.dtype) -> int:
