@@ -517,3 +517,106 @@ int oracle_gated_chunkwise(const double* q, const double* k, const double* v,
     }
     return err;
 }
+
+/*
+ * Backward pass by definition (gradients of L = sum_n dO_n . O_n from a zero
+ * initial state), differentiating the first-look sum of [RM] 保留机制初识,
+ * O_n = sum_{m<=n} w_nm (q_n . k_m) v_m with w_nm = gamma^(n-m):
+ *   dq_n = sum_{m<=n} w_nm (dO_n . v_m) k_m
+ *   dk_m = sum_{n>=m} w_nm (dO_n . v_m) q_n
+ *   dv_m = sum_{n>=m} w_nm (q_n . k_m) dO_n
+ *   dgamma_h = sum_{n>m} (n-m) gamma^(n-m-1) (q_n . k_m)(dO_n . v_m)
+ * dgamma may be NULL.
+ */
+int oracle_ret_backward(const double* q, const double* k, const double* v, const double* gamma,
+                        const double* dout, double* dq, double* dk_out, double* dv_out, double* dgamma,
+                        int B, int H, int N, int dk, int dv) {
+    if (bad_dims(B, H, N, dk, dv) || !q || !k || !v || !gamma || !dout || !dq || !dk_out || !dv_out)
+        return ORACLE_EBADARG;
+    if (dgamma) memset(dgamma, 0, sizeof(double) * (size_t)H);
+    double* dgam_bh = (double*)calloc((size_t)B * H, sizeof(double));
+    if (!dgam_bh) return ORACLE_ENOMEM;
+    #pragma omp parallel for schedule(static)
+    for (int bh = 0; bh < B * H; ++bh) {
+        const double gm = gamma[bh % H];
+        const double* Q = q + (size_t)bh * N * dk;
+        const double* K = k + (size_t)bh * N * dk;
+        const double* V = v + (size_t)bh * N * dv;
+        const double* DO = dout + (size_t)bh * N * dv;
+        double* DQ = dq + (size_t)bh * N * dk;
+        double* DK = dk_out + (size_t)bh * N * dk;
+        double* DV = dv_out + (size_t)bh * N * dv;
+        memset(DQ, 0, sizeof(double) * (size_t)N * dk);
+        memset(DK, 0, sizeof(double) * (size_t)N * dk);
+        memset(DV, 0, sizeof(double) * (size_t)N * dv);
+        double dg = 0.0;
+        for (int n = 0; n < N; ++n) {
+            for (int m = 0; m <= n; ++m) {
+                const double w = gpow(gm, n - m);
+                double s = 0.0, a = 0.0;
+                for (int d = 0; d < dk; ++d) s += Q[(size_t)n * dk + d] * K[(size_t)m * dk + d];
+                for (int c = 0; c < dv; ++c) a += DO[(size_t)n * dv + c] * V[(size_t)m * dv + c];
+                for (int d = 0; d < dk; ++d) {
+                    DQ[(size_t)n * dk + d] += w * a * K[(size_t)m * dk + d];
+                    DK[(size_t)m * dk + d] += w * a * Q[(size_t)n * dk + d];
+                }
+                for (int c = 0; c < dv; ++c) DV[(size_t)m * dv + c] += w * s * DO[(size_t)n * dv + c];
+                if (n > m) dg += (double)(n - m) * gpow(gm, n - m - 1) * s * a;
+            }
+        }
+        dgam_bh[bh] = dg;
+    }
+    if (dgamma)
+        for (int bh = 0; bh < B * H; ++bh) dgamma[bh % H] += dgam_bh[bh];
+    free(dgam_bh);
+    return ORACLE_OK;
+}
+
+/*
+ * Gated backward by definition ([GR] parallel_gate_retention: weights
+ * w_nm = exp(sum_{t=m+1..n} g_t)), from a zero initial state. dq, dk, dv as in
+ * oracle_ret_backward with these weights, and, since d w_nm / d g_t = w_nm for
+ * m < t <= n,
+ *   dg_t = sum over pairs n >= t > m of w_nm (q_n . k_m)(dO_n . v_m).
+ * dg may be NULL.
+ */
+int oracle_gated_backward(const double* q, const double* k, const double* v, const double* g,
+                          const double* dout, double* dq, double* dk_out, double* dv_out, double* dg,
+                          int B, int H, int N, int dk, int dv) {
+    if (bad_dims(B, H, N, dk, dv) || !q || !k || !v || !g || !dout || !dq || !dk_out || !dv_out)
+        return ORACLE_EBADARG;
+    #pragma omp parallel for schedule(static)
+    for (int bh = 0; bh < B * H; ++bh) {
+        const double* Q = q + (size_t)bh * N * dk;
+        const double* K = k + (size_t)bh * N * dk;
+        const double* V = v + (size_t)bh * N * dv;
+        const double* Gt = g + (size_t)bh * N;
+        const double* DO = dout + (size_t)bh * N * dv;
+        double* DQ = dq + (size_t)bh * N * dk;
+        double* DK = dk_out + (size_t)bh * N * dk;
+        double* DV = dv_out + (size_t)bh * N * dv;
+        double* DG = dg ? dg + (size_t)bh * N : NULL;
+        memset(DQ, 0, sizeof(double) * (size_t)N * dk);
+        memset(DK, 0, sizeof(double) * (size_t)N * dk);
+        memset(DV, 0, sizeof(double) * (size_t)N * dv);
+        if (DG) memset(DG, 0, sizeof(double) * (size_t)N);
+        for (int n = 0; n < N; ++n) {
+            for (int m = 0; m <= n; ++m) {
+                double run = 0.0;
+                for (int t = m + 1; t <= n; ++t) run += Gt[t];
+                const double w = exp(run);
+                double s = 0.0, a = 0.0;
+                for (int d = 0; d < dk; ++d) s += Q[(size_t)n * dk + d] * K[(size_t)m * dk + d];
+                for (int c = 0; c < dv; ++c) a += DO[(size_t)n * dv + c] * V[(size_t)m * dv + c];
+                for (int d = 0; d < dk; ++d) {
+                    DQ[(size_t)n * dk + d] += w * a * K[(size_t)m * dk + d];
+                    DK[(size_t)m * dk + d] += w * a * Q[(size_t)n * dk + d];
+                }
+                for (int c = 0; c < dv; ++c) DV[(size_t)m * dv + c] += w * s * DO[(size_t)n * dv + c];
+                if (DG)
+                    for (int t = m + 1; t <= n; ++t) DG[t] += w * s * a;
+            }
+        }
+    }
+    return ORACLE_OK;
+}

@@ -61,6 +61,8 @@ def _load():
                 "oracle_gated_parallel": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I],
                 "oracle_gated_recurrent": [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I],
                 "oracle_gated_chunkwise": [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I],
+                "oracle_ret_backward": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I],
+                "oracle_gated_backward": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I],
             }
             for name, argtypes in sig.items():
                 fn = getattr(lib, name)
@@ -210,3 +212,24 @@ def gated_chunkwise(q, k, v, g, chunk, state_in=None):
     _check(_load().oracle_gated_chunkwise(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(s_in), _ptr(s_out),
                                           _ptr(o), B, H, N, dk, dv, int(chunk)), "gated_chunkwise")
     return o, s_out
+
+
+def ret_backward(q, k, v, gamma, do):
+    """Gradients of L = sum dO . O (zero initial state) by definition: (dq, dk, dv, dgamma)."""
+    q, k, v, gamma, do = map(_f64, (q, k, v, gamma, do))
+    B, H, N, dk, dv = _dims(q, v)
+    dq, dkk, dvv = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+    dgam = np.empty(H)
+    _check(_load().oracle_ret_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(do), _ptr(dq), _ptr(dkk),
+                                       _ptr(dvv), _ptr(dgam), B, H, N, dk, dv), "ret_backward")
+    return dq, dkk, dvv, dgam
+
+
+def gated_backward(q, k, v, g, do):
+    """Gated gradients of L = sum dO . O (zero initial state) by definition: (dq, dk, dv, dg)."""
+    q, k, v, g, do = map(_f64, (q, k, v, g, do))
+    B, H, N, dk, dv = _dims(q, v)
+    dq, dkk, dvv, dg = np.empty_like(q), np.empty_like(k), np.empty_like(v), np.empty_like(g)
+    _check(_load().oracle_gated_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(do), _ptr(dq), _ptr(dkk),
+                                         _ptr(dvv), _ptr(dg), B, H, N, dk, dv), "gated_backward")
+    return dq, dkk, dvv, dg

@@ -308,6 +308,65 @@ def test_bad_arguments_rejected():
 
 # ---------------------------------------------------------------- planted mistakes
 
+# ---------------------------------------------------------------- backward pass
+
+def _fd(f, x, eps=1e-6):
+    """Central finite differences of the scalar function f at x (fp64)."""
+    g = np.zeros_like(x)
+    for idx in np.ndindex(x.shape):
+        xp, xm = x.copy(), x.copy()
+        xp[idx] += eps
+        xm[idx] -= eps
+        g[idx] = (f(xp) - f(xm)) / (2 * eps)
+    return g
+
+
+def test_backward_matches_finite_differences():
+    """Gradients of L = sum dO . O against central differences of the brute-force forward."""
+    q, k, v = _inputs(B=1, H=2, N=7, dk=3, dv=4, seed=30)
+    do = np.random.default_rng(31).standard_normal((1, 2, 7, 4))
+    gam = np.array([0.9, 0.6])
+    loss = lambda q_, k_, v_, g_: float(np.sum(do * O.ret_brute(q_, k_, v_, g_)))
+    dq, dk, dv, dgam = O.ret_backward(q, k, v, gam, do)
+    np.testing.assert_allclose(dq, _fd(lambda x: loss(x, k, v, gam), q), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dk, _fd(lambda x: loss(q, x, v, gam), k), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dv, _fd(lambda x: loss(q, k, x, gam), v), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dgam, _fd(lambda x: loss(q, k, v, x), gam), rtol=1e-6, atol=1e-8)
+
+
+def test_gated_backward_matches_finite_differences():
+    q, k, v = _inputs(B=1, H=2, N=7, dk=3, dv=4, seed=32)
+    do = np.random.default_rng(33).standard_normal((1, 2, 7, 4))
+    g = _gate(1, 2, 7, seed=34, scale=8.0)
+    loss = lambda q_, k_, v_, g_: float(np.sum(do * O.gated_brute(q_, k_, v_, g_)))
+    dq, dk, dv, dg = O.gated_backward(q, k, v, g, do)
+    np.testing.assert_allclose(dq, _fd(lambda x: loss(x, k, v, g), q), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dk, _fd(lambda x: loss(q, x, v, g), k), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dv, _fd(lambda x: loss(q, k, x, g), v), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dg, _fd(lambda x: loss(q, k, v, x), g), rtol=1e-6, atol=1e-8)
+
+
+def test_backward_gamma_zero_and_constant_gate():
+    """gamma = 0 leaves only the diagonal: dq_n = (dO_n . v_n) k_n, dv_n = (q_n . k_n) dO_n;
+    a constant gate g = ln gamma gives the fixed-gamma gradients."""
+    q, k, v = _inputs(B=1, H=2, N=9, dk=3, dv=4, seed=35)
+    do = np.random.default_rng(36).standard_normal((1, 2, 9, 4))
+    dq, dk, dv, _ = O.ret_backward(q, k, v, np.array([0.0, 0.0]), do)
+    a = np.einsum("bhnc,bhnc->bhn", do, v)
+    s = np.einsum("bhnd,bhnd->bhn", q, k)
+    np.testing.assert_allclose(dq, a[..., None] * k, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dk, a[..., None] * q, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dv, s[..., None] * do, rtol=1e-12, atol=1e-12)
+    gam = np.array([0.9, 0.75])
+    g = np.broadcast_to(np.log(gam)[None, :, None], (1, 2, 9)).copy()
+    ref = O.ret_backward(q, k, v, gam, do)
+    got = O.gated_backward(q, k, v, g, do)
+    for a_, b_ in zip(ref[:3], got[:3]):
+        np.testing.assert_allclose(b_, a_, rtol=1e-11, atol=1e-12)
+    # dL/dlog(gamma) = gamma dL/dgamma = sum over the sequence of dL/dg_t
+    np.testing.assert_allclose(got[3].sum(axis=2)[0], gam * ref[3], rtol=1e-10, atol=1e-12)
+
+
 _MUTANTS = {
     # the printed single gamma^c cross factor instead of the per-row gamma^(j+1)
     "uniform_cross_factor": ("const double r = gpow(gm, j + 1);", "const double r = gpow(gm, L);"),
@@ -324,6 +383,12 @@ _MUTANTS = {
     # gated parallel form with an exclusive instead of inclusive cumulative sum
     "gated_exclusive_cumsum": ("for (int n = 0; n < N; ++n) { acc += Gt[n]; G[n] = acc; }",
                                "for (int n = 0; n < N; ++n) { G[n] = acc; acc += Gt[n]; }"),
+    # backward: decay gradient exponent off by one
+    "backward_dgamma_power": ("if (n > m) dg += (double)(n - m) * gpow(gm, n - m - 1) * s * a;",
+                              "if (n > m) dg += (double)(n - m) * gpow(gm, n - m) * s * a;"),
+    # gated backward: gate gradient over the wrong range of t (includes t = m)
+    "backward_gate_range": ("for (int t = m + 1; t <= n; ++t) DG[t] += w * s * a;",
+                            "for (int t = m; t <= n; ++t) DG[t] += w * s * a;"),
 }
 
 
@@ -347,7 +412,8 @@ def _pins_pass_with(lib_path):
         sig_src = O._load()  # the real library carries the argtypes to copy
         for name in ("oracle_decay_matrix", "oracle_ret_brute", "oracle_ret_parallel", "oracle_ret_recurrent",
                      "oracle_ret_recurrent_step", "oracle_ret_chunkwise", "oracle_gated_brute",
-                     "oracle_gated_parallel", "oracle_gated_recurrent", "oracle_gated_chunkwise"):
+                     "oracle_gated_parallel", "oracle_gated_recurrent", "oracle_gated_chunkwise",
+                     "oracle_ret_backward", "oracle_gated_backward"):
             fn = getattr(lib, name)
             fn.argtypes = getattr(sig_src, name).argtypes
             fn.restype = ctypes.c_int
@@ -361,6 +427,8 @@ def _pins_pass_with(lib_path):
             lambda: test_chunkwise_matches_parallel_and_recurrent(7),
             lambda: test_gated_forms_agree(8),
             test_parallel_matches_brute_force,
+            test_backward_matches_finite_differences,
+            test_gated_backward_matches_finite_differences,
         ]
         for check in checks:
             try:
