@@ -142,6 +142,30 @@ RET_API const char* ret_status_str(ret_status s);
 RET_API ret_status ret_last_device_error(void* stream);
 
 /*
+ * Backward pass of ret_chunkwise / gated_ret_chunkwise from a zero initial
+ * state: gradients of L = sum_n dout_n . o_n, differentiating [RM] 保留机制初识's
+ * sum (o_n = sum_{m<=n} w_nm (q_n . k_m) v_m, w_nm = gamma^(n-m), or
+ * exp(G_n - G_m) with G the cumulative sum of g, [GR] parallel_gate_retention):
+ *   dq_n = sum_{m<=n} w_nm (dout_n . v_m) k_m,  dk_m = sum_{n>=m} w_nm (dout_n . v_m) q_n,
+ *   dv_m = sum_{n>=m} w_nm (q_n . k_m) dout_n,
+ *   dgamma_h (optional, [H] fp32) = d L / d gamma_h  (not defined for gamma_h = 0),
+ *   dg (optional, [B, H, N] fp32) = d L / d g.
+ * dout has v's layout; dq, dk, dv have q's, k's, v's (dtype dt). Computed with the
+ * forward kernels (dq directly, dk and dv on the time-reversed sequence, a dv wider
+ * than 256 contracted in pieces) and small kernels of this library; takes
+ * stream-ordered scratch (freed on the same stream). bf16 needs 16-byte aligned
+ * tensors. Requires dk <= 256.
+ */
+RET_API ret_status ret_chunkwise_backward(const void* q, const void* k, const void* v, const float* gamma,
+                                  const void* dout, void* dq, void* dk, void* dv, float* dgamma,
+                                  int B, int H, int N, int dk_dim, int dv_dim, int chunk,
+                                  ret_dtype dt, void* stream);
+RET_API ret_status gated_ret_chunkwise_backward(const void* q, const void* k, const void* v, const float* g,
+                                        const void* dout, void* dq, void* dk, void* dv, float* dg,
+                                        int B, int H, int N, int dk_dim, int dv_dim, int chunk,
+                                        ret_dtype dt, void* stream);
+
+/*
  * Sequence split into consecutive segments computed separately (for example
  * one per GPU, then one exchange of states), [RM] 块级循环 / [GR] cross_chunk:
  * the chunkwise recurrence composes over segments as

@@ -10,6 +10,7 @@
 #include "decode.cuh"
 #include "tc_chunk.cuh"
 #include "seqpar.cuh"
+#include "backward.cuh"
 
 using namespace ret;
 
@@ -111,6 +112,135 @@ ret_status chunkwise_state_entry(const void* k, const void* v, const float* deca
                                                           chunk, st);
     if (cudaFreeAsync(o, st) != cudaSuccess) return RET_ERR_CUDA;
     return r;
+}
+
+// ------------------------------------------------------------------ backward (see backward.cuh)
+
+inline int grid_for(size_t n) { return (int)std::min<size_t>((n + kBwdThreads - 1) / kBwdThreads, 8 * tc::sm_count()); }
+
+template <typename T>
+ret_status slice_flip(const void* src, void* dst, int BH, int N, int d_src, int c0, int w, bool flip, cudaStream_t st) {
+    const size_t total = (size_t)BH * N * w;
+    slice_flip_kernel<T><<<grid_for(total), kBwdThreads, 0, st>>>(static_cast<const T*>(src), static_cast<T*>(dst), N,
+                                                                  d_src, c0, w, flip, total);
+    return launch_status();
+}
+
+inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
+
+template <typename T, bool GATED>
+ret_status backward_impl(const void* q, const void* k, const void* v, const float* decay, const void* dout, void* dq,
+                         void* dk_out, void* dv_out, float* ddecay, int B, int H, int N, int dk, int dv, int chunk,
+                         ret_dtype dt, cudaStream_t st) {
+    const int BH = B * H;
+    const size_t nQ = (size_t)BH * N * dk, nV = (size_t)BH * N * dv;
+    const int pw = dv <= 256 ? dv : 256;  // width of one piece of the dv contraction
+    const int P = (dv + pw - 1) / pw;
+    // scratch: reversed Q, K, V, dO; two piece buffers; per-piece outputs; reversed dV; reversed gates
+    size_t off[9], bytes = 0;
+    const size_t sz[9] = {nQ * sizeof(T), nQ * sizeof(T), nV * sizeof(T), nV * sizeof(T),
+                          (size_t)BH * N * pw * sizeof(T), (size_t)BH * N * pw * sizeof(T), (size_t)P * nQ * sizeof(T),
+                          nV * sizeof(T), GATED ? (size_t)BH * N * sizeof(float) : 0};
+    for (int i = 0; i < 9; ++i) {
+        off[i] = bytes;
+        bytes += align256(sz[i]);
+    }
+    tc::keep_pool_memory();
+    uint8_t* sc = nullptr;
+    if (cudaMallocAsync(reinterpret_cast<void**>(&sc), bytes, st) != cudaSuccess) return RET_ERR_CUDA;
+    T* Qf = reinterpret_cast<T*>(sc + off[0]);
+    T* Kf = reinterpret_cast<T*>(sc + off[1]);
+    T* Vf = reinterpret_cast<T*>(sc + off[2]);
+    T* dOf = reinterpret_cast<T*>(sc + off[3]);
+    T* pa = reinterpret_cast<T*>(sc + off[4]);
+    T* pb = reinterpret_cast<T*>(sc + off[5]);
+    T* parts = reinterpret_cast<T*>(sc + off[6]);
+    T* Rf = reinterpret_cast<T*>(sc + off[7]);
+    float* gf = reinterpret_cast<float*>(sc + off[8]);
+    ret_status r = RET_OK;
+    auto ok = [&](ret_status x) { if (r == RET_OK) r = x; return r == RET_OK; };
+    auto fwd = [&](const void* fq, const void* fk, const void* fv, const float* dec, void* fo, int wq, int wv) {
+        return ok(chunkwise_entry<GATED>(fq, fk, fv, dec, fo, nullptr, nullptr, B, H, N, wq, wv, chunk, dt, st));
+    };
+    // dQ = forward(dO, V, K), the dv contraction in pieces
+    if (P == 1) {
+        fwd(dout, v, k, decay, dq, dv, dk);
+    } else {
+        for (int p = 0; p < P && r == RET_OK; ++p) {
+            const int c0 = p * pw, w = std::min(pw, dv - c0);
+            ok(slice_flip<T>(dout, pa, BH, N, dv, c0, w, false, st)) && ok(slice_flip<T>(v, pb, BH, N, dv, c0, w, false, st)) &&
+                fwd(pa, pb, k, decay, parts + (size_t)p * nQ, w, dk);
+        }
+        if (r == RET_OK) {
+            sum_flip_kernel<T><<<grid_for(nQ), kBwdThreads, 0, st>>>(parts, P, nQ, static_cast<T*>(dq), N, dk, false);
+            ok(launch_status());
+        }
+    }
+    // time-reversed copies (and gates reversed and shifted by one)
+    if (r == RET_OK) {
+        ok(slice_flip<T>(q, Qf, BH, N, dk, 0, dk, true, st)) && ok(slice_flip<T>(k, Kf, BH, N, dk, 0, dk, true, st)) &&
+            ok(slice_flip<T>(v, Vf, BH, N, dv, 0, dv, true, st)) && ok(slice_flip<T>(dout, dOf, BH, N, dv, 0, dv, true, st));
+        if (GATED && r == RET_OK) {
+            gate_flip_kernel<<<grid_for((size_t)BH * N), kBwdThreads, 0, st>>>(decay, gf, N, (size_t)BH * N);
+            ok(launch_status());
+        }
+    }
+    const float* dec_rev = GATED ? gf : decay;
+    // dK = reverse(forward(rev V, rev dO, rev Q)), in pieces
+    for (int p = 0; p < P && r == RET_OK; ++p) {
+        const int c0 = p * pw, w = std::min(pw, dv - c0);
+        if (P == 1) {
+            fwd(Vf, dOf, Qf, dec_rev, parts, dv, dk);
+        } else {
+            ok(slice_flip<T>(Vf, pa, BH, N, dv, c0, w, false, st)) && ok(slice_flip<T>(dOf, pb, BH, N, dv, c0, w, false, st)) &&
+                fwd(pa, pb, Qf, dec_rev, parts + (size_t)p * nQ, w, dk);
+        }
+    }
+    if (r == RET_OK) {
+        sum_flip_kernel<T><<<grid_for(nQ), kBwdThreads, 0, st>>>(parts, P, nQ, static_cast<T*>(dk_out), N, dk, true);
+        ok(launch_status());
+    }
+    // dV = reverse(forward(rev K, rev Q, rev dO))
+    if (r == RET_OK && fwd(Kf, Qf, dOf, dec_rev, Rf, dk, dv)) ok(slice_flip<T>(Rf, dv_out, BH, N, dv, 0, dv, true, st));
+    // decay gradient
+    if (r == RET_OK && ddecay) {
+        if (!GATED && cudaMemsetAsync(ddecay, 0, sizeof(float) * (size_t)H, st) != cudaSuccess) r = RET_ERR_CUDA;
+        if (r == RET_OK) {
+            decay_grad_kernel<T, GATED><<<BH, kBwdThreads, 0, st>>>(static_cast<const T*>(q), static_cast<const T*>(dq),
+                                                                    static_cast<const T*>(k),
+                                                                    static_cast<const T*>(dk_out), decay, ddecay, H, N,
+                                                                    dk);
+            ok(launch_status());
+        }
+    }
+    if (cudaFreeAsync(sc, st) != cudaSuccess && r == RET_OK) r = RET_ERR_CUDA;
+    return r;
+}
+
+template <bool GATED>
+ret_status backward_entry(const void* q, const void* k, const void* v, const float* decay, const void* dout, void* dq,
+                          void* dk_out, void* dv_out, float* ddecay, int B, int H, int N, int dk, int dv, int chunk,
+                          ret_dtype dt, void* stream) {
+    ret_status s = check_common(B, H, N, dk, dv, dt);
+    if (s != RET_OK) return s;
+    if (chunk <= 0) return RET_ERR_SHAPE;
+    if (dk > 256) return RET_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !decay || !dout || !dq || !dk_out || !dv_out) return RET_ERR_NULL;
+    cudaStream_t st = as_stream(stream);
+    if (N == 0) {
+        if (!GATED && ddecay && cudaMemsetAsync(ddecay, 0, sizeof(float) * (size_t)H, st) != cudaSuccess)
+            return RET_ERR_CUDA;
+        return RET_OK;
+    }
+    if (dt == RET_BF16) {
+        for (const void* p : {q, k, v, dout, static_cast<const void*>(dq), static_cast<const void*>(dk_out),
+                              static_cast<const void*>(dv_out)})
+            if (!aligned16(p)) return RET_ERR_ALIGN;
+        return backward_impl<__nv_bfloat16, GATED>(q, k, v, decay, dout, dq, dk_out, dv_out, ddecay, B, H, N, dk, dv,
+                                                   chunk, dt, st);
+    }
+    return backward_impl<float, GATED>(q, k, v, decay, dout, dq, dk_out, dv_out, ddecay, B, H, N, dk, dv, chunk, dt,
+                                       st);
 }
 
 template <typename T>
@@ -256,6 +386,18 @@ ret_status ret_selftest_wait_timeout(unsigned int limit_us, void* stream) {
     if (!tc::tc_device_ok()) return RET_ERR_UNSUPPORTED;
     tc::selftest_wait_kernel<<<1, 64, 0, as_stream(stream)>>>((unsigned long long)limit_us * 1000ull);
     return cudaGetLastError() == cudaSuccess ? RET_OK : RET_ERR_CUDA;
+}
+
+ret_status ret_chunkwise_backward(const void* q, const void* k, const void* v, const float* gamma, const void* dout,
+                                  void* dq, void* dk, void* dv, float* dgamma, int B, int H, int N, int dk_dim,
+                                  int dv_dim, int chunk, ret_dtype dt, void* stream) {
+    return backward_entry<false>(q, k, v, gamma, dout, dq, dk, dv, dgamma, B, H, N, dk_dim, dv_dim, chunk, dt, stream);
+}
+
+ret_status gated_ret_chunkwise_backward(const void* q, const void* k, const void* v, const float* g, const void* dout,
+                                        void* dq, void* dk, void* dv, float* dg, int B, int H, int N, int dk_dim,
+                                        int dv_dim, int chunk, ret_dtype dt, void* stream) {
+    return backward_entry<true>(q, k, v, g, dout, dq, dk, dv, dg, B, H, N, dk_dim, dv_dim, chunk, dt, stream);
 }
 
 int ret_chunkwise_state_launches(int B, int H, int N, int dk, int dv, int chunk, ret_dtype dt) {

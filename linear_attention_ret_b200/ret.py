@@ -28,7 +28,8 @@ STATUS = {0: "RET_OK", 1: "RET_ERR_NULL", 2: "RET_ERR_SHAPE", 3: "RET_ERR_DTYPE"
 SYMBOLS = ("ret_parallel", "ret_chunkwise", "ret_recurrent_step", "gated_ret_chunkwise", "ret_status_str",
            "ret_last_device_error", "ret_chunkwise_path", "ret_chunkwise_launches", "ret_version",
            "ret_chunkwise_noalloc", "ret_selftest_wait_timeout", "gated_ret_recurrent_step",
-           "ret_chunkwise_state", "gated_ret_chunkwise_state", "ret_state_prefix", "ret_chunkwise_state_launches")
+           "ret_chunkwise_state", "gated_ret_chunkwise_state", "ret_state_prefix", "ret_chunkwise_state_launches",
+           "ret_chunkwise_backward", "gated_ret_chunkwise_backward")
 
 _lock = threading.Lock()
 _lib = None
@@ -64,6 +65,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
         lib.gated_ret_chunkwise_state.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
         lib.ret_state_prefix.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
         lib.ret_chunkwise_state_launches.argtypes = [_i, _i, _i, _i, _i, _i, _i]
+        for fn in ("ret_chunkwise_backward", "gated_ret_chunkwise_backward"):
+            getattr(lib, fn).argtypes = [_vp] * 9 + [_i] * 7 + [_vp]
+            getattr(lib, fn).restype = _i
         lib.ret_chunkwise_state_launches.restype = _i
         for fn in ("ret_parallel", "ret_chunkwise", "gated_ret_chunkwise", "ret_recurrent_step",
                    "ret_chunkwise_noalloc", "gated_ret_recurrent_step", "ret_chunkwise_state",
@@ -208,6 +212,24 @@ def state_prefix(seg_states, seg_log2_decay, state_in=None, stream=None):
     _check("ret_state_prefix", load().ret_state_prefix(_ptr(seg_states), _ptr(seg_log2_decay), _ptr(state_in),
                                                        _ptr(starts), _ptr(end), R, B, H, dk, dv, _stream(stream)))
     return starts, end
+
+
+def chunkwise_backward(q, k, v, decay, dout, chunk, gated=False, ddecay=True, stream=None):
+    """Gradients of sum(dout * o) for o = ret_chunkwise(q, k, v, decay) (gated=True:
+    gated_ret_chunkwise with g = decay) from a zero initial state. Returns
+    (dq, dk, dv, ddecay) with ddecay = dgamma [H] or dg [B, H, N] (fp32), or None."""
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    dq, dkk, dvv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dd = None
+    if ddecay:
+        dd = torch.empty(B, H, N, dtype=torch.float32, device=q.device) if gated else \
+            torch.empty(H, dtype=torch.float32, device=q.device)
+    _cuda(q, k, v, decay, dout, dq, dkk, dvv, dd)
+    name = "gated_ret_chunkwise_backward" if gated else "ret_chunkwise_backward"
+    _check(name, getattr(load(), name)(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(dout), _ptr(dq), _ptr(dkk),
+                                       _ptr(dvv), _ptr(dd), B, H, N, dk, dv, int(chunk), _dt(q), _stream(stream)))
+    return dq, dkk, dvv, dd
 
 
 def last_device_error(stream=None) -> int:
