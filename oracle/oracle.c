@@ -620,3 +620,35 @@ int oracle_gated_backward(const double* q, const double* k, const double* v, con
     }
     return ORACLE_OK;
 }
+
+/*
+ * Multi-scale retention output epilogue. [RN] 3.2 adds a gate and a normalisation
+ * to retention; [GR]'s GateRetention module normalises each head with subln, an
+ * RMSNorm over the head dimension without affine weights, and gates with the
+ * swish of the g_proj projection:
+ *   y[b, n, h, :] = swish(gate[b, n, h, :]) * o[b, h, n, :] / sqrt(mean_c o[b, h, n, c]^2 + eps),
+ *   swish(x) = x / (1 + exp(-x)).
+ * o [B, H, N, dv] is the retention output; gate and y are token-major
+ * [B, N, H, dv], the layout of the module's projections.
+ */
+int oracle_msr_norm_gate(const double* o, const double* gate, double* y, int B, int H, int N, int dv, double eps) {
+    if (bad_dims(B, H, N, 1, dv) || !o || !gate || !y || eps < 0.0) return ORACLE_EBADARG;
+    #pragma omp parallel for schedule(static)
+    for (int bh = 0; bh < B * H; ++bh) {
+        const int b = bh / H, h = bh % H;
+        for (int n = 0; n < N; ++n) {
+            const double* orow = o + ((size_t)bh * N + n) * dv;
+            const size_t yoff = (((size_t)b * N + n) * H + h) * dv;
+            double ms = 0.0;
+            for (int c = 0; c < dv; ++c) ms += orow[c] * orow[c];
+            ms /= dv;
+            const double inv_rms = 1.0 / sqrt(ms + eps);
+            for (int c = 0; c < dv; ++c) {
+                const double x = gate[yoff + c];
+                const double swish = x / (1.0 + exp(-x));
+                y[yoff + c] = swish * orow[c] * inv_rms;
+            }
+        }
+    }
+    return ORACLE_OK;
+}

@@ -63,6 +63,7 @@ def _load():
                 "oracle_gated_chunkwise": [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I],
                 "oracle_ret_backward": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I],
                 "oracle_gated_backward": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I],
+                "oracle_msr_norm_gate": [_P, _P, _P, _I, _I, _I, _I, ctypes.c_double],
             }
             for name, argtypes in sig.items():
                 fn = getattr(lib, name)
@@ -233,3 +234,17 @@ def gated_backward(q, k, v, g, do):
     _check(_load().oracle_gated_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(do), _ptr(dq), _ptr(dkk),
                                          _ptr(dvv), _ptr(dg), B, H, N, dk, dv), "gated_backward")
     return dq, dkk, dvv, dg
+
+
+def msr_norm_gate(o, gate, eps=1e-5):
+    """Multi-scale retention output epilogue (explainer page 3.2; Gated RetNet page,
+    GateRetention's subln and swish gate): y[b, n, h] = swish(gate[b, n, h]) *
+    RMSNorm(o[b, h, n]) over dv, no affine weights. o [B, H, N, dv]; gate [B, N, H, dv];
+    returns y [B, N, H, dv]."""
+    o, gate = _f64(o), _f64(gate)
+    B, H, N, dv = o.shape
+    if gate.shape != (B, N, H, dv):
+        raise ValueError(f"gate shape {gate.shape} != {(B, N, H, dv)}")
+    y = np.empty_like(gate)
+    _check(_load().oracle_msr_norm_gate(_ptr(o), _ptr(gate), _ptr(y), B, H, N, dv, float(eps)), "msr_norm_gate")
+    return y

@@ -13,6 +13,7 @@ import tempfile
 import ctypes
 
 import numpy as np
+import torch
 import pytest
 
 from oracle import oracle as O
@@ -389,6 +390,15 @@ _MUTANTS = {
     # gated backward: gate gradient over the wrong range of t (includes t = m)
     "backward_gate_range": ("for (int t = m + 1; t <= n; ++t) DG[t] += w * s * a;",
                             "for (int t = m; t <= n; ++t) DG[t] += w * s * a;"),
+    # epilogue: eps added outside the square root
+    "norm_eps_outside": ("const double inv_rms = 1.0 / sqrt(ms + eps);", "const double inv_rms = 1.0 / (sqrt(ms) + eps);"),
+    # epilogue: sum of squares instead of the mean
+    "norm_sum_not_mean": ("    ms /= dv;\n", "\n"),
+    # epilogue: the gate's sigmoid instead of its swish
+    "gate_sigmoid": ("const double swish = x / (1.0 + exp(-x));", "const double swish = 1.0 / (1.0 + exp(-x));"),
+    # epilogue: y written head-major like o instead of token-major
+    "norm_layout": ("const size_t yoff = (((size_t)b * N + n) * H + h) * dv;",
+                    "const size_t yoff = ((size_t)bh * N + n) * dv;"),
 }
 
 
@@ -413,7 +423,7 @@ def _pins_pass_with(lib_path):
         for name in ("oracle_decay_matrix", "oracle_ret_brute", "oracle_ret_parallel", "oracle_ret_recurrent",
                      "oracle_ret_recurrent_step", "oracle_ret_chunkwise", "oracle_gated_brute",
                      "oracle_gated_parallel", "oracle_gated_recurrent", "oracle_gated_chunkwise",
-                     "oracle_ret_backward", "oracle_gated_backward"):
+                     "oracle_ret_backward", "oracle_gated_backward", "oracle_msr_norm_gate"):
             fn = getattr(lib, name)
             fn.argtypes = getattr(sig_src, name).argtypes
             fn.restype = ctypes.c_int
@@ -429,6 +439,8 @@ def _pins_pass_with(lib_path):
             test_parallel_matches_brute_force,
             test_backward_matches_finite_differences,
             test_gated_backward_matches_finite_differences,
+            lambda: test_golden_msr_norm_gate("two_heads_two_tokens_eps"),
+            lambda: test_golden_msr_norm_gate("one_row_eps0"),
         ]
         for check in checks:
             try:
@@ -450,3 +462,46 @@ def test_planted_mistake_is_caught(mutant):
 def test_unmutated_copy_passes_pins():
     with tempfile.TemporaryDirectory() as d:
         assert _pins_pass_with(_build_mutant(d, "#define ORACLE_OK 0", "#define ORACLE_OK 0"))
+
+
+# ---------------------------------------------------------------- multi-scale retention output epilogue
+
+NORM_GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "msr_norm_gate_hand_examples.json")
+
+
+@pytest.mark.parametrize("name", ["one_row_eps0", "two_heads_two_tokens_eps"])
+def test_golden_msr_norm_gate(name):
+    with open(NORM_GOLDEN, encoding="utf-8") as f:
+        ex = {e["name"]: e for e in json.load(f)["examples"]}[name]
+    ln3 = np.log(3.0)
+    y = O.msr_norm_gate(np.array(ex["o"], dtype=float), np.array(ex["gate_ln3"], dtype=float) * ln3, ex["eps"])
+    np.testing.assert_allclose(y, np.array(ex["y_ln3"]) * ln3, rtol=1e-14, atol=1e-15)
+
+
+def test_msr_norm_gate_matches_library_routines():
+    """Special case that reduces to library routines: torch's rms_norm (no weight) and silu, fp64."""
+    rng = np.random.default_rng(40)
+    o = rng.standard_normal((2, 3, 17, 24)) * 3.0
+    gate = rng.standard_normal((2, 17, 3, 24)) * 2.0
+    for eps in (0.0, 1e-5, 0.5):
+        y = O.msr_norm_gate(o, gate, eps)
+        ref = (torch.nn.functional.rms_norm(torch.from_numpy(o), (24,), eps=eps).permute(0, 2, 1, 3)
+               * torch.nn.functional.silu(torch.from_numpy(gate)))
+        np.testing.assert_allclose(y, ref.numpy(), rtol=1e-12, atol=1e-14)
+
+
+def test_msr_norm_gate_invariants():
+    """With eps = 0 the output is invariant to positive scaling of a head's row and odd in o;
+    with a large gate (swish(x) -> x) each row of y / gate has unit root mean square."""
+    rng = np.random.default_rng(41)
+    o = rng.standard_normal((1, 2, 5, 8))
+    gate = rng.standard_normal((1, 5, 2, 8))
+    y = O.msr_norm_gate(o, gate, 0.0)
+    np.testing.assert_allclose(O.msr_norm_gate(o * 7.5, gate, 0.0), y, rtol=1e-13)
+    np.testing.assert_allclose(O.msr_norm_gate(-o, gate, 0.0), -y, rtol=1e-13)
+    big = np.full((1, 5, 2, 8), 60.0)
+    r = O.msr_norm_gate(o, big, 0.0) / 60.0
+    np.testing.assert_allclose(np.sqrt((r ** 2).mean(axis=-1)), 1.0, rtol=1e-12)
+    # eps damps small rows: a row of zeros stays zero for any eps > 0
+    z = O.msr_norm_gate(np.zeros((1, 1, 2, 4)), np.ones((1, 2, 1, 4)), 1e-5)
+    assert np.all(z == 0.0)
