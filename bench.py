@@ -12,6 +12,10 @@ already resident in HBM:
   gated_decode      gated_ret_recurrent_step, same shapes, a fresh log-decay g [B, H] per step
   seqpar_6p7b       the retnet_6p7b_long sequence split across the ranks (strong scaling):
                     segment end states, one all-gather, start states, ret_chunkwise per segment
+  backward_1p3b     ret_chunkwise_backward on the retnet_1p3b shapes: dq, dk, dv and dgamma
+                    from q, k, v, gamma and an output gradient dO
+  msr_norm_1p3b     ret_msr_norm_gate on the retnet_1p3b output: per-head RMSNorm and swish gate
+  retention_msr_1p3b  ret_chunkwise then ret_msr_norm_gate on its output (retnet_1p3b shapes)
 For N > 1 (torchrun, one rank per GPU) every rank runs its own batch of the
 same shape (batch sharding, no collective on the data path): weak scaling.
 Rank 0 prints one JSON line. `--impl reference` times the fp64 CPU oracle on a
@@ -36,6 +40,7 @@ if ROOT not in sys.path:
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 L2_BYTES = 126 * 1024 * 1024
+NORM_EPS = 1e-5  # the norm epsilon the pages give as the module default
 
 
 # ----------------------------------------------------------------------------- workload arithmetic
@@ -49,6 +54,33 @@ def workload(name: str):
         spec = workload("retnet_6p7b_long")
         spec.update(kind="seqpar", metric="retention tokens/s (sequence-parallel chunkwise fwd)")
         return spec
+    if name == "backward_1p3b":
+        cfg = I.CONFIGS["retnet_1p3b"]
+        B, H, N, dk, dv, C = cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk
+        elt = 2
+        # reads q, k, v, dO; writes dq, dk, dv (dgamma is H floats)
+        io = B * H * N * (4 * dk + 3 * dv) * elt
+        # three contractions of the forward's shape: dQ (scores dO.v), dK (dO.v), dV (q.k)
+        flops = 3 * B * H * N * (2 * C * (dk + dv) + 4 * dk * dv)
+        return dict(cfg=cfg, kind="backward", units=B * N, unit="tokens/s",
+                    metric="retention tokens/s (chunkwise backward)", tokens=B * N, bytes=io, flops=flops,
+                    h2d=B * H * N * (2 * dk + 2 * dv) * elt, d2h=B * H * N * (2 * dk + dv) * elt + H * 4)
+    if name in ("msr_norm_1p3b", "retention_msr_1p3b"):
+        cfg = I.CONFIGS["retnet_1p3b"]
+        B, H, N, dk, dv, C = cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk
+        elt = 2
+        gy = 2 * B * H * N * dv * elt  # gate read, y written
+        if name == "msr_norm_1p3b":
+            return dict(cfg=cfg, kind="norm", units=B * N, unit="tokens/s",
+                        metric="tokens/s (multi-scale retention output epilogue)", tokens=B * N,
+                        bytes=B * H * N * dv * elt + gy, flops=0,
+                        h2d=2 * B * H * N * dv * elt, d2h=B * H * N * dv * elt)
+        # o stays an intermediate: the algorithmic bytes are q, k, v and the gate in, y out
+        return dict(cfg=cfg, kind="ret_norm", units=B * N, unit="tokens/s",
+                    metric="retention tokens/s (chunkwise fwd + output epilogue)", tokens=B * N,
+                    bytes=B * H * N * 2 * dk * elt + B * H * N * dv * elt + gy,
+                    flops=B * H * N * (2 * C * (dk + dv) + 4 * dk * dv),
+                    h2d=B * H * N * (2 * dk + 2 * dv) * elt, d2h=B * H * N * dv * elt)
     cfg = I.CONFIGS[name]
     B, H, N, dk, dv, C = cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk
     if name in ("decode", "gated_decode"):
@@ -78,10 +110,23 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
-def kernel_source_sha() -> str:
+# The sources each workload's measured kernels are compiled and launched from; a
+# traffic figure counts only while these files still hash to the value it was taken at.
+KERNEL_SOURCES = {
+    "chunk": ("common.cuh", "tc_chunk.cuh", "tc_wide.cuh"),
+    "decode": ("common.cuh", "decode.cuh"),
+    "norm": ("common.cuh", "norm.cuh"),
+    "backward": ("common.cuh", "tc_chunk.cuh", "tc_wide.cuh", "backward.cuh", "ret_api.cu"),
+}
+WORKLOAD_KERNELS = {"retnet_1p3b": "chunk", "retnet_6p7b_long": "chunk", "gated": "chunk", "seqpar_6p7b": "chunk",
+                    "decode": "decode", "gated_decode": "decode", "backward_1p3b": "backward",
+                    "msr_norm_1p3b": "norm", "retention_msr_1p3b": "chunk"}
+
+
+def kernel_source_sha(name: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "linear_attention_ret_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
+    for fn in KERNEL_SOURCES[WORKLOAD_KERNELS[name]]:
         with open(os.path.join(csrc, fn), "rb") as f:
             h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]
@@ -96,7 +141,7 @@ def ncu_traffic(name: str):
             rec = json.load(f).get(name)
     except (OSError, ValueError):
         return None
-    if not rec or rec.get("source_sha") != kernel_source_sha():
+    if not rec or rec.get("source_sha") != kernel_source_sha(name):
         return None
     return rec.get("traffic_bytes_per_launch")
 
@@ -235,7 +280,30 @@ def make_step(spec, dev, seed):
         def step():
             seqpar.sequence_parallel_chunkwise(x["q"], x["k"], x["v"], x["gamma"], cfg.chunk)
         return step, x, None, launches_per_call(spec)
+    if spec["kind"] == "norm":
+        x = {"o": I.retention_output(cfg.B, cfg.H, cfg.N, cfg.dv, cfg.dtype, seed=seed).to(dev),
+             "gate": I.gate_projection(cfg.B, cfg.H, cfg.N, cfg.dv, cfg.dtype, seed=seed).to(dev)}
+        y = torch.empty_like(x["gate"])
+
+        def step():
+            ret.msr_norm_gate(x["o"], x["gate"], NORM_EPS, y=y)
+        return step, x, y, launches_per_call(spec)
     x = {key: val.to(dev) for key, val in I.config_inputs(cfg, seed=seed).items()}
+    if spec["kind"] == "ret_norm":
+        x["gate"] = I.gate_projection(cfg.B, cfg.H, cfg.N, cfg.dv, cfg.dtype, seed=seed).to(dev)
+        o = torch.empty(cfg.B, cfg.H, cfg.N, cfg.dv, dtype=cfg.dtype, device=dev)
+        y = torch.empty_like(x["gate"])
+
+        def step():
+            ret.ret_chunkwise(x["q"], x["k"], x["v"], x["gamma"], cfg.chunk, o=o)
+            ret.msr_norm_gate(o, x["gate"], NORM_EPS, y=y)
+        return step, x, y, launches_per_call(spec)
+    if spec["kind"] == "backward":
+        x["do"] = I.output_grad(cfg.B, cfg.H, cfg.N, cfg.dv, cfg.dtype, seed=seed).to(dev)
+
+        def step():
+            ret.chunkwise_backward(x["q"], x["k"], x["v"], x["gamma"], x["do"], cfg.chunk)
+        return step, x, None, launches_per_call(spec)
     o = torch.empty(cfg.B, cfg.H, cfg.N, cfg.dv, dtype=cfg.dtype, device=dev)
     if spec["kind"] == "gated":
         def step():
@@ -260,6 +328,12 @@ def launches_per_call(spec) -> int:
     cfg = spec["cfg"]
     if spec["kind"] == "decode":
         return 1
+    if spec["kind"] == "norm":
+        return 1
+    if spec["kind"] == "ret_norm":
+        return ret.chunkwise_launches(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk, cfg.dtype) + 1
+    if spec["kind"] == "backward":
+        return ret.chunkwise_backward_launches(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk, cfg.dtype)
     if spec["kind"] == "seqpar":
         _, world, _ = dist_env()
         n = cfg.N // world + (1 if cfg.N % world else 0)
@@ -333,6 +407,9 @@ def run_ours(args, spec):
                 "peak_source": peak_src + " (MEASURED_PEAKS.json hbm_gbs, copy)" if peak_src == "measured"
                 else "fallback 6.65 TB/s",
                 "kernel_ms": round(kern_ms, 5),
+                "scope": ("the whole step: " + str(launches) + " launches (five calls of the forward kernel, "
+                          "slice/flip/sum copies, the decay gradient)") if spec["kind"] == "backward"
+                else "the step's launches",
                 "tensor_tflops": round(spec["flops"] / (kern_ms / 1e3) / 1e12, 2),
                 "tensor_frac_of_bf16_burst": round(spec["flops"] / (kern_ms / 1e3) / 1e12 / tf_burst, 4)}
     cfg = spec["cfg"]
@@ -400,6 +477,39 @@ def run_e2e(args, spec, dev, stream, world):
                 xd[key].copy_(xh[key], non_blocking=True)
             o, _ = seqpar.sequence_parallel_chunkwise(xd["q"], xd["k"], xd["v"], xd["gamma"], cfg.chunk)
             o_host.copy_(o, non_blocking=True)
+    elif spec["kind"] in ("norm", "ret_norm"):
+        seed = rank_seed(rank)
+        xh = ({"o": I.retention_output(cfg.B, cfg.H, cfg.N, cfg.dv, cfg.dtype, seed=seed)} if spec["kind"] == "norm"
+              else I.config_inputs(cfg, seed=seed))
+        xh["gate"] = I.gate_projection(cfg.B, cfg.H, cfg.N, cfg.dv, cfg.dtype, seed=seed)
+        xh = {k: t.pin_memory() for k, t in xh.items()}
+        xd = {k: torch.empty_like(t, device=dev) for k, t in xh.items()}
+        o = torch.empty(cfg.B, cfg.H, cfg.N, cfg.dv, dtype=cfg.dtype, device=dev)
+        y = torch.empty_like(xd["gate"])
+        y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+
+        def step():
+            for key in xh:
+                xd[key].copy_(xh[key], non_blocking=True)
+            if spec["kind"] == "norm":
+                ret.msr_norm_gate(xd["o"], xd["gate"], NORM_EPS, y=y)
+            else:
+                ret.ret_chunkwise(xd["q"], xd["k"], xd["v"], xd["gamma"], cfg.chunk, o=o)
+                ret.msr_norm_gate(o, xd["gate"], NORM_EPS, y=y)
+            y_host.copy_(y, non_blocking=True)
+    elif spec["kind"] == "backward":
+        xh = {k: t.pin_memory() for k, t in I.config_inputs(cfg, seed=rank_seed(rank)).items()}
+        xh["do"] = I.output_grad(cfg.B, cfg.H, cfg.N, cfg.dv, cfg.dtype, seed=rank_seed(rank)).pin_memory()
+        xd = {k: torch.empty_like(t, device=dev) for k, t in xh.items()}
+        outs_h = [torch.empty(xh[n].shape, dtype=cfg.dtype).pin_memory() for n in ("q", "k", "v")]
+        dgam_h = torch.empty(cfg.H, dtype=torch.float32).pin_memory()
+
+        def step():
+            for key in xh:
+                xd[key].copy_(xh[key], non_blocking=True)
+            grads = ret.chunkwise_backward(xd["q"], xd["k"], xd["v"], xd["gamma"], xd["do"], cfg.chunk)
+            for h, d in zip(outs_h + [dgam_h], grads):
+                h.copy_(d, non_blocking=True)
     else:
         xh = {k: t.pin_memory() for k, t in I.config_inputs(cfg, seed=rank_seed(rank)).items()}
         xd = {k: torch.empty_like(t, device=dev) for k, t in xh.items()}
@@ -458,8 +568,32 @@ def _oracle_sample_step(spec, heads, seed=0):
         def run():
             _, state[0] = O.ret_recurrent_step(qs, ks, vs, gam, state[0])
         return run, b_needed * cfg.H / (cfg.B * cfg.H)  # fraction of one decode step
+    if spec["kind"] == "norm":
+        o = I.retention_output(cfg.B, cfg.H, cfg.N, cfg.dv, cfg.dtype, seed=seed)
+        gate = I.gate_projection(cfg.B, cfg.H, cfg.N, cfg.dv, cfg.dtype, seed=seed)
+
+        def run():
+            O.msr_norm_gate(o, gate, NORM_EPS)
+        return run, cfg.B * cfg.N  # the whole workload: the epilogue is linear in its size
     x = I.config_inputs(cfg, seed=seed, B=max(1, -(-heads // cfg.H)))
+    if spec["kind"] == "ret_norm":
+        bh_idx = torch.arange(heads) % cfg.H
+        sl = {k: t.reshape(-1, *t.shape[2:])[:heads].unsqueeze(0) for k, t in x.items() if k != "gamma"}
+        gate = I.gate_projection(1, heads, cfg.N, cfg.dv, cfg.dtype, seed=seed)
+
+        def run():
+            o, _ = O.ret_chunkwise(sl["q"], sl["k"], sl["v"], x["gamma"][bh_idx], cfg.chunk)
+            O.msr_norm_gate(o, gate, NORM_EPS)
+        return run, heads * cfg.N / cfg.H
+    if spec["kind"] == "backward":
+        x["do"] = I.output_grad(x["q"].shape[0], cfg.H, cfg.N, cfg.dv, cfg.dtype, seed=seed)
     sl = {k: t.reshape(-1, *t.shape[2:])[:heads].unsqueeze(0) for k, t in x.items() if k != "gamma"}
+    if spec["kind"] == "backward":
+        gam = x["gamma"][torch.arange(heads) % cfg.H]
+
+        def run():
+            O.ret_backward(sl["q"], sl["k"], sl["v"], gam, sl["do"])
+        return run, heads * cfg.N / cfg.H
     if spec["kind"] == "gated":
         def run():
             O.gated_chunkwise(sl["q"], sl["k"], sl["v"], sl["g"], cfg.chunk)
@@ -546,7 +680,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="retnet_1p3b",
-                    choices=["retnet_1p3b", "retnet_6p7b_long", "gated", "decode", "gated_decode", "seqpar_6p7b"])
+                    choices=["retnet_1p3b", "retnet_6p7b_long", "gated", "decode", "gated_decode", "seqpar_6p7b",
+                             "backward_1p3b", "msr_norm_1p3b", "retention_msr_1p3b"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

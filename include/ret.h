@@ -153,8 +153,11 @@ RET_API ret_status ret_last_device_error(void* stream);
  * dout has v's layout; dq, dk, dv have q's, k's, v's (dtype dt). Computed with the
  * forward kernels (dq directly, dk and dv on the time-reversed sequence, a dv wider
  * than 256 contracted in pieces) and small kernels of this library; takes
- * stream-ordered scratch (freed on the same stream). bf16 needs 16-byte aligned
- * tensors. Requires dk <= 256.
+ * stream-ordered scratch (freed on the same stream). On the tensor-core path the
+ * pieces are read in place and run two at a time, the second on a library-owned
+ * stream of the current device forked from and joined back to `stream` with
+ * events, so all work stays ordered on `stream` (and can be captured in a graph).
+ * bf16 needs 16-byte aligned tensors. Requires dk <= 256.
  */
 RET_API ret_status ret_chunkwise_backward(const void* q, const void* k, const void* v, const float* gamma,
                                   const void* dout, void* dq, void* dk, void* dv, float* dgamma,
@@ -192,6 +195,33 @@ RET_API ret_status gated_ret_chunkwise_state(const void* k, const void* v, const
 /* Kernels one ret_chunkwise_state / gated_ret_chunkwise_state call launches (0 for
  * an empty segment, -1 if the arguments would be rejected). Host function. */
 RET_API int ret_chunkwise_state_launches(int B, int H, int N, int dk, int dv, int chunk, ret_dtype dt);
+
+/*
+ * Multi-scale retention output epilogue ("Retentive Network (RetNet) 详解",
+ * section 3.2: a gate and a normalisation on retention's output; the Gated
+ * RetNet page's GateRetention module: subln, an RMSNorm over each head's
+ * dimension without affine weights, and a swish gate fed by g_proj):
+ *   y[b, n, h, :] = swish(gate[b, n, h, :]) * o[b, h, n, :] / sqrt(mean_c o[b, h, n, c]^2 + eps),
+ *   swish(x) = x / (1 + exp(-x)).
+ * o: the retention output [B, H, N, dv] (as ret_chunkwise writes it); gate and y:
+ * token-major [B, N, H, dv], the layout of the module's projections. All three
+ * have dtype dt; sums and the scale are fp32. eps >= 0 (the pages' norm default
+ * is 1e-5). One pass: each element of o and gate is read once and y written once.
+ * y may be the gate buffer itself (in place); any other overlap of y with o or
+ * gate is rejected with RET_ERR_UNSUPPORTED. Errors: RET_ERR_SHAPE for invalid
+ * sizes or eps, RET_ERR_NULL for a missing pointer (N > 0), RET_ERR_DTYPE.
+ * Any dv and alignment; whole 16-byte rows with 16-byte aligned pointers take
+ * the vector kernel.
+ */
+RET_API ret_status ret_msr_norm_gate(const void* o, const void* gate, void* y, int B, int H, int N, int dv, float eps,
+                                     ret_dtype dt, void* stream);
+
+/* Kernels one ret_chunkwise_backward (gated = 0) or gated_ret_chunkwise_backward
+ * (gated = 1) call launches with these arguments, ddecay non-zero when the decay
+ * gradient is requested (0 for an empty sequence, -1 if the arguments would be
+ * rejected). The cudaMemsetAsync that zeroes dgamma is not counted. */
+RET_API int ret_chunkwise_backward_launches(int B, int H, int N, int dk, int dv, int chunk, ret_dtype dt, int gated,
+                                            int ddecay);
 
 /*
  * Start states of R consecutive segments from their end states and decays:

@@ -13,7 +13,8 @@
 // same gamma, or the reversed gates shifted by one (g'_i = g_{N-i}, g'_0 = 0).
 // The forward kernels take q/k widths up to 256, so a wider dv is contracted in
 // pieces (retention is linear in the scores q . k) whose outputs are summed.
-// This file holds the data-movement and reduction kernels of that composition.
+// This file holds the data-movement and reduction kernels of that composition:
+// one warp per row, whole 16-byte chunks where rows allow it.
 #pragma once
 
 #include "common.cuh"
@@ -21,37 +22,108 @@
 namespace ret {
 
 constexpr int kBwdThreads = 256;
+constexpr int kBwdWarps = kBwdThreads / 32;
 
-// dst[bh, t, c] = src[bh, flip ? N-1-t : t, c0 + c] for c < w (a contiguous column
-// slice, optionally time-reversed). src rows are d_src wide.
-template <typename T>
+// 16-byte chunks of a row: VEC when every row start and width is a whole number of
+// chunks (checked by the caller), else element by element.
+template <typename T, bool VEC>
+struct RowIo {
+    static constexpr int kE = VEC ? 16 / (int)sizeof(T) : 1;
+};
+
+// Rows one warp moves per iteration of the copy kernels (their loads all in flight
+// before the stores).
+constexpr int kCopyRows = 4;
+
+// dst[bh, t, :w] = src[bh, flip ? N-1-t : t, c0 : c0+w] (a column slice, optionally
+// time-reversed). src rows are d_src wide. A warp takes kCopyRows destination rows at a
+// time, 64 chunks of each per pass.
+template <typename T, bool VEC>
 __global__ void __launch_bounds__(kBwdThreads)
 slice_flip_kernel(const T* __restrict__ src, T* __restrict__ dst, int N, int d_src, int c0, int w, bool flip,
-                  size_t total) {
-    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
-        const int c = (int)(i % w);
-        const size_t row = i / w;  // bh * N + t
-        const int t = (int)(row % N);
-        const size_t bh = row / N;
-        const int ts = flip ? N - 1 - t : t;
-        dst[i] = src[(bh * N + ts) * d_src + c0 + c];
+                  size_t rows) {
+    const int lane = threadIdx.x & 31;
+    const size_t nw = (size_t)gridDim.x * kBwdWarps;
+    for (size_t r0 = ((size_t)blockIdx.x * kBwdWarps + (threadIdx.x >> 5)) * kCopyRows; r0 < rows;
+         r0 += nw * kCopyRows) {
+        if constexpr (VEC) {
+            constexpr int kE = RowIo<T, true>::kE;
+            const int cpr = w / kE;  // chunks per row
+            for (int cb = 0; cb < cpr; cb += 64) {
+                uint4 buf[kCopyRows][2];
+#pragma unroll
+                for (int i = 0; i < kCopyRows; ++i) {
+                    const size_t r = r0 + i;
+                    if (r >= rows) break;
+                    const size_t bh = r / N;
+                    const int t = (int)(r - bh * N);
+                    const uint4* s = reinterpret_cast<const uint4*>(src + (bh * N + (flip ? N - 1 - t : t)) * d_src + c0);
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int c = cb + lane + 32 * j;
+                        if (c < cpr) buf[i][j] = __ldcs(s + c);
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < kCopyRows; ++i) {
+                    const size_t r = r0 + i;
+                    if (r >= rows) break;
+                    uint4* d = reinterpret_cast<uint4*>(dst + r * w);
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int c = cb + lane + 32 * j;
+                        if (c < cpr) __stcs(d + c, buf[i][j]);
+                    }
+                }
+            }
+        } else {
+            for (int i = 0; i < kCopyRows && r0 + i < rows; ++i) {
+                const size_t r = r0 + i;
+                const size_t bh = r / N;
+                const int t = (int)(r - bh * N);
+                const T* s = src + (bh * N + (flip ? N - 1 - t : t)) * d_src + c0;
+                for (int c = lane; c < w; c += 32) dst[r * w + c] = s[c];
+            }
+        }
     }
 }
 
-// out[bh, t, c] = sum_p parts[p][bh, flip ? N-1-t : t, c], summed in fp32.
-template <typename T>
+// out[bh, t, :] = sum_p parts[p][bh, flip ? N-1-t : t, :], summed in fp32. One warp per row.
+template <typename T, bool VEC>
 __global__ void __launch_bounds__(kBwdThreads)
-sum_flip_kernel(const T* __restrict__ parts, int P, size_t part_elems, T* __restrict__ out, int N, int d, bool flip) {
-    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < part_elems;
-         i += (size_t)gridDim.x * blockDim.x) {
-        const int c = (int)(i % d);
-        const size_t row = i / d;
-        const int t = (int)(row % N);
-        const size_t bh = row / N;
-        const size_t src = (bh * N + (flip ? N - 1 - t : t)) * d + c;
-        float s = 0.f;
-        for (int p = 0; p < P; ++p) s += ld_elem(parts + (size_t)p * part_elems + src);
-        st_elem(out + i, s);
+sum_flip_kernel(const T* __restrict__ parts, int P, size_t part_elems, T* __restrict__ out, int N, int d, bool flip,
+                size_t rows) {
+    const int lane = threadIdx.x & 31;
+    for (size_t r = (size_t)blockIdx.x * kBwdWarps + (threadIdx.x >> 5); r < rows; r += (size_t)gridDim.x * kBwdWarps) {
+        const size_t bh = r / N;
+        const int t = (int)(r - bh * N);
+        const T* s = parts + (bh * N + (flip ? N - 1 - t : t)) * d;
+        T* o = out + r * d;
+        if constexpr (VEC) {
+            constexpr int kE = RowIo<T, true>::kE;
+            for (int c = lane; c < d / kE; c += 32) {
+                float acc[kE];
+#pragma unroll
+                for (int e = 0; e < kE; ++e) acc[e] = 0.f;
+                for (int p = 0; p < P; ++p) {
+                    const uint4 u = __ldcs(reinterpret_cast<const uint4*>(s + (size_t)p * part_elems) + c);
+                    const T* x = reinterpret_cast<const T*>(&u);
+#pragma unroll
+                    for (int e = 0; e < kE; ++e) acc[e] += ld_elem(x + e);
+                }
+                uint4 u;
+                T* y = reinterpret_cast<T*>(&u);
+#pragma unroll
+                for (int e = 0; e < kE; ++e) st_elem(y + e, acc[e]);
+                reinterpret_cast<uint4*>(o)[c] = u;
+            }
+        } else {
+            for (int c = lane; c < d; c += 32) {
+                float acc = 0.f;
+                for (int p = 0; p < P; ++p) acc += ld_elem(s + (size_t)p * part_elems + c);
+                st_elem(o + c, acc);
+            }
+        }
     }
 }
 
@@ -59,74 +131,100 @@ sum_flip_kernel(const T* __restrict__ parts, int P, size_t part_elems, T* __rest
 __global__ void __launch_bounds__(kBwdThreads)
 gate_flip_kernel(const float* __restrict__ g, float* __restrict__ gf, int N, size_t total) {
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
-        const int t = (int)(i % N);
         const size_t bh = i / N;
+        const int t = (int)(i - bh * N);
         gf[i] = t == 0 ? 0.f : g[bh * N + (N - t)];
     }
 }
 
-// Decay gradient from a_t = q_t . dQ_t - k_t . dK_t, one block per (b, h):
-// gated: dg[bh, t] = sum_{u >= t} a_u; fixed: atomically adds (1/gamma_h) sum_t t a_t
-// to dgamma[h] (zeroed by the caller). A warp computes each a_t; the block then scans
-// from the end of the sequence in tiles of kBwdThreads tokens with a running carry.
-template <typename T, bool GATED>
+// Tokens per block of the decay-gradient kernel.
+constexpr int kGradTokens = 64;
+
+// a_t = q_t . dQ_t - k_t . dK_t (= dL/dG_t) for a tile of kGradTokens tokens of one
+// (b, h) (grid: token tiles x B*H; one warp per token).
+// gated: out[bh, t] = a_t (the suffix sum follows in gate_grad_scan_kernel);
+// fixed: adds (1/gamma_h) sum_t t a_t of the tile to dgamma[h] (zeroed by the caller).
+template <typename T, bool VEC, bool GATED>
 __global__ void __launch_bounds__(kBwdThreads)
 decay_grad_kernel(const T* __restrict__ q, const T* __restrict__ dq, const T* __restrict__ k,
                   const T* __restrict__ dk, const float* __restrict__ decay, float* __restrict__ out, int H, int N,
                   int dk_dim) {
-    __shared__ float a_s[kBwdThreads];
-    __shared__ float warp_s[kBwdThreads / 32];
-    const int bh = blockIdx.x;
+    __shared__ float warp_s[kBwdWarps];
+    const int bh = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const size_t base = (size_t)bh * N * dk_dim;
-    float carry = 0.f;   // gated: sum of a_u over the tiles already scanned (later tokens)
-    float weighted = 0.f;  // fixed: this thread's share of sum_t t a_t
-    for (int tile_end = N; tile_end > 0; tile_end -= kBwdThreads) {
-        const int tile0 = max(0, tile_end - kBwdThreads);
-        const int len = tile_end - tile0;
-        for (int j = warp; j < len; j += kBwdThreads / 32) {
-            const size_t row = base + (size_t)(tile0 + j) * dk_dim;
-            float s = 0.f;
+    const int t0 = blockIdx.x * kGradTokens;
+    float weighted = 0.f;  // this warp's share of sum_t t a_t (fixed gamma)
+    for (int j = warp; j < kGradTokens && t0 + j < N; j += kBwdWarps) {
+        const int t = t0 + j;
+        const size_t row = ((size_t)bh * N + t) * dk_dim;
+        float s = 0.f;
+        if constexpr (VEC) {
+            constexpr int kE = RowIo<T, true>::kE;
+            for (int c = lane; c < dk_dim / kE; c += 32) {
+                const uint4 uq = __ldcs(reinterpret_cast<const uint4*>(q + row) + c);
+                const uint4 udq = __ldcs(reinterpret_cast<const uint4*>(dq + row) + c);
+                const uint4 uk = __ldcs(reinterpret_cast<const uint4*>(k + row) + c);
+                const uint4 udk = __ldcs(reinterpret_cast<const uint4*>(dk + row) + c);
+                const T* xq = reinterpret_cast<const T*>(&uq);
+                const T* xdq = reinterpret_cast<const T*>(&udq);
+                const T* xk = reinterpret_cast<const T*>(&uk);
+                const T* xdk = reinterpret_cast<const T*>(&udk);
+#pragma unroll
+                for (int e = 0; e < kE; ++e)
+                    s += ld_elem(xq + e) * ld_elem(xdq + e) - ld_elem(xk + e) * ld_elem(xdk + e);
+            }
+        } else {
             for (int c = lane; c < dk_dim; c += 32)
                 s += ld_elem(q + row + c) * ld_elem(dq + row + c) - ld_elem(k + row + c) * ld_elem(dk + row + c);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-            if (lane == 0) a_s[j] = s;
         }
-        __syncthreads();
-        const int j = threadIdx.x;
-        const float a = j < len ? a_s[j] : 0.f;
-        if (!GATED) {
-            weighted += (float)(tile0 + j) * a;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (GATED) {
+            if (lane == 0) out[(size_t)bh * N + t] = s;
         } else {
-            // inclusive suffix sum inside the tile: reverse index r = len - 1 - j
-            float x = a;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float y = __shfl_down_sync(0xffffffffu, x, o);
-                if (lane + o < 32) x += y;
-            }
-            if (lane == 0) warp_s[warp] = x;  // warp total (suffix sum at its first lane)
-            __syncthreads();
-            float later = 0.f;  // totals of the warps after this one
-            for (int w2 = warp + 1; w2 < kBwdThreads / 32; ++w2) later += warp_s[w2];
-            if (j < len) out[(size_t)bh * N + tile0 + j] = x + later + carry;
-            float total = 0.f;
-            for (int w2 = 0; w2 < kBwdThreads / 32; ++w2) total += warp_s[w2];
-            carry += total;
+            weighted += (float)t * s;
         }
-        __syncthreads();
     }
     if (!GATED) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) weighted += __shfl_xor_sync(0xffffffffu, weighted, o);
         if (lane == 0) warp_s[warp] = weighted;
         __syncthreads();
         if (threadIdx.x == 0) {
             float s = 0.f;
-            for (int w2 = 0; w2 < kBwdThreads / 32; ++w2) s += warp_s[w2];
+            for (int w2 = 0; w2 < kBwdWarps; ++w2) s += warp_s[w2];
             atomicAdd(out + bh % H, s / decay[bh % H]);
         }
+    }
+}
+
+// In place: dg[bh, t] = sum_{u >= t} a[bh, u] (a suffix sum, since G_u includes g_t for
+// every u >= t). One block per (b, h), tiles of kBwdThreads tokens from the end of the
+// sequence with a running carry.
+__global__ void __launch_bounds__(kBwdThreads) gate_grad_scan_kernel(float* __restrict__ dg, int N) {
+    __shared__ float warp_s[kBwdWarps];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float* a = dg + (size_t)blockIdx.x * N;
+    float carry = 0.f;
+    for (int tile_end = N; tile_end > 0; tile_end -= kBwdThreads) {
+        const int tile0 = max(0, tile_end - kBwdThreads);
+        const int len = tile_end - tile0;
+        const int j = threadIdx.x;
+        float x = j < len ? a[tile0 + j] : 0.f;
+        // inclusive suffix sum inside the warp
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_down_sync(0xffffffffu, x, o);
+            if (lane + o < 32) x += y;
+        }
+        if (lane == 0) warp_s[warp] = x;  // the warp's total
+        __syncthreads();
+        float later = 0.f, total = 0.f;
+        for (int w2 = 0; w2 < kBwdWarps; ++w2) {
+            if (w2 > warp) later += warp_s[w2];
+            total += warp_s[w2];
+        }
+        if (j < len) a[tile0 + j] = x + later + carry;
+        carry += total;
+        __syncthreads();
     }
 }
 

@@ -1,6 +1,7 @@
 // C ABI of libret.so (declared in include/ret.h): host-side validation, kernel
 // selection and launch. One translation unit holds every kernel so that they
 // share the module-scope device error word.
+#include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -11,6 +12,7 @@
 #include "tc_chunk.cuh"
 #include "seqpar.cuh"
 #include "backward.cuh"
+#include "norm.cuh"
 
 using namespace ret;
 
@@ -117,16 +119,91 @@ ret_status chunkwise_state_entry(const void* k, const void* v, const float* deca
 // ------------------------------------------------------------------ backward (see backward.cuh)
 
 inline int grid_for(size_t n) { return (int)std::min<size_t>((n + kBwdThreads - 1) / kBwdThreads, 8 * tc::sm_count()); }
+// Row kernels: one warp per `per_warp` rows, up to 32 blocks per SM.
+inline unsigned rows_grid(size_t rows, int per_warp = 1) {
+    const size_t warps = (rows + per_warp - 1) / per_warp;
+    return (unsigned)std::min<size_t>((warps + kBwdWarps - 1) / kBwdWarps, (size_t)32 * tc::sm_count());
+}
+inline bool whole_chunks(size_t elems, size_t elt) { return (elems * elt) % 16 == 0; }
 
 template <typename T>
-ret_status slice_flip(const void* src, void* dst, int BH, int N, int d_src, int c0, int w, bool flip, cudaStream_t st) {
-    const size_t total = (size_t)BH * N * w;
-    slice_flip_kernel<T><<<grid_for(total), kBwdThreads, 0, st>>>(static_cast<const T*>(src), static_cast<T*>(dst), N,
-                                                                  d_src, c0, w, flip, total);
+ret_status sum_flip(const T* parts, int P, size_t part_elems, T* out, int BH, int N, int d, bool flip, cudaStream_t st) {
+    const size_t rows = (size_t)BH * N;
+    if (whole_chunks(d, sizeof(T)) && whole_chunks(part_elems, sizeof(T)) && aligned16(parts) && aligned16(out))
+        sum_flip_kernel<T, true><<<rows_grid(rows), kBwdThreads, 0, st>>>(parts, P, part_elems, out, N, d, flip, rows);
+    else
+        sum_flip_kernel<T, false><<<rows_grid(rows), kBwdThreads, 0, st>>>(parts, P, part_elems, out, N, d, flip, rows);
     return launch_status();
 }
 
+template <typename T>
+ret_status slice_flip(const void* src, void* dst, int BH, int N, int d_src, int c0, int w, bool flip, cudaStream_t st) {
+    const size_t rows = (size_t)BH * N;
+    const T* s = static_cast<const T*>(src);
+    T* d = static_cast<T*>(dst);
+    if (whole_chunks(d_src, sizeof(T)) && whole_chunks(c0, sizeof(T)) && whole_chunks(w, sizeof(T)) && aligned16(s) &&
+        aligned16(d))
+        slice_flip_kernel<T, true><<<rows_grid(rows, kCopyRows), kBwdThreads, 0, st>>>(s, d, N, d_src, c0, w, flip,
+                                                                                       rows);
+    else
+        slice_flip_kernel<T, false><<<rows_grid(rows, kCopyRows), kBwdThreads, 0, st>>>(s, d, N, d_src, c0, w, flip,
+                                                                                        rows);
+    return launch_status();
+}
+
+template <typename T, bool GATED>
+ret_status decay_grad(const T* q, const T* dq, const T* k, const T* dk, const float* decay, float* out, int BH, int H,
+                      int N, int dk_dim, cudaStream_t st) {
+    if (!GATED && cudaMemsetAsync(out, 0, sizeof(float) * (size_t)H, st) != cudaSuccess) return RET_ERR_CUDA;
+    const dim3 grid((unsigned)((N + kGradTokens - 1) / kGradTokens), (unsigned)BH);
+    if (whole_chunks(dk_dim, sizeof(T)) && aligned16(q) && aligned16(dq) && aligned16(k) && aligned16(dk))
+        decay_grad_kernel<T, true, GATED><<<grid, kBwdThreads, 0, st>>>(q, dq, k, dk, decay, out, H, N, dk_dim);
+    else
+        decay_grad_kernel<T, false, GATED><<<grid, kBwdThreads, 0, st>>>(q, dq, k, dk, decay, out, H, N, dk_dim);
+    ret_status r = launch_status();
+    if (GATED && r == RET_OK) {
+        gate_grad_scan_kernel<<<(unsigned)BH, kBwdThreads, 0, st>>>(out, N);
+        r = launch_status();
+    }
+    return r;
+}
+
 inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
+
+// A second stream per device, with fork and join events, for the pieces of a dv
+// contraction that run side by side. Held under the mutex from fork to join, so calls
+// from several host threads do not interleave their events.
+struct AuxStream {
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+constexpr int kMaxDevices = 64;
+inline std::mutex& aux_mutex() {
+    static std::mutex m;
+    return m;
+}
+inline AuxStream* aux_stream() {
+    static AuxStream aux[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    AuxStream& a = aux[dev];
+    if (!a.s) {
+        if (cudaStreamCreateWithFlags(&a.s, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+        if (cudaEventCreateWithFlags(&a.fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&a.join, cudaEventDisableTiming) != cudaSuccess)
+            return nullptr;
+    }
+    return &a;
+}
+
+// The dv contraction of dQ and dK in pieces of 256: on the tensor-core path each piece is
+// read in place through row-strided tensor maps; otherwise it is copied out first.
+inline bool backward_pieces_in_place(int dk, int dv, int chunk, ret_dtype dt) {
+    if (dv <= 256 || dt != RET_BF16) return false;
+    for (int c0 = 0; c0 < dv; c0 += 256)
+        if (!tc_chunk_supported(std::min(256, dv - c0), dk, chunk, true)) return false;
+    return true;
+}
 
 template <typename T, bool GATED>
 ret_status backward_impl(const void* q, const void* k, const void* v, const float* decay, const void* dout, void* dq,
@@ -136,10 +213,12 @@ ret_status backward_impl(const void* q, const void* k, const void* v, const floa
     const size_t nQ = (size_t)BH * N * dk, nV = (size_t)BH * N * dv;
     const int pw = dv <= 256 ? dv : 256;  // width of one piece of the dv contraction
     const int P = (dv + pw - 1) / pw;
+    const bool in_place = backward_pieces_in_place(dk, dv, chunk, dt);
     // scratch: reversed Q, K, V, dO; two piece buffers; per-piece outputs; reversed dV; reversed gates
     size_t off[9], bytes = 0;
     const size_t sz[9] = {nQ * sizeof(T), nQ * sizeof(T), nV * sizeof(T), nV * sizeof(T),
-                          (size_t)BH * N * pw * sizeof(T), (size_t)BH * N * pw * sizeof(T), (size_t)P * nQ * sizeof(T),
+                          in_place ? 0 : (size_t)BH * N * pw * sizeof(T), in_place ? 0 : (size_t)BH * N * pw * sizeof(T),
+                          (size_t)P * nQ * sizeof(T),
                           nV * sizeof(T), GATED ? (size_t)BH * N * sizeof(float) : 0};
     for (int i = 0; i < 9; ++i) {
         off[i] = bytes;
@@ -162,18 +241,42 @@ ret_status backward_impl(const void* q, const void* k, const void* v, const floa
     auto fwd = [&](const void* fq, const void* fk, const void* fv, const float* dec, void* fo, int wq, int wv) {
         return ok(chunkwise_entry<GATED>(fq, fk, fv, dec, fo, nullptr, nullptr, B, H, N, wq, wv, chunk, dt, st));
     };
+    // All pieces of a dv contraction: forward(a[:, c0:c0+w], b[:, c0:c0+w], c) into parts[p],
+    // a and b dv wide. In place, odd pieces run on the second stream beside the even ones
+    // (each launch then sized for the SMs it shares); otherwise each piece is copied out.
+    auto pieces = [&](const void* a, const void* b, const void* c, const float* dec) {
+        if (!in_place) {
+            for (int p = 0; p < P && r == RET_OK; ++p) {
+                const int c0 = p * pw, w = std::min(pw, dv - c0);
+                ok(slice_flip<T>(a, pa, BH, N, dv, c0, w, false, st)) &&
+                    ok(slice_flip<T>(b, pb, BH, N, dv, c0, w, false, st)) &&
+                    fwd(pa, pb, c, dec, parts + (size_t)p * nQ, w, dk);
+            }
+            return r == RET_OK;
+        }
+        std::lock_guard<std::mutex> lock(aux_mutex());
+        AuxStream* aux = aux_stream();
+        if (!aux) return ok(RET_ERR_CUDA);
+        if (cudaEventRecord(aux->fork, st) != cudaSuccess || cudaStreamWaitEvent(aux->s, aux->fork, 0) != cudaSuccess)
+            return ok(RET_ERR_CUDA);
+        for (int p = 0; p < P && r == RET_OK; ++p) {
+            const int c0 = p * pw, w = std::min(pw, dv - c0);
+            ok(tc_chunk_launch<GATED>(static_cast<const T*>(a) + c0, static_cast<const T*>(b) + c0, c, dec,
+                                      parts + (size_t)p * nQ, nullptr, nullptr, B, H, N, w, dk, p % 2 ? aux->s : st,
+                                      dv, dv, 2));
+        }
+        // join even on failure, so the second stream never runs past this call
+        if ((cudaEventRecord(aux->join, aux->s) != cudaSuccess || cudaStreamWaitEvent(st, aux->join, 0) != cudaSuccess))
+            ok(RET_ERR_CUDA);
+        return r == RET_OK;
+    };
     // dQ = forward(dO, V, K), the dv contraction in pieces
     if (P == 1) {
         fwd(dout, v, k, decay, dq, dv, dk);
     } else {
-        for (int p = 0; p < P && r == RET_OK; ++p) {
-            const int c0 = p * pw, w = std::min(pw, dv - c0);
-            ok(slice_flip<T>(dout, pa, BH, N, dv, c0, w, false, st)) && ok(slice_flip<T>(v, pb, BH, N, dv, c0, w, false, st)) &&
-                fwd(pa, pb, k, decay, parts + (size_t)p * nQ, w, dk);
-        }
+        pieces(dout, v, k, decay);
         if (r == RET_OK) {
-            sum_flip_kernel<T><<<grid_for(nQ), kBwdThreads, 0, st>>>(parts, P, nQ, static_cast<T*>(dq), N, dk, false);
-            ok(launch_status());
+            ok(sum_flip<T>(parts, P, nQ, static_cast<T*>(dq), BH, N, dk, false, st));
         }
     }
     // time-reversed copies (and gates reversed and shifted by one)
@@ -187,32 +290,21 @@ ret_status backward_impl(const void* q, const void* k, const void* v, const floa
     }
     const float* dec_rev = GATED ? gf : decay;
     // dK = reverse(forward(rev V, rev dO, rev Q)), in pieces
-    for (int p = 0; p < P && r == RET_OK; ++p) {
-        const int c0 = p * pw, w = std::min(pw, dv - c0);
-        if (P == 1) {
+    if (r == RET_OK) {
+        if (P == 1)
             fwd(Vf, dOf, Qf, dec_rev, parts, dv, dk);
-        } else {
-            ok(slice_flip<T>(Vf, pa, BH, N, dv, c0, w, false, st)) && ok(slice_flip<T>(dOf, pb, BH, N, dv, c0, w, false, st)) &&
-                fwd(pa, pb, Qf, dec_rev, parts + (size_t)p * nQ, w, dk);
-        }
+        else
+            pieces(Vf, dOf, Qf, dec_rev);
     }
     if (r == RET_OK) {
-        sum_flip_kernel<T><<<grid_for(nQ), kBwdThreads, 0, st>>>(parts, P, nQ, static_cast<T*>(dk_out), N, dk, true);
-        ok(launch_status());
+        ok(sum_flip<T>(parts, P, nQ, static_cast<T*>(dk_out), BH, N, dk, true, st));
     }
     // dV = reverse(forward(rev K, rev Q, rev dO))
     if (r == RET_OK && fwd(Kf, Qf, dOf, dec_rev, Rf, dk, dv)) ok(slice_flip<T>(Rf, dv_out, BH, N, dv, 0, dv, true, st));
     // decay gradient
-    if (r == RET_OK && ddecay) {
-        if (!GATED && cudaMemsetAsync(ddecay, 0, sizeof(float) * (size_t)H, st) != cudaSuccess) r = RET_ERR_CUDA;
-        if (r == RET_OK) {
-            decay_grad_kernel<T, GATED><<<BH, kBwdThreads, 0, st>>>(static_cast<const T*>(q), static_cast<const T*>(dq),
-                                                                    static_cast<const T*>(k),
-                                                                    static_cast<const T*>(dk_out), decay, ddecay, H, N,
-                                                                    dk);
-            ok(launch_status());
-        }
-    }
+    if (r == RET_OK && ddecay)
+        ok(decay_grad<T, GATED>(static_cast<const T*>(q), static_cast<const T*>(dq), static_cast<const T*>(k),
+                                static_cast<const T*>(dk_out), decay, ddecay, BH, H, N, dk, st));
     if (cudaFreeAsync(sc, st) != cudaSuccess && r == RET_OK) r = RET_ERR_CUDA;
     return r;
 }
@@ -241,6 +333,46 @@ ret_status backward_entry(const void* q, const void* k, const void* v, const flo
     }
     return backward_impl<float, GATED>(q, k, v, decay, dout, dq, dk_out, dv_out, ddecay, B, H, N, dk, dv, chunk, dt,
                                        st);
+}
+
+// Multi-scale retention output epilogue: the vector kernel when rows are whole 16-byte
+// chunks (LPR lanes per row, CH chunks per lane), else the scalar kernel.
+template <typename T, int LPR, int CH>
+void launch_norm_vec(const T* o, const T* gate, T* y, int H, int N, int dv, float eps, size_t rows, cudaStream_t st) {
+    const size_t rows_per_block = (size_t)(kNormThreads / 32) * (32 / LPR);
+    const size_t blocks = std::min<size_t>((rows + rows_per_block - 1) / rows_per_block, (size_t)32 * tc::sm_count());
+    norm_gate_vec_kernel<T, LPR, CH><<<(unsigned)blocks, kNormThreads, 0, st>>>(o, gate, y, H, N, dv, eps, rows);
+}
+
+template <typename T>
+ret_status launch_norm_gate(const void* o_, const void* gate_, void* y_, int B, int H, int N, int dv, float eps,
+                            cudaStream_t st) {
+    const T* o = static_cast<const T*>(o_);
+    const T* gate = static_cast<const T*>(gate_);
+    T* y = static_cast<T*>(y_);
+    const size_t rows = (size_t)B * N * H;
+    const bool vec = ((size_t)dv * sizeof(T)) % 16 == 0 && aligned16(o) && aligned16(gate) && aligned16(y);
+    const int chunks = vec ? (int)((size_t)dv * sizeof(T) / 16) : 0;
+    if (vec && chunks <= 1) launch_norm_vec<T, 1, 1>(o, gate, y, H, N, dv, eps, rows, st);
+    else if (vec && chunks <= 2) launch_norm_vec<T, 2, 1>(o, gate, y, H, N, dv, eps, rows, st);
+    else if (vec && chunks <= 4) launch_norm_vec<T, 4, 1>(o, gate, y, H, N, dv, eps, rows, st);
+    else if (vec && chunks <= 8) launch_norm_vec<T, 8, 1>(o, gate, y, H, N, dv, eps, rows, st);
+    else if (vec && chunks <= 16) launch_norm_vec<T, 16, 1>(o, gate, y, H, N, dv, eps, rows, st);
+    else if (vec && chunks <= 32) launch_norm_vec<T, 32, 1>(o, gate, y, H, N, dv, eps, rows, st);
+    else if (vec && chunks <= 64) launch_norm_vec<T, 32, 2>(o, gate, y, H, N, dv, eps, rows, st);
+    else if (vec && chunks <= 128) launch_norm_vec<T, 32, 4>(o, gate, y, H, N, dv, eps, rows, st);
+    else if (vec && chunks <= 256) launch_norm_vec<T, 32, 8>(o, gate, y, H, N, dv, eps, rows, st);
+    else {
+        const size_t blocks = std::min<size_t>((rows + kNormThreads / 32 - 1) / (kNormThreads / 32),
+                                               (size_t)32 * tc::sm_count());
+        norm_gate_scalar_kernel<T><<<(unsigned)blocks, kNormThreads, 0, st>>>(o, gate, y, H, N, dv, eps, rows);
+    }
+    return launch_status();
+}
+
+inline bool ranges_overlap(const void* a, const void* b, size_t bytes) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), z = reinterpret_cast<uintptr_t>(b);
+    return x < z + bytes && z < x + bytes;
 }
 
 template <typename T>
@@ -405,6 +537,44 @@ int ret_chunkwise_state_launches(int B, int H, int N, int dk, int dv, int chunk,
     if (N == 0) return 0;
     // the decay kernel, then the state-only pass (+ prefix) or the CUDA-core chunkwise kernel
     return 1 + (tc_chunk_supported(dk, dv, chunk, dt == RET_BF16) ? tc_state_launches(B, H, N, dv) : 1);
+}
+
+ret_status ret_msr_norm_gate(const void* o, const void* gate, void* y, int B, int H, int N, int dv, float eps,
+                             ret_dtype dt, void* stream) {
+    ret_status s = check_common(B, H, N, 1, dv, dt);
+    if (s != RET_OK) return s;
+    if (!(eps >= 0.f) || !std::isfinite(eps)) return RET_ERR_SHAPE;
+    if (N == 0) return RET_OK;
+    if (!o || !gate || !y) return RET_ERR_NULL;
+    const size_t bytes = (size_t)B * H * N * dv * (dt == RET_BF16 ? 2 : 4);
+    // y may be the gate buffer itself; any other overlap would race
+    if (ranges_overlap(y, o, bytes) || (y != gate && ranges_overlap(y, gate, bytes))) return RET_ERR_UNSUPPORTED;
+    cudaStream_t st = as_stream(stream);
+    if (dt == RET_BF16) return launch_norm_gate<__nv_bfloat16>(o, gate, y, B, H, N, dv, eps, st);
+    return launch_norm_gate<float>(o, gate, y, B, H, N, dv, eps, st);
+}
+
+int ret_chunkwise_backward_launches(int B, int H, int N, int dk, int dv, int chunk, ret_dtype dt, int gated,
+                                    int ddecay) {
+    if (check_common(B, H, N, dk, dv, dt) != RET_OK || chunk <= 0 || dk > 256) return -1;
+    if (N == 0) return 0;
+    // mirrors backward_impl: forward calls, the slice / flip / sum kernels, the decay gradient
+    auto fwd = [&](int wq, int wv) { return ret_chunkwise_launches(B, H, N, wq, wv, chunk, dt); };
+    const int pw = dv <= 256 ? dv : 256, P = (dv + pw - 1) / pw;
+    const bool in_place = backward_pieces_in_place(dk, dv, chunk, dt);
+    int n = 0;
+    for (int p = 0; p < P; ++p) {
+        const int w = std::min(pw, dv - p * pw);
+        // in place: the pieces run two at a time, sized together; else two slices, then the forward
+        const int piece = in_place ? tc_chunk_launches(B, H, N, w, dk, 2) : 2 + fwd(w, dk);
+        n += P == 1 ? 2 * fwd(dv, dk) : 2 * piece;  // a dQ and a dK piece
+    }
+    n += P == 1 ? 0 : 1;                 // sum of the dQ pieces
+    n += 4 + (gated ? 1 : 0);            // reversed Q, K, V, dO (and gates)
+    n += 1;                              // sum + flip of the dK pieces
+    n += fwd(dk, dv) + 1;                // dV and its flip
+    n += ddecay ? (gated ? 2 : 1) : 0;   // decay gradient (gated: and its suffix sum)
+    return n;
 }
 
 const char* ret_version(void) { return "0.1.0"; }

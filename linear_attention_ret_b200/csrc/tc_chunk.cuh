@@ -973,12 +973,15 @@ inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 3D bf16 map over [BH][N][inner] with a 64 x 64 box and 128-byte swizzle.
-inline bool make_map(CUtensorMap* m, const void* base, int inner, int N, int BH) {
+// 3D bf16 map over [BH][N][inner] with a 64 x 64 box and 128-byte swizzle. Rows are
+// ld elements apart (ld = 0: dense, ld = inner), so a column slice of a wider tensor
+// can be read in place.
+inline bool make_map(CUtensorMap* m, const void* base, int inner, int N, int BH, int ld = 0) {
     auto fn = encode_fn();
     if (!fn) return false;
+    const cuuint64_t row = (cuuint64_t)(ld ? ld : inner);
     cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)N, (cuuint64_t)BH};
-    cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)inner * 2 * N};
+    cuuint64_t strides[2] = {row * 2, row * 2 * N};
     cuuint32_t box[3] = {64, 64, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
@@ -1016,9 +1019,11 @@ struct Plan {
     int subs() const { return F * (G - 1); }  // sub-segments whose end states the state-only pass writes
 };
 
-// sub_segments = false keeps one state-only CTA per segment (less scratch).
-inline Plan plan(int B, int H, int N, int dv, bool sub_segments = true) {
-    const int ctas = B * H * (dv / kDvS);
+// sub_segments = false keeps one state-only CTA per segment (less scratch). concurrent:
+// how many launches of this shape the caller runs at the same time on other streams
+// (their CTAs count towards filling the SMs).
+inline Plan plan(int B, int H, int N, int dv, bool sub_segments = true, int concurrent = 1) {
+    const int ctas = B * H * (dv / kDvS) * concurrent;
     const int nchunks = (N + kC - 1) / kC;
     int G = 1;
     if (2 * ctas <= sm_count()) G = std::min(std::min(sm_count() / ctas, kMaxSegments), nchunks / 4);
@@ -1062,10 +1067,10 @@ constexpr int kernel_smem() {
 template <int DK, bool GATED>
 ret_status launch_dk(const void* q, const void* k, const void* v, const float* decay, void* o,
                      const float* state_in, float* state_out, int B, int H, int N, int dv, const Plan& pl,
-                     void* scratch, cudaStream_t st) {
+                     void* scratch, cudaStream_t st, int ldq, int ldk) {
     const int BH = B * H;
     CUtensorMap mq, mk, mv, mo;
-    if (!make_map(&mq, q, DK, N, BH) || !make_map(&mk, k, DK, N, BH) || !make_map(&mv, v, dv, N, BH) ||
+    if (!make_map(&mq, q, DK, N, BH, ldq) || !make_map(&mk, k, DK, N, BH, ldk) || !make_map(&mv, v, dv, N, BH) ||
         !make_map(&mo, o, dv, N, BH))
         return RET_ERR_CUDA;
     Params prm{decay, state_in, state_out, nullptr, nullptr, H, N, dv, pl.seg_chunks, pl.F};
@@ -1102,21 +1107,29 @@ ret_status launch_dk(const void* q, const void* k, const void* v, const float* d
 }
 
 // Runs the tensor-core path with caller-provided scratch (at least scratch_bytes()).
+// ldq, ldk: row strides of q and k in elements (0: dense rows of dk).
 template <bool GATED>
 ret_status launch_with_scratch(const void* q, const void* k, const void* v, const float* decay, void* o,
                                const float* state_in, float* state_out, int B, int H, int N, int dk, int dv,
-                               const Plan& pl, void* scratch, cudaStream_t st) {
+                               const Plan& pl, void* scratch, cudaStream_t st, int ldq = 0, int ldk = 0) {
     switch (dk) {
-        case 64: return launch_dk<64, GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dv, pl, scratch, st);
-        case 128: return launch_dk<128, GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dv, pl, scratch, st);
-        case 256: return launch_dk<256, GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dv, pl, scratch, st);
+        case 64:
+            return launch_dk<64, GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dv, pl, scratch, st, ldq, ldk);
+        case 128:
+            return launch_dk<128, GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dv, pl, scratch, st, ldq,
+                                         ldk);
+        case 256:
+            return launch_dk<256, GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dv, pl, scratch, st, ldq,
+                                         ldk);
     }
     return RET_ERR_UNSUPPORTED;
 }
 
 }  // namespace tc
 
-inline int tc_chunk_launches(int B, int H, int N, int, int dv) { return tc::plan(B, H, N, dv).G > 1 ? 3 : 1; }
+inline int tc_chunk_launches(int B, int H, int N, int, int dv, int concurrent = 1) {
+    return tc::plan(B, H, N, dv, true, concurrent).G > 1 ? 3 : 1;
+}
 
 namespace tc {
 
@@ -1213,14 +1226,14 @@ inline int tc_state_launches(int B, int H, int N, int dv) {
 template <bool GATED>
 ret_status tc_chunk_launch(const void* q, const void* k, const void* v, const float* decay, void* o,
                            const float* state_in, float* state_out, int B, int H, int N, int dk, int dv,
-                           cudaStream_t st) {
-    const tc::Plan pl = tc::plan(B, H, N, dv);
+                           cudaStream_t st, int ldq = 0, int ldk = 0, int concurrent = 1) {
+    const tc::Plan pl = tc::plan(B, H, N, dv, true, concurrent);
     void* scratch = nullptr;
     const size_t bytes = tc::scratch_bytes(pl, B * H, dk, dv, state_in != nullptr && state_in == state_out);
     if (bytes) tc::keep_pool_memory();
     if (bytes && cudaMallocAsync(&scratch, bytes, st) != cudaSuccess) return RET_ERR_CUDA;
     const ret_status r = tc::launch_with_scratch<GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dk, dv,
-                                                        pl, scratch, st);
+                                                        pl, scratch, st, ldq, ldk);
     if (scratch && cudaFreeAsync(scratch, st) != cudaSuccess) return RET_ERR_CUDA;
     return r;
 }

@@ -9,6 +9,10 @@ Recipe (all draws on the CPU torch generator, in this order):
   x        ~ N(0, 1) and g = logsigmoid(x) / 16 for the gated form (the gate
              transform of the gated-RetNet module, upstream of the operator)
   S_0      ~ N(0, 0.01^2) (decode state, fp32)
+  dO       ~ N(0, 1) / sqrt(dv) (output gradient of the backward, own generator)
+  epilogue inputs (own generators): a retention output o [B, H, N, dv] ~ N(0, 1) times a
+             per-row scale e^z, z ~ N(0, 1) (rows of very different size, as the decays
+             make them), and a gate projection [B, N, H, dv] ~ N(0, 1)
 Per-head decays are the multi-scale schedules gamma_h = 1 - 2^(-5-h) and
 gamma_h = 1 - 2^(-5-h/3), h = 0..H-1, rounded to fp32.
 """
@@ -98,6 +102,25 @@ def config_inputs(cfg: RetConfig, seed: int | None = None, N: int | None = None,
     else:
         out["gamma"] = gammas(cfg.H, cfg.gamma_schedule)
     return out
+
+
+def output_grad(B: int, H: int, N: int, dv: int, dtype=torch.bfloat16, seed: int = 0) -> torch.Tensor:
+    """Output gradient dO [B, H, N, dv] ~ N(0, 1) / sqrt(dv) (seed + 104729), cast to dtype."""
+    g = _gen(seed + 104729)
+    return (torch.randn(B, H, N, dv, generator=g) / math.sqrt(dv)).to(dtype)
+
+
+def retention_output(B: int, H: int, N: int, dv: int, dtype=torch.bfloat16, seed: int = 0) -> torch.Tensor:
+    """Stand-in retention output o [B, H, N, dv]: N(0, 1) times e^z per row, z ~ N(0, 1) (seed + 7211)."""
+    g = _gen(seed + 7211)
+    x = torch.randn(B, H, N, dv, generator=g)
+    return (x * torch.exp(torch.randn(B, H, N, 1, generator=g))).to(dtype)
+
+
+def gate_projection(B: int, H: int, N: int, dv: int, dtype=torch.bfloat16, seed: int = 0) -> torch.Tensor:
+    """Gate projection output [B, N, H, dv] ~ N(0, 1) (seed + 9049), token-major."""
+    g = _gen(seed + 9049)
+    return torch.randn(B, N, H, dv, generator=g).to(dtype)
 
 
 def decode_state(B: int, H: int, dk: int, dv: int, seed: int = 0) -> torch.Tensor:

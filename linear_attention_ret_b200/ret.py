@@ -29,7 +29,8 @@ SYMBOLS = ("ret_parallel", "ret_chunkwise", "ret_recurrent_step", "gated_ret_chu
            "ret_last_device_error", "ret_chunkwise_path", "ret_chunkwise_launches", "ret_version",
            "ret_chunkwise_noalloc", "ret_selftest_wait_timeout", "gated_ret_recurrent_step",
            "ret_chunkwise_state", "gated_ret_chunkwise_state", "ret_state_prefix", "ret_chunkwise_state_launches",
-           "ret_chunkwise_backward", "gated_ret_chunkwise_backward")
+           "ret_chunkwise_backward", "gated_ret_chunkwise_backward", "ret_chunkwise_backward_launches",
+           "ret_msr_norm_gate")
 
 _lock = threading.Lock()
 _lib = None
@@ -65,6 +66,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
         lib.gated_ret_chunkwise_state.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
         lib.ret_state_prefix.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
         lib.ret_chunkwise_state_launches.argtypes = [_i, _i, _i, _i, _i, _i, _i]
+        lib.ret_chunkwise_backward_launches.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i, _i]
+        lib.ret_msr_norm_gate.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, ctypes.c_float, _i, _vp]
+        lib.ret_msr_norm_gate.restype = _i
         for fn in ("ret_chunkwise_backward", "gated_ret_chunkwise_backward"):
             getattr(lib, fn).argtypes = [_vp] * 9 + [_i] * 7 + [_vp]
             getattr(lib, fn).restype = _i
@@ -232,6 +236,23 @@ def chunkwise_backward(q, k, v, decay, dout, chunk, gated=False, ddecay=True, st
     return dq, dkk, dvv, dd
 
 
+def msr_norm_gate(o, gate, eps: float = 1e-5, y=None, stream=None):
+    """Multi-scale retention output epilogue: y[b, n, h] = swish(gate[b, n, h]) * RMSNorm(o[b, h, n])
+    over dv (no affine weights). o [B, H, N, dv]; gate [B, N, H, dv] (same dtype);
+    returns y [B, N, H, dv] (may be `gate` itself for an in-place update)."""
+    B, H, N, dv = o.shape
+    if tuple(gate.shape) != (B, N, H, dv):
+        raise ValueError(f"gate must be [B, N, H, dv] = {(B, N, H, dv)}, got {tuple(gate.shape)}")
+    if y is None:
+        y = torch.empty_like(gate)
+    if gate.dtype != o.dtype or y.dtype != o.dtype or tuple(y.shape) != tuple(gate.shape):
+        raise ValueError("o, gate and y must share one dtype; y has gate's shape")
+    _cuda(o, gate, y)
+    _check("ret_msr_norm_gate", load().ret_msr_norm_gate(_ptr(o), _ptr(gate), _ptr(y), B, H, N, dv, float(eps), _dt(o),
+                                                         _stream(stream)))
+    return y
+
+
 def last_device_error(stream=None) -> int:
     return int(load().ret_last_device_error(_stream(stream)))
 
@@ -248,6 +269,13 @@ def chunkwise_launches(B: int, H: int, N: int, dk: int, dv: int, chunk: int, dty
 def chunkwise_state_launches(B: int, H: int, N: int, dk: int, dv: int, chunk: int, dtype: torch.dtype) -> int:
     return int(load().ret_chunkwise_state_launches(B, H, N, dk, dv, chunk,
                                                    RET_BF16 if dtype == torch.bfloat16 else RET_F32))
+
+
+def chunkwise_backward_launches(B: int, H: int, N: int, dk: int, dv: int, chunk: int, dtype: torch.dtype,
+                                gated: bool = False, ddecay: bool = True) -> int:
+    return int(load().ret_chunkwise_backward_launches(B, H, N, dk, dv, chunk,
+                                                      RET_BF16 if dtype == torch.bfloat16 else RET_F32,
+                                                      int(gated), int(ddecay)))
 
 
 def chunkwise_path(dk: int, dv: int, chunk: int, dtype: torch.dtype) -> int:
