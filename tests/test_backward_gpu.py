@@ -82,3 +82,22 @@ def test_backward_gradient_of_forward_by_directional_derivative(cuda_lib):
     fd = (loss(eps) - loss(-eps)) / (2 * eps)
     an = sum(float((g.double().cpu() * e.double()).sum()) for g, e in zip((dq, dkk, dvv), dirs))
     assert abs(fd - an) <= 1e-3 * abs(an), (fd, an)
+
+
+def test_backward_full_size_sampled_heads(cuda_lib):
+    """The 1.3B-shaped workload (B4 H8 N2048 dk256 dv512) as bench.py times it; the oracle
+    computes head 7 of every batch element (its dgamma sums over the batch) and head 0
+    of batch element 0, each by definition."""
+    cfg = I.CONFIGS["retnet_1p3b"]
+    x = I.config_inputs(cfg, seed=0)
+    do = I.output_grad(cfg.B, cfg.H, cfg.N, cfg.dv, cfg.dtype, seed=0)
+    dq, dkk, dvv, dgam = cuda_lib.chunkwise_backward(*(x[n].to(DEV) for n in ("q", "k", "v", "gamma")),
+                                                     do.to(DEV), cfg.chunk)
+    assert cuda_lib.last_device_error() == 0
+    for h, bs in ((7, range(cfg.B)), (0, range(1))):
+        sel = lambda t: t[list(bs), h:h + 1]
+        want = O.ret_backward(sel(x["q"]), sel(x["k"]), sel(x["v"]), x["gamma"][h:h + 1], sel(do))
+        for got, ref, what in zip((dq, dkk, dvv), want[:3], ("dq", "dk", "dv")):
+            _check(sel(got.cpu()), ref, cfg.dtype, f"{what} head {h}")
+        if h == 7:
+            _check(dgam[h:h + 1], want[3], cfg.dtype, "dgamma head 7", tol=5e-2)
