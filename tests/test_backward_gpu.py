@@ -20,6 +20,8 @@ BWD_CASES = [
     (1, 2, 200, 128, 128, torch.bfloat16),   # tensor-core path
     (1, 2, 257, 256, 512, torch.bfloat16),   # dv = 512: the dq/dk contraction in two pieces
     (2, 1, 64, 64, 128, torch.bfloat16),
+    (1, 2, 130, 64, 512, torch.bfloat16),   # dv pieces copied out (value width 64 is off the tensor-core path)
+    (1, 1, 70, 32, 300, torch.float32),     # fp32 pieces of 256 and a ragged 44
 ]
 
 
