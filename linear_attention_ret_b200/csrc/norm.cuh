@@ -56,10 +56,16 @@ template <> struct Vec16<__nv_bfloat16> {
     }
 };
 
-// swish(x) = x / (1 + e^-x) with the fast exponential and divide. The fast exponential's
-// documented error is 2 + 1.17|x| ulp, under 1e-5 relative for |x| < 80; an e^-x that
-// overflows to infinity gives -0, the limit.
-__device__ __forceinline__ float swish(float x) { return __fdividef(x, 1.f + __expf(-x)); }
+// swish(x) = x / (1 + e^-x) = x * rcp(1 + 2^(-x log2 e)) with the hardware ex2 and rcp
+// (flush-to-zero forms; relative errors about 2^-22 and 1 ulp): five instructions. The
+// flushes only touch e^-x below 2^-126 (where 1 + e^-x rounds to 1 anyway) and results
+// below 2^-126 in magnitude (x < -87, where swish(x) is under 1e-36).
+__device__ __forceinline__ float swish(float x) {
+    float e, r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-x * kLog2e));
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.f + e));
+    return x * r;
+}
 
 // Source row of o and destination row of y for token-major row index r = (b N + n) H + h.
 __device__ __forceinline__ void norm_rows(size_t r, int H, int N, size_t& o_row, size_t& y_row) {
