@@ -624,6 +624,8 @@ def cpu_baseline(spec, budget_s: float = 12.0):
     el = time.perf_counter() - t0
     value = units * reps / el
     what = "decode steps" if spec["kind"] == "decode" else f"{cfg.N} tokens"
+    if spec["kind"] == "norm":
+        heads = total_heads  # the epilogue sample is the whole workload
     return {"value": round(value, 3), "unit": spec["unit"], "cores": threads, "kind": "oracle",
             "sample": f"{reps} run(s) of the fp64 oracle on {heads} of {total_heads} (b,h) heads x {what} "
                       f"({el:.1f} s wall, OpenMP over heads)",
@@ -658,6 +660,8 @@ def run_reference(args, spec):
     el = time.perf_counter() - t0
     value = units * args.steps / el
     what = "decode steps" if spec["kind"] == "decode" else f"{cfg.N} tokens"
+    if spec["kind"] == "norm":
+        heads = cfg.B * cfg.H  # the epilogue sample is the whole workload
     sample = (f"each step: fp64 oracle on {heads} of {cfg.B * cfg.H} (b,h) heads x {what}, "
               f"OpenMP over heads")
     line = {"impl": "reference", "metric": spec["metric"], "value": round(value, 4), "unit": spec["unit"],

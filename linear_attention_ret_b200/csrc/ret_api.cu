@@ -187,11 +187,16 @@ inline AuxStream* aux_stream() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
     AuxStream& a = aux[dev];
-    if (!a.s) {
-        if (cudaStreamCreateWithFlags(&a.s, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
-        if (cudaEventCreateWithFlags(&a.fork, cudaEventDisableTiming) != cudaSuccess ||
-            cudaEventCreateWithFlags(&a.join, cudaEventDisableTiming) != cudaSuccess)
+    if (!a.s) {  // publish the stream only once its events exist too
+        AuxStream n;
+        if (cudaStreamCreateWithFlags(&n.s, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+        if (cudaEventCreateWithFlags(&n.fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&n.join, cudaEventDisableTiming) != cudaSuccess) {
+            if (n.fork) cudaEventDestroy(n.fork);
+            cudaStreamDestroy(n.s);
             return nullptr;
+        }
+        a = n;
     }
     return &a;
 }
@@ -541,8 +546,9 @@ int ret_chunkwise_state_launches(int B, int H, int N, int dk, int dv, int chunk,
 
 ret_status ret_msr_norm_gate(const void* o, const void* gate, void* y, int B, int H, int N, int dv, float eps,
                              ret_dtype dt, void* stream) {
-    ret_status s = check_common(B, H, N, 1, dv, dt);
-    if (s != RET_OK) return s;
+    if (dt != RET_F32 && dt != RET_BF16) return RET_ERR_DTYPE;
+    // the kernels stride over rows, so B * H has no grid limit here
+    if (B <= 0 || H <= 0 || N < 0 || dv <= 0) return RET_ERR_SHAPE;
     if (!(eps >= 0.f) || !std::isfinite(eps)) return RET_ERR_SHAPE;
     if (N == 0) return RET_OK;
     if (!o || !gate || !y) return RET_ERR_NULL;

@@ -36,6 +36,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <utility>
+
 #include "common.cuh"
 
 namespace ret {
@@ -334,6 +336,10 @@ template <int DK, bool GATED, bool STATE_ONLY>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, Params p) {
+    // Launched as a programmatic dependent of the previous kernel in the stream: the CTAs
+    // may be placed while that kernel drains, and wait here until it has completed and its
+    // writes are visible, before any global memory is touched.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     // Heads with gamma close to 1 take the 128-token body (tc_wide.cuh); the choice is per
     // CTA, so one launch serves a mix of heads.
     if constexpr (wide_capable(DK, GATED, STATE_ONLY)) {
@@ -1064,6 +1070,24 @@ constexpr int kernel_smem() {
         return Layout<DK>::kSmemAlloc;
 }
 
+// Launches a tensor-core kernel with programmatic stream serialization: its CTAs may start
+// while the previous kernel in the stream finishes, and wait (griddepcontrol.wait, the
+// kernel's first instruction) until that kernel has completed.
+template <typename... P, typename... A>
+inline cudaError_t launch_dependent(void (*kernel)(P...), dim3 grid, size_t smem, cudaStream_t st, A&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
+}
+
 template <int DK, bool GATED>
 ret_status launch_dk(const void* q, const void* k, const void* v, const float* decay, void* o,
                      const float* state_in, float* state_out, int B, int H, int N, int dv, const Plan& pl,
@@ -1091,8 +1115,8 @@ ret_status launch_dk(const void* q, const void* k, const void* v, const float* d
             return RET_ERR_CUDA;
         Params prm1 = prm;  // the state-only pass runs over the sub-segments
         prm1.seg_chunks = pl.seg_chunks / pl.F;
-        k1<<<dim3(dv / kDvS, BH, pl.subs()), kThreads, smem1, st>>>(mq, mk, mv, mo, prm1);
-        if (cudaGetLastError() != cudaSuccess) return RET_ERR_CUDA;
+        if (launch_dependent(k1, dim3(dv / kDvS, BH, pl.subs()), smem1, st, mq, mk, mv, mo, prm1) != cudaSuccess)
+            return RET_ERR_CUDA;
         const int n4 = BH * DK * dv / 4;
         seg_prefix_kernel<<<std::min((n4 + 255) / 256, 4 * sm_count()), 256, 0, st>>>(
             prm.state_in, prm.seg_state, prm.seg_ldec, pl.subs() + 1, BH, DK * dv);
@@ -1102,8 +1126,8 @@ ret_status launch_dk(const void* q, const void* k, const void* v, const float* d
     constexpr int smem2 = kernel_smem<DK, GATED, false>();
     if (cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2) != cudaSuccess)
         return RET_ERR_CUDA;
-    k2<<<dim3(dv / kDvS, BH, pl.G), kThreads, smem2, st>>>(mq, mk, mv, mo, prm);
-    return cudaGetLastError() == cudaSuccess ? RET_OK : RET_ERR_CUDA;
+    return launch_dependent(k2, dim3(dv / kDvS, BH, pl.G), smem2, st, mq, mk, mv, mo, prm) == cudaSuccess ? RET_OK
+                                                                                                     : RET_ERR_CUDA;
 }
 
 // Runs the tensor-core path with caller-provided scratch (at least scratch_bytes()).
@@ -1180,8 +1204,8 @@ ret_status launch_state_dk(const void* k, const void* v, const float* decay, flo
     constexpr int smem1 = kernel_smem<DK, GATED, true>();
     if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1) != cudaSuccess)
         return RET_ERR_CUDA;
-    k1<<<dim3(dv / kDvS, BH, subs), kThreads, smem1, st>>>(mk, mk, mv, mv, prm);
-    if (cudaGetLastError() != cudaSuccess) return RET_ERR_CUDA;
+    if (launch_dependent(k1, dim3(dv / kDvS, BH, subs), smem1, st, mk, mk, mv, mv, prm) != cudaSuccess)
+        return RET_ERR_CUDA;
     if (subs > 1) {
         const int n4 = BH * DK * dv / 4;
         seg_prefix_kernel<<<std::min((n4 + 255) / 256, 4 * sm_count()), 256, 0, st>>>(nullptr, states, ldec, subs + 1,
