@@ -74,3 +74,57 @@ def test_parallel_and_step_validation(lib):
     assert lib.ret_recurrent_step(None, None, None, None, None, None, 1, 1, 8, 8, 0, None) == 1
     assert lib.ret_recurrent_step(None, None, None, None, None, None, 1, 1, 5000, 8, 0, None) == 4
     assert lib.ret_recurrent_step(None, None, None, None, None, None, 1, 1, 8, 8, 2, None) == 3
+
+
+@pytest.mark.parametrize("fn", ["ret_chunkwise_backward", "gated_ret_chunkwise_backward"])
+def test_backward_validation(lib, fn):
+    def call(B=1, H=1, N=8, dk=64, dv=64, chunk=64, dt=1):
+        return getattr(lib, fn)(*([None] * 9), B, H, N, dk, dv, chunk, dt, None)
+    assert call(B=0) == 2
+    assert call(N=-3) == 2
+    assert call(chunk=0) == 2
+    assert call(dt=9) == 3
+    assert call(dk=512) == 4
+    assert call() == 1  # NULL tensors
+
+
+def test_backward_launch_count_validation(lib):
+    f = lib.ret_chunkwise_backward_launches
+    assert f(0, 1, 8, 64, 64, 64, 1, 0, 1) == -1
+    assert f(1, 1, 8, 300, 64, 64, 1, 0, 1) == -1
+    assert f(1, 1, 0, 64, 64, 64, 1, 0, 1) == 0
+    n_fixed, n_gated = f(1, 2, 100, 32, 40, 64, 0, 0, 1), f(1, 2, 100, 32, 40, 64, 0, 1, 1)
+    assert n_fixed > 0 and n_gated == n_fixed + 2  # the reversed gates and the gate-gradient suffix sum
+    assert f(1, 2, 100, 32, 40, 64, 0, 0, 0) == n_fixed - 1  # no decay gradient
+
+
+def test_norm_gate_validation(lib):
+    import ctypes
+    f = lib.ret_msr_norm_gate
+    p = lambda x: ctypes.c_void_p(x)
+    args = lambda o, g, y, B=1, H=2, N=8, dv=64, eps=1e-5, dt=1: (o, g, y, B, H, N, dv, eps, dt, None)
+    assert f(*args(None, None, None, dt=4)) == 3
+    assert f(*args(None, None, None, B=0)) == 2
+    assert f(*args(None, None, None, dv=0)) == 2
+    assert f(*args(None, None, None, eps=-1.0)) == 2
+    assert f(*args(None, None, None, eps=float("nan"))) == 2
+    assert f(*args(None, None, None, N=0)) == 0  # empty: nothing to do, nothing launched
+    assert f(*args(None, None, None)) == 1
+    # overlaps are rejected before any launch (the addresses are never dereferenced)
+    base = 1 << 40
+    nbytes = 1 * 2 * 8 * 64 * 2
+    assert f(*args(p(base), p(base + 4 * nbytes), p(base + 64))) == 4           # y inside o
+    assert f(*args(p(base), p(base + 4 * nbytes), p(base + 4 * nbytes + 32))) == 4  # y inside gate, not gate
+
+
+def test_bindings_refuse_host_tensors(lib):
+    """The product path has no CPU fallback: host tensors are refused before the library is called."""
+    import torch
+    from linear_attention_ret_b200 import ret
+    q = torch.zeros(1, 1, 4, 8)
+    with pytest.raises(ValueError):
+        ret.chunkwise_backward(q, q, q, torch.ones(1), q, 64)
+    with pytest.raises(ValueError):
+        ret.msr_norm_gate(q, torch.zeros(1, 4, 1, 8))
+    with pytest.raises(ValueError):
+        ret.ret_chunkwise(q, q, q, torch.ones(1), 64)
