@@ -170,30 +170,37 @@ ret_status decay_grad(const T* q, const T* dq, const T* k, const T* dk, const fl
 
 inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
-// A second stream per device, with fork and join events, for the pieces of a dv
-// contraction that run side by side. Held under the mutex from fork to join, so calls
-// from several host threads do not interleave their events.
-struct AuxStream {
-    cudaStream_t s = nullptr;
-    cudaEvent_t fork = nullptr, join = nullptr;
+// Two library streams per device, with events, for the steps of the backward that run side
+// by side. Held under the mutex from the first fork to the last join, so calls from several
+// host threads do not interleave their events.
+constexpr int kAuxEvents = 7;
+struct AuxStreams {
+    cudaStream_t s[2] = {nullptr, nullptr};
+    cudaEvent_t ev[kAuxEvents] = {};
 };
 constexpr int kMaxDevices = 64;
 inline std::mutex& aux_mutex() {
     static std::mutex m;
     return m;
 }
-inline AuxStream* aux_stream() {
-    static AuxStream aux[kMaxDevices];
+inline void destroy_aux(AuxStreams& n) {
+    for (cudaEvent_t e : n.ev)
+        if (e) cudaEventDestroy(e);
+    for (cudaStream_t x : n.s)
+        if (x) cudaStreamDestroy(x);
+}
+inline AuxStreams* aux_streams() {
+    static AuxStreams aux[kMaxDevices];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    AuxStream& a = aux[dev];
-    if (!a.s) {  // publish the stream only once its events exist too
-        AuxStream n;
-        if (cudaStreamCreateWithFlags(&n.s, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
-        if (cudaEventCreateWithFlags(&n.fork, cudaEventDisableTiming) != cudaSuccess ||
-            cudaEventCreateWithFlags(&n.join, cudaEventDisableTiming) != cudaSuccess) {
-            if (n.fork) cudaEventDestroy(n.fork);
-            cudaStreamDestroy(n.s);
+    AuxStreams& a = aux[dev];
+    if (!a.s[0]) {  // publish only once every stream and event exists
+        AuxStreams n;
+        bool ok = true;
+        for (cudaStream_t& x : n.s) ok = ok && cudaStreamCreateWithFlags(&x, cudaStreamNonBlocking) == cudaSuccess;
+        for (cudaEvent_t& e : n.ev) ok = ok && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
+        if (!ok) {
+            destroy_aux(n);
             return nullptr;
         }
         a = n;
@@ -210,6 +217,107 @@ inline bool backward_pieces_in_place(int dk, int dv, int chunk, ret_dtype dt) {
     return true;
 }
 
+// The backward on the tensor-core path with dv in pieces read in place, as a small graph of
+// steps on the caller's stream st and two library streams s1, s2:
+//   st: dQ piece 0 | wait s1 -> dq = sum of the dQ pieces | wait s2 -> dV forward, reverse -> | wait s2 -> dgamma/dg
+//   s1: dQ piece 1 |                  wait s2 (reversals) -> dK piece 1 ------------------------>|
+//   s2: reversed Q, K, V, dO (and gates) -> dK piece 0 | wait s1 -> dk = reverse(sum of dK pieces)
+// (more pieces alternate between the two streams of their row). The reversals run beside the
+// dQ pieces and the dV forward beside the dK pieces, filling the SMs each leaves idle.
+template <typename T, bool GATED>
+ret_status backward_concurrent(const void* q, const void* k, const void* v, const float* decay, const void* dout,
+                               void* dq, void* dk_out, void* dv_out, float* ddecay, int B, int H, int N, int dk, int dv,
+                               int chunk, ret_dtype dt, cudaStream_t st) {
+    const int BH = B * H;
+    const size_t nQ = (size_t)BH * N * dk, nV = (size_t)BH * N * dv;
+    const int pw = 256, P = (dv + pw - 1) / pw;
+    // scratch: reversed Q, K, V, dO; dQ pieces; dK pieces; reversed dV; reversed gates
+    size_t off[8], bytes = 0;
+    const size_t sz[8] = {nQ * sizeof(T), nQ * sizeof(T), nV * sizeof(T), nV * sizeof(T), (size_t)P * nQ * sizeof(T),
+                          (size_t)P * nQ * sizeof(T), nV * sizeof(T), GATED ? (size_t)BH * N * sizeof(float) : 0};
+    for (int i = 0; i < 8; ++i) {
+        off[i] = bytes;
+        bytes += align256(sz[i]);
+    }
+    tc::keep_pool_memory();
+    uint8_t* sc = nullptr;
+    if (cudaMallocAsync(reinterpret_cast<void**>(&sc), bytes, st) != cudaSuccess) return RET_ERR_CUDA;
+    T* Qf = reinterpret_cast<T*>(sc + off[0]);
+    T* Kf = reinterpret_cast<T*>(sc + off[1]);
+    T* Vf = reinterpret_cast<T*>(sc + off[2]);
+    T* dOf = reinterpret_cast<T*>(sc + off[3]);
+    T* partsQ = reinterpret_cast<T*>(sc + off[4]);
+    T* partsK = reinterpret_cast<T*>(sc + off[5]);
+    T* Rf = reinterpret_cast<T*>(sc + off[6]);
+    float* gf = reinterpret_cast<float*>(sc + off[7]);
+    const float* dec_rev = GATED ? gf : decay;
+
+    ret_status r = RET_OK;
+    auto ok = [&](ret_status x) { if (r == RET_OK) r = x; return r == RET_OK; };
+    auto cu = [&](cudaError_t e) { return ok(e == cudaSuccess ? RET_OK : RET_ERR_CUDA); };
+    std::lock_guard<std::mutex> lock(aux_mutex());
+    AuxStreams* a = aux_streams();
+    if (!a) {
+        cudaFreeAsync(sc, st);
+        return RET_ERR_CUDA;
+    }
+    cudaStream_t s1 = a->s[0], s2 = a->s[1];
+    cudaEvent_t ev_fork = a->ev[0], ev_dq = a->ev[1], ev_rev = a->ev[2], ev_dk1 = a->ev[3], ev_dk = a->ev[4],
+                ev_j1 = a->ev[5], ev_j2 = a->ev[6];
+    auto piece = [&](const void* x, const void* y, const void* z, const float* dec, T* fo, int p, cudaStream_t s) {
+        const int c0 = p * pw, w = std::min(pw, dv - c0);
+        return ok(tc_chunk_launch<GATED>(static_cast<const T*>(x) + c0, static_cast<const T*>(y) + c0, z, dec,
+                                         fo + (size_t)p * nQ, nullptr, nullptr, B, H, N, w, dk, s, dv, dv, 2));
+    };
+    // fork
+    if (cu(cudaEventRecord(ev_fork, st))) {
+        cu(cudaStreamWaitEvent(s1, ev_fork, 0));
+        cu(cudaStreamWaitEvent(s2, ev_fork, 0));
+    }
+    // dQ = forward(dO, V, K) in pieces on st and s1; the reversals on s2
+    for (int p = 0; p < P && r == RET_OK; ++p) piece(dout, v, k, decay, partsQ, p, p % 2 ? s1 : st);
+    if (r == RET_OK) {
+        ok(slice_flip<T>(q, Qf, BH, N, dk, 0, dk, true, s2)) && ok(slice_flip<T>(k, Kf, BH, N, dk, 0, dk, true, s2)) &&
+            ok(slice_flip<T>(v, Vf, BH, N, dv, 0, dv, true, s2)) &&
+            ok(slice_flip<T>(dout, dOf, BH, N, dv, 0, dv, true, s2));
+        if (GATED && r == RET_OK) {
+            gate_flip_kernel<<<grid_for((size_t)BH * N), kBwdThreads, 0, s2>>>(decay, gf, N, (size_t)BH * N);
+            ok(launch_status());
+        }
+    }
+    if (r == RET_OK) cu(cudaEventRecord(ev_rev, s2));
+    // dq on st, once s1's pieces are done
+    if (r == RET_OK && cu(cudaEventRecord(ev_dq, s1)) && cu(cudaStreamWaitEvent(st, ev_dq, 0)))
+        ok(sum_flip<T>(partsQ, P, nQ, static_cast<T*>(dq), BH, N, dk, false, st));
+    // dK = reverse(forward(rev V, rev dO, rev Q)) in pieces on s2 and s1, after the reversals
+    if (r == RET_OK) cu(cudaStreamWaitEvent(s1, ev_rev, 0));
+    for (int p = 0; p < P && r == RET_OK; ++p) piece(Vf, dOf, Qf, dec_rev, partsK, p, p % 2 ? s1 : s2);
+    // dV = reverse(forward(rev K, rev Q, rev dO)) on st, beside the dK pieces
+    if (r == RET_OK && cu(cudaStreamWaitEvent(st, ev_rev, 0)) &&
+        ok(chunkwise_entry<GATED>(Kf, Qf, dOf, dec_rev, Rf, nullptr, nullptr, B, H, N, dk, dv, chunk, dt, st)))
+        ok(slice_flip<T>(Rf, dv_out, BH, N, dv, 0, dv, true, st));
+    // dk on s2 once s1's pieces are done
+    if (r == RET_OK && cu(cudaEventRecord(ev_dk1, s1)) && cu(cudaStreamWaitEvent(s2, ev_dk1, 0)) &&
+        ok(sum_flip<T>(partsK, P, nQ, static_cast<T*>(dk_out), BH, N, dk, true, s2)))
+        cu(cudaEventRecord(ev_dk, s2));
+    // decay gradient on st, after dq (st) and dk (s2)
+    if (r == RET_OK && ddecay && cu(cudaStreamWaitEvent(st, ev_dk, 0)))
+        ok(decay_grad<T, GATED>(static_cast<const T*>(q), static_cast<const T*>(dq), static_cast<const T*>(k),
+                                static_cast<const T*>(dk_out), decay, ddecay, BH, H, N, dk, st));
+    // join both library streams back into st whatever happened, then release the scratch on st
+    const bool joined = cudaEventRecord(ev_j1, s1) == cudaSuccess && cudaEventRecord(ev_j2, s2) == cudaSuccess &&
+                        cudaStreamWaitEvent(st, ev_j1, 0) == cudaSuccess &&
+                        cudaStreamWaitEvent(st, ev_j2, 0) == cudaSuccess;
+    if (!joined) {
+        // the library streams could not be ordered before st: wait for them before freeing
+        cudaStreamSynchronize(s1);
+        cudaStreamSynchronize(s2);
+        ok(RET_ERR_CUDA);
+    }
+    if (cudaFreeAsync(sc, st) != cudaSuccess) ok(RET_ERR_CUDA);
+    return r;
+}
+
 template <typename T, bool GATED>
 ret_status backward_impl(const void* q, const void* k, const void* v, const float* decay, const void* dout, void* dq,
                          void* dk_out, void* dv_out, float* ddecay, int B, int H, int N, int dk, int dv, int chunk,
@@ -218,11 +326,13 @@ ret_status backward_impl(const void* q, const void* k, const void* v, const floa
     const size_t nQ = (size_t)BH * N * dk, nV = (size_t)BH * N * dv;
     const int pw = dv <= 256 ? dv : 256;  // width of one piece of the dv contraction
     const int P = (dv + pw - 1) / pw;
-    const bool in_place = backward_pieces_in_place(dk, dv, chunk, dt);
+    if (backward_pieces_in_place(dk, dv, chunk, dt))
+        return backward_concurrent<T, GATED>(q, k, v, decay, dout, dq, dk_out, dv_out, ddecay, B, H, N, dk, dv, chunk,
+                                             dt, st);
     // scratch: reversed Q, K, V, dO; two piece buffers; per-piece outputs; reversed dV; reversed gates
     size_t off[9], bytes = 0;
     const size_t sz[9] = {nQ * sizeof(T), nQ * sizeof(T), nV * sizeof(T), nV * sizeof(T),
-                          in_place ? 0 : (size_t)BH * N * pw * sizeof(T), in_place ? 0 : (size_t)BH * N * pw * sizeof(T),
+                          P > 1 ? (size_t)BH * N * pw * sizeof(T) : 0, P > 1 ? (size_t)BH * N * pw * sizeof(T) : 0,
                           (size_t)P * nQ * sizeof(T),
                           nV * sizeof(T), GATED ? (size_t)BH * N * sizeof(float) : 0};
     for (int i = 0; i < 9; ++i) {
@@ -246,33 +356,15 @@ ret_status backward_impl(const void* q, const void* k, const void* v, const floa
     auto fwd = [&](const void* fq, const void* fk, const void* fv, const float* dec, void* fo, int wq, int wv) {
         return ok(chunkwise_entry<GATED>(fq, fk, fv, dec, fo, nullptr, nullptr, B, H, N, wq, wv, chunk, dt, st));
     };
-    // All pieces of a dv contraction: forward(a[:, c0:c0+w], b[:, c0:c0+w], c) into parts[p],
-    // a and b dv wide. In place, odd pieces run on the second stream beside the even ones
-    // (each launch then sized for the SMs it shares); otherwise each piece is copied out.
+    // All pieces of a dv contraction, copied out first: forward(a[:, c0:c0+w], b[:, c0:c0+w], c)
+    // into parts[p], a and b dv wide.
     auto pieces = [&](const void* a, const void* b, const void* c, const float* dec) {
-        if (!in_place) {
-            for (int p = 0; p < P && r == RET_OK; ++p) {
-                const int c0 = p * pw, w = std::min(pw, dv - c0);
-                ok(slice_flip<T>(a, pa, BH, N, dv, c0, w, false, st)) &&
-                    ok(slice_flip<T>(b, pb, BH, N, dv, c0, w, false, st)) &&
-                    fwd(pa, pb, c, dec, parts + (size_t)p * nQ, w, dk);
-            }
-            return r == RET_OK;
-        }
-        std::lock_guard<std::mutex> lock(aux_mutex());
-        AuxStream* aux = aux_stream();
-        if (!aux) return ok(RET_ERR_CUDA);
-        if (cudaEventRecord(aux->fork, st) != cudaSuccess || cudaStreamWaitEvent(aux->s, aux->fork, 0) != cudaSuccess)
-            return ok(RET_ERR_CUDA);
         for (int p = 0; p < P && r == RET_OK; ++p) {
             const int c0 = p * pw, w = std::min(pw, dv - c0);
-            ok(tc_chunk_launch<GATED>(static_cast<const T*>(a) + c0, static_cast<const T*>(b) + c0, c, dec,
-                                      parts + (size_t)p * nQ, nullptr, nullptr, B, H, N, w, dk, p % 2 ? aux->s : st,
-                                      dv, dv, 2));
+            ok(slice_flip<T>(a, pa, BH, N, dv, c0, w, false, st)) &&
+                ok(slice_flip<T>(b, pb, BH, N, dv, c0, w, false, st)) &&
+                fwd(pa, pb, c, dec, parts + (size_t)p * nQ, w, dk);
         }
-        // join even on failure, so the second stream never runs past this call
-        if ((cudaEventRecord(aux->join, aux->s) != cudaSuccess || cudaStreamWaitEvent(st, aux->join, 0) != cudaSuccess))
-            ok(RET_ERR_CUDA);
         return r == RET_OK;
     };
     // dQ = forward(dO, V, K), the dv contraction in pieces

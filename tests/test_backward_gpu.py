@@ -103,3 +103,16 @@ def test_backward_full_size_sampled_heads(cuda_lib):
             _check(sel(got.cpu()), ref, cfg.dtype, f"{what} head {h}")
         if h == 7:
             _check(dgam[h:h + 1], want[3], cfg.dtype, "dgamma head 7", tol=5e-2)
+
+
+@pytest.mark.parametrize("gated", [False, True])
+def test_backward_without_decay_gradient(cuda_lib, gated):
+    """ddecay=False: the same dq, dk, dv (the tensor-core path with dv in pieces)."""
+    q, k, v, do, gen = _case(1, 2, 190, 256, 512, torch.bfloat16, seed=21)
+    decay = I.gate(1, 2, 190, gen) * 4.0 if gated else torch.tensor([0.97, 0.9])
+    d = [t.to(DEV) for t in (q, k, v, decay, do)]
+    full = cuda_lib.chunkwise_backward(*d, 64, gated=gated)
+    part = cuda_lib.chunkwise_backward(*d, 64, gated=gated, ddecay=False)
+    assert part[3] is None
+    for a, b in zip(full[:3], part[:3]):
+        assert torch.equal(a, b)
