@@ -10,11 +10,13 @@
  *        块级循环 (chunkwise recurrent form: parallel inside a chunk, state
  *        passed between chunks).
  *   [RN] 171host.com, "Retentive Network (RetNet) 详解": section 3.1 (the three
- *        equivalent forms) and 3.2 (multi-scale retention: one gamma per head).
+ *        equivalent forms) and 3.2 (multi-scale retention: one gamma per head,
+ *        plus a gate and a normalisation).
  *   [GR] pwwt.cn, "unilm RetNet 技术指南 ... Gated RetNet 的源码解析": the gated
  *        form with a per-token, per-head log-decay g (parallel_gate_retention,
  *        chunk_gate_retention = cross_chunk + inner_chunk,
- *        recurrent_gate_retention).
+ *        recurrent_gate_retention), and the GateRetention module (subln, an
+ *        RMSNorm over the head dimension; g_proj feeding a swish gate).
  *
  * Conventions shared by every entry point
  *   - Pointers are DEVICE pointers owned by the caller. The library never frees
@@ -27,9 +29,14 @@
  *   - No 1/sqrt(dk) scale is applied: callers pass pre-scaled q or k.
  *   - Calls are asynchronous on `stream` (a cudaStream_t cast to void*;
  *     NULL = the legacy default stream). Arguments are validated on the host
- *     before anything is launched; a non-RET_OK status means nothing ran.
+ *     before anything is launched: a validation status (RET_ERR_NULL, _SHAPE,
+ *     _DTYPE, _UNSUPPORTED, _ALIGN, _SCRATCH) means nothing ran. RET_ERR_CUDA
+ *     from a call that launches several kernels may follow some of them; the
+ *     outputs are then undefined.
  *   - Errors are returned, never raised: no exit(), no device trap.
- *   - Calls keep no state between calls and are safe from several host threads.
+ *   - Calls keep no per-call state (the library holds only per-device helpers
+ *     it creates once: the no-allocation scratch buffer, and two streams with
+ *     their events for the backward) and are safe from several host threads.
  *   - N == 0 is a valid empty problem: nothing is launched, state_out (if
  *     given) receives state_in (or zeros).
  */
