@@ -684,8 +684,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="retnet_1p3b",
-                    choices=["retnet_1p3b", "retnet_6p7b_long", "gated", "decode", "gated_decode", "seqpar_6p7b",
-                             "backward_1p3b", "msr_norm_1p3b", "retention_msr_1p3b"])
+                    choices=list(WORKLOAD_KERNELS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

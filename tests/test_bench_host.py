@@ -39,7 +39,8 @@ def test_every_workload_has_sources_and_a_cli_choice():
         for f in bench.KERNEL_SOURCES[group]:
             assert os.path.exists(os.path.join(csrc, f)), f
         assert len(bench.kernel_source_sha(w)) == 16
-    # every workload is accepted on the command line
+    # the command line accepts exactly these workloads, and each has its arithmetic
+    assert sorted(bench.WORKLOAD_KERNELS) == sorted(WORKLOADS)
     for w in WORKLOADS:
         spec = bench.workload(w)
         assert spec["unit"] in ("tokens/s", "steps/s") and spec["bytes"] > 0
