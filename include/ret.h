@@ -246,7 +246,7 @@ RET_API ret_status ret_state_prefix(const float* seg_states, const float* seg_lo
                             int R, int B, int H, int dk, int dv, void* stream);
 
 /*
- * Self-test of the failure path (the paper has no counterpart; a diagnostic).
+ * Self-test of the failure path (the pages have no counterpart; a diagnostic).
  * Launches one CTA on `stream` that takes tensor memory as the tensor-core
  * kernels do, waits on an mbarrier that nothing completes with the kernels'
  * bounded wait limited to limit_us microseconds (1 .. 1,000,000), sets the
@@ -273,7 +273,7 @@ RET_API int ret_chunkwise_path(int dk, int dv, int chunk, ret_dtype dt);
 RET_API int ret_chunkwise_launches(int B, int H, int N, int dk, int dv, int chunk, ret_dtype dt);
 
 /*
- * ret_chunkwise without any device allocation. The paper has no counterpart for
+ * ret_chunkwise without any device allocation. The pages have no counterpart for
  * this entry point: it is an interface for callers, not part of the method.
  *
  * ret_chunkwise may take stream-ordered scratch from the device's default
