@@ -1,0 +1,99 @@
+"""The factorisations the tensor-core kernel's fixed-decay bodies compute with, modelled in
+fp64 and checked against the oracle's chunkwise form ("RetNet retention mechanism" page,
+section 块级循环):
+
+128-token body (gamma >= 2^-0.75): with zeta_m = gamma^(L-1-m) over a tile of L tokens and
+the state held as S = kappa T (a scalar kappa and a matrix T),
+    kappa <- kappa gamma^L                         (the decay of the carried state, on the scalar)
+    o_j    = (kappa / zeta_j) [ q_j T + sum_{m<=j} (q_j . k_m) zeta_m v_m / kappa ]
+    T     <- T + sum_m zeta_m k_m^T v_m / kappa
+and T is rescaled (T <- kappa T, kappa <- 1) when kappa falls below 2^-40.
+
+64-token merged accumulator (gamma in [1/2, 1]): with zeta'_j = gamma^(63-j),
+    gamma^(j-m) = zeta'_m / zeta'_j  and  gamma^(j+1) = gamma^64 / zeta'_j,
+so o_j = (1/zeta'_j) [ q_j (gamma^64 S) + sum_{m<=j} zeta'_m (q_j . k_m) v_m ] over 64-token chunks
+(a ragged last chunk is zero padding: its rows past the end contribute nothing).
+"""
+import numpy as np
+import pytest
+
+from oracle import oracle as O
+
+
+def _tile_model_128(q, k, v, gamma, renorm=2.0 ** -40):
+    N = q.shape[0]
+    T = np.zeros((q.shape[1], v.shape[1]))
+    kappa = 1.0
+    out = np.zeros((N, v.shape[1]))
+    for t0 in range(0, N, 128):
+        L = min(128, N - t0)
+        qs, ks, vs = q[t0:t0 + L], k[t0:t0 + L], v[t0:t0 + L]
+        zeta = gamma ** (L - 1 - np.arange(L))
+        if kappa * gamma ** L < renorm:
+            T, kappa = kappa * T, 1.0
+        kappa *= gamma ** L
+        A = np.tril(qs @ ks.T)
+        zv = zeta[:, None] * vs / kappa
+        out[t0:t0 + L] = (kappa / zeta)[:, None] * (qs @ T + A @ zv)
+        T = T + ks.T @ zv
+    return out, kappa * T
+
+
+def _merged_model_64(q, k, v, gamma):
+    N = q.shape[0]
+    S = np.zeros((q.shape[1], v.shape[1]))
+    zp = gamma ** (63 - np.arange(64))
+    out = np.zeros((N, v.shape[1]))
+    for t0 in range(0, N, 64):
+        L = min(64, N - t0)
+        qs = np.zeros((64, q.shape[1])); ks = np.zeros((64, k.shape[1])); vs = np.zeros((64, v.shape[1]))
+        qs[:L], ks[:L], vs[:L] = q[t0:t0 + L], k[t0:t0 + L], v[t0:t0 + L]  # zero padding past the end
+        P = np.tril(qs @ ks.T) * zp[None, :]
+        acc = qs @ (gamma ** 64 * S) + P @ vs
+        out[t0:t0 + L] = (acc / zp[:, None])[:L]
+        # the state update over the chunk's true length L: S <- gamma^L S + sum gamma^(L-1-m) k_m^T v_m
+        w = gamma ** (L - 1 - np.arange(L))
+        S = gamma ** L * S + (ks[:L] * w[:, None]).T @ vs[:L]
+    return out, S
+
+
+@pytest.mark.parametrize("gamma", [0.999, 0.96875, 2.0 ** -0.75])
+@pytest.mark.parametrize("N", [128, 300, 517])
+def test_128_token_factorisation_equals_chunkwise(gamma, N):
+    rng = np.random.default_rng(N)
+    q, k, v = (rng.standard_normal((N, d)) / 3 for d in (6, 6, 5))
+    o, s = _tile_model_128(q, k, v, gamma)
+    want_o, want_s = O.ret_chunkwise(q[None, None], k[None, None], v[None, None], np.array([gamma]), 128)
+    np.testing.assert_allclose(o, want_o[0, 0], rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(s, want_s[0, 0], rtol=1e-9, atol=1e-11)
+
+
+def test_128_token_rescaling_keeps_the_result():
+    """A sequence long enough that kappa crosses 2^-40 several times (gamma^128 = 2^-96 per tile)."""
+    gamma, N = 2.0 ** -0.75, 1000
+    rng = np.random.default_rng(3)
+    q, k, v = (rng.standard_normal((N, 4)) for _ in range(3))
+    o, s = _tile_model_128(q, k, v, gamma)
+    want_o, want_s = O.ret_chunkwise(q[None, None], k[None, None], v[None, None], np.array([gamma]), 64)
+    np.testing.assert_allclose(o, want_o[0, 0], rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(s, want_s[0, 0], rtol=1e-9, atol=1e-11)
+
+
+@pytest.mark.parametrize("gamma", [0.5, 0.75, 0.999])
+@pytest.mark.parametrize("N", [64, 100, 257])
+def test_64_token_merged_accumulator_equals_chunkwise(gamma, N):
+    rng = np.random.default_rng(N + 7)
+    q, k, v = (rng.standard_normal((N, d)) / 3 for d in (6, 6, 5))
+    o, s = _merged_model_64(q, k, v, gamma)
+    want_o, want_s = O.ret_chunkwise(q[None, None], k[None, None], v[None, None], np.array([gamma]), 64)
+    np.testing.assert_allclose(o, want_o[0, 0], rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(s, want_s[0, 0], rtol=1e-9, atol=1e-11)
+
+
+def test_merged_factors_stay_in_range():
+    """For gamma in [1/2, 1] every factor of the merged 64-token form lies in [2^-64, 2^63],
+    inside the normal range of bf16 and fp32."""
+    for gamma in (0.5, 0.6, 0.9, 1.0):
+        zp = gamma ** (63 - np.arange(64))
+        factors = np.concatenate([zp, 1 / zp, [gamma ** 64]])
+        assert factors.min() >= 2.0 ** -64 and factors.max() <= 2.0 ** 63
