@@ -13,11 +13,12 @@ v and o [B, H, N, dv], states [B, H, dk, dv] fp32, bf16 or fp32 inputs):
 * ``ret.ret_recurrent_step`` / ``ret.gated_ret_recurrent_step``: one decode step,
   updating the state in place.
 * ``ret.ret_parallel``: the parallel form, for checking.
-* ``ret.chunkwise_backward``: dq, dk, dv and dgamma (or dg) of either chunkwise form.
+* ``ret.chunkwise_backward``: dq, dk, dv and dgamma (or dg) of either chunkwise form;
+  ``autograd.chunkwise_retention`` wraps forward and backward as a differentiable torch op.
 * ``ret.msr_norm_gate``: the output epilogue, swish(gate) * per-head RMSNorm(o),
   token-major.
 * ``ret.chunkwise_state`` and ``ret.state_prefix``: segment end states and start
   states for a sequence split across calls or GPUs; ``seqpar.sequence_parallel_chunkwise``
   runs the whole split over a torch.distributed group.
 """
-__all__ = ["ret", "inputs", "build", "seqpar"]
+__all__ = ["ret", "inputs", "build", "seqpar", "autograd"]

@@ -116,15 +116,67 @@ def _stream(stream):
 
 
 def _cuda(*ts):
+    dev = None
     for t in ts:
-        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+        if t is None:
+            continue
+        if not t.is_cuda or not t.is_contiguous():
             raise ValueError("tensors must be contiguous CUDA tensors")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"tensors must be on one device, got {dev} and {t.device}")
+
+
+def _expect(name, t, shape, dtype=None):
+    """Shape (and dtype) every tensor must have given the leading one, checked before any
+    pointer reaches the library: a wrong size there would read past an allocation."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _rank(name, t, n):
+    if t.dim() != n:
+        raise ValueError(f"{name} must have {n} dimensions, got shape {tuple(t.shape)}")
+
+
+def _seq_args(q, k, v, decay, gated, o=None, state_in=None, state_out=None):
+    """q, k [B, H, N, dk]; v, o [B, H, N, dv] (q's dtype); gamma [H] or g [B, H, N] fp32;
+    states [B, H, dk, dv] fp32. Returns (B, H, N, dk, dv)."""
+    _rank("q", q, 4)
+    _rank("v", v, 4)
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    _expect("k", k, (B, H, N, dk), q.dtype)
+    _expect("v", v, (B, H, N, dv), q.dtype)
+    _expect("g" if gated else "gamma", decay, (B, H, N) if gated else (H,), torch.float32)
+    _expect("o", o, (B, H, N, dv), q.dtype)
+    _expect("state_in", state_in, (B, H, dk, dv), torch.float32)
+    _expect("state_out", state_out, (B, H, dk, dv), torch.float32)
+    return B, H, N, dk, dv
+
+
+def _step_args(q, k, v, decay, state, o, gated):
+    """q, k [B, H, dk]; v, o [B, H, dv]; gamma [H] or g [B, H] fp32; state [B, H, dk, dv] fp32."""
+    _rank("q", q, 3)
+    _rank("v", v, 3)
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    _expect("k", k, (B, H, dk), q.dtype)
+    _expect("v", v, (B, H, dv), q.dtype)
+    _expect("g" if gated else "gamma", decay, (B, H) if gated else (H,), torch.float32)
+    _expect("state", state, (B, H, dk, dv), torch.float32)
+    _expect("o", o, (B, H, dv), q.dtype)
+    return B, H, dk, dv
 
 
 def ret_parallel(q, k, v, gamma, o=None, stream=None):
     """O = (Q K^T (.) D) V. Returns o [B, H, N, dv] (dtype of q)."""
-    B, H, N, dk = q.shape
-    dv = v.shape[-1]
+    B, H, N, dk, dv = _seq_args(q, k, v, gamma, False, o)
     o = torch.empty(B, H, N, dv, dtype=q.dtype, device=q.device) if o is None else o
     _cuda(q, k, v, gamma, o)
     _check("ret_parallel", load().ret_parallel(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(o),
@@ -134,8 +186,7 @@ def ret_parallel(q, k, v, gamma, o=None, stream=None):
 
 def ret_chunkwise(q, k, v, gamma, chunk, state_in=None, state_out=None, o=None, stream=None):
     """Chunkwise retention. Returns o; writes the final state into state_out if given."""
-    B, H, N, dk = q.shape
-    dv = v.shape[-1]
+    B, H, N, dk, dv = _seq_args(q, k, v, gamma, False, o, state_in, state_out)
     o = torch.empty(B, H, N, dv, dtype=q.dtype, device=q.device) if o is None else o
     _cuda(q, k, v, gamma, o, state_in, state_out)
     _check("ret_chunkwise", load().ret_chunkwise(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(o),
@@ -147,8 +198,7 @@ def ret_chunkwise(q, k, v, gamma, chunk, state_in=None, state_out=None, o=None, 
 def ret_chunkwise_noalloc(q, k, v, gamma, chunk, state_in=None, state_out=None, o=None, stream=None):
     """ret_chunkwise without device allocation by the library: scratch comes from a
     fixed 16 MiB buffer inside libret.so (see include/ret.h). Returns o."""
-    B, H, N, dk = q.shape
-    dv = v.shape[-1]
+    B, H, N, dk, dv = _seq_args(q, k, v, gamma, False, o, state_in, state_out)
     o = torch.empty(B, H, N, dv, dtype=q.dtype, device=q.device) if o is None else o
     _cuda(q, k, v, gamma, o, state_in, state_out)
     _check("ret_chunkwise_noalloc", load().ret_chunkwise_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(o),
@@ -159,8 +209,7 @@ def ret_chunkwise_noalloc(q, k, v, gamma, chunk, state_in=None, state_out=None, 
 
 def gated_ret_chunkwise(q, k, v, g, chunk, state_in=None, state_out=None, o=None, stream=None):
     """Gated chunkwise retention (per-token log-decay g). Returns o."""
-    B, H, N, dk = q.shape
-    dv = v.shape[-1]
+    B, H, N, dk, dv = _seq_args(q, k, v, g, True, o, state_in, state_out)
     o = torch.empty(B, H, N, dv, dtype=q.dtype, device=q.device) if o is None else o
     _cuda(q, k, v, g, o, state_in, state_out)
     _check("gated_ret_chunkwise", load().gated_ret_chunkwise(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(o),
@@ -171,8 +220,7 @@ def gated_ret_chunkwise(q, k, v, g, chunk, state_in=None, state_out=None, o=None
 
 def ret_recurrent_step(q, k, v, gamma, state, o=None, stream=None):
     """One decode step; updates state [B, H, dk, dv] in place and returns o [B, H, dv]."""
-    B, H, dk = q.shape
-    dv = v.shape[-1]
+    B, H, dk, dv = _step_args(q, k, v, gamma, state, o, False)
     o = torch.empty(B, H, dv, dtype=q.dtype, device=q.device) if o is None else o
     _cuda(q, k, v, gamma, state, o)
     _check("ret_recurrent_step", load().ret_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(state),
@@ -182,8 +230,7 @@ def ret_recurrent_step(q, k, v, gamma, state, o=None, stream=None):
 
 def gated_ret_recurrent_step(q, k, v, g, state, o=None, stream=None):
     """One gated decode step with log-decay g [B, H] (fp32); updates state in place, returns o [B, H, dv]."""
-    B, H, dk = q.shape
-    dv = v.shape[-1]
+    B, H, dk, dv = _step_args(q, k, v, g, state, o, True)
     o = torch.empty(B, H, dv, dtype=q.dtype, device=q.device) if o is None else o
     _cuda(q, k, v, g, state, o)
     _check("gated_ret_recurrent_step", load().gated_ret_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g),
@@ -195,8 +242,8 @@ def gated_ret_recurrent_step(q, k, v, g, state, o=None, stream=None):
 def chunkwise_state(k, v, decay, chunk, gated=False, state_out=None, log2_decay=None, stream=None):
     """End state U [B, H, dk, dv] of a segment from a zero start and log2 of its total decay
     [B, H] (decay: gamma [H], or g [B, H, N] with gated=True). Returns (U, log2_decay)."""
-    B, H, N, dk = k.shape
-    dv = v.shape[-1]
+    B, H, N, dk, dv = _seq_args(k, k, v, decay, gated, None, None, state_out)
+    _expect("log2_decay", log2_decay, (B, H), torch.float32)
     state_out = torch.empty(B, H, dk, dv, dtype=torch.float32, device=k.device) if state_out is None else state_out
     log2_decay = torch.empty(B, H, dtype=torch.float32, device=k.device) if log2_decay is None else log2_decay
     _cuda(k, v, decay, state_out, log2_decay)
@@ -209,7 +256,11 @@ def chunkwise_state(k, v, decay, chunk, gated=False, state_out=None, log2_decay=
 def state_prefix(seg_states, seg_log2_decay, state_in=None, stream=None):
     """Start states [R, B, H, dk, dv] of R consecutive segments and the state after all of
     them, from their end states U [R, B, H, dk, dv] and log2 decays [R, B, H]."""
+    _rank("seg_states", seg_states, 5)
     R, B, H, dk, dv = seg_states.shape
+    _expect("seg_states", seg_states, (R, B, H, dk, dv), torch.float32)
+    _expect("seg_log2_decay", seg_log2_decay, (R, B, H), torch.float32)
+    _expect("state_in", state_in, (B, H, dk, dv), torch.float32)
     starts = torch.empty_like(seg_states)
     end = torch.empty(B, H, dk, dv, dtype=torch.float32, device=seg_states.device)
     _cuda(seg_states, seg_log2_decay, state_in, starts, end)
@@ -222,8 +273,8 @@ def chunkwise_backward(q, k, v, decay, dout, chunk, gated=False, ddecay=True, st
     """Gradients of sum(dout * o) for o = ret_chunkwise(q, k, v, decay) (gated=True:
     gated_ret_chunkwise with g = decay) from a zero initial state. Returns
     (dq, dk, dv, ddecay) with ddecay = dgamma [H] or dg [B, H, N] (fp32), or None."""
-    B, H, N, dk = q.shape
-    dv = v.shape[-1]
+    B, H, N, dk, dv = _seq_args(q, k, v, decay, gated)
+    _expect("dout", dout, (B, H, N, dv), q.dtype)
     dq, dkk, dvv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     dd = None
     if ddecay:
@@ -240,6 +291,7 @@ def msr_norm_gate(o, gate, eps: float = 1e-5, y=None, stream=None):
     """Multi-scale retention output epilogue: y[b, n, h] = swish(gate[b, n, h]) * RMSNorm(o[b, h, n])
     over dv (no affine weights). o [B, H, N, dv]; gate [B, N, H, dv] (same dtype);
     returns y [B, N, H, dv] (may be `gate` itself for an in-place update)."""
+    _rank("o", o, 4)
     B, H, N, dv = o.shape
     if tuple(gate.shape) != (B, N, H, dv):
         raise ValueError(f"gate must be [B, N, H, dv] = {(B, N, H, dv)}, got {tuple(gate.shape)}")
