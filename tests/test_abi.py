@@ -128,3 +128,15 @@ def test_bindings_refuse_host_tensors(lib):
         ret.msr_norm_gate(q, torch.zeros(1, 4, 1, 8))
     with pytest.raises(ValueError):
         ret.ret_chunkwise(q, q, q, torch.ones(1), 64)
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """No fallback: without libret.so every call raises instead of computing anything on the host."""
+    import torch
+    from linear_attention_ret_b200 import ret
+    monkeypatch.setattr(ret, "_lib", None)
+    monkeypatch.setattr(ret, "LIB_PATH", str(tmp_path / "absent" / "libret.so"))
+    with pytest.raises(RuntimeError, match="libret.so not found"):
+        ret.load()
+    with pytest.raises(RuntimeError, match="libret.so not found"):
+        ret.chunkwise_launches(1, 1, 8, 64, 64, 64, torch.bfloat16)
