@@ -416,6 +416,7 @@ def run_ours(args, spec):
     line = {
         "metric": spec["metric"], "value": round(value, 2), "unit": spec["unit"], "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "ms_per_step_median": round(statistics.median(per_step), 5),  # this rank's CUDA-event times per step
         "higher_is_better": True, "scaling": "strong" if strong else "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1)/sqrt(dk); " + ("one sequence split across ranks)" if strong
                                                         else "per-rank seeds)"),
@@ -430,6 +431,8 @@ def run_ours(args, spec):
         "gpu_launches": args.steps * launches,
         "launches_per_step": launches,
     }
+    if spec["kind"] == "decode":
+        line["ms_per_1024_steps"] = round(1024 * ms_per_step, 3)  # a 1024-token generation
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(spec, budget_s=args.cpu_seconds)
     if rank == 0:
@@ -607,13 +610,8 @@ def _oracle_sample_step(spec, heads, seed=0):
     return run, heads * cfg.N / cfg.H  # tokens (all heads of a token count once)
 
 
-def cpu_baseline(spec, budget_s: float = 12.0):
-    from oracle import oracle as O
-    threads = O.max_threads()
-    cfg = spec["cfg"]
-    total_heads = cfg.B * cfg.H
-    heads = min(total_heads, threads)
-    run, units = _oracle_sample_step(spec, heads)
+def _time_oracle(run, budget_s):
+    """Runs `run` at least once and until about budget_s seconds; returns (reps, seconds)."""
     t0 = time.perf_counter()
     run()
     t = time.perf_counter() - t0
@@ -621,14 +619,38 @@ def cpu_baseline(spec, budget_s: float = 12.0):
     while time.perf_counter() - t0 + t <= budget_s and reps < 64:
         run()
         reps += 1
-    el = time.perf_counter() - t0
+    return reps, time.perf_counter() - t0
+
+
+def cpu_baseline(spec, budget_s: float = 12.0, single_budget_s: float = 4.0):
+    """The fp64 oracle on the host cores (OpenMP over heads) on a bounded sample, plus the
+    same oracle on one thread and one head for the per-core figure."""
+    from oracle import oracle as O
+    threads = O.max_threads()
+    cfg = spec["cfg"]
+    total_heads = cfg.B * cfg.H
+    heads = min(total_heads, threads)
+    run, units = _oracle_sample_step(spec, heads)
+    reps, el = _time_oracle(run, budget_s)
     value = units * reps / el
     what = "decode steps" if spec["kind"] == "decode" else f"{cfg.N} tokens"
-    if spec["kind"] == "norm":
-        heads = total_heads  # the epilogue sample is the whole workload
+    covered = lambda n: (total_heads if spec["kind"] == "norm"  # the epilogue sample is the whole workload
+                         else max(1, -(-n // cfg.H)) * cfg.H if spec["kind"] == "decode"  # whole batch rows
+                         else n)
+    heads = covered(heads)
+    O.set_threads(1)
+    try:
+        run1, units1 = _oracle_sample_step(spec, 1)
+        reps1, el1 = _time_oracle(run1, single_budget_s)
+    finally:
+        O.set_threads(threads)
+    heads1 = covered(1)
     return {"value": round(value, 3), "unit": spec["unit"], "cores": threads, "kind": "oracle",
             "sample": f"{reps} run(s) of the fp64 oracle on {heads} of {total_heads} (b,h) heads x {what} "
                       f"({el:.1f} s wall, OpenMP over heads)",
+            "single_thread": {"value": round(units1 * reps1 / el1, 3), "unit": spec["unit"], "cores": 1,
+                              "sample": f"{reps1} run(s) on {heads1} of {total_heads} (b,h) heads x {what} "
+                                        f"({el1:.1f} s wall, one thread)"},
             "cpu": _cpu_model()}
 
 
