@@ -97,3 +97,60 @@ def test_merged_factors_stay_in_range():
         zp = gamma ** (63 - np.arange(64))
         factors = np.concatenate([zp, 1 / zp, [gamma ** 64]])
         assert factors.min() >= 2.0 ** -64 and factors.max() <= 2.0 ** 63
+
+
+# ---------------------------------------------------------------- anti-causal tiles (a reversed kernel)
+#
+# The backward's dK and dV are anti-causal sums, R_m = sum_{n>=m} w_nm (a_m . b_n) c_n (dV: a=k, b=q, c=dO;
+# dK: a=v, b=dO, c=q). Without reversing the sequence in memory they can be computed over the forward's
+# tiles visited from the last to the first, carrying S' = sum over later tokens of w b_n^T c_n:
+#   fixed gamma, a tile of L tokens, local index j:  row factor gamma^(L-j), key weight gamma^i,
+#       state decay gamma^L, intra weights gamma^(i-j) for i >= j (upper triangle);
+#   gated:  row factor exp(sum of g over (j, L-1]), key weight exp(sum of g over [0, i]),
+#       state decay exp(sum of g over the tile), intra weights exp(sum of g over (j, i]).
+
+def _anticausal_model(a, b, c, tile, gamma=None, g=None):
+    N = a.shape[0]
+    S = np.zeros((b.shape[1], c.shape[1]))
+    out = np.zeros((N, c.shape[1]))
+    starts = list(range(0, N, tile))
+    for t0 in reversed(starts):
+        L = min(tile, N - t0)
+        A, Bm, C = a[t0:t0 + L], b[t0:t0 + L], c[t0:t0 + L]
+        idx = np.arange(L)
+        if g is None:
+            row = gamma ** (L - idx)
+            key = gamma ** idx
+            decay = gamma ** L
+            W = np.where(idx[None, :] >= idx[:, None], gamma ** np.maximum(idx[None, :] - idx[:, None], 0), 0.0)
+        else:
+            gl = g[t0:t0 + L]
+            inc = np.cumsum(gl)                      # sum over [0, i]
+            row = np.exp(inc[-1] - inc)              # sum over (j, L-1]
+            key = np.exp(inc)
+            decay = np.exp(inc[-1])
+            W = np.where(idx[None, :] >= idx[:, None], np.exp(inc[None, :] - inc[:, None]), 0.0)
+        scores = (A @ Bm.T) * W                      # [j, i]: (a_j . b_i) w_ji for i >= j
+        out[t0:t0 + L] = scores @ C + row[:, None] * (A @ S)
+        S = decay * S + (Bm * key[:, None]).T @ C
+    return out
+
+
+@pytest.mark.parametrize("N,tile", [(128, 64), (300, 64), (517, 128), (77, 128)])
+@pytest.mark.parametrize("gated", [False, True])
+def test_anticausal_tiles_give_dk_and_dv(N, tile, gated):
+    rng = np.random.default_rng(N + tile)
+    q, k = rng.standard_normal((N, 5)), rng.standard_normal((N, 5))
+    v, do = rng.standard_normal((N, 6)), rng.standard_normal((N, 6))
+    if gated:
+        g = -np.abs(rng.standard_normal(N)) / 4
+        want = O.gated_backward(q[None, None], k[None, None], v[None, None], g[None, None], do[None, None])
+        dv = _anticausal_model(k, q, do, tile, g=g)
+        dk = _anticausal_model(v, do, q, tile, g=g)
+    else:
+        gamma = 0.97
+        want = O.ret_backward(q[None, None], k[None, None], v[None, None], np.array([gamma]), do[None, None])
+        dv = _anticausal_model(k, q, do, tile, gamma=gamma)
+        dk = _anticausal_model(v, do, q, tile, gamma=gamma)
+    np.testing.assert_allclose(dv, want[2][0, 0], rtol=1e-9, atol=1e-10)
+    np.testing.assert_allclose(dk, want[1][0, 0], rtol=1e-9, atol=1e-10)
