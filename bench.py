@@ -1,10 +1,13 @@
 #!/usr/bin/env python
 """Throughput benchmark of the B200 retention library.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--also A,B] [--impl ours|reference]
 
-One step is one call of the hot path on one batch of seeded synthetic input
-already resident in HBM:
+With no --workload the line's top-level figures are retnet_1p3b's and the line
+carries a "workloads" object with one sub-record each for decode,
+retnet_6p7b_long and gated, measured the same way (own timed region, roofline,
+e2e, clocks and CPU baseline). One step is one call of the hot path on one
+batch of seeded synthetic input already resident in HBM:
   retnet_1p3b       (default) ret_chunkwise, B=4 H=8 N=2048 dk=256 dv=512 chunk 64, bf16
   retnet_6p7b_long  ret_chunkwise, B=1 H=16 N=8192 dk=256 dv=512 chunk 128, bf16
   gated             gated_ret_chunkwise, B=2 H=8 N=16384 dk=dv=128 chunk 64, bf16
@@ -342,6 +345,117 @@ def launches_per_call(spec) -> int:
     return ret.chunkwise_launches(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk, cfg.dtype)
 
 
+DTYPE_NAMES = {"torch.bfloat16": "bf16", "torch.float32": "f32"}
+
+# Workloads measured beside the headline one in the default line (each as a sub-record
+# with its own roofline, e2e, clocks and CPU baseline): the recurrent decode step, the
+# 6.7B-shaped long sequence and the gated form.
+DEFAULT_ALSO = ("decode", "retnet_6p7b_long", "gated")
+
+
+def dtype_name(cfg) -> str:
+    """The arithmetic type of the inputs and outputs (accumulation and state are fp32)."""
+    return DTYPE_NAMES[str(cfg.dtype)]
+
+
+def measure(args, name, spec, dev, stream, world, steps, cpu_budget):
+    """One workload on this rank: warm-up, clock-sampled burn-in, K timed steps (CUDA
+    events on the launch stream, max over ranks), then the end-to-end figure. Returns
+    the record rank 0 prints (every rank takes the same collective steps)."""
+    import torch
+    from linear_attention_ret_b200 import ret
+    rank = dist_env()[0]
+    step, x, o, launches = make_step(spec, dev, rank_seed(rank))
+    # nvidia-smi samples every 100 ms while a timed region lasts milliseconds, so sampling
+    # starts before the warm-up and an untimed burn-in keeps the same load for about a
+    # second; the samples then describe the clocks the timed region runs at.
+    clocks = ClockSampler(gpu_uuid(dev.index))
+    clocks.start()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    err = ret.last_device_error()
+    if err != 0:
+        raise SystemExit(f"{name}: device error word set after warm-up: {err}")
+    t_burn = time.perf_counter()
+    while time.perf_counter() - t_burn < args.burn_in:
+        for _ in range(10):
+            step()
+        torch.cuda.synchronize()
+
+    # timed region: K steps, barrier + synchronize on both sides, events per step on the launch stream
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    barrier(world, dev)
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for i in range(steps):
+        step()
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    clk = clocks.stop()
+    per_step = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+    total_ms = ev[0].elapsed_time(ev[-1])
+    max_ms = max_over_ranks(total_ms, world, dev)
+    if ret.last_device_error() != 0:
+        raise SystemExit(f"{name}: device error word set in the timed region")
+    del x, o
+    e2e = run_e2e(args, spec, dev, stream, world)
+
+    ms_per_step = max_ms / steps
+    strong = spec["kind"] == "seqpar"  # one sequence split across the ranks
+    if spec["kind"] == "decode":
+        value = world * 1e3 / ms_per_step
+    else:
+        value = spec["units"] * (1 if strong else world) / (ms_per_step / 1e3)
+    hbm, tf_burst, tf_sust, peak_src = measured_peaks()
+    # the step's mean duration on this rank: a step is one launch of the dominant kernel
+    # (plus, for split sequences, two short launches whose share the ncu launch list records)
+    kern_ms = statistics.mean(per_step)
+    achieved = spec["bytes"] / (kern_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "traffic": ncu_traffic(name),
+                "traffic_note": "dram__bytes_read.sum + dram__bytes_write.sum per step from one ncu capture "
+                                "(null unless the kernel sources are unchanged since); the write count misses "
+                                "output rows still in L2 when the kernel ends",
+                "algorithmic_bytes": spec["bytes"],
+                "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs, copy)" if peak_src == "measured"
+                else "fallback 6.65 TB/s",
+                "kernel_ms": round(kern_ms, 5),
+                "scope": ("the whole step: " + str(launches) + " launches (five calls of the forward kernel, "
+                          "slice/flip/sum copies, the decay gradient)") if spec["kind"] == "backward"
+                else "the step's launches",
+                "tensor_tflops": round(spec["flops"] / (kern_ms / 1e3) / 1e12, 2),
+                "tensor_frac_of_bf16_burst": round(spec["flops"] / (kern_ms / 1e3) / 1e12 / tf_burst, 4),
+                "tensor_frac_of_bf16_sustained": round(spec["flops"] / (kern_ms / 1e3) / 1e12 / tf_sust, 4)}
+    cfg = spec["cfg"]
+    rec = {
+        "metric": spec["metric"], "value": round(value, 2), "unit": spec["unit"], "n_gpus": world,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "ms_per_step_median": round(statistics.median(per_step), 5),  # this rank's CUDA-event times per step
+        "higher_is_better": True, "scaling": "strong" if strong else "weak", "vs_baseline": None,
+        "dtype": dtype_name(cfg),
+        "data": "synthetic (seeded N(0,1)/sqrt(dk); " + ("one sequence split across ranks)" if strong
+                                                        else "per-rank seeds)"),
+        "config": {"workload": name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "dk": cfg.dk, "dv": cfg.dv,
+                   "chunk": cfg.chunk, "state": "fp32", "accumulate": "fp32",
+                   "l2": f"working set {spec['bytes'] / 1e6:.0f} MB per step > 126 MB L2 (no flush)",
+                   "parallelism": (f"sequence-parallel x{world} (one all-gather of segment states)" if strong
+                                   else f"batch-sharded x{world}") if world > 1 else "single GPU"},
+        "roofline": roofline,
+        "clocks": dict(clk, window="warm-up, ~1 s untimed burn-in and the timed region") if clk else None,
+        "e2e": e2e,
+        "gpu_launches": steps * launches,
+        "launches_per_step": launches,
+    }
+    if spec["kind"] == "decode":
+        rec["ms_per_1024_steps"] = round(1024 * ms_per_step, 3)  # a 1024-token generation
+        rec["tokens_per_s"] = round(world * cfg.B * 1e3 / ms_per_step, 1)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rec["cpu_baseline"] = cpu_baseline(spec, budget_s=cpu_budget, single_budget_s=max(1.0, cpu_budget / 3))
+    return rec
+
+
 def run_ours(args, spec):
     import torch
     rank, world, local = dist_env()
@@ -354,87 +468,15 @@ def run_ours(args, spec):
     ret.load()
     stream = torch.cuda.current_stream(dev)
 
-    step, x, o, launches = make_step(spec, dev, rank_seed(rank))
-    # nvidia-smi samples every 100 ms while a timed region lasts milliseconds, so sampling
-    # starts before the warm-up and an untimed burn-in keeps the same load for about a
-    # second; the samples then describe the clocks the timed region runs at.
-    clocks = ClockSampler(gpu_uuid(local))
-    clocks.start()
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    err = ret.last_device_error()
-    if err != 0:
-        raise SystemExit(f"device error word set after warm-up: {err}")
-    t_burn = time.perf_counter()
-    while time.perf_counter() - t_burn < args.burn_in:
-        for _ in range(10):
-            step()
-        torch.cuda.synchronize()
-
-    # timed region: K steps, barrier + synchronize on both sides, events per step on the launch stream
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
-    barrier(world, dev)
-    torch.cuda.synchronize()
-    ev[0].record(stream)
-    for i in range(args.steps):
-        step()
-        ev[i + 1].record(stream)
-    torch.cuda.synchronize()
-    barrier(world, dev)
-    clk = clocks.stop()
-    per_step = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
-    total_ms = ev[0].elapsed_time(ev[-1])
-    max_ms = max_over_ranks(total_ms, world, dev)
-    if ret.last_device_error() != 0:
-        raise SystemExit("device error word set in the timed region")
-
-    e2e = run_e2e(args, spec, dev, stream, world)
-
-    ms_per_step = max_ms / args.steps
-    strong = spec["kind"] == "seqpar"  # one sequence split across the ranks
-    if spec["kind"] == "decode":
-        value = world * 1e3 / ms_per_step
-    else:
-        value = spec["units"] * (1 if strong else world) / (ms_per_step / 1e3)
-    hbm, tf_burst, tf_sust, peak_src = measured_peaks()
-    # the dominant kernel's duration: a step is one launch of it (plus, for split
-    # sequences, two short launches whose share the ncu launch list records)
-    kern_ms = statistics.mean(per_step)
-    achieved = spec["bytes"] / (kern_ms / 1e3) / 1e9
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                "frac": round(achieved / hbm, 4), "traffic": ncu_traffic(args.workload),
-                "peak_source": peak_src + " (MEASURED_PEAKS.json hbm_gbs, copy)" if peak_src == "measured"
-                else "fallback 6.65 TB/s",
-                "kernel_ms": round(kern_ms, 5),
-                "scope": ("the whole step: " + str(launches) + " launches (five calls of the forward kernel, "
-                          "slice/flip/sum copies, the decay gradient)") if spec["kind"] == "backward"
-                else "the step's launches",
-                "tensor_tflops": round(spec["flops"] / (kern_ms / 1e3) / 1e12, 2),
-                "tensor_frac_of_bf16_burst": round(spec["flops"] / (kern_ms / 1e3) / 1e12 / tf_burst, 4)}
-    cfg = spec["cfg"]
-    line = {
-        "metric": spec["metric"], "value": round(value, 2), "unit": spec["unit"], "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
-        "ms_per_step_median": round(statistics.median(per_step), 5),  # this rank's CUDA-event times per step
-        "higher_is_better": True, "scaling": "strong" if strong else "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1)/sqrt(dk); " + ("one sequence split across ranks)" if strong
-                                                        else "per-rank seeds)"),
-        "config": {"workload": args.workload, "B": cfg.B, "H": cfg.H, "N": cfg.N, "dk": cfg.dk, "dv": cfg.dv,
-                   "chunk": cfg.chunk, "state": "fp32",
-                   "l2": f"working set {spec['bytes'] / 1e6:.0f} MB per step > 126 MB L2 (no flush)",
-                   "parallelism": (f"sequence-parallel x{world} (one all-gather of segment states)" if strong
-                                   else f"batch-sharded x{world}") if world > 1 else "single GPU"},
-        "roofline": roofline,
-        "clocks": dict(clk, window="warm-up, ~1 s untimed burn-in and the timed region") if clk else None,
-        "e2e": e2e,
-        "gpu_launches": args.steps * launches,
-        "launches_per_step": launches,
-    }
-    if spec["kind"] == "decode":
-        line["ms_per_1024_steps"] = round(1024 * ms_per_step, 3)  # a 1024-token generation
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(spec, budget_s=args.cpu_seconds)
+    line = measure(args, args.workload, spec, dev, stream, world, args.steps, args.cpu_seconds)
+    also = [w for w in args.also if w != args.workload]
+    if also:
+        # the other headline workloads, each measured the same way, as sub-records of this line
+        line["workloads"] = {}
+        for name in also:
+            sub = measure(args, name, workload(name), dev, stream, world, args.steps, args.cpu_seconds / 2)
+            line["workloads"][name] = sub
+            torch.cuda.empty_cache()
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -705,8 +747,12 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="retnet_1p3b",
-                    choices=list(WORKLOAD_KERNELS))
+    ap.add_argument("--workload", default=None, choices=list(WORKLOAD_KERNELS),
+                    help="one workload (default: retnet_1p3b, with decode, retnet_6p7b_long and gated "
+                         "as sub-records of the same line)")
+    ap.add_argument("--also", default=None,
+                    help="comma-separated workloads measured as sub-records of the line "
+                         "(default: none with --workload, else " + ",".join(DEFAULT_ALSO) + ")")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -715,6 +761,15 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.also is None:
+        args.also = [] if args.workload else list(DEFAULT_ALSO)
+    else:
+        args.also = [w for w in args.also.split(",") if w]
+        for w in args.also:
+            if w not in WORKLOAD_KERNELS:
+                ap.error(f"--also: unknown workload {w!r}")
+    if args.workload is None:
+        args.workload = "retnet_1p3b"
     spec = workload(args.workload)
     if args.impl == "reference":
         run_reference(args, spec)

@@ -36,7 +36,9 @@
  *   - Errors are returned, never raised: no exit(), no device trap.
  *   - Calls keep no per-call state (the library holds only per-device helpers
  *     it creates once: the no-allocation scratch buffer, and two streams with
- *     their events for the backward) and are safe from several host threads.
+ *     their events for the backward) and are safe from several host threads,
+ *     except ret_chunkwise_noalloc, whose calls all share one scratch buffer:
+ *     calls of it that overlap on the GPU race (see its declaration).
  *   - N == 0 is a valid empty problem: nothing is launched, state_out (if
  *     given) receives state_in (or zeros).
  */
@@ -288,7 +290,10 @@ RET_API int ret_chunkwise_launches(int B, int H, int N, int dk, int dv, int chun
  *
  *  - The first call on a device, with that device current, looks up the
  *    buffer's device address (cudaGetSymbolAddress) and caches it. Make that
- *    first call before any stream capture.
+ *    first call before any stream capture. The cached address belongs to the
+ *    device's current context: after cudaDeviceReset (or any reset of the
+ *    primary context) in the same process it is stale, so do not call this
+ *    entry point again in that process after such a reset.
  *  - A problem whose scratch would exceed the buffer is rejected on the host
  *    with RET_ERR_SCRATCH before anything is launched. Passing state_in and
  *    state_out as the same buffer needs an extra copy of the state in scratch.
@@ -307,6 +312,17 @@ RET_API ret_status ret_chunkwise_noalloc(const void* q, const void* k, const voi
                                  void* o, const float* state_in, float* state_out,
                                  int B, int H, int N, int dk, int dv, int chunk,
                                  ret_dtype dt, void* stream);
+
+/*
+ * Scratch bytes of the fixed buffer that ret_chunkwise_noalloc would use for these
+ * sizes (in_place != 0: state_in and state_out are one buffer), 0 when the call needs
+ * none, -1 for sizes the call rejects as invalid. A value above
+ * RET_NOALLOC_SCRATCH_BYTES means the call returns RET_ERR_SCRATCH. The figure depends
+ * on the current device's SM count (the plan splits long sequences of few heads into
+ * segments to fill the SMs). Host-only: launches nothing. No counterpart on the pages.
+ */
+RET_API long long ret_chunkwise_noalloc_scratch_bytes(int B, int H, int N, int dk, int dv, int chunk,
+                                              ret_dtype dt, int in_place);
 
 /* Library version, "major.minor.patch". */
 RET_API const char* ret_version(void);

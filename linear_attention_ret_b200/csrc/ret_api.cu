@@ -708,7 +708,24 @@ void* noalloc_scratch() {
     return g_noalloc_ptr[dev];
 }
 
+// The segment plan of a no-allocation call: ret_chunkwise's, or, when that does not fit
+// the fixed buffer, one state-only piece per segment (less scratch, same result up to
+// rounding order).
+tc::Plan noalloc_plan(int B, int H, int N, int dk, int dv, bool alias) {
+    tc::Plan pl = tc::plan(B, H, N, dv);
+    if (tc::scratch_bytes(pl, B * H, dk, dv, alias) > RET_NOALLOC_SCRATCH_BYTES) pl = tc::plan(B, H, N, dv, false);
+    return pl;
+}
+
 }  // namespace
+
+extern "C" long long ret_chunkwise_noalloc_scratch_bytes(int B, int H, int N, int dk, int dv, int chunk, ret_dtype dt,
+                                                         int in_place) {
+    if (check_common(B, H, N, dk, dv, dt) != RET_OK || chunk <= 0 || dk > 256) return -1;
+    if (N == 0 || !tc_chunk_supported(dk, dv, chunk, dt == RET_BF16)) return 0;
+    const tc::Plan pl = noalloc_plan(B, H, N, dk, dv, in_place != 0);
+    return (long long)tc::scratch_bytes(pl, B * H, dk, dv, in_place != 0);
+}
 
 extern "C" ret_status ret_chunkwise_noalloc(const void* q, const void* k, const void* v, const float* gamma,
                                             void* o, const float* state_in, float* state_out, int B, int H, int N,
@@ -729,8 +746,7 @@ extern "C" ret_status ret_chunkwise_noalloc(const void* q, const void* k, const 
     }
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RET_ERR_ALIGN;
     const bool alias = state_in != nullptr && state_in == state_out;
-    tc::Plan pl = tc::plan(B, H, N, dv);
-    if (tc::scratch_bytes(pl, B * H, dk, dv, alias) > RET_NOALLOC_SCRATCH_BYTES) pl = tc::plan(B, H, N, dv, false);
+    const tc::Plan pl = noalloc_plan(B, H, N, dk, dv, alias);
     const size_t bytes = tc::scratch_bytes(pl, B * H, dk, dv, alias);
     if (bytes > RET_NOALLOC_SCRATCH_BYTES) return RET_ERR_SCRATCH;
     void* scratch = nullptr;

@@ -33,6 +33,7 @@
 #pragma once
 
 #include <algorithm>
+#include <atomic>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -955,16 +956,34 @@ __global__ void __launch_bounds__(64, 1) selftest_wait_kernel(unsigned long long
 
 // ------------------------------------------------------------------ host side
 
+// Per-device facts the host code needs on every call, cached per device (a process may
+// drive several GPUs from several threads). Racing first lookups store the same value,
+// so plain atomics suffice.
+constexpr int kMaxDevices = 64;
+
+inline int current_device() {
+    int dev = 0;
+    return (cudaGetDevice(&dev) == cudaSuccess && dev >= 0) ? dev : -1;
+}
+
+// 1 if the current device is sm_100 (the tensor-core path's target), else 0.
 inline bool tc_device_ok() {
-    static int cached = -1;
-    if (cached < 0) {
-        int dev = 0, major = 0, minor = 0;
-        cached = (cudaGetDevice(&dev) == cudaSuccess &&
-                  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess &&
-                  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) == cudaSuccess &&
-                  major == 10 && minor == 0) ? 1 : 0;
+    static std::atomic<int> cached[kMaxDevices];  // 0 = unknown, 1 = yes, 2 = no
+    const int dev = current_device();
+    if (dev < 0) return false;
+    auto query = [dev] {
+        int major = 0, minor = 0;
+        return cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess &&
+               cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) == cudaSuccess &&
+               major == 10 && minor == 0;
+    };
+    if (dev >= kMaxDevices) return query();
+    int c = cached[dev].load(std::memory_order_relaxed);
+    if (c == 0) {
+        c = query() ? 1 : 2;
+        cached[dev].store(c, std::memory_order_relaxed);
     }
-    return cached == 1;
+    return c == 1;
 }
 
 inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -1006,12 +1025,21 @@ inline bool tc_chunk_supported(int dk, int dv, int chunk, bool bf16) {
 
 namespace tc {
 
+// Streaming multiprocessors of the current device (148 on a B200 if the query fails).
 inline int sm_count() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    static std::atomic<int> cached[kMaxDevices];
+    const int dev = current_device();
+    auto query = [dev] {
+        int n = 0;
+        if (dev < 0 || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
             n = 148;
+        return n;
+    };
+    if (dev < 0 || dev >= kMaxDevices) return query();
+    int n = cached[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
+        n = query();
+        cached[dev].store(n, std::memory_order_relaxed);
     }
     return n;
 }
@@ -1162,10 +1190,9 @@ namespace tc {
 // call would map fresh memory. Raise it once per device so that repeated calls
 // reuse the pool's memory.
 inline void keep_pool_memory() {
-    static bool done[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || done[dev]) return;
-    done[dev] = true;
+    static std::atomic<bool> done[kMaxDevices];
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices || done[dev].exchange(true)) return;
     cudaMemPool_t pool;
     if (cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
         uint64_t threshold = UINT64_MAX;

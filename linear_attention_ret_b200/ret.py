@@ -30,7 +30,7 @@ SYMBOLS = ("ret_parallel", "ret_chunkwise", "ret_recurrent_step", "gated_ret_chu
            "ret_chunkwise_noalloc", "ret_selftest_wait_timeout", "gated_ret_recurrent_step",
            "ret_chunkwise_state", "gated_ret_chunkwise_state", "ret_state_prefix", "ret_chunkwise_state_launches",
            "ret_chunkwise_backward", "gated_ret_chunkwise_backward", "ret_chunkwise_backward_launches",
-           "ret_msr_norm_gate")
+           "ret_msr_norm_gate", "ret_chunkwise_noalloc_scratch_bytes")
 
 _lock = threading.Lock()
 _lib = None
@@ -87,6 +87,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
         lib.ret_chunkwise_path.restype = _i
         lib.ret_chunkwise_launches.argtypes = [_i, _i, _i, _i, _i, _i, _i]
         lib.ret_chunkwise_launches.restype = _i
+        lib.ret_chunkwise_noalloc_scratch_bytes.argtypes = [_i] * 8
+        lib.ret_chunkwise_noalloc_scratch_bytes.restype = ctypes.c_longlong
         lib.ret_version.argtypes = []
         lib.ret_version.restype = ctypes.c_char_p
         _lib = lib
@@ -332,3 +334,15 @@ def chunkwise_backward_launches(B: int, H: int, N: int, dk: int, dv: int, chunk:
 
 def chunkwise_path(dk: int, dv: int, chunk: int, dtype: torch.dtype) -> int:
     return int(load().ret_chunkwise_path(dk, dv, chunk, RET_BF16 if dtype == torch.bfloat16 else RET_F32))
+
+
+def noalloc_scratch_bytes(B: int, H: int, N: int, dk: int, dv: int, chunk: int, dtype: torch.dtype,
+                          in_place: bool = False) -> int:
+    """Bytes of the fixed buffer ret_chunkwise_noalloc would use on the current device (0: none,
+    -1: invalid sizes); above NOALLOC_SCRATCH_BYTES the call is rejected with RET_ERR_SCRATCH."""
+    return int(load().ret_chunkwise_noalloc_scratch_bytes(B, H, N, dk, dv, chunk,
+                                                          RET_BF16 if dtype == torch.bfloat16 else RET_F32,
+                                                          int(in_place)))
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20  # RET_NOALLOC_SCRATCH_BYTES in include/ret.h

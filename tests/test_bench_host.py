@@ -55,3 +55,17 @@ def test_traffic_records_are_well_formed_and_reported_only_while_current():
         # a figure is reported only while the measured kernel's sources hash as at capture
         assert bench.ncu_traffic(w) == (r["traffic_bytes_per_launch"] if r["source_sha"] == bench.kernel_source_sha(w)
                                         else None)
+
+
+def test_default_line_covers_every_headline_workload():
+    # the default run's line carries the decode step, the 6.7B-shaped sequence and the gated
+    # form as sub-records beside the 1.3B-shaped headline, each with its own roofline
+    assert set(bench.DEFAULT_ALSO) == {"decode", "retnet_6p7b_long", "gated"}
+    for w in bench.DEFAULT_ALSO:
+        assert w in bench.WORKLOAD_KERNELS
+    # the dtype field names the inputs' arithmetic type, per workload
+    from linear_attention_ret_b200 import inputs as I
+    assert bench.dtype_name(I.CONFIGS["retnet_1p3b"]) == "bf16"
+    assert bench.dtype_name(I.CONFIGS["tiny"]) == "f32"
+    d = bench.workload("decode")
+    assert d["unit"] == "steps/s" and d["bytes"] == 2 * 64 * 16 * 256 * 512 * 4 + 64 * 16 * (2 * 256 + 2 * 512) * 2

@@ -167,3 +167,50 @@ def test_segments_compose_on_gpu(cuda_lib, B, H, lengths, dk, dv, dtype, gated):
     assert cuda_lib.last_device_error() == 0
     assert_close(torch.cat(outs, dim=2), want_o, dtype, "o over all segments")
     assert rel_l2(end, want_s) <= tol_for(dtype), "final state"
+
+
+# ------------------------------------------------------------------ GPU: the product orchestration end to end
+
+ORCH_CASES = [
+    # B, H, N, dk, dv, dtype, gated
+    (1, 4, 2100, 256, 256, torch.bfloat16, False),   # tensor-core path, split sequence inside the state pass
+    (1, 2, 1333, 128, 128, torch.bfloat16, True),    # tensor-core gated path, ragged tail
+    (1, 2, 111, 32, 40, torch.float32, False),       # CUDA-core path
+    (1, 2, 97, 32, 40, torch.float32, True),
+]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("with_group", [False, True])
+@pytest.mark.parametrize("B,H,N,dk,dv,dtype,gated", ORCH_CASES)
+def test_sequence_parallel_library_ops_on_gpu(cuda_lib, B, H, N, dk, dv, dtype, gated, with_group):
+    """seqpar.sequence_parallel_chunkwise with the library's own kernels (LibraryOps) in one
+    process: without a process group, and inside a one-rank NCCL group, where the
+    all-gather of (U, log2 D) and the pick of this rank's start state run for real."""
+    import torch.distributed as dist
+    from linear_attention_ret_b200 import inputs as I
+    from linear_attention_ret_b200 import seqpar
+    from oracle import oracle as O
+    from tests.parity import assert_close, rel_l2, tol_for
+    dev = "cuda:0"
+    gen = torch.Generator().manual_seed(N + dk + int(gated))
+    q, k, v = I.qkv(B, H, N, dk, dv, dtype, gen=gen)
+    S0 = torch.randn(B, H, dk, dv, generator=gen) * 0.05
+    if gated:
+        decay = I.gate(B, H, N, gen) * 4.0
+        want_o, want_s = O.gated_chunkwise(q, k, v, decay, 64, state_in=S0)
+    else:
+        decay = torch.tensor([0.9, 0.96875, 0.999, 0.5][:H], dtype=torch.float32)
+        want_o, want_s = O.ret_chunkwise(q, k, v, decay, 64, state_in=S0)
+    if with_group:
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0, world_size=1)
+    try:
+        o, end = seqpar.sequence_parallel_chunkwise(q.to(dev), k.to(dev), v.to(dev), decay.to(dev), 64,
+                                                    gated=gated, state_in=S0.to(dev))
+        torch.cuda.synchronize()
+    finally:
+        if with_group:
+            dist.destroy_process_group()
+    assert cuda_lib.last_device_error() == 0
+    assert_close(o, want_o, dtype, "o")
+    assert rel_l2(end, want_s) <= tol_for(dtype), "final state"
