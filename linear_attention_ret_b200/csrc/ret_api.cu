@@ -208,49 +208,51 @@ inline AuxStreams* aux_streams() {
     return &a;
 }
 
-// The dv contraction of dQ and dK in pieces of 256: on the tensor-core path each piece is
-// read in place through row-strided tensor maps; otherwise it is copied out first.
-inline bool backward_pieces_in_place(int dk, int dv, int chunk, ret_dtype dt) {
-    if (dv <= 256 || dt != RET_BF16) return false;
+// The backward on the tensor-core path: every launch (the dQ pieces, the dK pieces and dV,
+// each with q/k widths of at most 256 read in place through row-strided tensor maps) is a
+// tensor-core launch. dK and dV run on the time-reversed kernels, so nothing is copied.
+inline bool backward_on_tensor_cores(int dk, int dv, int chunk, ret_dtype dt) {
+    if (dt != RET_BF16 || !tc_chunk_supported(dk, dv, chunk, true)) return false;  // dV: widths dk, values dv
     for (int c0 = 0; c0 < dv; c0 += 256)
-        if (!tc_chunk_supported(std::min(256, dv - c0), dk, chunk, true)) return false;
+        if (!tc_chunk_supported(std::min(256, dv - c0), dk, chunk, true)) return false;  // dQ, dK pieces
     return true;
 }
 
-// The backward on the tensor-core path with dv in pieces read in place, as a small graph of
-// steps on the caller's stream st and two library streams s1, s2:
-//   st: dQ piece 0 | wait s1 -> dq = sum of the dQ pieces | wait s2 -> dV forward, reverse -> | wait s2 -> dgamma/dg
-//   s1: dQ piece 1 |                  wait s2 (reversals) -> dK piece 1 ------------------------>|
-//   s2: reversed Q, K, V, dO (and gates) -> dK piece 0 | wait s1 -> dk = reverse(sum of dK pieces)
-// (more pieces alternate between the two streams of their row). The reversals run beside the
-// dQ pieces and the dV forward beside the dK pieces, filling the SMs each leaves idle.
+// Kernel launches of one backward call on the tensor-core path.
+inline int backward_tc_launches(int B, int H, int N, int dk, int dv, bool gated, bool ddecay) {
+    const int P = (dv + 255) / 256, conc = 2 * P + 1;
+    int n = 0;
+    for (int p = 0; p < P; ++p) n += 2 * tc_chunk_launches(B, H, N, std::min(256, dv - 256 * p), dk, conc);
+    n += tc_chunk_launches(B, H, N, dk, dv, conc);  // dV
+    n += P > 1 ? 2 : 0;                             // sums of the dQ and dK pieces
+    n += ddecay ? (gated ? 2 : 1) : 0;              // decay gradient (gated: and its suffix sum)
+    return n;
+}
+
+// The backward on the tensor-core path as a small graph of steps on the caller's stream st
+// and two library streams s1, s2:
+//   st: dQ piece 0 | wait s1 -> dq = sum of the dQ pieces | wait s2 -> dgamma/dg
+//   s1: dQ piece 1 | dK piece 1 (reversed)
+//   s2: dK piece 0 (reversed) | dV (reversed) | wait s1 -> dk = sum of the dK pieces
+// (more pieces alternate between the streams of their row; with one piece the dQ and dK
+// calls write dq and dk directly). dQ = forward(dO, V, K); dK = reversed forward(V, dO, Q);
+// dV = reversed forward(K, Q, dO), each with the caller's gamma or gates as they are.
 template <typename T, bool GATED>
-ret_status backward_concurrent(const void* q, const void* k, const void* v, const float* decay, const void* dout,
-                               void* dq, void* dk_out, void* dv_out, float* ddecay, int B, int H, int N, int dk, int dv,
-                               int chunk, ret_dtype dt, cudaStream_t st) {
+ret_status backward_tc(const void* q, const void* k, const void* v, const float* decay, const void* dout,
+                       void* dq, void* dk_out, void* dv_out, float* ddecay, int B, int H, int N, int dk, int dv,
+                       cudaStream_t st) {
     const int BH = B * H;
-    const size_t nQ = (size_t)BH * N * dk, nV = (size_t)BH * N * dv;
-    const int pw = 256, P = (dv + pw - 1) / pw;
-    // scratch: reversed Q, K, V, dO; dQ pieces; dK pieces; reversed dV; reversed gates
-    size_t off[8], bytes = 0;
-    const size_t sz[8] = {nQ * sizeof(T), nQ * sizeof(T), nV * sizeof(T), nV * sizeof(T), (size_t)P * nQ * sizeof(T),
-                          (size_t)P * nQ * sizeof(T), nV * sizeof(T), GATED ? (size_t)BH * N * sizeof(float) : 0};
-    for (int i = 0; i < 8; ++i) {
-        off[i] = bytes;
-        bytes += align256(sz[i]);
-    }
-    tc::keep_pool_memory();
+    const size_t nQ = (size_t)BH * N * dk;
+    const int pw = 256, P = (dv + pw - 1) / pw, conc = 2 * P + 1;
+    // scratch (P > 1 only): the dQ and dK pieces
+    const size_t part_bytes = align256((size_t)P * nQ * sizeof(T));
     uint8_t* sc = nullptr;
-    if (cudaMallocAsync(reinterpret_cast<void**>(&sc), bytes, st) != cudaSuccess) return RET_ERR_CUDA;
-    T* Qf = reinterpret_cast<T*>(sc + off[0]);
-    T* Kf = reinterpret_cast<T*>(sc + off[1]);
-    T* Vf = reinterpret_cast<T*>(sc + off[2]);
-    T* dOf = reinterpret_cast<T*>(sc + off[3]);
-    T* partsQ = reinterpret_cast<T*>(sc + off[4]);
-    T* partsK = reinterpret_cast<T*>(sc + off[5]);
-    T* Rf = reinterpret_cast<T*>(sc + off[6]);
-    float* gf = reinterpret_cast<float*>(sc + off[7]);
-    const float* dec_rev = GATED ? gf : decay;
+    if (P > 1) {
+        tc::keep_pool_memory();
+        if (cudaMallocAsync(reinterpret_cast<void**>(&sc), 2 * part_bytes, st) != cudaSuccess) return RET_ERR_CUDA;
+    }
+    T* partsQ = P > 1 ? reinterpret_cast<T*>(sc) : static_cast<T*>(dq);
+    T* partsK = P > 1 ? reinterpret_cast<T*>(sc + part_bytes) : static_cast<T*>(dk_out);
 
     ret_status r = RET_OK;
     auto ok = [&](ret_status x) { if (r == RET_OK) r = x; return r == RET_OK; };
@@ -258,50 +260,41 @@ ret_status backward_concurrent(const void* q, const void* k, const void* v, cons
     std::lock_guard<std::mutex> lock(aux_mutex());
     AuxStreams* a = aux_streams();
     if (!a) {
-        cudaFreeAsync(sc, st);
+        if (sc) cudaFreeAsync(sc, st);
         return RET_ERR_CUDA;
     }
     cudaStream_t s1 = a->s[0], s2 = a->s[1];
-    cudaEvent_t ev_fork = a->ev[0], ev_dq = a->ev[1], ev_rev = a->ev[2], ev_dk1 = a->ev[3], ev_dk = a->ev[4],
-                ev_j1 = a->ev[5], ev_j2 = a->ev[6];
-    auto piece = [&](const void* x, const void* y, const void* z, const float* dec, T* fo, int p, cudaStream_t s) {
+    cudaEvent_t ev_fork = a->ev[0], ev_q1 = a->ev[1], ev_k1 = a->ev[2], ev_k = a->ev[3], ev_j1 = a->ev[4],
+                ev_j2 = a->ev[5];
+    // one piece of a dv contraction: queries x[:, c0:c0+w], keys y[:, c0:c0+w] (rows dv apart), values z
+    auto piece = [&](bool rev, const void* x, const void* y, const void* z, T* fo, int p, cudaStream_t s) {
         const int c0 = p * pw, w = std::min(pw, dv - c0);
-        return ok(tc_chunk_launch<GATED>(static_cast<const T*>(x) + c0, static_cast<const T*>(y) + c0, z, dec,
-                                         fo + (size_t)p * nQ, nullptr, nullptr, B, H, N, w, dk, s, dv, dv, 2));
+        const void* xp = static_cast<const T*>(x) + c0;
+        const void* yp = static_cast<const T*>(y) + c0;
+        T* out = fo + (size_t)p * nQ;
+        return ok(rev ? tc_chunk_launch<GATED, true>(xp, yp, z, decay, out, nullptr, nullptr, B, H, N, w, dk, s, dv,
+                                                     dv, conc)
+                      : tc_chunk_launch<GATED, false>(xp, yp, z, decay, out, nullptr, nullptr, B, H, N, w, dk, s, dv,
+                                                      dv, conc));
     };
-    // fork
     if (cu(cudaEventRecord(ev_fork, st))) {
         cu(cudaStreamWaitEvent(s1, ev_fork, 0));
         cu(cudaStreamWaitEvent(s2, ev_fork, 0));
     }
-    // dQ = forward(dO, V, K) in pieces on st and s1; the reversals on s2
-    for (int p = 0; p < P && r == RET_OK; ++p) piece(dout, v, k, decay, partsQ, p, p % 2 ? s1 : st);
-    if (r == RET_OK) {
-        ok(slice_flip<T>(q, Qf, BH, N, dk, 0, dk, true, s2)) && ok(slice_flip<T>(k, Kf, BH, N, dk, 0, dk, true, s2)) &&
-            ok(slice_flip<T>(v, Vf, BH, N, dv, 0, dv, true, s2)) &&
-            ok(slice_flip<T>(dout, dOf, BH, N, dv, 0, dv, true, s2));
-        if (GATED && r == RET_OK) {
-            gate_flip_kernel<<<grid_for((size_t)BH * N), kBwdThreads, 0, s2>>>(decay, gf, N, (size_t)BH * N);
-            ok(launch_status());
-        }
-    }
-    if (r == RET_OK) cu(cudaEventRecord(ev_rev, s2));
-    // dq on st, once s1's pieces are done
-    if (r == RET_OK && cu(cudaEventRecord(ev_dq, s1)) && cu(cudaStreamWaitEvent(st, ev_dq, 0)))
+    // dQ pieces on st and s1, then dK pieces on s2 and s1, dV on s2
+    for (int p = 0; p < P && r == RET_OK; ++p) piece(false, dout, v, k, partsQ, p, p % 2 ? s1 : st);
+    if (r == RET_OK) cu(cudaEventRecord(ev_q1, s1));  // s1's dQ pieces
+    for (int p = 0; p < P && r == RET_OK; ++p) piece(true, v, dout, q, partsK, p, p % 2 ? s1 : s2);
+    if (r == RET_OK) cu(cudaEventRecord(ev_k1, s1));  // s1's dK pieces
+    if (r == RET_OK)
+        ok(tc_chunk_launch<GATED, true>(k, q, dout, decay, dv_out, nullptr, nullptr, B, H, N, dk, dv, s2, 0, 0, conc));
+    // dq = sum of the dQ pieces on st, dk = sum of the dK pieces on s2, each once s1's pieces are done
+    if (r == RET_OK && cu(cudaStreamWaitEvent(st, ev_q1, 0)) && P > 1)
         ok(sum_flip<T>(partsQ, P, nQ, static_cast<T*>(dq), BH, N, dk, false, st));
-    // dK = reverse(forward(rev V, rev dO, rev Q)) in pieces on s2 and s1, after the reversals
-    if (r == RET_OK) cu(cudaStreamWaitEvent(s1, ev_rev, 0));
-    for (int p = 0; p < P && r == RET_OK; ++p) piece(Vf, dOf, Qf, dec_rev, partsK, p, p % 2 ? s1 : s2);
-    // dV = reverse(forward(rev K, rev Q, rev dO)) on st, beside the dK pieces
-    if (r == RET_OK && cu(cudaStreamWaitEvent(st, ev_rev, 0)) &&
-        ok(chunkwise_entry<GATED>(Kf, Qf, dOf, dec_rev, Rf, nullptr, nullptr, B, H, N, dk, dv, chunk, dt, st)))
-        ok(slice_flip<T>(Rf, dv_out, BH, N, dv, 0, dv, true, st));
-    // dk on s2 once s1's pieces are done
-    if (r == RET_OK && cu(cudaEventRecord(ev_dk1, s1)) && cu(cudaStreamWaitEvent(s2, ev_dk1, 0)) &&
-        ok(sum_flip<T>(partsK, P, nQ, static_cast<T*>(dk_out), BH, N, dk, true, s2)))
-        cu(cudaEventRecord(ev_dk, s2));
-    // decay gradient on st, after dq (st) and dk (s2)
-    if (r == RET_OK && ddecay && cu(cudaStreamWaitEvent(st, ev_dk, 0)))
+    if (r == RET_OK && cu(cudaStreamWaitEvent(s2, ev_k1, 0)) && P > 1)
+        ok(sum_flip<T>(partsK, P, nQ, static_cast<T*>(dk_out), BH, N, dk, false, s2));
+    // decay gradient on st, after dq (st, s1) and dk (s1, s2)
+    if (r == RET_OK && cu(cudaEventRecord(ev_k, s2)) && ddecay && cu(cudaStreamWaitEvent(st, ev_k, 0)))
         ok(decay_grad<T, GATED>(static_cast<const T*>(q), static_cast<const T*>(dq), static_cast<const T*>(k),
                                 static_cast<const T*>(dk_out), decay, ddecay, BH, H, N, dk, st));
     // join both library streams back into st whatever happened, then release the scratch on st
@@ -314,7 +307,7 @@ ret_status backward_concurrent(const void* q, const void* k, const void* v, cons
         cudaStreamSynchronize(s2);
         ok(RET_ERR_CUDA);
     }
-    if (cudaFreeAsync(sc, st) != cudaSuccess) ok(RET_ERR_CUDA);
+    if (sc && cudaFreeAsync(sc, st) != cudaSuccess) ok(RET_ERR_CUDA);
     return r;
 }
 
@@ -326,9 +319,8 @@ ret_status backward_impl(const void* q, const void* k, const void* v, const floa
     const size_t nQ = (size_t)BH * N * dk, nV = (size_t)BH * N * dv;
     const int pw = dv <= 256 ? dv : 256;  // width of one piece of the dv contraction
     const int P = (dv + pw - 1) / pw;
-    if (backward_pieces_in_place(dk, dv, chunk, dt))
-        return backward_concurrent<T, GATED>(q, k, v, decay, dout, dq, dk_out, dv_out, ddecay, B, H, N, dk, dv, chunk,
-                                             dt, st);
+    if (backward_on_tensor_cores(dk, dv, chunk, dt))
+        return backward_tc<T, GATED>(q, k, v, decay, dout, dq, dk_out, dv_out, ddecay, B, H, N, dk, dv, st);
     // scratch: reversed Q, K, V, dO; two piece buffers; per-piece outputs; reversed dV; reversed gates
     size_t off[9], bytes = 0;
     const size_t sz[9] = {nQ * sizeof(T), nQ * sizeof(T), nV * sizeof(T), nV * sizeof(T),
@@ -656,16 +648,15 @@ int ret_chunkwise_backward_launches(int B, int H, int N, int dk, int dv, int chu
                                     int ddecay) {
     if (check_common(B, H, N, dk, dv, dt) != RET_OK || chunk <= 0 || dk > 256) return -1;
     if (N == 0) return 0;
-    // mirrors backward_impl: forward calls, the slice / flip / sum kernels, the decay gradient
+    if (backward_on_tensor_cores(dk, dv, chunk, dt)) return backward_tc_launches(B, H, N, dk, dv, gated, ddecay);
+    // mirrors backward_impl's copying path: forward calls, the slice / flip / sum kernels, the decay gradient
     auto fwd = [&](int wq, int wv) { return ret_chunkwise_launches(B, H, N, wq, wv, chunk, dt); };
     const int pw = dv <= 256 ? dv : 256, P = (dv + pw - 1) / pw;
-    const bool in_place = backward_pieces_in_place(dk, dv, chunk, dt);
     int n = 0;
     for (int p = 0; p < P; ++p) {
         const int w = std::min(pw, dv - p * pw);
-        // in place: the pieces run two at a time, sized together; else two slices, then the forward
-        const int piece = in_place ? tc_chunk_launches(B, H, N, w, dk, 2) : 2 + fwd(w, dk);
-        n += P == 1 ? 2 * fwd(dv, dk) : 2 * piece;  // a dQ and a dK piece
+        // two slices, then the forward, for a dQ and a dK piece
+        n += P == 1 ? 2 * fwd(dv, dk) : 2 * (2 + fwd(w, dk));
     }
     n += P == 1 ? 0 : 1;                 // sum of the dQ pieces
     n += 4 + (gated ? 1 : 0);            // reversed Q, K, V, dO (and gates)

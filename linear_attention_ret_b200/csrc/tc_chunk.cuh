@@ -290,6 +290,7 @@ struct Params {
     int H, N, dv;
     int seg_chunks;          // chunks per sequence segment (blockIdx.z = segment)
     int sub_per_seg;         // state-only sub-segments per full-pass segment (their start states are in seg_state)
+    int units;               // segments the sequence is cut into at seg_chunks each (REV counts them from the end)
 };
 
 // In-chunk inclusive cumulative sum of the gate in log2 units, by one warp:
@@ -333,7 +334,16 @@ constexpr bool wide_capable(int dk, bool gated, bool state_only) {
 // decay to the scratch buffers. seg_prefix_kernel then turns them into the
 // segment start states S_in(g) = decay_{g-1} S_in(g-1) + U_{g-1}, S_in(0) =
 // state_in, and the full pass starts each segment from its S_in.
-template <int DK, bool GATED, bool STATE_ONLY>
+// REV: the time-reversed direction, O_j = sum over later tokens i >= j of w_ij (q_j . k_i)
+// v_i with the same weights (gamma^(i-j), or exp(G_i - G_j) for the gated form); the
+// gradients dK and dV are such sums. The chunks are visited from the last back and the
+// state is referenced at the token before the current chunk, R = sum_{i >= t0} w(i, t0-1)
+// k_i^T v_i. With Gl the chunk's inclusive cumulative log-decay (L tokens) the factors
+// mirror the forward's: key weights exp(Gl_i) instead of exp(Gl_{L-1} - Gl_i), cross-term
+// row factors exp(Gl_{L-1} - Gl_j) instead of exp(Gl_j), the same chunk decay
+// exp(Gl_{L-1}), and the upper triangle i >= j of the mask. Segments of a split sequence
+// are chained from the last back too (blockIdx.z counts them from the end).
+template <int DK, bool GATED, bool STATE_ONLY, bool REV>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, Params p) {
@@ -346,7 +356,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if constexpr (wide_capable(DK, GATED, STATE_ONLY)) {
         const float lgw = log2f(p.decay_in[blockIdx.y % p.H]);
         if (lgw >= kWideMinLog2 && lgw <= 0.f) {
-            wide_body<DK>(tm_q, tm_k, tm_v, tm_o, p, lgw);
+            wide_body<DK, REV>(tm_q, tm_k, tm_v, tm_o, p, lgw);
             return;
         }
     }
@@ -361,10 +371,21 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int slice = blockIdx.x, bh = blockIdx.y;
     const int dv0 = slice * kDvS;
-    const int seg = blockIdx.z;
-    const int cbase = seg * p.seg_chunks;                          // first chunk of this segment
+    const int seg = blockIdx.z;                                    // place in the chain of segments
+    const int tseg = REV ? p.units - 1 - seg : seg;                // place in time
+    const int cbase = tseg * p.seg_chunks;                         // first chunk of this segment
     const int nchunks = min(p.seg_chunks, (p.N + kC - 1) / kC - cbase);
-    const bool last_seg = (cbase + nchunks) * kC >= p.N;
+    const bool last_seg = seg == p.units - 1;                      // the chain's last: writes state_out
+    // token start of the i-th chunk visited (REV: from the segment's last chunk back)
+    auto chunk_t0 = [&](int i) { return (cbase + (REV ? nchunks - 1 - i : i)) * kC; };
+    if (STATE_ONLY && nchunks <= 0) {
+        // REV only: a sub-segment past the end of a short last segment holds no tokens; its
+        // local state is zero and its decay one
+        float* so = p.seg_state + ((size_t)seg * gridDim.y + bh) * DK * p.dv + dv0;
+        for (int e = threadIdx.x; e < DK * kDvS; e += blockDim.x) so[(size_t)(e / kDvS) * p.dv + e % kDvS] = 0.f;
+        if (slice == 0 && threadIdx.x == 0) p.seg_ldec[(size_t)seg * gridDim.y + bh] = 0.f;
+        return;
+    }
 
     if (threadIdx.x == 0) {
         for (int b = 0; b < Lay::kNumBars; ++b) mbar_init(bar(b), 1);
@@ -411,7 +432,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (i >= NS && !mbar_wait(bar(kEmpty0 + s), ((i / NS) - 1) & 1, abort_flag)) break;
                 const uint32_t st = sbase + Lay::kStage0 + s * Lay::kStageBytes;
                 mbar_expect_tx(bar(kFull0 + s), STATE_ONLY ? Lay::kKBytes + Lay::kVBytes : Lay::kStageBytes);
-                const int t0 = (cbase + i) * kC;
+                const int t0 = chunk_t0(i);
 #pragma unroll
                 for (int kb = 0; kb < DK / 64; ++kb) {
                     if (!STATE_ONLY) tma_load_3d(st + kb * kTile64, &tm_q, kb * 64, t0, bh, bar(kFull0 + s));
@@ -532,31 +553,39 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             group_sync(1);
             return *abort_flag == 0;
         };
+        // row factors of the drain: per buffer where they depend on the chunk (gated; REV
+        // split, whose factor gamma^(L-1-j) depends on the chunk's length), else one table
+        constexpr bool kRowPerChunk = GATED || REV;
         if (!GATED) {
             if (te <= kC) pw[te] = pow_int_log2(lg, te);
             group_sync(1);
-            if (te < kC) rr[te] = merged ? pow_int_log2(-lg, kC - 1 - te) : pw[te + 1];
+            if (te < kC) rr[te] = merged ? pow_int_log2(-lg, REV ? te : kC - 1 - te) : pw[te + 1];
         }
         float g0 = 0.f, g1 = 0.f;  // gated: prefetched gate values of the next chunk (first warp)
         if (GATED && te < 32) {
-            const int a = cbase * kC + 2 * te;
+            const int a = chunk_t0(0) + 2 * te;
             g0 = (a < p.N ? G[a] : 0.f) * kLog2e;
             g1 = (a + 1 < p.N ? G[a + 1] : 0.f) * kLog2e;
         }
         // ---------------- P = mask(Q K^T) of chunk c in bf16 (its attention buffer): row j, 32 columns per thread
         auto do_p = [&](int ci) {
             const int b = abuf(ci);
-            const int t0 = (cbase + ci) * kC;
+            const int t0 = chunk_t0(ci);
             float* cumb = cum + b * kC;
             if (GATED) {
                 if (te < 32) {
                     warp_cumsum64(g0, g1, lane, cumb);
-                    const int a = t0 + kC + 2 * te;
+                    // prefetch the next chunk's gates (none past the last chunk: a >= N reads zero)
+                    const int a = (ci + 1 < nchunks ? chunk_t0(ci + 1) : p.N) + 2 * te;
                     g0 = (a < p.N ? G[a] : 0.f) * kLog2e;
                     g1 = (a + 1 < p.N ? G[a + 1] : 0.f) * kLog2e;
                 }
                 group_sync(1);
-                if (te < kC) rr[b * kC + te] = exp2f(cumb[te]);
+                // forward exp(Gl_j); REV exp(Gl_last - Gl_j) (gates past N are zero, so Gl_63 = Gl_{L-1})
+                if (te < kC) rr[b * kC + te] = exp2f(REV ? cumb[kC - 1] - cumb[te] : cumb[te]);
+            } else if (REV && !merged) {
+                const int L = min(kC, p.N - t0);
+                if (te < kC) rr[b * kC + te] = te < L ? pw[L - 1 - te] : 0.f;
             }
             if (!wait_all(kAFull0 + b, ause(ci) & 1)) return false;
             tc_fence_after();
@@ -570,11 +599,18 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (GATED) {
                     const float cj = cumb[j];
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) w[c] = cj - cumb[m0 + c];
+                    for (int c = 0; c < 32; ++c) w[c] = REV ? cumb[m0 + c] - cj : cj - cumb[m0 + c];
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
                         const int m = m0 + c;
-                        w[c] = m > j ? 0.f : (m == j ? 1.f : exp2f(w[c]));
+                        w[c] = (REV ? m < j : m > j) ? 0.f : (m == j ? 1.f : exp2f(w[c]));
+                    }
+                } else if (REV) {
+                    // split: gamma^(m-j); merged: zeta'_m = gamma^m
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const int m = m0 + c;
+                        w[c] = m < j ? 0.f : pw[merged ? m : m - j];
                     }
                 } else {
                     // split: gamma^(j-m); merged: zeta'_m = gamma^(63-m)
@@ -611,8 +647,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // ---------------- O = O_intra + r_j O_inter of chunk c -> bf16 -> staging -> TMA store
         auto do_drain = [&](int ci) {
             const int b = abuf(ci);
-            const int t0 = (cbase + ci) * kC;
-            const float* rrb = GATED ? rr + b * kC : rr;
+            const int t0 = chunk_t0(ci);
+            const float* rrb = (kRowPerChunk && (GATED || !merged)) ? rr + b * kC : rr;
             const uint32_t tA = tmem + lane_off + Lay::kColA + bcols * b;
             if (te == 0) tma_store_wait_read();  // the previous chunk's O store has read the staging tile
             if (!wait_all(kOFull0 + b, ause(ci) & 1)) return false;
@@ -716,7 +752,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         };
         float g0 = 0.f, g1 = 0.f;
         if (GATED && ts < 32) {
-            const int a = cbase * kC + 2 * ts;
+            const int a = chunk_t0(0) + 2 * ts;
             g0 = (a < p.N ? G[a] : 0.f) * kLog2e;
             g1 = (a + 1 < p.N ? G[a + 1] : 0.f) * kLog2e;
         }
@@ -729,22 +765,22 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // zeta-scaled V of chunk c into ZV buffer c & 1, divided by the scale c_{next} that
         // make_zv picks from c_prev (the current scale) and the chunk's decay.
         auto make_zv = [&](int c, float c_prev, bool force_renorm, float& decay, bool& renorm, float& c_next) {
-            const int t0 = (cbase + c) * kC, L = min(kC, p.N - t0);
+            const int t0 = chunk_t0(c), L = min(kC, p.N - t0);
             if (GATED) {
                 if (ts < 32) {
                     warp_cumsum64(g0, g1, lane, cum);
-                    const int a = t0 + kC + 2 * ts;
+                    const int a = (c + 1 < nchunks ? chunk_t0(c + 1) : p.N) + 2 * ts;
                     g0 = (a < p.N ? G[a] : 0.f) * kLog2e;
                     g1 = (a + 1 < p.N ? G[a + 1] : 0.f) * kLog2e;
                 }
                 group_sync(2);
-                if (ts < kC) zeta[ts] = ts < L ? exp2f(cum[L - 1] - cum[ts]) : 0.f;
+                if (ts < kC) zeta[ts] = ts < L ? exp2f(REV ? cum[ts] : cum[L - 1] - cum[ts]) : 0.f;
                 if (ts == 0) {
                     dec[0] = exp2f(cum[L - 1]);
                     dec[1] = cum[L - 1];
                 }
             } else {
-                if (ts < kC) zeta[ts] = ts < L ? pow_int_log2(lg, L - 1 - ts) : 0.f;
+                if (ts < kC) zeta[ts] = ts < L ? pow_int_log2(lg, REV ? ts + 1 : L - 1 - ts) : 0.f;
                 if (ts == 0) {
                     dec[0] = pow_int_log2(lg, L);
                     dec[1] = lg * (float)L;
@@ -784,8 +820,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             return true;
         };
 
-        // The bf16 state copy is S (split output accumulators) or gamma^64 S (merged).
-        const float sop = merged ? pow_int_log2(lg, kC) : 1.f;
+        // The bf16 state copy feeding chunk c's cross term is S (split output accumulators)
+        // or, merged, gamma^64 S (forward) or gamma^(L_c - 1) S (REV, L_c the chunk's length).
+        auto sop_of = [&](int c) {
+            return !merged ? 1.f : REV ? pow_int_log2(lg, min(kC, p.N - chunk_t0(c)) - 1) : pow_int_log2(lg, kC);
+        };
+        const float sop = sop_of(0);
         float dec0 = 0.f, c_cur = 1.f;
         bool renorm = true;
         bool ok = make_zv(0, 1.f, true, dec0, renorm, c_cur);
@@ -841,7 +881,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 // S_op = bf16(sop c_i T_i) for the next cross term; on renormalisation also
                 // T <- c_i d_{i+1} T_i so that the next update (scaled by 1/c_{i+1} = 1) adds onto it.
                 // The state-only pass needs no S_op and touches T only to renormalise.
-                const float tscale = c_cur * dec_next, hscale = c_cur * sop;
+                const float tscale = c_cur * dec_next, hscale = c_cur * sop_of(i + 1);
 #pragma unroll 1
                 for (int cb = 0; cb < DK / 64; ++cb) {
                     uint32_t w0[32], w1[32], h[16];
@@ -1116,7 +1156,7 @@ inline cudaError_t launch_dependent(void (*kernel)(P...), dim3 grid, size_t smem
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
 }
 
-template <int DK, bool GATED>
+template <int DK, bool GATED, bool REV>
 ret_status launch_dk(const void* q, const void* k, const void* v, const float* decay, void* o,
                      const float* state_in, float* state_out, int B, int H, int N, int dv, const Plan& pl,
                      void* scratch, cudaStream_t st, int ldq, int ldk) {
@@ -1125,7 +1165,7 @@ ret_status launch_dk(const void* q, const void* k, const void* v, const float* d
     if (!make_map(&mq, q, DK, N, BH, ldq) || !make_map(&mk, k, DK, N, BH, ldk) || !make_map(&mv, v, dv, N, BH) ||
         !make_map(&mo, o, dv, N, BH))
         return RET_ERR_CUDA;
-    Params prm{decay, state_in, state_out, nullptr, nullptr, H, N, dv, pl.seg_chunks, pl.F};
+    Params prm{decay, state_in, state_out, nullptr, nullptr, H, N, dv, pl.seg_chunks, pl.F, pl.G};
     if (pl.G > 1) {
         uint8_t* sc = static_cast<uint8_t*>(scratch);
         prm.seg_state = reinterpret_cast<float*>(sc);
@@ -1137,12 +1177,13 @@ ret_status launch_dk(const void* q, const void* k, const void* v, const float* d
                 return RET_ERR_CUDA;
             prm.state_in = copy;
         }
-        auto k1 = chunk_tc_kernel<DK, GATED, true>;
+        auto k1 = chunk_tc_kernel<DK, GATED, true, REV>;
         constexpr int smem1 = kernel_smem<DK, GATED, true>();
         if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1) != cudaSuccess)
             return RET_ERR_CUDA;
         Params prm1 = prm;  // the state-only pass runs over the sub-segments
         prm1.seg_chunks = pl.seg_chunks / pl.F;
+        prm1.units = pl.F * pl.G;
         if (launch_dependent(k1, dim3(dv / kDvS, BH, pl.subs()), smem1, st, mq, mk, mv, mo, prm1) != cudaSuccess)
             return RET_ERR_CUDA;
         const int n4 = BH * DK * dv / 4;
@@ -1150,7 +1191,7 @@ ret_status launch_dk(const void* q, const void* k, const void* v, const float* d
             prm.state_in, prm.seg_state, prm.seg_ldec, pl.subs() + 1, BH, DK * dv);
         if (cudaGetLastError() != cudaSuccess) return RET_ERR_CUDA;
     }
-    auto k2 = chunk_tc_kernel<DK, GATED, false>;
+    auto k2 = chunk_tc_kernel<DK, GATED, false, REV>;
     constexpr int smem2 = kernel_smem<DK, GATED, false>();
     if (cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2) != cudaSuccess)
         return RET_ERR_CUDA;
@@ -1159,20 +1200,22 @@ ret_status launch_dk(const void* q, const void* k, const void* v, const float* d
 }
 
 // Runs the tensor-core path with caller-provided scratch (at least scratch_bytes()).
-// ldq, ldk: row strides of q and k in elements (0: dense rows of dk).
-template <bool GATED>
+// ldq, ldk: row strides of q and k in elements (0: dense rows of dk). REV: the
+// time-reversed direction (sums over later tokens), see chunk_tc_kernel.
+template <bool GATED, bool REV = false>
 ret_status launch_with_scratch(const void* q, const void* k, const void* v, const float* decay, void* o,
                                const float* state_in, float* state_out, int B, int H, int N, int dk, int dv,
                                const Plan& pl, void* scratch, cudaStream_t st, int ldq = 0, int ldk = 0) {
     switch (dk) {
         case 64:
-            return launch_dk<64, GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dv, pl, scratch, st, ldq, ldk);
+            return launch_dk<64, GATED, REV>(q, k, v, decay, o, state_in, state_out, B, H, N, dv, pl, scratch, st,
+                                             ldq, ldk);
         case 128:
-            return launch_dk<128, GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dv, pl, scratch, st, ldq,
-                                         ldk);
+            return launch_dk<128, GATED, REV>(q, k, v, decay, o, state_in, state_out, B, H, N, dv, pl, scratch, st,
+                                              ldq, ldk);
         case 256:
-            return launch_dk<256, GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dv, pl, scratch, st, ldq,
-                                         ldk);
+            return launch_dk<256, GATED, REV>(q, k, v, decay, o, state_in, state_out, B, H, N, dv, pl, scratch, st,
+                                              ldq, ldk);
     }
     return RET_ERR_UNSUPPORTED;
 }
@@ -1226,8 +1269,8 @@ ret_status launch_state_dk(const void* k, const void* v, const float* decay, flo
     uint8_t* sc = static_cast<uint8_t*>(scratch);
     float* states = subs > 1 ? reinterpret_cast<float*>(sc) : state_out;
     float* ldec = reinterpret_cast<float*>(sc + (subs > 1 ? sizeof(float) * (size_t)subs * BH * DK * dv : 0));
-    Params prm{decay, nullptr, nullptr, states, ldec, H, N, dv, sub_chunks, 1};
-    auto k1 = chunk_tc_kernel<DK, GATED, true>;
+    Params prm{decay, nullptr, nullptr, states, ldec, H, N, dv, sub_chunks, 1, subs};
+    auto k1 = chunk_tc_kernel<DK, GATED, true, false>;
     constexpr int smem1 = kernel_smem<DK, GATED, true>();
     if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1) != cudaSuccess)
         return RET_ERR_CUDA;
@@ -1274,7 +1317,7 @@ inline int tc_state_launches(int B, int H, int N, int dv) {
 
 // Tensor-core path; a split sequence takes its scratch from the stream-ordered
 // allocator and returns it on the same stream after the two launches.
-template <bool GATED>
+template <bool GATED, bool REV = false>
 ret_status tc_chunk_launch(const void* q, const void* k, const void* v, const float* decay, void* o,
                            const float* state_in, float* state_out, int B, int H, int N, int dk, int dv,
                            cudaStream_t st, int ldq = 0, int ldk = 0, int concurrent = 1) {
@@ -1283,8 +1326,8 @@ ret_status tc_chunk_launch(const void* q, const void* k, const void* v, const fl
     const size_t bytes = tc::scratch_bytes(pl, B * H, dk, dv, state_in != nullptr && state_in == state_out);
     if (bytes) tc::keep_pool_memory();
     if (bytes && cudaMallocAsync(&scratch, bytes, st) != cudaSuccess) return RET_ERR_CUDA;
-    const ret_status r = tc::launch_with_scratch<GATED>(q, k, v, decay, o, state_in, state_out, B, H, N, dk, dv,
-                                                        pl, scratch, st, ldq, ldk);
+    const ret_status r = tc::launch_with_scratch<GATED, REV>(q, k, v, decay, o, state_in, state_out, B, H, N, dk,
+                                                             dv, pl, scratch, st, ldq, ldk);
     if (scratch && cudaFreeAsync(scratch, st) != cudaSuccess) return RET_ERR_CUDA;
     return r;
 }

@@ -28,6 +28,13 @@
 //   Z^T  = T_op^T Q^T       M=128 N=128 K=dk           TS (bf16 T copy in TMEM) -> R
 //   Z^T += (zeta V / kappa)^T P^T  M=128 N=128 K=128   SS, P = causal mask of A (bf16)
 // TMEM: S^T (dk columns), its bf16 copy (dk/2), R (128 columns) -- 512 at dk = 256.
+//
+// REV (time-reversed direction, used for the gradients dK and dV): O_j = sum over later
+// tokens i >= j of gamma^(i-j) (q_j . k_i) v_i. The tiles are visited from the last to
+// the first and the state, referenced at the token before the current tile, is
+// R = sum_{i >= t0} gamma^(i-t0+1) k_i^T v_i. Everything above holds with
+// zeta_i = gamma^(i+1) (i the token's place in its tile) and the mask i >= j: the cross
+// factor gamma^(L-1-j) R_next = kappa T / zeta_j with kappa T = gamma^L R_next.
 // Shared memory: one Q, K and V tile, each with its own full/empty barriers so that it
 // reloads as soon as its last reader is done (K after the update, Q after the cross
 // term, V after O_intra), and one P tile that is also the staging tile of the O store.
@@ -77,7 +84,7 @@ __device__ __forceinline__ float lazy_next_scale(float kappa, float decay, bool 
     return renorm ? 1.f : kappa * decay;
 }
 
-template <int DK>
+template <int DK, bool REV>
 __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                                           const CUtensorMap& tm_o, const Params& p, float lg) {
     using Lay = WideLayout<DK>;
@@ -89,13 +96,18 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Lay::kTmemSlot);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // seg: place of this segment in the order the segments are chained (its start state is
+    // the chain's seg-th); tseg: its place in time (REV chains them from the last back)
     const int slice = blockIdx.x, bh = blockIdx.y, seg = blockIdx.z;
+    const int tseg = REV ? p.units - 1 - seg : seg;
     const int dv0 = slice * kDvS;
-    const int tbeg = seg * p.seg_chunks * kC;                 // first token of this segment
+    const int tbeg = tseg * p.seg_chunks * kC;                // first token of this segment
     const int tend = min(tbeg + p.seg_chunks * kC, p.N);      // one past its last token
     const int ntiles = (tend - tbeg + kW - 1) / kW;
-    const bool last_seg = tend >= p.N;
-    auto tile_len = [&](int c) { return min(kW, tend - (tbeg + c * kW)); };
+    const bool last_seg = seg == p.units - 1;                 // the chain's last: writes state_out
+    // token start of the c-th tile visited (REV: from the last tile of the segment back)
+    auto tile_t0 = [&](int c) { return tbeg + (REV ? ntiles - 1 - c : c) * kW; };
+    auto tile_len = [&](int c) { return min(kW, tend - tile_t0(c)); };
 
     if (threadIdx.x == 0) {
         for (int b = 0; b < Lay::kNumBars; ++b) mbar_init(bar(b), 1);
@@ -124,7 +136,7 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
             // past N read as zero.
             int issued[3] = {-1, -1, -1};  // K, Q, V: last tile whose copies were issued
             for (int c = 0; c < ntiles; ++c) {
-                const int t0 = tbeg + c * kW;
+                const int t0 = tile_t0(c);
                 const uint32_t ph = (c - 1) & 1;
                 if (c > 0 && !mbar_wait(bar(wKEmpty), ph, abort_flag)) break;
                 mbar_expect_tx(bar(wKFull), DK / 64 * kBlk);
@@ -230,12 +242,13 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
         };
         float kappa = 1.f;
         for (int c = 0; c < ntiles; ++c) {
-            const int t0 = tbeg + c * kW, L = tile_len(c);
+            const int t0 = tile_t0(c), L = tile_len(c);
             if (c > 0) {
                 bool rn;
                 kappa = lazy_next_scale(kappa, pow_int_log2(lg, L), false, rn);
             }
-            // ---------------- P = causal mask of A in bf16, row j = r (K-major, 128-byte swizzle)
+            // ---------------- P = causal mask of A in bf16, row j = r (K-major, 128-byte swizzle);
+            // REV keeps the upper triangle m >= j instead
             if (!wait_all(wAFull, c & 1)) break;
             tc_fence_after();
             uint32_t pk[64];
@@ -248,10 +261,11 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
                     const int m = hh * 64 + 2 * u;
-                    pk[hh * 32 + u] = pack_bf16(m <= r ? __uint_as_float(a0[2 * u]) : 0.f,
-                                                m + 1 <= r ? __uint_as_float(a0[2 * u + 1]) : 0.f);
-                    pk[hh * 32 + 16 + u] = pack_bf16(m + 32 <= r ? __uint_as_float(a1[2 * u]) : 0.f,
-                                                     m + 33 <= r ? __uint_as_float(a1[2 * u + 1]) : 0.f);
+                    auto keep = [&](int mm) { return REV ? mm >= r : mm <= r; };
+                    pk[hh * 32 + u] = pack_bf16(keep(m) ? __uint_as_float(a0[2 * u]) : 0.f,
+                                                keep(m + 1) ? __uint_as_float(a0[2 * u + 1]) : 0.f);
+                    pk[hh * 32 + 16 + u] = pack_bf16(keep(m + 32) ? __uint_as_float(a1[2 * u]) : 0.f,
+                                                     keep(m + 33) ? __uint_as_float(a1[2 * u + 1]) : 0.f);
                 }
             }
             // A is in registers: the cross term may overwrite R. The previous tile's O store
@@ -271,7 +285,7 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
             group_sync(1);
             if (te == 0) mbar_arrive(bar(wPReady));
             // ---------------- O_j = (kappa / zeta_j) Z_j -> bf16 -> staging -> TMA store
-            rowf[te] = te < L ? kappa * pow_int_log2(-lg, L - 1 - te) : 0.f;
+            rowf[te] = te < L ? kappa * pow_int_log2(-lg, REV ? te + 1 : L - 1 - te) : 0.f;
             if (!wait_all(wOFull, c & 1)) break;
             tc_fence_after();
             {
@@ -344,7 +358,7 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
         // two 16 KB blocks of 128 token rows, so the token of a chunk is (ci mod 1024) / 8.
         auto build_zv = [&](int c, float kappa) {
             const int L = tile_len(c);
-            zk[ts] = ts < L ? pow_int_log2(lg, L - 1 - ts) * (1.f / kappa) : 0.f;
+            zk[ts] = ts < L ? pow_int_log2(lg, REV ? ts + 1 : L - 1 - ts) * (1.f / kappa) : 0.f;
             if (!wait_all(wVFull, c & 1)) return false;
             uint8_t* vt = sm + Lay::kV;
 #pragma unroll

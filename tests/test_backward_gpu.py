@@ -38,6 +38,51 @@ def _check(got, want, dtype, what, tol=None):
     assert err <= tol, f"{what}: rel-L2 {err:.3e} > {tol:.0e}"
 
 
+def _f64(t):
+    return t.detach().to("cpu", torch.float64).numpy() if hasattr(t, "detach") else np.asarray(t, np.float64)
+
+
+def _check_decay_grad(got, q, k, decay, dq, dk, want, want_dq, want_dk, dtype, gated, what):
+    """dgamma (fixed) or dg (gated), which the library forms from a_t = q_t . dQ_t - k_t . dK_t:
+    dgamma_h = (1 / gamma_h) sum_{b,t} t a_t, dg_t = sum_{u>=t} a_u.
+
+    (1) The decay-gradient step itself: the result equals that formula evaluated in fp64 on
+        the library's own dq and dk, to fp32 summation error (1e-4 of the summed magnitudes).
+    (2) Against the oracle: the formula is exact, so the error is what the errors of dq and dk
+        propagate to. Their check allows ||dQ - dQ_ref|| <= tol ||dQ_ref||; by Cauchy-Schwarz
+        |sum_t w_t q_t . (dQ - dQ_ref)_t| <= ||w_t |q_t| || tol ||dQ_ref|| (w_t = t / gamma for
+        dgamma, the suffix indicator for dg), and the same for k and dK. That sum cancels
+        (sum_t a_t = 0): the bound grows with N (1 - gamma^2) while dgamma does not, so the
+        check allows the larger of the bound and tol_decay ||ref||.
+    """
+    tol = TOL_F32 if dtype == torch.float32 else TOL_BF16
+    tol_decay = 1e-3 if dtype == torch.float32 else 5e-2
+    q, k, dq, dk = (_f64(t) for t in (q, k, dq, dk))
+    a = (q * dq).sum(-1) - (k * dk).sum(-1)                    # [B, H, N]
+    mag = np.abs(q * dq).sum(-1) + np.abs(k * dk).sum(-1)
+    qn, kn = np.linalg.norm(q, axis=-1), np.linalg.norm(k, axis=-1)
+    eq, ek = tol * np.linalg.norm(_f64(want_dq)), tol * np.linalg.norm(_f64(want_dk))
+    got, want = _f64(got), _f64(want)
+    N = q.shape[2]
+    if gated:
+        formula = np.flip(np.cumsum(np.flip(a, -1), -1), -1)
+        scale = np.flip(np.cumsum(np.flip(mag, -1), -1), -1)
+        # every suffix sum is bounded through the whole sequence's norms
+        per_row = np.linalg.norm(qn, axis=-1) * eq + np.linalg.norm(kn, axis=-1) * ek   # [B, H]
+        bound = np.sqrt(N * (per_row ** 2).sum())
+    else:
+        t = np.arange(N, dtype=np.float64)
+        gam = _f64(decay)
+        formula = (t * a).sum((0, 2)) / gam
+        scale = (t * mag).sum((0, 2)) / gam
+        per_head = (np.sqrt(((t * qn) ** 2).sum((0, 2))) * eq + np.sqrt(((t * kn) ** 2).sum((0, 2))) * ek) / gam
+        bound = np.linalg.norm(per_head)
+    assert np.all(np.abs(got - formula) <= 1e-4 * scale + 1e-30), f"{what}: differs from its formula on dq, dk"
+    err = np.linalg.norm(got - want)
+    allowed = max(bound, tol_decay * np.linalg.norm(want))
+    assert err <= allowed, f"{what}: error {err:.3e} > {allowed:.3e} (rel-L2 {err / np.linalg.norm(want):.3e})"
+
+
 @pytest.mark.parametrize("B,H,N,dk,dv,dtype", BWD_CASES)
 def test_backward_matches_oracle(cuda_lib, B, H, N, dk, dv, dtype):
     q, k, v, do, _ = _case(B, H, N, dk, dv, dtype, seed=N + dv)
@@ -48,8 +93,7 @@ def test_backward_matches_oracle(cuda_lib, B, H, N, dk, dv, dtype):
     _check(dq, want[0], dtype, "dq")
     _check(dkk, want[1], dtype, "dk")
     _check(dvv, want[2], dtype, "dv")
-    # dgamma is a sum over the sequence of differences q.dq - k.dk: allow for the cancellation
-    _check(dgam, want[3], dtype, "dgamma", tol=1e-3 if dtype == torch.float32 else 5e-2)
+    _check_decay_grad(dgam, q, k, gam, dq, dkk, want[3], want[0], want[1], dtype, False, "dgamma")
 
 
 @pytest.mark.parametrize("B,H,N,dk,dv,dtype", BWD_CASES)
@@ -62,7 +106,7 @@ def test_gated_backward_matches_oracle(cuda_lib, B, H, N, dk, dv, dtype):
     _check(dq, want[0], dtype, "dq")
     _check(dkk, want[1], dtype, "dk")
     _check(dvv, want[2], dtype, "dv")
-    _check(dg, want[3], dtype, "dg", tol=1e-3 if dtype == torch.float32 else 5e-2)
+    _check_decay_grad(dg, q, k, g, dq, dkk, want[3], want[0], want[1], dtype, True, "dg")
 
 
 def test_backward_gradient_of_forward_by_directional_derivative(cuda_lib):
@@ -116,3 +160,47 @@ def test_backward_without_decay_gradient(cuda_lib, gated):
     assert part[3] is None
     for a, b in zip(full[:3], part[:3]):
         assert torch.equal(a, b)
+
+
+# The dK and dV sums run over later tokens; on the tensor-core path they are computed by the
+# time-reversed forward kernels (chunks visited from the last back, upper-triangular mask,
+# mirrored decay factors). These cases reach each body of that kernel: the 128-token body
+# (gamma >= 0.595 with widths 128 or 256), the 64-token body with the merged output
+# accumulator (gamma in [0.5, 0.595)) and with split accumulators (gamma < 0.5, gated), on
+# sequences long enough for few heads to be cut into segments chained from the end, with
+# ragged last chunks.
+REV_CASES = [
+    # B, H, N, dk, dv, gammas (None: gated)
+    (1, 4, 450, 128, 128, [0.3, 0.55, 0.9, 0.999]),
+    (1, 2, 300, 256, 256, [0.2, 0.45]),
+    (2, 2, 700, 256, 512, [0.5, 0.7]),
+    (1, 2, 1333, 128, 128, None),
+    (1, 1, 2049, 256, 256, None),
+]
+
+
+@pytest.mark.parametrize("B,H,N,dk,dv,gams", REV_CASES)
+def test_backward_reversed_kernels_match_oracle(cuda_lib, B, H, N, dk, dv, gams):
+    dtype = torch.bfloat16
+    q, k, v, do, gen = _case(B, H, N, dk, dv, dtype, seed=5 * N + dk)
+    if gams is None:
+        decay = I.gate(B, H, N, gen) * 4.0
+        want = O.gated_backward(q, k, v, decay, do)
+    else:
+        decay = torch.tensor(gams, dtype=torch.float32)
+        want = O.ret_backward(q, k, v, decay, do)
+    got = cuda_lib.chunkwise_backward(*(t.to(DEV) for t in (q, k, v, decay, do)), 64, gated=gams is None)
+    assert cuda_lib.last_device_error() == 0
+    for g, w, what in zip(got[:3], want[:3], ("dq", "dk", "dv")):
+        _check(g, w, dtype, what)
+    _check_decay_grad(got[3], q, k, decay, got[0], got[1], want[3], want[0], want[1], dtype, gams is None,
+                      "dgamma" if gams else "dg")
+
+
+def test_backward_launches_on_tensor_cores(cuda_lib):
+    """The 1.3B-shaped backward launches two dQ pieces, two reversed dK pieces, the reversed
+    dV call, the two piece sums and the decay gradient: no copies of reversed operands."""
+    assert cuda_lib.chunkwise_backward_launches(4, 8, 2048, 256, 512, 64, torch.bfloat16) == 8
+    assert cuda_lib.chunkwise_backward_launches(4, 8, 2048, 256, 512, 64, torch.bfloat16, ddecay=False) == 7
+    # one piece (dv <= 256): dQ and dK write dq and dk directly, no sums
+    assert cuda_lib.chunkwise_backward_launches(4, 8, 2048, 128, 256, 64, torch.bfloat16) == 4

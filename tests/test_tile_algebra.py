@@ -154,3 +154,83 @@ def test_anticausal_tiles_give_dk_and_dv(N, tile, gated):
         dk = _anticausal_model(v, do, q, tile, gamma=gamma)
     np.testing.assert_allclose(dv, want[2][0, 0], rtol=1e-9, atol=1e-10)
     np.testing.assert_allclose(dk, want[1][0, 0], rtol=1e-9, atol=1e-10)
+
+
+# ---------------------------------------------------------------- the reversed kernel's own factors
+#
+# The time-reversed kernel references its carried state at the token before the current tile
+# (the convention of the gated model above): R = sum_{n >= t0} w(n, t0 - 1) b_n^T c_n, so for
+# fixed gamma the key weights are gamma^(i+1), the cross-term row factors gamma^(L-1-j) and the
+# tile decay gamma^L. Its two fixed-decay bodies factor these like the forward's:
+#   128-token body: zeta_i = gamma^(i+1), R = kappa T, kappa T = gamma^L R_next before the update,
+#       o_j = (kappa / zeta_j) [ a_j T + sum_{i>=j} (a_j . b_i) zeta_i c_i / kappa ];
+#   64-token merged accumulator: zeta'_i = gamma^i, the state copy scaled by gamma^(L-1),
+#       o_j = (1 / zeta'_j) [ a_j (gamma^(L-1) R_next) + sum_{i>=j} zeta'_i (a_j . b_i) c_i ].
+
+def _rev_tile_model_128(a, b, c, gamma, renorm=2.0 ** -40):
+    N = a.shape[0]
+    T = np.zeros((b.shape[1], c.shape[1]))
+    kappa = 1.0
+    out = np.zeros((N, c.shape[1]))
+    for t0 in reversed(range(0, N, 128)):
+        L = min(128, N - t0)
+        A_, B_, C_ = a[t0:t0 + L], b[t0:t0 + L], c[t0:t0 + L]
+        zeta = gamma ** (np.arange(L) + 1)
+        if kappa * gamma ** L < renorm:
+            T, kappa = kappa * T, 1.0
+        kappa *= gamma ** L
+        scores = np.triu(A_ @ B_.T)                  # i >= j
+        zc = zeta[:, None] * C_ / kappa
+        out[t0:t0 + L] = (kappa / zeta)[:, None] * (A_ @ T + scores @ zc)
+        T = T + B_.T @ zc
+    return out
+
+
+def _rev_merged_model_64(a, b, c, gamma):
+    N = a.shape[0]
+    R = np.zeros((b.shape[1], c.shape[1]))
+    out = np.zeros((N, c.shape[1]))
+    for t0 in reversed(range(0, N, 64)):
+        L = min(64, N - t0)
+        zp = gamma ** np.arange(L)
+        A_, B_, C_ = a[t0:t0 + L], b[t0:t0 + L], c[t0:t0 + L]
+        P = np.triu(A_ @ B_.T) * zp[None, :]
+        acc = A_ @ (gamma ** (L - 1) * R) + P @ C_
+        out[t0:t0 + L] = acc / zp[:, None]
+        R = gamma ** L * R + (B_ * (gamma ** (np.arange(L) + 1))[:, None]).T @ C_
+    return out
+
+
+@pytest.mark.parametrize("gamma", [0.999, 0.9, 2.0 ** -0.75])
+@pytest.mark.parametrize("N", [128, 300, 517, 1100])
+def test_reversed_128_token_factors_give_dk_and_dv(gamma, N):
+    rng = np.random.default_rng(N + 11)
+    q, k = rng.standard_normal((N, 5)) / 2, rng.standard_normal((N, 5)) / 2
+    v, do = rng.standard_normal((N, 6)) / 2, rng.standard_normal((N, 6)) / 2
+    want = O.ret_backward(q[None, None], k[None, None], v[None, None], np.array([gamma]), do[None, None])
+    np.testing.assert_allclose(_rev_tile_model_128(k, q, do, gamma), want[2][0, 0], rtol=1e-9, atol=1e-10)
+    np.testing.assert_allclose(_rev_tile_model_128(v, do, q, gamma), want[1][0, 0], rtol=1e-9, atol=1e-10)
+
+
+@pytest.mark.parametrize("gamma", [0.5, 0.55, 0.999])
+@pytest.mark.parametrize("N", [64, 100, 257])
+def test_reversed_64_token_merged_factors_give_dk_and_dv(gamma, N):
+    rng = np.random.default_rng(N + 13)
+    q, k = rng.standard_normal((N, 5)) / 2, rng.standard_normal((N, 5)) / 2
+    v, do = rng.standard_normal((N, 6)) / 2, rng.standard_normal((N, 6)) / 2
+    want = O.ret_backward(q[None, None], k[None, None], v[None, None], np.array([gamma]), do[None, None])
+    np.testing.assert_allclose(_rev_merged_model_64(k, q, do, gamma), want[2][0, 0], rtol=1e-9, atol=1e-10)
+    np.testing.assert_allclose(_rev_merged_model_64(v, do, q, gamma), want[1][0, 0], rtol=1e-9, atol=1e-10)
+
+
+def test_reversed_factors_stay_in_range():
+    """128-token body (log2 gamma >= -0.75) and merged 64-token form (gamma >= 1/2): every
+    factor of the reversed direction lies within the normal range of bf16 and fp32."""
+    for gamma in (2.0 ** -0.75, 0.9, 1.0):
+        zeta = gamma ** (np.arange(128) + 1)
+        f = np.log2(np.concatenate([zeta, 1 / zeta, [gamma ** 128]]))
+        assert f.min() >= -96 - 1e-9 and f.max() <= 96 + 1e-9
+    for gamma in (0.5, 0.6, 1.0):
+        zp = gamma ** np.arange(64)
+        f = np.log2(np.concatenate([zp, 1 / zp, [gamma ** 63]]))
+        assert f.min() >= -64 - 1e-9 and f.max() <= 63 + 1e-9
