@@ -311,6 +311,7 @@ __device__ __forceinline__ void warp_cumsum64(float g0, float g1, int lane, floa
 }  // namespace ret
 
 #include "tc_wide.cuh"
+#include "tc_state.cuh"
 
 namespace ret {
 namespace tc {
@@ -933,32 +934,67 @@ constexpr int kMaxSegments = 16;  // segments of a split sequence, at most
 // Segment start states of a split sequence, between the two passes: seg_state[g] holds
 // U_g (segment g's end state from a zero start) on entry and S_in(g + 1) = Gamma_g S_in(g)
 // + U_g on exit, with S_in(0) = state_in (or zero) and Gamma_g = 2^seg_ldec[g]. One thread
-// per 4 consecutive state elements; all of a thread's G - 1 loads are issued before the
-// sequential recurrence, so every full-pass CTA then reads one state instead of folding
-// all earlier segments itself. seg_state is the library's scratch (16-byte aligned);
-// state_in is read element by element (only 4-byte alignment is required of it).
+// per 4 consecutive state elements (no grid-stride loop: the kernel is latency-bound, so
+// every thread issues its NS loads at once and the grid covers the states in one pass);
+// NS = G - 1 states is a template argument so that exactly those loads are in flight.
+// Every full-pass CTA then reads one state instead of folding all earlier segments
+// itself. seg_state is the library's scratch (16-byte aligned); state_in is read element
+// by element (only 4-byte alignment is required of it).
+template <int NS>
 __global__ void __launch_bounds__(256)
 seg_prefix_kernel(const float* __restrict__ state_in, float* __restrict__ seg_state, const float* __restrict__ seg_ldec,
-                  int G, int BH, int per_bh) {
+                  int BH, int per_bh) {
     const size_t n4 = (size_t)BH * per_bh / 4;
-    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
-        const int bh = (int)(i * 4 / per_bh);
-        float4 u[kMaxSegments - 1];
+    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n4) return;
+    const int bh = (int)(i * 4 / per_bh);
+    float4 u[NS];
+    float gam[NS];
 #pragma unroll
-        for (int g = 0; g < kMaxSegments - 1; ++g)
-            if (g < G - 1) u[g] = reinterpret_cast<const float4*>(seg_state + (size_t)g * BH * per_bh)[i];
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (state_in) x = make_float4(state_in[4 * i], state_in[4 * i + 1], state_in[4 * i + 2], state_in[4 * i + 3]);
-#pragma unroll
-        for (int g = 0; g < kMaxSegments - 1; ++g) {
-            if (g < G - 1) {
-                const float gam = exp2f(seg_ldec[(size_t)g * BH + bh]);
-                x = make_float4(fmaf(gam, x.x, u[g].x), fmaf(gam, x.y, u[g].y), fmaf(gam, x.z, u[g].z),
-                                fmaf(gam, x.w, u[g].w));
-                reinterpret_cast<float4*>(seg_state + (size_t)g * BH * per_bh)[i] = x;
-            }
-        }
+    for (int g = 0; g < NS; ++g) {
+        u[g] = __ldcs(reinterpret_cast<const float4*>(seg_state + (size_t)g * BH * per_bh) + i);
+        gam[g] = seg_ldec[(size_t)g * BH + bh];
     }
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (state_in) x = make_float4(state_in[4 * i], state_in[4 * i + 1], state_in[4 * i + 2], state_in[4 * i + 3]);
+#pragma unroll
+    for (int g = 0; g < NS; ++g) {
+        const float d = exp2f(gam[g]);
+        x = make_float4(fmaf(d, x.x, u[g].x), fmaf(d, x.y, u[g].y), fmaf(d, x.z, u[g].z), fmaf(d, x.w, u[g].w));
+        reinterpret_cast<float4*>(seg_state + (size_t)g * BH * per_bh)[i] = x;
+    }
+}
+
+template <int NS>
+inline void launch_seg_prefix_n(const float* state_in, float* seg_state, const float* seg_ldec, int BH, int per_bh,
+                                unsigned blocks, cudaStream_t st) {
+    seg_prefix_kernel<NS><<<blocks, 256, 0, st>>>(state_in, seg_state, seg_ldec, BH, per_bh);
+}
+
+// Launches the prefix over `ns` segment states (1 <= ns < kMaxSegments).
+inline cudaError_t launch_seg_prefix(const float* state_in, float* seg_state, const float* seg_ldec, int ns, int BH,
+                                     int per_bh, cudaStream_t st) {
+    const size_t n4 = (size_t)BH * per_bh / 4;
+    const unsigned blocks = (unsigned)((n4 + 255) / 256);
+    switch (ns) {
+        case 1: launch_seg_prefix_n<1>(state_in, seg_state, seg_ldec, BH, per_bh, blocks, st); break;
+        case 2: launch_seg_prefix_n<2>(state_in, seg_state, seg_ldec, BH, per_bh, blocks, st); break;
+        case 3: launch_seg_prefix_n<3>(state_in, seg_state, seg_ldec, BH, per_bh, blocks, st); break;
+        case 4: launch_seg_prefix_n<4>(state_in, seg_state, seg_ldec, BH, per_bh, blocks, st); break;
+        case 5: launch_seg_prefix_n<5>(state_in, seg_state, seg_ldec, BH, per_bh, blocks, st); break;
+        case 6: launch_seg_prefix_n<6>(state_in, seg_state, seg_ldec, BH, per_bh, blocks, st); break;
+        case 7: launch_seg_prefix_n<7>(state_in, seg_state, seg_ldec, BH, per_bh, blocks, st); break;
+        case 8: launch_seg_prefix_n<8>(state_in, seg_state, seg_ldec, BH, per_bh, blocks, st); break;
+        case 9: launch_seg_prefix_n<9>(state_in, seg_state, seg_ldec, BH, per_bh, blocks, st); break;
+        case 10: launch_seg_prefix_n<10>(state_in, seg_state, seg_ldec, BH, per_bh, blocks, st); break;
+        case 11: launch_seg_prefix_n<11>(state_in, seg_state, seg_ldec, BH, per_bh, blocks, st); break;
+        case 12: launch_seg_prefix_n<12>(state_in, seg_state, seg_ldec, BH, per_bh, blocks, st); break;
+        case 13: launch_seg_prefix_n<13>(state_in, seg_state, seg_ldec, BH, per_bh, blocks, st); break;
+        case 14: launch_seg_prefix_n<14>(state_in, seg_state, seg_ldec, BH, per_bh, blocks, st); break;
+        case 15: launch_seg_prefix_n<15>(state_in, seg_state, seg_ldec, BH, per_bh, blocks, st); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
 }
 
 // Self-test of the failure path: one CTA takes TMEM like the chunk kernels, waits with
@@ -1142,10 +1178,11 @@ constexpr int kernel_smem() {
 // while the previous kernel in the stream finishes, and wait (griddepcontrol.wait, the
 // kernel's first instruction) until that kernel has completed.
 template <typename... P, typename... A>
-inline cudaError_t launch_dependent(void (*kernel)(P...), dim3 grid, size_t smem, cudaStream_t st, A&&... args) {
+inline cudaError_t launch_dependent(void (*kernel)(P...), dim3 grid, int threads, size_t smem, cudaStream_t st,
+                                    A&&... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -1177,25 +1214,23 @@ ret_status launch_dk(const void* q, const void* k, const void* v, const float* d
                 return RET_ERR_CUDA;
             prm.state_in = copy;
         }
-        auto k1 = chunk_tc_kernel<DK, GATED, true, REV>;
-        constexpr int smem1 = kernel_smem<DK, GATED, true>();
+        auto k1 = state_tc_kernel<DK, GATED, REV>;
+        constexpr int smem1 = StateLayout<DK>::kSmemAlloc;
         if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1) != cudaSuccess)
             return RET_ERR_CUDA;
         Params prm1 = prm;  // the state-only pass runs over the sub-segments
         prm1.seg_chunks = pl.seg_chunks / pl.F;
         prm1.units = pl.F * pl.G;
-        if (launch_dependent(k1, dim3(dv / kDvS, BH, pl.subs()), smem1, st, mq, mk, mv, mo, prm1) != cudaSuccess)
+        if (launch_dependent(k1, dim3(dv / kDvS, BH, pl.subs()), kSThreads, smem1, st, mk, mv, prm1) != cudaSuccess)
             return RET_ERR_CUDA;
-        const int n4 = BH * DK * dv / 4;
-        seg_prefix_kernel<<<std::min((n4 + 255) / 256, 4 * sm_count()), 256, 0, st>>>(
-            prm.state_in, prm.seg_state, prm.seg_ldec, pl.subs() + 1, BH, DK * dv);
-        if (cudaGetLastError() != cudaSuccess) return RET_ERR_CUDA;
+        if (launch_seg_prefix(prm.state_in, prm.seg_state, prm.seg_ldec, pl.subs(), BH, DK * dv, st) != cudaSuccess)
+            return RET_ERR_CUDA;
     }
     auto k2 = chunk_tc_kernel<DK, GATED, false, REV>;
     constexpr int smem2 = kernel_smem<DK, GATED, false>();
     if (cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2) != cudaSuccess)
         return RET_ERR_CUDA;
-    return launch_dependent(k2, dim3(dv / kDvS, BH, pl.G), smem2, st, mq, mk, mv, mo, prm) == cudaSuccess ? RET_OK
+    return launch_dependent(k2, dim3(dv / kDvS, BH, pl.G), kThreads, smem2, st, mq, mk, mv, mo, prm) == cudaSuccess ? RET_OK
                                                                                                      : RET_ERR_CUDA;
 }
 
@@ -1270,17 +1305,14 @@ ret_status launch_state_dk(const void* k, const void* v, const float* decay, flo
     float* states = subs > 1 ? reinterpret_cast<float*>(sc) : state_out;
     float* ldec = reinterpret_cast<float*>(sc + (subs > 1 ? sizeof(float) * (size_t)subs * BH * DK * dv : 0));
     Params prm{decay, nullptr, nullptr, states, ldec, H, N, dv, sub_chunks, 1, subs};
-    auto k1 = chunk_tc_kernel<DK, GATED, true, false>;
-    constexpr int smem1 = kernel_smem<DK, GATED, true>();
+    auto k1 = state_tc_kernel<DK, GATED, false>;
+    constexpr int smem1 = StateLayout<DK>::kSmemAlloc;
     if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1) != cudaSuccess)
         return RET_ERR_CUDA;
-    if (launch_dependent(k1, dim3(dv / kDvS, BH, subs), smem1, st, mk, mk, mv, mv, prm) != cudaSuccess)
+    if (launch_dependent(k1, dim3(dv / kDvS, BH, subs), kSThreads, smem1, st, mk, mv, prm) != cudaSuccess)
         return RET_ERR_CUDA;
     if (subs > 1) {
-        const int n4 = BH * DK * dv / 4;
-        seg_prefix_kernel<<<std::min((n4 + 255) / 256, 4 * sm_count()), 256, 0, st>>>(nullptr, states, ldec, subs + 1,
-                                                                                       BH, DK * dv);
-        if (cudaGetLastError() != cudaSuccess) return RET_ERR_CUDA;
+        if (launch_seg_prefix(nullptr, states, ldec, subs, BH, DK * dv, st) != cudaSuccess) return RET_ERR_CUDA;
         if (cudaMemcpyAsync(state_out, states + (size_t)(subs - 1) * BH * DK * dv, sizeof(float) * (size_t)BH * DK * dv,
                             cudaMemcpyDeviceToDevice, st) != cudaSuccess)
             return RET_ERR_CUDA;

@@ -1,0 +1,290 @@
+// State-only pass of a split sequence (sm_100a): the end state of each sub-segment from a
+// zero start and its total decay, without outputs. Included by tc_chunk.cuh.
+//
+// Method: "RetNet retention mechanism" (aiqz.cc), section 块级循环 (the state carried
+// between chunks, S_i = decay_i S_{i-1} + K_i^T diag(zeta) V_i), and the Gated RetNet
+// page's cross_chunk update with per-token decays. Only the update product runs here:
+//   S^T += (zeta V / kappa)^T K     M = 128 (dv slice)  N = dk  K = 128 tokens   (SS, both MN-major)
+// over 128-token tiles, with the state held as S = kappa T (T in TMEM, the scalar kappa in
+// registers; T is rescaled in place only when kappa would fall below 2^-40).
+//
+// Roles (192 threads): warp 0 issues the TMA loads (2 or 3 stages of a K tile and a V
+// tile), warp 1 allocates TMEM and issues the products, warps 2-5 turn each V tile into
+// zeta V / kappa in place and finally write kappa T. REV visits the tiles from the last
+// back with the reversed direction's key weights (see chunk_tc_kernel). All waits are
+// bounded like the other bodies'.
+#pragma once
+
+namespace ret {
+namespace tc {
+
+constexpr int kSThreads = 192;
+
+template <int DK>
+struct StateLayout {
+    static constexpr int kKBytes = DK / 64 * kBlk;             // 128 token rows x DK
+    static constexpr int kVBytes = 2 * kBlk;                    // 128 token rows x 128 dv
+    static constexpr int kStageBytes = kKBytes + kVBytes;
+    static constexpr int kStages = (3 * kStageBytes <= 200 * 1024) ? 3 : 2;
+    static constexpr int kBar = kStages * kStageBytes;
+    static constexpr int kNumBars = 12;                         // full[3], empty[3], zv[3], upd, drain
+    static constexpr int kTab = kBar + kNumBars * 8;            // zeta / kappa [128], gated cumsum [128]
+    static constexpr int kTmemSlot = kTab + 2 * kW * 4;
+    static constexpr int kAbort = kTmemSlot + 4;
+    static constexpr int kBytes = kAbort + 4;
+    static constexpr int kSmemAlloc = kBytes + 1024;            // slack to align the base to 1024 B
+    static constexpr int kTmemCols = DK <= 32 ? 32 : DK <= 64 ? 64 : DK <= 128 ? 128 : 256;
+    static_assert(kSmemAlloc <= 227 * 1024, "shared memory overflow");
+};
+
+enum StateBar { sFull0 = 0, sEmpty0 = 3, sZV0 = 6, sUpd = 9, sDrain = 10 };
+
+// Inclusive cumulative sum over 128 values in log2 units by one warp: lane l holds
+// x[4l .. 4l+3]; writes cum[0..127].
+__device__ __forceinline__ void warp_cumsum128(const float (&x)[4], int lane, float* cum) {
+    const float p1 = x[0] + x[1], p2 = p1 + x[2], p3 = p2 + x[3];
+    float incl = p3;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    const float excl = incl - p3;
+    cum[4 * lane] = excl + x[0];
+    cum[4 * lane + 1] = excl + p1;
+    cum[4 * lane + 2] = excl + p2;
+    cum[4 * lane + 3] = excl + p3;
+}
+
+// Grid: (dv / 128, B*H, sub-segments). p.seg_chunks: 64-token chunks per sub-segment;
+// p.units: sub-segments the whole sequence is cut into (REV counts them from the end).
+// Writes sub-segment z's end state to seg_state[z] and log2 of its total decay to
+// seg_ldec[z].
+template <int DK, bool GATED, bool REV>
+__global__ void __launch_bounds__(kSThreads, 1)
+state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, Params p) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    using Lay = StateLayout<DK>;
+    constexpr int NS = Lay::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    auto bar = [&](int b) { return sbase + Lay::kBar + 8 * b; };
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Lay::kAbort);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Lay::kTmemSlot);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int slice = blockIdx.x, bh = blockIdx.y, seg = blockIdx.z;
+    const int dv0 = slice * kDvS;
+    const int tseg = REV ? p.units - 1 - seg : seg;
+    const int tbeg = tseg * p.seg_chunks * kC;
+    const int tend = min(tbeg + p.seg_chunks * kC, p.N);
+    const int ntiles = tend > tbeg ? (tend - tbeg + kW - 1) / kW : 0;
+    float* so = p.seg_state + ((size_t)seg * gridDim.y + bh) * DK * p.dv + dv0;
+    if (ntiles == 0) {
+        // REV only: a sub-segment past the end of a short last segment: zero state, no decay
+        for (int e = threadIdx.x; e < DK * kDvS; e += blockDim.x) so[(size_t)(e / kDvS) * p.dv + e % kDvS] = 0.f;
+        if (slice == 0 && threadIdx.x == 0) p.seg_ldec[(size_t)seg * gridDim.y + bh] = 0.f;
+        return;
+    }
+    auto tile_t0 = [&](int c) { return tbeg + (REV ? ntiles - 1 - c : c) * kW; };
+    auto tile_len = [&](int c) { return min(kW, tend - tile_t0(c)); };
+
+    if (threadIdx.x == 0) {
+        for (int b = 0; b < Lay::kNumBars; ++b) mbar_init(bar(b), 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_k)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_v)) : "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(tmem_slot)), "r"(Lay::kTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int issued = -1;
+            for (int c = 0; c < ntiles; ++c) {
+                const int s = c % NS;
+                if (c >= NS && !mbar_wait(bar(sEmpty0 + s), ((c / NS) - 1) & 1, abort_flag)) break;
+                const uint32_t st = sbase + s * Lay::kStageBytes;
+                const int t0 = tile_t0(c);
+                mbar_expect_tx(bar(sFull0 + s), Lay::kStageBytes);
+#pragma unroll
+                for (int kb = 0; kb < DK / 64; ++kb)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        tma_load_3d(st + kb * kBlk + h * kTile64, &tm_k, kb * 64, t0 + 64 * h, bh, bar(sFull0 + s));
+#pragma unroll
+                for (int db = 0; db < 2; ++db)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        tma_load_3d(st + Lay::kKBytes + db * kBlk + h * kTile64, &tm_v, dv0 + 64 * db, t0 + 64 * h, bh,
+                                    bar(sFull0 + s));
+                issued = c;
+            }
+            if (*abort_flag && issued >= 0) {
+                // drain the copies in flight before the CTA may exit
+                for (int c = std::max(issued - NS + 1, 0); c <= issued; ++c)
+                    mbar_drain(bar(sFull0 + c % NS), (c / NS) & 1);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t id_up = idesc(128, DK, 1, 1);
+            for (int c = 0; c < ntiles; ++c) {
+                const int s = c % NS;
+                const uint32_t sK = sbase + s * Lay::kStageBytes, sZ = sK + Lay::kKBytes;
+                if (!mbar_wait(bar(sFull0 + s), (c / NS) & 1, abort_flag) ||
+                    !mbar_wait(bar(sZV0 + s), (c / NS) & 1, abort_flag))
+                    break;
+                tc_fence_after();
+                // S^T += (zeta V / kappa)^T K: A = the scaled V tile MN-major (dv blocks 16 KB apart),
+                // B = K tile MN-major (dk blocks 16 KB apart), 16 tokens per step
+#pragma unroll
+                for (int ks = 0; ks < kW / 16; ++ks)
+                    mma_ss(tmem, sdesc(sZ + ks * 2048, kBlk, 1024), sdesc(sK + ks * 2048, kBlk, 1024), id_up,
+                           (c > 0 || ks > 0) ? 1u : 0u);
+                mma_commit(bar(sEmpty0 + s));
+                mma_commit(bar(sUpd));
+            }
+            mma_commit(bar(sDrain));
+            mbar_drain(bar(sDrain), 0);
+        }
+    } else {
+        // ------------------------------------------------------------ state epilogue (warps 2..5)
+        const int ts = threadIdx.x - 64;  // 0..127
+        const int quarter = warp & 3;     // TMEM lane quarter this warp may access
+        const int d = quarter * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        float* zk = reinterpret_cast<float*>(sm + Lay::kTab);   // zeta_m / kappa of the current tile
+        float* cum = zk + kW;                                    // gated: in-tile cumulative log2 decay
+        auto wait_all = [&](int b, uint32_t parity) {
+            mbar_wait(bar(b), parity, abort_flag);
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            return *abort_flag == 0;
+        };
+        const float lg = GATED ? 0.f : log2f(p.decay_in[bh % p.H]);
+        const float* G = GATED ? p.decay_in + (size_t)bh * p.N : nullptr;
+        float gx[4] = {0.f, 0.f, 0.f, 0.f};  // gated: this lane's four gates of the next tile (warp 2)
+        auto load_gates = [&](int c) {
+            if (GATED && ts < 32) {
+                const int t0 = tile_t0(c), L = tile_len(c);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) gx[i] = 4 * ts + i < L ? G[t0 + 4 * ts + i] * kLog2e : 0.f;
+            }
+        };
+        load_gates(0);
+        float kappa = 1.f, ldec_sum = 0.f;
+        bool ok = true;
+        for (int c = 0; c < ntiles && ok; ++c) {
+            const int s = c % NS, L = tile_len(c);
+            // tile decay (log2) and key weights
+            float ldec;
+            if (GATED) {
+                if (ts < 32) {
+                    warp_cumsum128(gx, lane, cum);
+                    if (c + 1 < ntiles) load_gates(c + 1);
+                }
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                ldec = cum[L - 1];
+            } else {
+                ldec = lg * (float)L;
+            }
+            const float dec = GATED ? exp2f(ldec) : pow_int_log2(lg, L);
+            bool renorm;
+            const float k_next = lazy_next_scale(kappa, dec, false, renorm);
+            if (renorm && c > 0) {
+                // T <- kappa dec T once the previous update has landed, so that with kappa = 1 the
+                // next update adds onto the decayed state
+                if (!wait_all(sUpd, (c - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const float sc = kappa * dec;
+#pragma unroll 1
+                for (int cb = 0; cb < DK / 32; ++cb) {
+                    uint32_t w[32];
+                    tmem_ld32(tmem + lane_off + cb * 32, w);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * sc);
+                    tmem_st32(tmem + lane_off + cb * 32, w);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+            }
+            kappa = k_next;
+            ldec_sum += ldec;
+            {
+                const float inv = 1.f / kappa;
+                float z;
+                if (GATED) z = REV ? exp2f(cum[ts]) : exp2f(cum[L - 1] - cum[ts]);
+                else z = pow_int_log2(lg, REV ? ts + 1 : L - 1 - ts);
+                zk[ts] = ts < L ? z * inv : 0.f;
+            }
+            if (!wait_all(sFull0 + s, (c / NS) & 1)) {  // the V tile landed (and zk is complete)
+                ok = false;
+                break;
+            }
+            uint8_t* vt = sm + s * Lay::kStageBytes + Lay::kKBytes;
+#pragma unroll
+            for (int pass = 0; pass < 2; ++pass) {
+                uint4 x[8];
+                float z[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {  // all loads before any store
+                    const int ci = (pass * 8 + e) * 128 + ts;
+                    z[e] = zk[(ci & 1023) >> 3];
+                    x[e] = *reinterpret_cast<const uint4*>(vt + ci * 16);
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    float2 f;
+                    f = unpack_bf16(x[e].x); x[e].x = pack_bf16(f.x * z[e], f.y * z[e]);
+                    f = unpack_bf16(x[e].y); x[e].y = pack_bf16(f.x * z[e], f.y * z[e]);
+                    f = unpack_bf16(x[e].z); x[e].z = pack_bf16(f.x * z[e], f.y * z[e]);
+                    f = unpack_bf16(x[e].w); x[e].w = pack_bf16(f.x * z[e], f.y * z[e]);
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) *reinterpret_cast<uint4*>(vt + ((pass * 8 + e) * 128 + ts) * 16) = x[e];
+            }
+            fence_proxy_async();
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (ts == 0) mbar_arrive(bar(sZV0 + s));
+        }
+        // the end state S = kappa T, rows dk of column dv0 + d, and the total decay
+        if (ok && wait_all(sUpd, (ntiles - 1) & 1)) {
+            tc_fence_after();
+#pragma unroll 1
+            for (int cb = 0; cb < DK / 32; ++cb) {
+                uint32_t w[32];
+                tmem_ld32(tmem + lane_off + cb * 32, w);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) so[(size_t)(cb * 32 + i) * p.dv + d] = __uint_as_float(w[i]) * kappa;
+            }
+            if (slice == 0 && ts == 0) p.seg_ldec[(size_t)seg * gridDim.y + bh] = ldec_sum;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(Lay::kTmemCols)
+                     : "memory");
+    }
+}
+
+}  // namespace tc
+}  // namespace ret
