@@ -66,6 +66,7 @@ struct WideLayout {
     static constexpr int kColR = DK + DK / 2;
     static constexpr int kTmemCols = kColR + kW <= 256 ? 256 : 512;
     static_assert(kColR + kW <= 512, "TMEM overflow");
+    static_assert(kAgTab % 16 == 0 && kSgTab % 16 == 0, "row-factor tables are read as float4");
     static_assert(kSmemAlloc <= 227 * 1024, "shared memory overflow");
 };
 
@@ -289,41 +290,43 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
             if (!wait_all(wOFull, c & 1)) break;
             tc_fence_after();
             {
-                uint32_t z[4][32];
+                // Z^T (dv lanes x 128 token columns) read as 16-lane x 8-column fragments:
+                // z[hf][th] holds lanes quarter*32 + 16 hf + {g, g + 8} (g = lane / 4) and token
+                // columns 64 th + 8k + 2 (lane % 4) + {0, 1}, k = 0..7 -- pairs of adjacent tokens
+                // of one dv column, the register layout stmatrix .trans writes as 8 x 8 blocks of
+                // (token rows x dv columns) into the staging tiles.
+                uint32_t z[2][2][32];
 #pragma unroll
-                for (int h = 0; h < 4; ++h) tmem_ld32(tR + h * 32, z[h]);
+                for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+                    for (int th = 0; th < 2; ++th) tmem_ld16x256b_x8(tR + ((uint32_t)(16 * hf) << 16) + 64 * th, z[hf][th]);
                 tmem_wait_ld();
                 tc_fence_before();
                 group_sync(1);
                 if (te == 0) mbar_arrive(bar(wOFree));
-                // row factors into registers before the first shared store (aliasing)
+                const int g = lane >> 2, i2 = 2 * (lane & 3);
 #pragma unroll
-                for (int h = 0; h < 4; ++h)
+                for (int th = 0; th < 2; ++th) {
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj)
-                        z[h][jj] = __float_as_uint(rowf[h * 32 + jj] * __uint_as_float(z[h][jj]));
-                // Thread r owns dv column d = r for all 128 tokens. A lane-pair shuffle packs two
-                // adjacent dv columns into one 4-byte store: even lanes store token j, odd lanes
-                // token j + 4 (disjoint banks under the 128-byte swizzle). Staging block
-                // (token half th, dv half db) is the 64 x 64 box at kP + (2 th + db) * 8 KB.
-                const bool odd = lane & 1;
-                const int cb = ((r & 63) & ~1) * 2;  // byte offset of the dv pair inside a 128-byte row
+                    for (int k = 0; k < 8; k += 2) {
+                        // row factors of tokens 64 th + 8k' + i2 + {0, 1}, k' = k, k + 1
+                        const float2 f0 = reinterpret_cast<const float2*>(rowf)[(64 * th + 8 * k + i2) >> 1];
+                        const float2 f1 = reinterpret_cast<const float2*>(rowf)[(64 * th + 8 * k + 8 + i2) >> 1];
+                        // block b = 2 (k' - k) + (dv half of the 16 lanes); thread lane supplies the
+                        // address of block lane / 8, row lane % 8 (token 64 th + 8 (k + b / 2) + lane % 8)
+                        const int b = lane >> 3, q = lane & 7;
+                        const int jr = 8 * (k + (b >> 1)) + q;  // token row inside the 64-token box
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    uint8_t* ost = sm + Lay::kP + ((h >> 1) * 2 + (r >> 6)) * kTile64;
-                    const float* o = reinterpret_cast<const float*>(z[h]);
-                    uint32_t w[16];
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) {
-                        const int ja = 8 * (u >> 2) + (u & 3);  // token pair (ja, ja + 4) inside the 32-token block
-                        const float send = odd ? o[ja] : o[ja + 4];
-                        const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-                        w[u] = odd ? pack_bf16(recv, o[ja + 4]) : pack_bf16(o[ja], recv);
-                    }
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) {
-                        const int jr = (h & 1) * 32 + 8 * (u >> 2) + (u & 3) + (odd ? 4 : 0);  // row in the box
-                        *reinterpret_cast<uint32_t*>(ost + jr * 128 + ((((cb >> 4) ^ (jr & 7)) << 4) | (cb & 15))) = w[u];
+                        for (int hf = 0; hf < 2; ++hf) {
+                            const uint32_t* zz = z[hf][th];
+                            const uint32_t r0 = pack_bf16(f0.x * __uint_as_float(zz[4 * k]), f0.y * __uint_as_float(zz[4 * k + 1]));
+                            const uint32_t r1 = pack_bf16(f0.x * __uint_as_float(zz[4 * k + 2]), f0.y * __uint_as_float(zz[4 * k + 3]));
+                            const uint32_t r2 = pack_bf16(f1.x * __uint_as_float(zz[4 * k + 4]), f1.y * __uint_as_float(zz[4 * k + 5]));
+                            const uint32_t r3 = pack_bf16(f1.x * __uint_as_float(zz[4 * k + 6]), f1.y * __uint_as_float(zz[4 * k + 7]));
+                            const int dvb = quarter * 32 + 16 * hf + 8 * (b & 1);  // first dv column of the block
+                            const uint32_t box = sbase + Lay::kP + (2 * th + (dvb >> 6)) * kTile64;
+                            stmatrix_x4_trans(box + jr * 128 + (((((dvb & 63) >> 3) ^ (jr & 7))) << 4), r0, r1, r2, r3);
+                        }
                     }
                 }
             }
