@@ -680,62 +680,42 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (!wait_all(kOFull0 + b, ause(ci) & 1)) return false;
             tc_fence_after();
             {
-                // Each thread owns dv column d for all 64 tokens. A lane-pair shuffle packs two
-                // adjacent dv columns into one 4-byte store: even lanes store token j, odd lanes
-                // token j + 4. With the 128-byte swizzle those two rows hit disjoint banks.
-                const bool odd = lane & 1;
-                const int cb = ((d & 63) & ~1) * 2;  // byte offset of the dv pair inside a 128-byte row
-                uint8_t* ost = sm + Lay::kOst + (d >> 6) * kTile64;
-                // The accumulators of all 64 tokens into registers first, then release the TMEM
-                // columns so the next chunk's Q K^T can start while this drain finishes.
-                uint32_t oi[2][32];
-                if (merged) {
+                // The output accumulators read as 16-lane x 8-column fragments: lanes quarter*32 +
+                // 16 hf + {g, g + 8} (g = lane / 4), token columns 8k + 2 (lane % 4) + {0, 1}, i.e.
+                // pairs of adjacent tokens of one dv column, which stmatrix .trans writes as 8 x 8
+                // blocks of (token rows x dv columns) into the two staging boxes (dv halves).
+                // All of them are read before the TMEM columns are released to the next chunk.
+                uint32_t zi[2][32], ze[2][32];  // merged: the one accumulator; split: O_intra, O_inter
 #pragma unroll
-                    for (int jb = 0; jb < 2; ++jb) tmem_ld32(tA + jb * 32, oi[jb]);
-                    tmem_wait_ld();
-                    tc_fence_before();
-                    group_sync(1);
-                    if (te == 0) mbar_arrive(bar(kOFree0 + b));
-                    // O_j = Z_j / zeta'_j, every table read before the first shared store (aliasing)
-#pragma unroll
-                    for (int jb = 0; jb < 2; ++jb)
-#pragma unroll
-                        for (int jj = 0; jj < 32; ++jj)
-                            oi[jb][jj] = __float_as_uint(rrb[jb * 32 + jj] * __uint_as_float(oi[jb][jj]));
-                } else {
-                    uint32_t oe[2][32];
-#pragma unroll
-                    for (int jb = 0; jb < 2; ++jb) {
-                        tmem_ld32(tA + kC + jb * 32, oi[jb]);
-                        tmem_ld32(tA + jb * 32, oe[jb]);
-                    }
-                    tmem_wait_ld();
-                    tc_fence_before();
-                    group_sync(1);
-                    if (te == 0) mbar_arrive(bar(kOFree0 + b));
-                    // O = O_intra + r_j O_inter in place, every table read before the first shared store
-#pragma unroll
-                    for (int jb = 0; jb < 2; ++jb)
-#pragma unroll
-                        for (int jj = 0; jj < 32; ++jj)
-                            oi[jb][jj] = __float_as_uint(
-                                fmaf(rrb[jb * 32 + jj], __uint_as_float(oe[jb][jj]), __uint_as_float(oi[jb][jj])));
+                for (int hf = 0; hf < 2; ++hf) {
+                    const uint32_t lh = (uint32_t)(16 * hf) << 16;
+                    tmem_ld16x256b_x8(tA + lh + (merged ? 0 : kC), zi[hf]);
+                    if (!merged) tmem_ld16x256b_x8(tA + lh, ze[hf]);
                 }
+                tmem_wait_ld();
+                tc_fence_before();
+                group_sync(1);
+                if (te == 0) mbar_arrive(bar(kOFree0 + b));
+                const int i2 = 2 * (lane & 3), bk = lane >> 3, q = lane & 7;
 #pragma unroll
-                for (int jb = 0; jb < 2; ++jb) {
-                    const float* o = reinterpret_cast<const float*>(oi[jb]);
-                    uint32_t w[16];
+                for (int k = 0; k < 8; k += 2) {
+                    // row factors of tokens 8k' + i2 + {0, 1}, k' = k, k + 1 (read before any shared store)
+                    const float2 f0 = reinterpret_cast<const float2*>(rrb)[(8 * k + i2) >> 1];
+                    const float2 f1 = reinterpret_cast<const float2*>(rrb)[(8 * k + 8 + i2) >> 1];
+                    const int jr = 8 * (k + (bk >> 1)) + q;  // token row of the block row this lane addresses
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) {
-                        const int ja = 8 * (u >> 2) + (u & 3);  // token pair (ja, ja + 4) inside the block
-                        const float send = odd ? o[ja] : o[ja + 4];
-                        const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-                        w[u] = odd ? pack_bf16(recv, o[ja + 4]) : pack_bf16(o[ja], recv);
-                    }
+                    for (int hf = 0; hf < 2; ++hf) {
+                        float o[8];
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) {
-                        const int j = jb * 32 + 8 * (u >> 2) + (u & 3) + (odd ? 4 : 0);
-                        *reinterpret_cast<uint32_t*>(ost + j * 128 + ((((cb >> 4) ^ (j & 7)) << 4) | (cb & 15))) = w[u];
+                        for (int e = 0; e < 8; ++e) {
+                            const float f = e < 4 ? ((e & 1) ? f0.y : f0.x) : ((e & 1) ? f1.y : f1.x);
+                            const float a = __uint_as_float(zi[hf][4 * k + e]);
+                            o[e] = merged ? f * a : fmaf(f, __uint_as_float(ze[hf][4 * k + e]), a);
+                        }
+                        const int dvb = quarter * 32 + 16 * hf + 8 * (bk & 1);  // first dv column of the block
+                        const uint32_t box = sbase + Lay::kOst + (dvb >> 6) * kTile64;
+                        stmatrix_x4_trans(box + jr * 128 + ((((dvb & 63) >> 3) ^ (jr & 7)) << 4), pack_bf16(o[0], o[1]),
+                                          pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]), pack_bf16(o[6], o[7]));
                     }
                 }
             }
