@@ -27,7 +27,7 @@ struct StateLayout {
     static constexpr int kStageBytes = kKBytes + kVBytes;
     static constexpr int kStages = (3 * kStageBytes <= 200 * 1024) ? 3 : 2;
     static constexpr int kBar = kStages * kStageBytes;
-    static constexpr int kNumBars = 12;                         // full[3], empty[3], zv[3], upd, drain
+    static constexpr int kNumBars = 13;                         // full[3], empty[3], zv[3], upd[3], drain
     static constexpr int kTab = kBar + kNumBars * 8;            // zeta / kappa [128], gated cumsum [128]
     static constexpr int kTmemSlot = kTab + 2 * kW * 4;
     static constexpr int kAbort = kTmemSlot + 4;
@@ -37,7 +37,11 @@ struct StateLayout {
     static_assert(kSmemAlloc <= 227 * 1024, "shared memory overflow");
 };
 
-enum StateBar { sFull0 = 0, sEmpty0 = 3, sZV0 = 6, sUpd = 9, sDrain = 10 };
+// upd[s]: the update of a tile in stage s has completed. One per stage, like the others, so
+// that a wait for a given tile's update is never more than one phase behind: the epilogue
+// waits on it only now and then (renormalisation, the end), and a single barrier could by
+// then have completed two phases, which a parity wait cannot tell from none.
+enum StateBar { sFull0 = 0, sEmpty0 = 3, sZV0 = 6, sUpd0 = 9, sDrain = 12 };
 
 // Inclusive cumulative sum over 128 values in log2 units by one warp: lane l holds
 // x[4l .. 4l+3]; writes cum[0..127].
@@ -154,7 +158,7 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     mma_ss(tmem, sdesc(sZ + ks * 2048, kBlk, 1024), sdesc(sK + ks * 2048, kBlk, 1024), id_up,
                            (c > 0 || ks > 0) ? 1u : 0u);
                 mma_commit(bar(sEmpty0 + s));
-                mma_commit(bar(sUpd));
+                mma_commit(bar(sUpd0 + s));
             }
             mma_commit(bar(sDrain));
             mbar_drain(bar(sDrain), 0);
@@ -205,7 +209,7 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             if (renorm && c > 0) {
                 // T <- kappa dec T once the previous update has landed, so that with kappa = 1 the
                 // next update adds onto the decayed state
-                if (!wait_all(sUpd, (c - 1) & 1)) {
+                if (!wait_all(sUpd0 + (c - 1) % NS, ((c - 1) / NS) & 1)) {
                     ok = false;
                     break;
                 }
@@ -263,7 +267,7 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             if (ts == 0) mbar_arrive(bar(sZV0 + s));
         }
         // the end state S = kappa T, rows dk of column dv0 + d, and the total decay
-        if (ok && wait_all(sUpd, (ntiles - 1) & 1)) {
+        if (ok && wait_all(sUpd0 + (ntiles - 1) % NS, ((ntiles - 1) / NS) & 1)) {
             tc_fence_after();
 #pragma unroll 1
             for (int cb = 0; cb < DK / 32; ++cb) {
