@@ -116,10 +116,10 @@ def measured_peaks():
 # The sources each workload's measured kernels are compiled and launched from; a
 # traffic figure counts only while these files still hash to the value it was taken at.
 KERNEL_SOURCES = {
-    "chunk": ("common.cuh", "tc_chunk.cuh", "tc_wide.cuh"),
+    "chunk": ("common.cuh", "tc_chunk.cuh", "tc_wide.cuh", "tc_state.cuh"),
     "decode": ("common.cuh", "decode.cuh"),
     "norm": ("common.cuh", "norm.cuh"),
-    "backward": ("common.cuh", "tc_chunk.cuh", "tc_wide.cuh", "backward.cuh", "ret_api.cu"),
+    "backward": ("common.cuh", "tc_chunk.cuh", "tc_wide.cuh", "tc_state.cuh", "backward.cuh", "ret_api.cu"),
 }
 WORKLOAD_KERNELS = {"retnet_1p3b": "chunk", "retnet_6p7b_long": "chunk", "gated": "chunk", "seqpar_6p7b": "chunk",
                     "decode": "decode", "gated_decode": "decode", "backward_1p3b": "backward",
@@ -422,8 +422,8 @@ def measure(args, name, spec, dev, stream, world, steps, cpu_budget):
                 "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs, copy)" if peak_src == "measured"
                 else "fallback 6.65 TB/s",
                 "kernel_ms": round(kern_ms, 5),
-                "scope": ("the whole step: " + str(launches) + " launches (five calls of the forward kernel, "
-                          "slice/flip/sum copies, the decay gradient)") if spec["kind"] == "backward"
+                "scope": ("the whole step: " + str(launches) + " launches (the dQ and dK pieces, dV, the piece "
+                          "sums, the decay gradient)") if spec["kind"] == "backward"
                 else "the step's launches",
                 "tensor_tflops": round(spec["flops"] / (kern_ms / 1e3) / 1e12, 2),
                 "tensor_frac_of_bf16_burst": round(spec["flops"] / (kern_ms / 1e3) / 1e12 / tf_burst, 4),

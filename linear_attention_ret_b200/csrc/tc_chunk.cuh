@@ -299,6 +299,12 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Two bf16 products in one instruction (each rounded to bf16 once).
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
+    __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+
 __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
     __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&u);
     return __bfloat1622float2(h);
@@ -812,11 +818,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                float2 f;
-                f = unpack_bf16(x[e].x); x[e].x = pack_bf16(f.x * z[e], f.y * z[e]);
-                f = unpack_bf16(x[e].y); x[e].y = pack_bf16(f.x * z[e], f.y * z[e]);
-                f = unpack_bf16(x[e].z); x[e].z = pack_bf16(f.x * z[e], f.y * z[e]);
-                f = unpack_bf16(x[e].w); x[e].w = pack_bf16(f.x * z[e], f.y * z[e]);
+                // bf16 pair products: the factor rounded to bf16, each product rounded once
+                const uint32_t z2 = pack_bf16(z[e], z[e]);
+                x[e].x = mul_bf16x2(x[e].x, z2);
+                x[e].y = mul_bf16x2(x[e].y, z2);
+                x[e].z = mul_bf16x2(x[e].z, z2);
+                x[e].w = mul_bf16x2(x[e].w, z2);
             }
 #pragma unroll
             for (int e = 0; e < 8; ++e) *reinterpret_cast<uint4*>(zv + (e * kEpiThreads + ts) * 16) = x[e];

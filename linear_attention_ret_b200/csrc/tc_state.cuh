@@ -253,11 +253,12 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 }
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    float2 f;
-                    f = unpack_bf16(x[e].x); x[e].x = pack_bf16(f.x * z[e], f.y * z[e]);
-                    f = unpack_bf16(x[e].y); x[e].y = pack_bf16(f.x * z[e], f.y * z[e]);
-                    f = unpack_bf16(x[e].z); x[e].z = pack_bf16(f.x * z[e], f.y * z[e]);
-                    f = unpack_bf16(x[e].w); x[e].w = pack_bf16(f.x * z[e], f.y * z[e]);
+                    // bf16 pair products: the factor rounded to bf16, each product rounded once
+                    const uint32_t z2 = pack_bf16(z[e], z[e]);
+                    x[e].x = mul_bf16x2(x[e].x, z2);
+                    x[e].y = mul_bf16x2(x[e].y, z2);
+                    x[e].z = mul_bf16x2(x[e].z, z2);
+                    x[e].w = mul_bf16x2(x[e].w, z2);
                 }
 #pragma unroll
                 for (int e = 0; e < 8; ++e) *reinterpret_cast<uint4*>(vt + ((pass * 8 + e) * 128 + ts) * 16) = x[e];

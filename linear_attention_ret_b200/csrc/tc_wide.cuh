@@ -35,9 +35,13 @@
 // R = sum_{i >= t0} gamma^(i-t0+1) k_i^T v_i. Everything above holds with
 // zeta_i = gamma^(i+1) (i the token's place in its tile) and the mask i >= j: the cross
 // factor gamma^(L-1-j) R_next = kappa T / zeta_j with kappa T = gamma^L R_next.
-// Shared memory: one Q, K and V tile, each with its own full/empty barriers so that it
+// Shared memory: one Q and one K tile, each with its own full/empty barriers so that it
 // reloads as soon as its last reader is done (K after the update, Q after the cross
-// term, V after O_intra), and one P tile that is also the staging tile of the O store.
+// term); two V tiles (tile c in buffer c & 1, loaded right after K, so that V(c+1) lands
+// and becomes zeta V / kappa while tile c's products still read ZV(c)); and one P tile
+// that is also the staging tile of the O store (224 KB at dk = 256). zeta V / kappa is
+// formed with bf16 pair products (the factor rounded to bf16, each product rounded once:
+// the operand's rounding error grows from 2^-8 to about 2^-7, relative).
 #pragma once
 
 namespace ret {
@@ -51,11 +55,12 @@ template <int DK>
 struct WideLayout {
     static constexpr int kQ = 0;                        // Q tile: DK/64 blocks (rows = tokens)
     static constexpr int kK = kQ + DK / 64 * kBlk;      // K tile
-    static constexpr int kV = kK + DK / 64 * kBlk;      // V tile, then zeta V / kappa (2 blocks of 64 dv columns)
-    static constexpr int kP = kV + 2 * kBlk;            // P (2 blocks of 64 m columns); O staging (4 x 64 x 64)
+    static constexpr int kV = kK + DK / 64 * kBlk;      // two V tiles, each then zeta V / kappa (2 blocks of 64 dv columns)
+    static constexpr int kVBuf = 2 * kBlk;              // bytes of one V tile
+    static constexpr int kP = kV + 2 * kVBuf;           // P (2 blocks of 64 m columns); O staging (4 x 64 x 64)
     static constexpr int kBar = kP + 2 * kBlk;
-    static constexpr int kNumBars = 16;
-    static constexpr int kAgTab = kBar + kNumBars * 8;  // attention group: drain row factors [128]
+    static constexpr int kNumBars = 19;
+    static constexpr int kAgTab = (kBar + kNumBars * 8 + 15) & ~15;  // attention group: drain row factors [128]
     static constexpr int kSgTab = kAgTab + kW * 4;      // state group: zeta / kappa [128]
     static constexpr int kTmemSlot = kSgTab + kW * 4;
     static constexpr int kAbort = kTmemSlot + 4;
@@ -71,9 +76,10 @@ struct WideLayout {
 };
 
 enum WideBar {
-    wQFull = 0, wKFull, wVFull, wQEmpty, wKEmpty, wVEmpty,
+    wQFull = 0, wKFull, wQEmpty, wKEmpty,
+    wVFull0, wVFull1, wVEmpty0, wVEmpty1,      // per V buffer (tile c uses buffer c & 1)
     wAFull, wARead, wPReady, wOFull, wOFree,
-    wSFull, wSReady, wZV, wDrain
+    wSFull, wSReady, wZV0, wZV1, wDrain
 };
 
 // Lazy decay normalisation (S = kappa T). Given the current kappa and the next tile's
@@ -147,6 +153,20 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
                     for (int h = 0; h < 2; ++h)
                         tma_load_3d(sbase + Lay::kK + kb * kBlk + h * kTile64, &tm_k, kb * 64, t0 + 64 * h, bh, bar(wKFull));
                 issued[0] = c;
+                // V tile c into buffer c & 1 (free once O_intra(c - 2) has read it), before Q: the
+                // state epilogue turns it into zeta V / kappa while tile c - 1 is still running
+                {
+                    const int vb = c & 1;
+                    if (c > 1 && !mbar_wait(bar(wVEmpty0 + vb), ((c >> 1) - 1) & 1, abort_flag)) break;
+                    mbar_expect_tx(bar(wVFull0 + vb), Lay::kVBuf);
+#pragma unroll
+                    for (int db = 0; db < 2; ++db)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            tma_load_3d(sbase + Lay::kV + vb * Lay::kVBuf + db * kBlk + h * kTile64, &tm_v, dv0 + 64 * db,
+                                        t0 + 64 * h, bh, bar(wVFull0 + vb));
+                }
+                issued[2] = c;
                 if (c > 0 && !mbar_wait(bar(wQEmpty), ph, abort_flag)) break;
                 mbar_expect_tx(bar(wQFull), DK / 64 * kBlk);
 #pragma unroll
@@ -155,21 +175,12 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
                     for (int h = 0; h < 2; ++h)
                         tma_load_3d(sbase + Lay::kQ + kb * kBlk + h * kTile64, &tm_q, kb * 64, t0 + 64 * h, bh, bar(wQFull));
                 issued[1] = c;
-                if (c > 0 && !mbar_wait(bar(wVEmpty), ph, abort_flag)) break;
-                mbar_expect_tx(bar(wVFull), 2 * kBlk);
-#pragma unroll
-                for (int db = 0; db < 2; ++db)
-#pragma unroll
-                    for (int h = 0; h < 2; ++h)
-                        tma_load_3d(sbase + Lay::kV + db * kBlk + h * kTile64, &tm_v, dv0 + 64 * db, t0 + 64 * h, bh,
-                                    bar(wVFull));
-                issued[2] = c;
             }
             if (*abort_flag) {
                 // drain the copies in flight before the CTA may exit
                 if (issued[0] >= 0) mbar_drain(bar(wKFull), issued[0] & 1);
                 if (issued[1] >= 0) mbar_drain(bar(wQFull), issued[1] & 1);
-                if (issued[2] >= 0) mbar_drain(bar(wVFull), issued[2] & 1);
+                for (int c = std::max(issued[2] - 1, 0); c <= issued[2]; ++c) mbar_drain(bar(wVFull0 + (c & 1)), (c >> 1) & 1);
             }
         }
     } else if (warp == 1) {
@@ -180,7 +191,7 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
             constexpr uint32_t id_ov = idesc(128, kW, 1, 0);
             constexpr uint32_t id_up = idesc(128, DK, 1, 1);
             const uint32_t tS = tmem + Lay::kColS, tSop = tmem + Lay::kColSop, tR = tmem + Lay::kColR;
-            const uint32_t sQ = sbase + Lay::kQ, sK = sbase + Lay::kK, sZ = sbase + Lay::kV, sP = sbase + Lay::kP;
+            const uint32_t sQ = sbase + Lay::kQ, sK = sbase + Lay::kK, sP = sbase + Lay::kP;
             for (int c = 0; c < ntiles; ++c) {
                 const uint32_t ph = c & 1;
                 // A = Q K^T (both K-major; 16-element K steps, 64-column blocks 16 KB apart);
@@ -196,7 +207,10 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
                 mma_commit(bar(wAFull));
                 // S^T += (zeta V / kappa)^T K while the epilogue reads A: A operand = the
                 // scaled V tile MN-major (dv blocks 16 KB apart), B = K tile MN-major.
-                if (!mbar_wait(bar(wZV), ph, abort_flag) || !mbar_wait(bar(wSReady), ph, abort_flag)) break;
+                const int vb = c & 1;
+                const uint32_t sZ = sbase + Lay::kV + vb * Lay::kVBuf;  // this tile's zeta V / kappa
+                if (!mbar_wait(bar(wZV0 + vb), (c >> 1) & 1, abort_flag) || !mbar_wait(bar(wSReady), ph, abort_flag))
+                    break;
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < kW / 16; ++ks)
@@ -222,7 +236,7 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
                     mma_ss(tR, sdesc(sZ + ks * 2048, kBlk, 1024), sdesc(sP + (ks >> 2) * kBlk + (ks & 3) * 32, 16, 1024),
                            id_ov, 1);
                 mma_commit(bar(wOFull));
-                mma_commit(bar(wVEmpty));
+                mma_commit(bar(wVEmpty0 + vb));
             }
             // every issued MMA must complete before TMEM can be released
             mma_commit(bar(wDrain));
@@ -362,8 +376,8 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
         auto build_zv = [&](int c, float kappa) {
             const int L = tile_len(c);
             zk[ts] = ts < L ? pow_int_log2(lg, REV ? ts + 1 : L - 1 - ts) * (1.f / kappa) : 0.f;
-            if (!wait_all(wVFull, c & 1)) return false;
-            uint8_t* vt = sm + Lay::kV;
+            if (!wait_all(wVFull0 + (c & 1), (c >> 1) & 1)) return false;
+            uint8_t* vt = sm + Lay::kV + (c & 1) * Lay::kVBuf;
 #pragma unroll
             for (int pass = 0; pass < 2; ++pass) {
                 uint4 x[8];
@@ -376,11 +390,12 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
                 }
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    float2 f;
-                    f = unpack_bf16(x[e].x); x[e].x = pack_bf16(f.x * z[e], f.y * z[e]);
-                    f = unpack_bf16(x[e].y); x[e].y = pack_bf16(f.x * z[e], f.y * z[e]);
-                    f = unpack_bf16(x[e].z); x[e].z = pack_bf16(f.x * z[e], f.y * z[e]);
-                    f = unpack_bf16(x[e].w); x[e].w = pack_bf16(f.x * z[e], f.y * z[e]);
+                    // bf16 pair products (the factor rounded to bf16, the product rounded once)
+                    const uint32_t z2 = pack_bf16(z[e], z[e]);
+                    x[e].x = mul_bf16x2(x[e].x, z2);
+                    x[e].y = mul_bf16x2(x[e].y, z2);
+                    x[e].z = mul_bf16x2(x[e].z, z2);
+                    x[e].w = mul_bf16x2(x[e].w, z2);
                 }
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
@@ -388,7 +403,7 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
             }
             fence_proxy_async();
             group_sync(2);
-            if (ts == 0) mbar_arrive(bar(wZV));
+            if (ts == 0) mbar_arrive(bar(wZV0 + (c & 1)));
             return true;
         };
 
