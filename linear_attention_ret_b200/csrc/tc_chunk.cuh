@@ -1227,7 +1227,7 @@ ret_status launch_dk(const void* q, const void* k, const void* v, const float* d
             prm.state_in = copy;
         }
         auto k1 = state_tc_kernel<DK, GATED, REV>;
-        constexpr int smem1 = StateLayout<DK>::kSmemAlloc;
+        constexpr int smem1 = StateLayout<DK, state_tile(GATED)>::kSmemAlloc;
         if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1) != cudaSuccess)
             return RET_ERR_CUDA;
         Params prm1 = prm;  // the state-only pass runs over the sub-segments
@@ -1318,7 +1318,7 @@ ret_status launch_state_dk(const void* k, const void* v, const float* decay, flo
     float* ldec = reinterpret_cast<float*>(sc + (subs > 1 ? sizeof(float) * (size_t)subs * BH * DK * dv : 0));
     Params prm{decay, nullptr, nullptr, states, ldec, H, N, dv, sub_chunks, 1, subs};
     auto k1 = state_tc_kernel<DK, GATED, false>;
-    constexpr int smem1 = StateLayout<DK>::kSmemAlloc;
+    constexpr int smem1 = StateLayout<DK, state_tile(GATED)>::kSmemAlloc;
     if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1) != cudaSuccess)
         return RET_ERR_CUDA;
     if (launch_dependent(k1, dim3(dv / kDvS, BH, subs), kSThreads, smem1, st, mk, mv, prm) != cudaSuccess)

@@ -4,44 +4,48 @@
 // Method: "RetNet retention mechanism" (aiqz.cc), section 块级循环 (the state carried
 // between chunks, S_i = decay_i S_{i-1} + K_i^T diag(zeta) V_i), and the Gated RetNet
 // page's cross_chunk update with per-token decays. Only the update product runs here:
-//   S^T += (zeta V / kappa)^T K     M = 128 (dv slice)  N = dk  K = 128 tokens   (SS, both MN-major)
-// over 128-token tiles, with the state held as S = kappa T (T in TMEM, the scalar kappa in
+//   S^T += (zeta V / kappa)^T K     M = 128 (dv slice)  N = dk  K = TT tokens   (SS, both MN-major)
+// over tiles of TT tokens, with the state held as S = kappa T (T in TMEM, the scalar kappa in
 // registers; T is rescaled in place only when kappa would fall below 2^-40).
 //
-// Roles (192 threads): warp 0 issues the TMA loads (2 or 3 stages of a K tile and a V
-// tile), warp 1 allocates TMEM and issues the products, warps 2-5 turn each V tile into
-// zeta V / kappa in place and finally write kappa T. REV visits the tiles from the last
-// back with the reversed direction's key weights (see chunk_tc_kernel). All waits are
-// bounded like the other bodies'.
+// Roles (192 threads): warp 0 issues the TMA loads (a ring of stages of a K tile and a V
+// tile, 192 KB in all: the pass is bound by how fast copies arrive, so it keeps many in
+// flight), warp 1 allocates TMEM and issues the products, warps 2-5 turn each V tile into
+// zeta V / kappa in place and finally write kappa T. Tiles are 64 tokens for a fixed decay
+// (four stages at dk = 256: more copies in flight) and 128 tokens for the gated form, whose
+// per-tile work (a scan of the gates, exponentials, more frequent rescaling) is better
+// amortised over longer tiles; its gates are read 256 tokens ahead, since their latency
+// exceeds a tile's work. REV visits the tiles from the last back with the reversed
+// direction's key weights (see chunk_tc_kernel). All waits are bounded like the other
+// bodies'.
 #pragma once
 
 namespace ret {
 namespace tc {
 
 constexpr int kSThreads = 192;
+constexpr int kMaxSStages = 8;
 
-template <int DK>
+// tokens per tile of the state-only pass
+__host__ __device__ constexpr int state_tile(bool gated) { return gated ? 128 : 64; }
+
+template <int DK, int TT>
 struct StateLayout {
-    static constexpr int kKBytes = DK / 64 * kBlk;             // 128 token rows x DK
-    static constexpr int kVBytes = 2 * kBlk;                    // 128 token rows x 128 dv
+    static constexpr int kRowBlk = TT * 128;                    // one TT-row x 64-column block (128-byte rows)
+    static constexpr int kKBytes = DK / 64 * kRowBlk;           // TT token rows x DK
+    static constexpr int kVBytes = 2 * kRowBlk;                 // TT token rows x 128 dv
     static constexpr int kStageBytes = kKBytes + kVBytes;
-    static constexpr int kStages = (3 * kStageBytes <= 200 * 1024) ? 3 : 2;
+    static constexpr int kStages = std::min(kMaxSStages, 192 * 1024 / kStageBytes);
     static constexpr int kBar = kStages * kStageBytes;
-    static constexpr int kNumBars = 13;                         // full[3], empty[3], zv[3], upd[3], drain
-    static constexpr int kTab = kBar + kNumBars * 8;            // zeta / kappa [128], gated cumsum [128]
-    static constexpr int kTmemSlot = kTab + 2 * kW * 4;
+    static constexpr int kNumBars = 4 * kStages + 1;            // full, empty, zv, upd per stage; drain
+    static constexpr int kTab = kBar + kNumBars * 8;            // zeta / kappa [TT], gated cumsum [TT]
+    static constexpr int kTmemSlot = kTab + 2 * TT * 4;
     static constexpr int kAbort = kTmemSlot + 4;
     static constexpr int kBytes = kAbort + 4;
     static constexpr int kSmemAlloc = kBytes + 1024;            // slack to align the base to 1024 B
     static constexpr int kTmemCols = DK <= 32 ? 32 : DK <= 64 ? 64 : DK <= 128 ? 128 : 256;
     static_assert(kSmemAlloc <= 227 * 1024, "shared memory overflow");
 };
-
-// upd[s]: the update of a tile in stage s has completed. One per stage, like the others, so
-// that a wait for a given tile's update is never more than one phase behind: the epilogue
-// waits on it only now and then (renormalisation, the end), and a single barrier could by
-// then have completed two phases, which a parity wait cannot tell from none.
-enum StateBar { sFull0 = 0, sEmpty0 = 3, sZV0 = 6, sUpd0 = 9, sDrain = 12 };
 
 // Inclusive cumulative sum over 128 values in log2 units by one warp: lane l holds
 // x[4l .. 4l+3]; writes cum[0..127].
@@ -60,6 +64,14 @@ __device__ __forceinline__ void warp_cumsum128(const float (&x)[4], int lane, fl
     cum[4 * lane + 3] = excl + p3;
 }
 
+// upd[s]: the update of a tile in stage s has completed. One per stage, like the others, so
+// that a wait for a given tile's update is never more than one phase behind: the epilogue
+// waits on it only now and then (renormalisation, the end), and a single barrier could by
+// then have completed two phases, which a parity wait cannot tell from none.
+// barrier index of (kind, stage) for NS stages
+__host__ __device__ constexpr int sbar(int kind, int stage, int ns) { return kind * ns + stage; }
+enum StateBarKind { sFull = 0, sEmpty = 1, sZV = 2, sUpd = 3 };
+
 // Grid: (dv / 128, B*H, sub-segments). p.seg_chunks: 64-token chunks per sub-segment;
 // p.units: sub-segments the whole sequence is cut into (REV counts them from the end).
 // Writes sub-segment z's end state to seg_state[z] and log2 of its total decay to
@@ -68,7 +80,8 @@ template <int DK, bool GATED, bool REV>
 __global__ void __launch_bounds__(kSThreads, 1)
 state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, Params p) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    using Lay = StateLayout<DK>;
+    constexpr int kST = state_tile(GATED);
+    using Lay = StateLayout<DK, kST>;
     constexpr int NS = Lay::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -83,7 +96,7 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int tseg = REV ? p.units - 1 - seg : seg;
     const int tbeg = tseg * p.seg_chunks * kC;
     const int tend = min(tbeg + p.seg_chunks * kC, p.N);
-    const int ntiles = tend > tbeg ? (tend - tbeg + kW - 1) / kW : 0;
+    const int ntiles = tend > tbeg ? (tend - tbeg + kST - 1) / kST : 0;
     float* so = p.seg_state + ((size_t)seg * gridDim.y + bh) * DK * p.dv + dv0;
     if (ntiles == 0) {
         // REV only: a sub-segment past the end of a short last segment: zero state, no decay
@@ -91,8 +104,8 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         if (slice == 0 && threadIdx.x == 0) p.seg_ldec[(size_t)seg * gridDim.y + bh] = 0.f;
         return;
     }
-    auto tile_t0 = [&](int c) { return tbeg + (REV ? ntiles - 1 - c : c) * kW; };
-    auto tile_len = [&](int c) { return min(kW, tend - tile_t0(c)); };
+    auto tile_t0 = [&](int c) { return tbeg + (REV ? ntiles - 1 - c : c) * kST; };
+    auto tile_len = [&](int c) { return min(kST, tend - tile_t0(c)); };
 
     if (threadIdx.x == 0) {
         for (int b = 0; b < Lay::kNumBars; ++b) mbar_init(bar(b), 1);
@@ -117,27 +130,28 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             int issued = -1;
             for (int c = 0; c < ntiles; ++c) {
                 const int s = c % NS;
-                if (c >= NS && !mbar_wait(bar(sEmpty0 + s), ((c / NS) - 1) & 1, abort_flag)) break;
+                if (c >= NS && !mbar_wait(bar(sbar(sEmpty, s, NS)), ((c / NS) - 1) & 1, abort_flag)) break;
                 const uint32_t st = sbase + s * Lay::kStageBytes;
                 const int t0 = tile_t0(c);
-                mbar_expect_tx(bar(sFull0 + s), Lay::kStageBytes);
+                const uint32_t fb = bar(sbar(sFull, s, NS));
+                mbar_expect_tx(fb, Lay::kStageBytes);
 #pragma unroll
                 for (int kb = 0; kb < DK / 64; ++kb)
 #pragma unroll
-                    for (int h = 0; h < 2; ++h)
-                        tma_load_3d(st + kb * kBlk + h * kTile64, &tm_k, kb * 64, t0 + 64 * h, bh, bar(sFull0 + s));
+                    for (int h = 0; h < kST / 64; ++h)
+                        tma_load_3d(st + kb * Lay::kRowBlk + h * kTile64, &tm_k, kb * 64, t0 + 64 * h, bh, fb);
 #pragma unroll
                 for (int db = 0; db < 2; ++db)
 #pragma unroll
-                    for (int h = 0; h < 2; ++h)
-                        tma_load_3d(st + Lay::kKBytes + db * kBlk + h * kTile64, &tm_v, dv0 + 64 * db, t0 + 64 * h, bh,
-                                    bar(sFull0 + s));
+                    for (int h = 0; h < kST / 64; ++h)
+                        tma_load_3d(st + Lay::kKBytes + db * Lay::kRowBlk + h * kTile64, &tm_v, dv0 + 64 * db,
+                                    t0 + 64 * h, bh, fb);
                 issued = c;
             }
             if (*abort_flag && issued >= 0) {
                 // drain the copies in flight before the CTA may exit
                 for (int c = std::max(issued - NS + 1, 0); c <= issued; ++c)
-                    mbar_drain(bar(sFull0 + c % NS), (c / NS) & 1);
+                    mbar_drain(bar(sbar(sFull, c % NS, NS)), (c / NS) & 1);
             }
         }
     } else if (warp == 1) {
@@ -147,21 +161,21 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             for (int c = 0; c < ntiles; ++c) {
                 const int s = c % NS;
                 const uint32_t sK = sbase + s * Lay::kStageBytes, sZ = sK + Lay::kKBytes;
-                if (!mbar_wait(bar(sFull0 + s), (c / NS) & 1, abort_flag) ||
-                    !mbar_wait(bar(sZV0 + s), (c / NS) & 1, abort_flag))
+                if (!mbar_wait(bar(sbar(sFull, s, NS)), (c / NS) & 1, abort_flag) ||
+                    !mbar_wait(bar(sbar(sZV, s, NS)), (c / NS) & 1, abort_flag))
                     break;
                 tc_fence_after();
-                // S^T += (zeta V / kappa)^T K: A = the scaled V tile MN-major (dv blocks 16 KB apart),
-                // B = K tile MN-major (dk blocks 16 KB apart), 16 tokens per step
+                // S^T += (zeta V / kappa)^T K: A = the scaled V tile MN-major (dv blocks kRowBlk apart),
+                // B = K tile MN-major (dk blocks kRowBlk apart), 16 tokens per step
 #pragma unroll
-                for (int ks = 0; ks < kW / 16; ++ks)
-                    mma_ss(tmem, sdesc(sZ + ks * 2048, kBlk, 1024), sdesc(sK + ks * 2048, kBlk, 1024), id_up,
-                           (c > 0 || ks > 0) ? 1u : 0u);
-                mma_commit(bar(sEmpty0 + s));
-                mma_commit(bar(sUpd0 + s));
+                for (int ks = 0; ks < kST / 16; ++ks)
+                    mma_ss(tmem, sdesc(sZ + ks * 2048, Lay::kRowBlk, 1024), sdesc(sK + ks * 2048, Lay::kRowBlk, 1024),
+                           id_up, (c > 0 || ks > 0) ? 1u : 0u);
+                mma_commit(bar(sbar(sEmpty, s, NS)));
+                mma_commit(bar(sbar(sUpd, s, NS)));
             }
-            mma_commit(bar(sDrain));
-            mbar_drain(bar(sDrain), 0);
+            mma_commit(bar(4 * NS));
+            mbar_drain(bar(4 * NS), 0);
         }
     } else {
         // ------------------------------------------------------------ state epilogue (warps 2..5)
@@ -170,7 +184,7 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         const int d = quarter * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         float* zk = reinterpret_cast<float*>(sm + Lay::kTab);   // zeta_m / kappa of the current tile
-        float* cum = zk + kW;                                    // gated: in-tile cumulative log2 decay
+        float* cum = zk + kST;                                   // gated: in-tile cumulative log2 decay
         auto wait_all = [&](int b, uint32_t parity) {
             mbar_wait(bar(b), parity, abort_flag);
             asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -178,15 +192,24 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         };
         const float lg = GATED ? 0.f : log2f(p.decay_in[bh % p.H]);
         const float* G = GATED ? p.decay_in + (size_t)bh * p.N : nullptr;
-        float gx[4] = {0.f, 0.f, 0.f, 0.f};  // gated: this lane's four gates of the next tile (warp 2)
-        auto load_gates = [&](int c) {
-            if (GATED && ts < 32) {
+        // gated: lane l of warp 2 holds gates GPL l .. GPL l + GPL - 1 of tiles c .. c + PF - 1
+        // (read 256 tokens ahead)
+        constexpr int GPL = kST / 32, PF = 256 / kST;
+        float gq[PF][GPL];
+        auto load_tile_gates = [&](int c, float (&x)[GPL]) {
+#pragma unroll
+            for (int i = 0; i < GPL; ++i) x[i] = 0.f;
+            if (c < ntiles) {
                 const int t0 = tile_t0(c), L = tile_len(c);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) gx[i] = 4 * ts + i < L ? G[t0 + 4 * ts + i] * kLog2e : 0.f;
+                for (int i = 0; i < GPL; ++i)
+                    if (GPL * ts + i < L) x[i] = G[t0 + GPL * ts + i] * kLog2e;
             }
         };
-        load_gates(0);
+        if (GATED && ts < 32) {
+#pragma unroll
+            for (int f = 0; f < PF; ++f) load_tile_gates(f, gq[f]);
+        }
         float kappa = 1.f, ldec_sum = 0.f;
         bool ok = true;
         for (int c = 0; c < ntiles && ok; ++c) {
@@ -195,8 +218,13 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             float ldec;
             if (GATED) {
                 if (ts < 32) {
-                    warp_cumsum128(gx, lane, cum);
-                    if (c + 1 < ntiles) load_gates(c + 1);
+                    if constexpr (kST == 64) warp_cumsum64(gq[0][0], gq[0][1], lane, cum);
+                    else warp_cumsum128(gq[0], lane, cum);
+#pragma unroll
+                    for (int f = 0; f + 1 < PF; ++f)
+#pragma unroll
+                        for (int i = 0; i < GPL; ++i) gq[f][i] = gq[f + 1][i];
+                    load_tile_gates(c + PF, gq[PF - 1]);
                 }
                 asm volatile("bar.sync 1, 128;" ::: "memory");
                 ldec = cum[L - 1];
@@ -209,7 +237,7 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             if (renorm && c > 0) {
                 // T <- kappa dec T once the previous update has landed, so that with kappa = 1 the
                 // next update adds onto the decayed state
-                if (!wait_all(sUpd0 + (c - 1) % NS, ((c - 1) / NS) & 1)) {
+                if (!wait_all(sbar(sUpd, (c - 1) % NS, NS), ((c - 1) / NS) & 1)) {
                     ok = false;
                     break;
                 }
@@ -229,26 +257,28 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             }
             kappa = k_next;
             ldec_sum += ldec;
-            {
+            if (ts < kST) {
                 const float inv = 1.f / kappa;
                 float z;
                 if (GATED) z = REV ? exp2f(cum[ts]) : exp2f(cum[L - 1] - cum[ts]);
                 else z = pow_int_log2(lg, REV ? ts + 1 : L - 1 - ts);
                 zk[ts] = ts < L ? z * inv : 0.f;
             }
-            if (!wait_all(sFull0 + s, (c / NS) & 1)) {  // the V tile landed (and zk is complete)
+            if (!wait_all(sbar(sFull, s, NS), (c / NS) & 1)) {  // the V tile landed (and zk is complete)
                 ok = false;
                 break;
             }
             uint8_t* vt = sm + s * Lay::kStageBytes + Lay::kKBytes;
 #pragma unroll
-            for (int pass = 0; pass < 2; ++pass) {
+            for (int pass = 0; pass < kST / 64; ++pass) {
+                // 16-byte chunks ci = e * 128 + ts of the two dv blocks (TT token rows of 128 bytes
+                // each), so the token of a chunk is (ci mod 8 TT) / 8. All loads before any store.
                 uint4 x[8];
                 float z[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {  // all loads before any store
+                for (int e = 0; e < 8; ++e) {
                     const int ci = (pass * 8 + e) * 128 + ts;
-                    z[e] = zk[(ci & 1023) >> 3];
+                    z[e] = zk[(ci & (8 * kST - 1)) >> 3];
                     x[e] = *reinterpret_cast<const uint4*>(vt + ci * 16);
                 }
 #pragma unroll
@@ -265,10 +295,10 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             }
             fence_proxy_async();
             asm volatile("bar.sync 1, 128;" ::: "memory");
-            if (ts == 0) mbar_arrive(bar(sZV0 + s));
+            if (ts == 0) mbar_arrive(bar(sbar(sZV, s, NS)));
         }
         // the end state S = kappa T, rows dk of column dv0 + d, and the total decay
-        if (ok && wait_all(sUpd0 + (ntiles - 1) % NS, ((ntiles - 1) / NS) & 1)) {
+        if (ok && wait_all(sbar(sUpd, (ntiles - 1) % NS, NS), ((ntiles - 1) / NS) & 1)) {
             tc_fence_after();
 #pragma unroll 1
             for (int cb = 0; cb < DK / 32; ++cb) {

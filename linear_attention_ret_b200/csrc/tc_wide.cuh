@@ -318,7 +318,7 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
                 tc_fence_before();
                 group_sync(1);
                 if (te == 0) mbar_arrive(bar(wOFree));
-                const int g = lane >> 2, i2 = 2 * (lane & 3);
+                const int i2 = 2 * (lane & 3);
 #pragma unroll
                 for (int th = 0; th < 2; ++th) {
 #pragma unroll
