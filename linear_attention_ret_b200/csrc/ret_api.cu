@@ -224,90 +224,77 @@ inline int backward_tc_launches(int B, int H, int N, int dk, int dv, bool gated,
     int n = 0;
     for (int p = 0; p < P; ++p) n += 2 * tc_chunk_launches(B, H, N, std::min(256, dv - 256 * p), dk, conc);
     n += tc_chunk_launches(B, H, N, dk, dv, conc);  // dV
-    n += P > 1 ? 2 : 0;                             // sums of the dQ and dK pieces
     n += ddecay ? (gated ? 2 : 1) : 0;              // decay gradient (gated: and its suffix sum)
     return n;
 }
 
 // The backward on the tensor-core path as a small graph of steps on the caller's stream st
 // and two library streams s1, s2:
-//   st: dQ piece 0 | wait s1 -> dq = sum of the dQ pieces | wait s2 -> dgamma/dg
-//   s1: dQ piece 1 | dK piece 1 (reversed)
-//   s2: dK piece 0 (reversed) | dV (reversed) | wait s1 -> dk = sum of the dK pieces
+//   st: zero dq, dk | dQ piece 0 (adds onto dq) | wait s1, s2 -> dgamma/dg
+//   s1: dQ piece 1 (adds onto dq) | dK piece 1 (reversed, adds onto dk)
+//   s2: dK piece 0 (reversed, adds onto dk) | dV (reversed) | wait s1
 // (more pieces alternate between the streams of their row; with one piece the dQ and dK
-// calls write dq and dk directly). dQ = forward(dO, V, K); dK = reversed forward(V, dO, Q);
-// dV = reversed forward(K, Q, dO), each with the caller's gamma or gates as they are.
+// calls store dq and dk directly, with no zeroing). dQ = forward(dO, V, K); dK = reversed
+// forward(V, dO, Q); dV = reversed forward(K, Q, dO), each with the caller's gamma or gates
+// as they are.
 template <typename T, bool GATED>
 ret_status backward_tc(const void* q, const void* k, const void* v, const float* decay, const void* dout,
                        void* dq, void* dk_out, void* dv_out, float* ddecay, int B, int H, int N, int dk, int dv,
                        cudaStream_t st) {
-    const int BH = B * H;
-    const size_t nQ = (size_t)BH * N * dk;
+    const size_t nQ = (size_t)B * H * N * dk;
     const int pw = 256, P = (dv + pw - 1) / pw, conc = 2 * P + 1;
-    // scratch (P > 1 only): the dQ and dK pieces
-    const size_t part_bytes = align256((size_t)P * nQ * sizeof(T));
-    uint8_t* sc = nullptr;
-    if (P > 1) {
-        tc::keep_pool_memory();
-        if (cudaMallocAsync(reinterpret_cast<void**>(&sc), 2 * part_bytes, st) != cudaSuccess) return RET_ERR_CUDA;
-    }
-    T* partsQ = P > 1 ? reinterpret_cast<T*>(sc) : static_cast<T*>(dq);
-    T* partsK = P > 1 ? reinterpret_cast<T*>(sc + part_bytes) : static_cast<T*>(dk_out);
-
     ret_status r = RET_OK;
     auto ok = [&](ret_status x) { if (r == RET_OK) r = x; return r == RET_OK; };
     auto cu = [&](cudaError_t e) { return ok(e == cudaSuccess ? RET_OK : RET_ERR_CUDA); };
     std::lock_guard<std::mutex> lock(aux_mutex());
     AuxStreams* a = aux_streams();
-    if (!a) {
-        if (sc) cudaFreeAsync(sc, st);
-        return RET_ERR_CUDA;
-    }
+    if (!a) return RET_ERR_CUDA;
     cudaStream_t s1 = a->s[0], s2 = a->s[1];
     cudaEvent_t ev_fork = a->ev[0], ev_q1 = a->ev[1], ev_k1 = a->ev[2], ev_k = a->ev[3], ev_j1 = a->ev[4],
                 ev_j2 = a->ev[5];
+    // With several pieces, dq and dk start at zero and every piece adds its output tiles onto
+    // them (in L2, in bf16, rounded once per addition): with two pieces each element is
+    // round(a + b), whatever order the pieces' additions take.
+    if (P > 1) {
+        cu(cudaMemsetAsync(dq, 0, nQ * sizeof(T), st));
+        cu(cudaMemsetAsync(dk_out, 0, nQ * sizeof(T), st));
+    }
     // one piece of a dv contraction: queries x[:, c0:c0+w], keys y[:, c0:c0+w] (rows dv apart), values z
-    auto piece = [&](bool rev, const void* x, const void* y, const void* z, T* fo, int p, cudaStream_t s) {
+    auto piece = [&](bool rev, const void* x, const void* y, const void* z, void* out, int p, cudaStream_t s) {
         const int c0 = p * pw, w = std::min(pw, dv - c0);
         const void* xp = static_cast<const T*>(x) + c0;
         const void* yp = static_cast<const T*>(y) + c0;
-        T* out = fo + (size_t)p * nQ;
         return ok(rev ? tc_chunk_launch<GATED, true>(xp, yp, z, decay, out, nullptr, nullptr, B, H, N, w, dk, s, dv,
-                                                     dv, conc)
+                                                     dv, conc, P > 1)
                       : tc_chunk_launch<GATED, false>(xp, yp, z, decay, out, nullptr, nullptr, B, H, N, w, dk, s, dv,
-                                                      dv, conc));
+                                                      dv, conc, P > 1));
     };
-    if (cu(cudaEventRecord(ev_fork, st))) {
+    if (r == RET_OK && cu(cudaEventRecord(ev_fork, st))) {
         cu(cudaStreamWaitEvent(s1, ev_fork, 0));
         cu(cudaStreamWaitEvent(s2, ev_fork, 0));
     }
     // dQ pieces on st and s1, then dK pieces on s2 and s1, dV on s2
-    for (int p = 0; p < P && r == RET_OK; ++p) piece(false, dout, v, k, partsQ, p, p % 2 ? s1 : st);
+    for (int p = 0; p < P && r == RET_OK; ++p) piece(false, dout, v, k, dq, p, p % 2 ? s1 : st);
     if (r == RET_OK) cu(cudaEventRecord(ev_q1, s1));  // s1's dQ pieces
-    for (int p = 0; p < P && r == RET_OK; ++p) piece(true, v, dout, q, partsK, p, p % 2 ? s1 : s2);
+    for (int p = 0; p < P && r == RET_OK; ++p) piece(true, v, dout, q, dk_out, p, p % 2 ? s1 : s2);
     if (r == RET_OK) cu(cudaEventRecord(ev_k1, s1));  // s1's dK pieces
     if (r == RET_OK)
         ok(tc_chunk_launch<GATED, true>(k, q, dout, decay, dv_out, nullptr, nullptr, B, H, N, dk, dv, s2, 0, 0, conc));
-    // dq = sum of the dQ pieces on st, dk = sum of the dK pieces on s2, each once s1's pieces are done
-    if (r == RET_OK && cu(cudaStreamWaitEvent(st, ev_q1, 0)) && P > 1)
-        ok(sum_flip<T>(partsQ, P, nQ, static_cast<T*>(dq), BH, N, dk, false, st));
-    if (r == RET_OK && cu(cudaStreamWaitEvent(s2, ev_k1, 0)) && P > 1)
-        ok(sum_flip<T>(partsK, P, nQ, static_cast<T*>(dk_out), BH, N, dk, false, s2));
-    // decay gradient on st, after dq (st, s1) and dk (s1, s2)
-    if (r == RET_OK && cu(cudaEventRecord(ev_k, s2)) && ddecay && cu(cudaStreamWaitEvent(st, ev_k, 0)))
+    // decay gradient on st once dq (st, s1) and dk (s2, s1) are complete
+    if (r == RET_OK && ddecay && cu(cudaStreamWaitEvent(s2, ev_k1, 0)) && cu(cudaEventRecord(ev_k, s2)) &&
+        cu(cudaStreamWaitEvent(st, ev_q1, 0)) && cu(cudaStreamWaitEvent(st, ev_k, 0)))
         ok(decay_grad<T, GATED>(static_cast<const T*>(q), static_cast<const T*>(dq), static_cast<const T*>(k),
-                                static_cast<const T*>(dk_out), decay, ddecay, BH, H, N, dk, st));
-    // join both library streams back into st whatever happened, then release the scratch on st
+                                static_cast<const T*>(dk_out), decay, ddecay, B * H, H, N, dk, st));
+    // join both library streams back into st whatever happened
     const bool joined = cudaEventRecord(ev_j1, s1) == cudaSuccess && cudaEventRecord(ev_j2, s2) == cudaSuccess &&
                         cudaStreamWaitEvent(st, ev_j1, 0) == cudaSuccess &&
                         cudaStreamWaitEvent(st, ev_j2, 0) == cudaSuccess;
     if (!joined) {
-        // the library streams could not be ordered before st: wait for them before freeing
+        // the library streams could not be ordered before st: wait for them
         cudaStreamSynchronize(s1);
         cudaStreamSynchronize(s2);
         ok(RET_ERR_CUDA);
     }
-    if (sc && cudaFreeAsync(sc, st) != cudaSuccess) ok(RET_ERR_CUDA);
     return r;
 }
 

@@ -171,6 +171,20 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, int x, int 
                  ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(src)
                  : "memory");
 }
+// Adds the tile into global memory instead of storing it (the addition is done in L2,
+// element by element in the tensor's type, rounded once).
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, int x, int y, int z, uint32_t src) {
+    asm volatile("cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2, %3}], [%4];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(src)
+                 : "memory");
+}
+// The output tile copy: a store, or an addition onto what the output already holds.
+__device__ __forceinline__ void tma_out_3d(bool add, const CUtensorMap* map, int x, int y, int z, uint32_t src) {
+    if (add)
+        tma_reduce_add_3d(map, x, y, z, src);
+    else
+        tma_store_3d(map, x, y, z, src);
+}
 __device__ __forceinline__ void tma_store_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void tma_store_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
@@ -322,6 +336,7 @@ struct Params {
     int seg_chunks;          // chunks per sequence segment (blockIdx.z = segment)
     int sub_per_seg;         // state-only sub-segments per full-pass segment (their start states are in seg_state)
     int units;               // segments the sequence is cut into at seg_chunks each (REV counts them from the end)
+    int o_add;               // nonzero: output tiles are added onto o (which the caller has initialised)
 };
 
 // In-chunk inclusive cumulative sum of the gate in log2 units, by one warp:
@@ -728,8 +743,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             fence_proxy_async();
             group_sync(1);
             if (te == 0) {
-                tma_store_3d(&tm_o, dv0, t0, bh, sbase + Lay::kOst);
-                tma_store_3d(&tm_o, dv0 + 64, t0, bh, sbase + Lay::kOst + kTile64);
+                tma_out_3d(p.o_add, &tm_o, dv0, t0, bh, sbase + Lay::kOst);
+                tma_out_3d(p.o_add, &tm_o, dv0 + 64, t0, bh, sbase + Lay::kOst + kTile64);
                 tma_store_commit();
             }
             return true;
@@ -1208,13 +1223,13 @@ inline cudaError_t launch_dependent(void (*kernel)(P...), dim3 grid, int threads
 template <int DK, bool GATED, bool REV>
 ret_status launch_dk(const void* q, const void* k, const void* v, const float* decay, void* o,
                      const float* state_in, float* state_out, int B, int H, int N, int dv, const Plan& pl,
-                     void* scratch, cudaStream_t st, int ldq, int ldk) {
+                     void* scratch, cudaStream_t st, int ldq, int ldk, bool o_add) {
     const int BH = B * H;
     CUtensorMap mq, mk, mv, mo;
     if (!make_map(&mq, q, DK, N, BH, ldq) || !make_map(&mk, k, DK, N, BH, ldk) || !make_map(&mv, v, dv, N, BH) ||
         !make_map(&mo, o, dv, N, BH))
         return RET_ERR_CUDA;
-    Params prm{decay, state_in, state_out, nullptr, nullptr, H, N, dv, pl.seg_chunks, pl.F, pl.G};
+    Params prm{decay, state_in, state_out, nullptr, nullptr, H, N, dv, pl.seg_chunks, pl.F, pl.G, o_add ? 1 : 0};
     if (pl.G > 1) {
         uint8_t* sc = static_cast<uint8_t*>(scratch);
         prm.seg_state = reinterpret_cast<float*>(sc);
@@ -1248,21 +1263,23 @@ ret_status launch_dk(const void* q, const void* k, const void* v, const float* d
 
 // Runs the tensor-core path with caller-provided scratch (at least scratch_bytes()).
 // ldq, ldk: row strides of q and k in elements (0: dense rows of dk). REV: the
-// time-reversed direction (sums over later tokens), see chunk_tc_kernel.
+// time-reversed direction (sums over later tokens), see chunk_tc_kernel. o_add: add the
+// output onto o instead of storing it.
 template <bool GATED, bool REV = false>
 ret_status launch_with_scratch(const void* q, const void* k, const void* v, const float* decay, void* o,
                                const float* state_in, float* state_out, int B, int H, int N, int dk, int dv,
-                               const Plan& pl, void* scratch, cudaStream_t st, int ldq = 0, int ldk = 0) {
+                               const Plan& pl, void* scratch, cudaStream_t st, int ldq = 0, int ldk = 0,
+                               bool o_add = false) {
     switch (dk) {
         case 64:
             return launch_dk<64, GATED, REV>(q, k, v, decay, o, state_in, state_out, B, H, N, dv, pl, scratch, st,
-                                             ldq, ldk);
+                                             ldq, ldk, o_add);
         case 128:
             return launch_dk<128, GATED, REV>(q, k, v, decay, o, state_in, state_out, B, H, N, dv, pl, scratch, st,
-                                              ldq, ldk);
+                                              ldq, ldk, o_add);
         case 256:
             return launch_dk<256, GATED, REV>(q, k, v, decay, o, state_in, state_out, B, H, N, dv, pl, scratch, st,
-                                              ldq, ldk);
+                                              ldq, ldk, o_add);
     }
     return RET_ERR_UNSUPPORTED;
 }
@@ -1364,14 +1381,14 @@ inline int tc_state_launches(int B, int H, int N, int dv) {
 template <bool GATED, bool REV = false>
 ret_status tc_chunk_launch(const void* q, const void* k, const void* v, const float* decay, void* o,
                            const float* state_in, float* state_out, int B, int H, int N, int dk, int dv,
-                           cudaStream_t st, int ldq = 0, int ldk = 0, int concurrent = 1) {
+                           cudaStream_t st, int ldq = 0, int ldk = 0, int concurrent = 1, bool o_add = false) {
     const tc::Plan pl = tc::plan(B, H, N, dv, true, concurrent);
     void* scratch = nullptr;
     const size_t bytes = tc::scratch_bytes(pl, B * H, dk, dv, state_in != nullptr && state_in == state_out);
     if (bytes) tc::keep_pool_memory();
     if (bytes && cudaMallocAsync(&scratch, bytes, st) != cudaSuccess) return RET_ERR_CUDA;
     const ret_status r = tc::launch_with_scratch<GATED, REV>(q, k, v, decay, o, state_in, state_out, B, H, N, dk,
-                                                             dv, pl, scratch, st, ldq, ldk);
+                                                             dv, pl, scratch, st, ldq, ldk, o_add);
     if (scratch && cudaFreeAsync(scratch, st) != cudaSuccess) return RET_ERR_CUDA;
     return r;
 }

@@ -352,8 +352,8 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
 #pragma unroll
                 for (int th = 0; th < 2; ++th) {
                     if (th * 64 >= L) break;
-                    tma_store_3d(&tm_o, dv0, t0 + 64 * th, bh, sbase + Lay::kP + (2 * th) * kTile64);
-                    tma_store_3d(&tm_o, dv0 + 64, t0 + 64 * th, bh, sbase + Lay::kP + (2 * th + 1) * kTile64);
+                    tma_out_3d(p.o_add, &tm_o, dv0, t0 + 64 * th, bh, sbase + Lay::kP + (2 * th) * kTile64);
+                    tma_out_3d(p.o_add, &tm_o, dv0 + 64, t0 + 64 * th, bh, sbase + Lay::kP + (2 * th + 1) * kTile64);
                 }
                 tma_store_commit();
             }

@@ -151,7 +151,8 @@ def test_backward_full_size_sampled_heads(cuda_lib):
 
 @pytest.mark.parametrize("gated", [False, True])
 def test_backward_without_decay_gradient(cuda_lib, gated):
-    """ddecay=False: the same dq, dk, dv (the tensor-core path with dv in pieces)."""
+    """ddecay=False: the same dq, dk, dv, bit for bit (the tensor-core path with dv in two
+    pieces whose tiles add onto dq and dk in either order: each element is round(a + b))."""
     q, k, v, do, gen = _case(1, 2, 190, 256, 512, torch.bfloat16, seed=21)
     decay = I.gate(1, 2, 190, gen) * 4.0 if gated else torch.tensor([0.97, 0.9])
     d = [t.to(DEV) for t in (q, k, v, decay, do)]
@@ -198,9 +199,10 @@ def test_backward_reversed_kernels_match_oracle(cuda_lib, B, H, N, dk, dv, gams)
 
 
 def test_backward_launches_on_tensor_cores(cuda_lib):
-    """The 1.3B-shaped backward launches two dQ pieces, two reversed dK pieces, the reversed
-    dV call, the two piece sums and the decay gradient: no copies of reversed operands."""
-    assert cuda_lib.chunkwise_backward_launches(4, 8, 2048, 256, 512, 64, torch.bfloat16) == 8
-    assert cuda_lib.chunkwise_backward_launches(4, 8, 2048, 256, 512, 64, torch.bfloat16, ddecay=False) == 7
-    # one piece (dv <= 256): dQ and dK write dq and dk directly, no sums
+    """The 1.3B-shaped backward launches two dQ pieces, two reversed dK pieces (each adding its
+    tiles onto the zeroed dq or dk), the reversed dV call and the decay gradient: no copies
+    of reversed operands and no separate sums of the pieces."""
+    assert cuda_lib.chunkwise_backward_launches(4, 8, 2048, 256, 512, 64, torch.bfloat16) == 6
+    assert cuda_lib.chunkwise_backward_launches(4, 8, 2048, 256, 512, 64, torch.bfloat16, ddecay=False) == 5
+    # one piece (dv <= 256): dQ and dK store dq and dk directly
     assert cuda_lib.chunkwise_backward_launches(4, 8, 2048, 128, 256, 64, torch.bfloat16) == 4
