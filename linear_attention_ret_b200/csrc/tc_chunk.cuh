@@ -608,11 +608,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             group_sync(1);
             if (te < kC) rr[te] = merged ? pow_int_log2(-lg, REV ? te : kC - 1 - te) : pw[te + 1];
         }
-        float g0 = 0.f, g1 = 0.f;  // gated: prefetched gate values of the next chunk (first warp)
+        // gated: the next chunk's gates, prefetched by the first warp as they are in memory and
+        // scaled to log2 units only where the chunk's scan reads them, so that no instruction
+        // waits for the load before the group barrier
+        float g0 = 0.f, g1 = 0.f;
         if (GATED && te < 32) {
             const int a = chunk_t0(0) + 2 * te;
-            g0 = (a < p.N ? G[a] : 0.f) * kLog2e;
-            g1 = (a + 1 < p.N ? G[a + 1] : 0.f) * kLog2e;
+            g0 = a < p.N ? G[a] : 0.f;
+            g1 = a + 1 < p.N ? G[a + 1] : 0.f;
         }
         // ---------------- P = mask(Q K^T) of chunk c in bf16 (its attention buffer): row j, 32 columns per thread
         auto do_p = [&](int ci) {
@@ -621,11 +624,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             float* cumb = cum + b * kC;
             if (GATED) {
                 if (te < 32) {
-                    warp_cumsum64(g0, g1, lane, cumb);
+                    warp_cumsum64(g0 * kLog2e, g1 * kLog2e, lane, cumb);
                     // prefetch the next chunk's gates (none past the last chunk: a >= N reads zero)
                     const int a = (ci + 1 < nchunks ? chunk_t0(ci + 1) : p.N) + 2 * te;
-                    g0 = (a < p.N ? G[a] : 0.f) * kLog2e;
-                    g1 = (a + 1 < p.N ? G[a + 1] : 0.f) * kLog2e;
+                    g0 = a < p.N ? G[a] : 0.f;
+                    g1 = a + 1 < p.N ? G[a + 1] : 0.f;
                 }
                 group_sync(1);
                 // forward exp(Gl_j); REV exp(Gl_last - Gl_j) (gates past N are zero, so Gl_63 = Gl_{L-1})
@@ -777,11 +780,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             group_sync(2);
             return *abort_flag == 0;
         };
-        float g0 = 0.f, g1 = 0.f;
+        float g0 = 0.f, g1 = 0.f;  // gated: the next chunk's gates, prefetched as in the attention group
         if (GATED && ts < 32) {
             const int a = chunk_t0(0) + 2 * ts;
-            g0 = (a < p.N ? G[a] : 0.f) * kLog2e;
-            g1 = (a + 1 < p.N ? G[a + 1] : 0.f) * kLog2e;
+            g0 = a < p.N ? G[a] : 0.f;
+            g1 = a + 1 < p.N ? G[a + 1] : 0.f;
         }
         float ldec_sum = 0.f;  // log2 of the decay accumulated over this segment
         // Lazy decay. The state is held as S_i = c_i * T_i with T in TMEM and the scalar c_i in
@@ -795,10 +798,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const int t0 = chunk_t0(c), L = min(kC, p.N - t0);
             if (GATED) {
                 if (ts < 32) {
-                    warp_cumsum64(g0, g1, lane, cum);
+                    warp_cumsum64(g0 * kLog2e, g1 * kLog2e, lane, cum);
                     const int a = (c + 1 < nchunks ? chunk_t0(c + 1) : p.N) + 2 * ts;
-                    g0 = (a < p.N ? G[a] : 0.f) * kLog2e;
-                    g1 = (a + 1 < p.N ? G[a + 1] : 0.f) * kLog2e;
+                    g0 = a < p.N ? G[a] : 0.f;
+                    g1 = a + 1 < p.N ? G[a + 1] : 0.f;
                 }
                 group_sync(2);
                 if (ts < kC) zeta[ts] = ts < L ? exp2f(REV ? cum[ts] : cum[L - 1] - cum[ts]) : 0.f;

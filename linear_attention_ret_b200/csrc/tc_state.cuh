@@ -193,7 +193,8 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         const float lg = GATED ? 0.f : log2f(p.decay_in[bh % p.H]);
         const float* G = GATED ? p.decay_in + (size_t)bh * p.N : nullptr;
         // gated: lane l of warp 2 holds gates GPL l .. GPL l + GPL - 1 of tiles c .. c + PF - 1
-        // (read 256 tokens ahead)
+        // (read 256 tokens ahead, kept as they are in memory and scaled to log2 units where the
+        // tile's scan reads them, so that no instruction waits for a load before it is needed)
         constexpr int GPL = kST / 32, PF = 256 / kST;
         float gq[PF][GPL];
         auto load_tile_gates = [&](int c, float (&x)[GPL]) {
@@ -203,7 +204,7 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 const int t0 = tile_t0(c), L = tile_len(c);
 #pragma unroll
                 for (int i = 0; i < GPL; ++i)
-                    if (GPL * ts + i < L) x[i] = G[t0 + GPL * ts + i] * kLog2e;
+                    if (GPL * ts + i < L) x[i] = G[t0 + GPL * ts + i];
             }
         };
         if (GATED && ts < 32) {
@@ -218,8 +219,11 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             float ldec;
             if (GATED) {
                 if (ts < 32) {
-                    if constexpr (kST == 64) warp_cumsum64(gq[0][0], gq[0][1], lane, cum);
-                    else warp_cumsum128(gq[0], lane, cum);
+                    float y[GPL];
+#pragma unroll
+                    for (int i = 0; i < GPL; ++i) y[i] = gq[0][i] * kLog2e;
+                    if constexpr (kST == 64) warp_cumsum64(y[0], y[1], lane, cum);
+                    else warp_cumsum128(y, lane, cum);
 #pragma unroll
                     for (int f = 0; f + 1 < PF; ++f)
 #pragma unroll
