@@ -595,6 +595,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         float* cum = reinterpret_cast<float*>(sm + Lay::kAgTab);  // gated: in-chunk cumsum (log2 units), per buffer
         float* rr = cum + 2 * kC;  // row factor of the drain, per buffer: r_j (split), 1 / zeta'_j (merged)
         float* pw = rr + 2 * kC;                                  // fixed gamma: gamma^t, t = 0..64
+        float* gcol = pw;  // gated (pw unused): column factors [64] of the current chunk, then max |c|
         auto wait_all = [&](int b, uint32_t parity) {  // every thread reaches the barrier; uniform result
             mbar_wait(bar(b), parity, abort_flag);
             group_sync(1);
@@ -625,6 +626,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (GATED) {
                 if (te < 32) {
                     warp_cumsum64(g0 * kLog2e, g1 * kLog2e, lane, cumb);
+                    // largest |cumulative log2-decay| of the chunk (this lane's two values, just written)
+                    float mx = fmaxf(fabsf(cumb[2 * lane]), fabsf(cumb[2 * lane + 1]));
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                    if (lane == 0) gcol[kC] = mx;
                     // prefetch the next chunk's gates (none past the last chunk: a >= N reads zero)
                     const int a = (ci + 1 < nchunks ? chunk_t0(ci + 1) : p.N) + 2 * te;
                     g0 = a < p.N ? G[a] : 0.f;
@@ -633,6 +639,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 group_sync(1);
                 // forward exp(Gl_j); REV exp(Gl_last - Gl_j) (gates past N are zero, so Gl_63 = Gl_{L-1})
                 if (te < kC) rr[b * kC + te] = exp2f(REV ? cumb[kC - 1] - cumb[te] : cumb[te]);
+                // column factors of the weights exp2(c_j - c_m) = exp2(c_j) exp2(-c_m) (REV: the
+                // mirror), used when every |c| of the chunk is at most 100 so that both factors
+                // and their products with Q K^T stay inside the fp32 range
+                if (te < kC) gcol[te] = exp2f(REV ? cumb[te] : -cumb[te]);
             } else if (REV && !merged) {
                 const int L = min(kC, p.N - t0);
                 if (te < kC) rr[b * kC + te] = te < L ? pw[L - 1 - te] : 0.f;
@@ -648,12 +658,21 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 float w[32];
                 if (GATED) {
                     const float cj = cumb[j];
+                    if (gcol[kC] <= 100.f) {  // uniform over the group: one value per chunk
+                        const float rj = exp2f(REV ? -cj : cj);
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) w[c] = REV ? cumb[m0 + c] - cj : cj - cumb[m0 + c];
+                        for (int c = 0; c < 32; ++c) {
+                            const int m = m0 + c;
+                            w[c] = (REV ? m < j : m > j) ? 0.f : (m == j ? 1.f : gcol[m] * rj);
+                        }
+                    } else {
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const int m = m0 + c;
-                        w[c] = (REV ? m < j : m > j) ? 0.f : (m == j ? 1.f : exp2f(w[c]));
+                        for (int c = 0; c < 32; ++c) w[c] = REV ? cumb[m0 + c] - cj : cj - cumb[m0 + c];
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            const int m = m0 + c;
+                            w[c] = (REV ? m < j : m > j) ? 0.f : (m == j ? 1.f : exp2f(w[c]));
+                        }
                     }
                 } else if (REV) {
                     // split: gamma^(m-j); merged: zeta'_m = gamma^m

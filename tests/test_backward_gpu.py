@@ -109,6 +109,22 @@ def test_gated_backward_matches_oracle(cuda_lib, B, H, N, dk, dv, dtype):
     _check_decay_grad(dg, q, k, g, dq, dkk, want[3], want[0], want[1], dtype, True, "dg")
 
 
+def test_gated_backward_steep_and_mild_gates(cuda_lib):
+    """The reversed gated kernels form their mask weights from a row and a column factor when
+    the chunk's cumulative log2-decay stays within +-100, else element by element; dq, dk and
+    dv must match the oracle with both kinds of chunk in one call."""
+    q, k, v, do, gen = _case(1, 4, 300, 64, 128, torch.bfloat16, seed=78)
+    g = I.gate(1, 4, 300, gen)
+    g[:, 1] *= 200.0
+    g[:, 2, 150:] *= 200.0
+    dq, dkk, dvv, _ = cuda_lib.chunkwise_backward(*(t.to(DEV) for t in (q, k, v, g, do)), 64, gated=True)
+    assert cuda_lib.last_device_error() == 0
+    want = O.gated_backward(q, k, v, g, do)
+    _check(dq, want[0], torch.bfloat16, "dq")
+    _check(dkk, want[1], torch.bfloat16, "dk")
+    _check(dvv, want[2], torch.bfloat16, "dv")
+
+
 def test_backward_gradient_of_forward_by_directional_derivative(cuda_lib):
     """Independent of the oracle's backward: for a random direction (Q', K', V') the
     directional derivative of sum(dO * O) computed from the GPU forward by central

@@ -98,6 +98,34 @@ def test_gated_chunkwise_matches_oracle(cuda_lib, B, H, N, dk, dv, chunk, dtype)
     assert_close(s_out, want_s, dtype, "state")
 
 
+def _steep_and_mild_gates(B, H, N, gen):
+    """Gates whose in-chunk cumulative log2-decay stays far inside +-100 on some heads and
+    chunks and passes it on others (about -9 per token), with both kinds inside one head."""
+    g = I.gate(B, H, N, gen)
+    g[:, 1] *= 200.0
+    g[:, 2, N // 2:] *= 200.0
+    return g
+
+
+def test_gated_steep_and_mild_gates(cuda_lib):
+    """The gated mask weights exp(G_j - G_m) are formed from a row and a column factor when the
+    chunk's cumulative log2-decay stays within +-100, else element by element; one call mixes
+    both kinds of chunk (ragged tail, initial state) and must match the oracle."""
+    B, H, N, dk, dv = 1, 4, 300, 64, 128
+    gen = torch.Generator().manual_seed(77)
+    q, k, v = I.qkv(B, H, N, dk, dv, torch.bfloat16, gen=gen)
+    g = _steep_and_mild_gates(B, H, N, gen)
+    S0 = torch.randn(B, H, dk, dv, generator=gen) * 0.05
+    qd, kd, vd, gdv, S0d = _dev(q, k, v, g, S0)
+    s_out = torch.empty_like(S0d)
+    o = cuda_lib.gated_ret_chunkwise(qd, kd, vd, gdv, 64, state_in=S0d, state_out=s_out)
+    assert cuda_lib.last_device_error() == 0
+    want_o, want_s = O.gated_chunkwise(q, k, v, g, 64, state_in=S0)
+    for h in range(H):
+        assert rel_l2(o[0, h].cpu(), want_o[0, h]) <= TOL_BF16, ("o", h)
+        assert rel_l2(s_out[0, h].cpu(), want_s[0, h]) <= TOL_BF16, ("state", h)
+
+
 def test_chunkwise_no_state_and_in_place_state(cuda_lib):
     B, H, N, dk, dv = 2, 2, 96, 64, 128
     q, k, v = _rand_inputs(B, H, N, dk, dv, torch.bfloat16, seed=11)
