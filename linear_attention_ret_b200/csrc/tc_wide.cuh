@@ -62,7 +62,8 @@ struct WideLayout {
     static constexpr int kNumBars = 19;
     static constexpr int kAgTab = (kBar + kNumBars * 8 + 15) & ~15;  // attention group: drain row factors [128]
     static constexpr int kSgTab = kAgTab + kW * 4;      // state group: zeta / kappa [128]
-    static constexpr int kTmemSlot = kSgTab + kW * 4;
+    static constexpr int kBc = kSgTab + kW * 4;         // gated: the state group's tile decay, broadcast
+    static constexpr int kTmemSlot = kBc + 16;
     static constexpr int kAbort = kTmemSlot + 4;
     static constexpr int kBytes = kAbort + 4;
     static constexpr int kSmemAlloc = kBytes + 1024;    // slack to align the base to 1024 B
@@ -91,9 +92,40 @@ __device__ __forceinline__ float lazy_next_scale(float kappa, float decay, bool 
     return renorm ? 1.f : kappa * decay;
 }
 
-template <int DK, bool REV>
+// Gated: raw gates 4l .. 4l+3 (natural-log units) of the 128-token tile starting at t0, for
+// lane l of one warp; zero at and past the segment end tend.
+__device__ __forceinline__ void load_gates4(const float* G, int t0, int tend, int lane, float (&g)[4]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int t = t0 + 4 * lane + i;
+        g[i] = t < tend ? G[t] : 0.f;
+    }
+}
+
+// Gated: in-tile inclusive cumulative log2-decay c of a 128-token tile by one warp, from the
+// raw gates load_gates4 gave lane l; lane l gets c at tokens 4l .. 4l+3. Returns the tile's
+// total, c after token 127 (equal to c after the last valid token: gates past it are zero).
+__device__ __forceinline__ float tile_scan128(const float (&g)[4], float (&c)[4], int lane) {
+    const float y0 = g[0] * kLog2e, y1 = g[1] * kLog2e, y2 = g[2] * kLog2e, y3 = g[3] * kLog2e;
+    const float p1 = y0 + y1, p2 = p1 + y2, p3 = p2 + y3;
+    float incl = p3;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    const float excl = incl - p3;
+    c[0] = excl + y0;
+    c[1] = excl + p1;
+    c[2] = excl + p2;
+    c[3] = excl + p3;
+    return __shfl_sync(0xffffffffu, c[3], 31);
+}
+
+template <int DK, bool REV, bool GATED = false>
 __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                                           const CUtensorMap& tm_o, const Params& p, float lg) {
+    static_assert(!(GATED && REV), "the time-reversed gated form takes the 64-token body");
     using Lay = WideLayout<DK>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -115,6 +147,10 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
     // token start of the c-th tile visited (REV: from the last tile of the segment back)
     auto tile_t0 = [&](int c) { return tbeg + (REV ? ntiles - 1 - c : c) * kW; };
     auto tile_len = [&](int c) { return min(kW, tend - tile_t0(c)); };
+    // gated: this head's gates g [N] (log-decay per token); the tile factors below replace
+    // gamma^L by the tile decay exp2(c_last) and gamma^(L-1-m) by zeta_m = exp2(c_last - c_m),
+    // with c the tile's inclusive cumulative log2-decay
+    const float* G = GATED ? p.decay_in + (size_t)bh * p.N : nullptr;
 
     if (threadIdx.x == 0) {
         for (int b = 0; b < Lay::kNumBars; ++b) mbar_init(bar(b), 1);
@@ -256,9 +292,23 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
             return *abort_flag == 0;
         };
         float kappa = 1.f;
+        // gated: the group's first warp scans each tile's gates (prefetched one tile ahead, raw)
+        // and alone holds kappa; the other threads only read the row factors it writes
+        float gnext[4] = {0.f, 0.f, 0.f, 0.f};
+        if (GATED && te < 32) load_gates4(G, tile_t0(0), tend, lane, gnext);
         for (int c = 0; c < ntiles; ++c) {
             const int t0 = tile_t0(c), L = tile_len(c);
-            if (c > 0) {
+            float gc[4] = {0.f, 0.f, 0.f, 0.f}, gl = 0.f;
+            if constexpr (GATED) {
+                if (te < 32) {
+                    gl = tile_scan128(gnext, gc, lane);
+                    if (c + 1 < ntiles) load_gates4(G, tile_t0(c + 1), tend, lane, gnext);
+                    if (c > 0) {
+                        bool rn;
+                        kappa = lazy_next_scale(kappa, exp2f(gl), false, rn);
+                    }
+                }
+            } else if (c > 0) {
                 bool rn;
                 kappa = lazy_next_scale(kappa, pow_int_log2(lg, L), false, rn);
             }
@@ -300,7 +350,17 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
             group_sync(1);
             if (te == 0) mbar_arrive(bar(wPReady));
             // ---------------- O_j = (kappa / zeta_j) Z_j -> bf16 -> staging -> TMA store
-            rowf[te] = te < L ? kappa * pow_int_log2(-lg, REV ? te + 1 : L - 1 - te) : 0.f;
+            if constexpr (GATED) {
+                if (te < 32) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int tok = 4 * lane + i;
+                        rowf[tok] = tok < L ? kappa * exp2f(gc[i] - gl) : 0.f;  // kappa / zeta_j
+                    }
+                }
+            } else {
+                rowf[te] = te < L ? kappa * pow_int_log2(-lg, REV ? te + 1 : L - 1 - te) : 0.f;
+            }
             if (!wait_all(wOFull, c & 1)) break;
             tc_fence_after();
             {
@@ -366,6 +426,9 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
         const int d = quarter * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         float* zk = reinterpret_cast<float*>(sm + Lay::kSgTab);  // zeta_m / kappa
+        float* bc = reinterpret_cast<float*>(sm + Lay::kBc);     // gated: the next tile's decay
+        // gated: the group's first warp scans the next tile's gates (prefetched one tile ahead)
+        float graw[4] = {0.f, 0.f, 0.f, 0.f}, sgc[4] = {0.f, 0.f, 0.f, 0.f}, sgl = 0.f;
         auto wait_all = [&](int b, uint32_t parity) {
             mbar_wait(bar(b), parity, abort_flag);
             group_sync(2);
@@ -375,7 +438,17 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
         // two 16 KB blocks of 128 token rows, so the token of a chunk is (ci mod 1024) / 8.
         auto build_zv = [&](int c, float kappa) {
             const int L = tile_len(c);
-            zk[ts] = ts < L ? pow_int_log2(lg, REV ? ts + 1 : L - 1 - ts) * (1.f / kappa) : 0.f;
+            if constexpr (GATED) {
+                if (ts < 32) {  // sgc, sgl: the scan of tile c
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int tok = 4 * lane + i;
+                        zk[tok] = tok < L ? exp2f(sgl - sgc[i]) * (1.f / kappa) : 0.f;
+                    }
+                }
+            } else {
+                zk[ts] = ts < L ? pow_int_log2(lg, REV ? ts + 1 : L - 1 - ts) * (1.f / kappa) : 0.f;
+            }
             if (!wait_all(wVFull0 + (c & 1), (c >> 1) & 1)) return false;
             uint8_t* vt = sm + Lay::kV + (c & 1) * Lay::kVBuf;
 #pragma unroll
@@ -412,7 +485,19 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
         float kappa;
         {
             bool rn;
-            const float dec0 = pow_int_log2(lg, tile_len(0));
+            float dec0;
+            if constexpr (GATED) {
+                if (ts < 32) {
+                    load_gates4(G, tile_t0(0), tend, lane, graw);
+                    sgl = tile_scan128(graw, sgc, lane);
+                    if (lane == 0) bc[0] = exp2f(sgl);
+                    if (ntiles > 1) load_gates4(G, tile_t0(1), tend, lane, graw);
+                }
+                group_sync(2);
+                dec0 = bc[0];
+            } else {
+                dec0 = pow_int_log2(lg, tile_len(0));
+            }
             kappa = lazy_next_scale(1.f, dec0, true, rn);
             const float* sin = segment_start_state(p, seg, bh, DK, dv0 + d);
 #pragma unroll 1
@@ -438,10 +523,22 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
             bool rn = false;
             float dec_next = 0.f, k_next = 1.f;
             if (!last) {
-                dec_next = pow_int_log2(lg, tile_len(c + 1));
-                k_next = lazy_next_scale(kappa, dec_next, false, rn);
+                if constexpr (GATED) {
+                    if (ts < 32) {  // scan tile c + 1; its decay reaches the group at the barrier below
+                        sgl = tile_scan128(graw, sgc, lane);
+                        if (c + 2 < ntiles) load_gates4(G, tile_t0(c + 2), tend, lane, graw);
+                        if (lane == 0) bc[0] = exp2f(sgl);
+                    }
+                } else {
+                    dec_next = pow_int_log2(lg, tile_len(c + 1));
+                    k_next = lazy_next_scale(kappa, dec_next, false, rn);
+                }
             }
             if (!wait_all(wSFull, c & 1)) break;
+            if (GATED && !last) {
+                dec_next = bc[0];
+                k_next = lazy_next_scale(kappa, dec_next, false, rn);
+            }
             tc_fence_after();
             if (last) {
                 float* so = last_seg ? p.state_out : nullptr;

@@ -126,6 +126,37 @@ def test_gated_steep_and_mild_gates(cuda_lib):
         assert rel_l2(s_out[0, h].cpu(), want_s[0, h]) <= TOL_BF16, ("state", h)
 
 
+GATED_WIDE_CASES = [
+    # B, H, N, dk, dv
+    (1, 2, 300, 128, 128),   # ragged last tile
+    (2, 3, 1000, 256, 256),  # two dv slices; the lazy scale renormalises along the sequence
+    (1, 1, 2053, 128, 128),  # one head: the sequence is cut into segments
+]
+
+
+@pytest.mark.parametrize("B,H,N,dk,dv", GATED_WIDE_CASES)
+def test_gated_128_token_body_matches_oracle(cuda_lib, B, H, N, dk, dv):
+    """Gated segments whose every gate lies in [-0.52, 0] (log2-decay of at most 0.75 per
+    token) run the 128-token body, with the tile decay exp2(c_last) and the key weights
+    exp2(c_last - c_m) in place of gamma's powers. One gate of head 0 is set outside that
+    range, so that head's segment takes the 64-token body in the same call."""
+    gen = torch.Generator().manual_seed(N + dk)
+    q, k, v = I.qkv(B, H, N, dk, dv, torch.bfloat16, gen=gen)
+    g = I.gate(B, H, N, gen)
+    assert float(g.min()) > -0.5 and float(g.max()) <= 0.0
+    g[0, 0, N // 3] = -1.0
+    S0 = torch.randn(B, H, dk, dv, generator=gen) * 0.05
+    qd, kd, vd, gdv, S0d = _dev(q, k, v, g, S0)
+    s_out = torch.empty_like(S0d)
+    o = cuda_lib.gated_ret_chunkwise(qd, kd, vd, gdv, 64, state_in=S0d, state_out=s_out)
+    assert cuda_lib.last_device_error() == 0
+    want_o, want_s = O.gated_chunkwise(q, k, v, g, 64, state_in=S0)
+    for b in range(B):
+        for h in range(H):
+            assert rel_l2(o[b, h].cpu(), want_o[b, h]) <= TOL_BF16, ("o", b, h)
+            assert rel_l2(s_out[b, h].cpu(), want_s[b, h]) <= TOL_BF16, ("state", b, h)
+
+
 def test_chunkwise_no_state_and_in_place_state(cuda_lib):
     B, H, N, dk, dv = 2, 2, 96, 64, 128
     q, k, v = _rand_inputs(B, H, N, dk, dv, torch.bfloat16, seed=11)
