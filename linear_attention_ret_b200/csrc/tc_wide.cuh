@@ -36,8 +36,8 @@
 // zeta_i = gamma^(i+1) (i the token's place in its tile) and the mask i >= j: the cross
 // factor gamma^(L-1-j) R_next = kappa T / zeta_j with kappa T = gamma^L R_next.
 // Shared memory: one Q and one K tile, each with its own full/empty barriers so that it
-// reloads as soon as its last reader is done (K after the update, Q after the cross
-// term); two V tiles (tile c in buffer c & 1, loaded right after K, so that V(c+1) lands
+// reloads as soon as its last reader is done (K after the update, each dk half of Q after
+// the cross term's steps over it); two V tiles (tile c in buffer c & 1, loaded right after K, so that V(c+1) lands
 // and becomes zeta V / kappa while tile c's products still read ZV(c)); and one P tile
 // that is also the staging tile of the O store (224 KB at dk = 256). zeta V / kappa is
 // formed with bf16 pair products (the factor rounded to bf16, each product rounded once:
@@ -59,7 +59,7 @@ struct WideLayout {
     static constexpr int kVBuf = 2 * kBlk;              // bytes of one V tile
     static constexpr int kP = kV + 2 * kVBuf;           // P (2 blocks of 64 m columns); O staging (4 x 64 x 64)
     static constexpr int kBar = kP + 2 * kBlk;
-    static constexpr int kNumBars = 19;
+    static constexpr int kNumBars = 20;
     static constexpr int kAgTab = (kBar + kNumBars * 8 + 15) & ~15;  // attention group: drain row factors [128]
     static constexpr int kSgTab = kAgTab + kW * 4;      // state group: zeta / kappa [128]
     static constexpr int kBc = kSgTab + kW * 4;         // gated: the state group's tile decay, broadcast
@@ -77,10 +77,11 @@ struct WideLayout {
 };
 
 enum WideBar {
-    wQFull = 0, wKFull, wQEmpty, wKEmpty,
+    wQFull = 0, wKFull, wQEmpty, wKEmpty,      // wQFull, wQEmpty: the low dk half of Q (wQFullHi, wQEmptyHi: the high)
     wVFull0, wVFull1, wVEmpty0, wVEmpty1,      // per V buffer (tile c uses buffer c & 1)
     wAFull, wARead, wPReady, wOFull, wOFree,
-    wSFull, wSReady, wZV0, wZV1, wDrain
+    wSFull, wSReady, wZV0, wZV1, wDrain,
+    wQFullHi, wQEmptyHi
 };
 
 // Lazy decay normalisation (S = kappa T). Given the current kappa and the next tile's
@@ -127,6 +128,10 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
                                           const CUtensorMap& tm_o, const Params& p, float lg) {
     static_assert(!(GATED && REV), "the time-reversed gated form takes the 64-token body");
     using Lay = WideLayout<DK>;
+    // dk = 256: Q in two dk halves with their own barriers (each reloads once the cross term
+    // has read it); at dk = 128 one Q barrier measured faster
+    constexpr bool kQHalves = DK == 256;
+    constexpr int kQLo = kQHalves ? DK / 128 : DK / 64;  // dk blocks of the low part (all of Q without halves)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
@@ -177,7 +182,7 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
             // 64 x 64 boxes; two of them (tokens t0 and t0 + 64) fill one 128-row block.
             // Rows past the segment end are loaded too and masked by the epilogues; rows
             // past N read as zero.
-            int issued[3] = {-1, -1, -1};  // K, Q, V: last tile whose copies were issued
+            int issued[4] = {-1, -1, -1, -1};  // K, Q low half, V, Q high half: last tile whose copies were issued
             for (int c = 0; c < ntiles; ++c) {
                 const int t0 = tile_t0(c);
                 const uint32_t ph = (c - 1) & 1;
@@ -203,19 +208,32 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
                                         t0 + 64 * h, bh, bar(wVFull0 + vb));
                 }
                 issued[2] = c;
+                // Q: the low part (all of Q without halves), then the high half
                 if (c > 0 && !mbar_wait(bar(wQEmpty), ph, abort_flag)) break;
-                mbar_expect_tx(bar(wQFull), DK / 64 * kBlk);
+                mbar_expect_tx(bar(wQFull), kQLo * kBlk);
 #pragma unroll
-                for (int kb = 0; kb < DK / 64; ++kb)
+                for (int kb = 0; kb < kQLo; ++kb)
 #pragma unroll
                     for (int h = 0; h < 2; ++h)
                         tma_load_3d(sbase + Lay::kQ + kb * kBlk + h * kTile64, &tm_q, kb * 64, t0 + 64 * h, bh, bar(wQFull));
                 issued[1] = c;
+                if constexpr (kQHalves) {
+                    if (c > 0 && !mbar_wait(bar(wQEmptyHi), ph, abort_flag)) break;
+                    mbar_expect_tx(bar(wQFullHi), (DK / 64 - kQLo) * kBlk);
+#pragma unroll
+                    for (int kb = kQLo; kb < DK / 64; ++kb)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            tma_load_3d(sbase + Lay::kQ + kb * kBlk + h * kTile64, &tm_q, kb * 64, t0 + 64 * h, bh,
+                                        bar(wQFullHi));
+                    issued[3] = c;
+                }
             }
             if (*abort_flag) {
                 // drain the copies in flight before the CTA may exit
                 if (issued[0] >= 0) mbar_drain(bar(wKFull), issued[0] & 1);
                 if (issued[1] >= 0) mbar_drain(bar(wQFull), issued[1] & 1);
+                if (kQHalves && issued[3] >= 0) mbar_drain(bar(wQFullHi), issued[3] & 1);
                 for (int c = std::max(issued[2] - 1, 0); c <= issued[2]; ++c) mbar_drain(bar(wVFull0 + (c & 1)), (c >> 1) & 1);
             }
         }
@@ -236,9 +254,18 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
                 if (c > 0 && !mbar_wait(bar(wOFree), (c - 1) & 1, abort_flag)) break;
                 tc_fence_after();
 #pragma unroll
-                for (int ks = 0; ks < DK / 16; ++ks) {
+                for (int ks = 0; ks < 4 * kQLo; ++ks) {  // the low part of Q
                     const uint32_t off = (ks >> 2) * kBlk + (ks & 3) * 32;
                     mma_ss(tR, sdesc(sQ + off, 16, 1024), sdesc(sK + off, 16, 1024), id_qk, ks > 0);
+                }
+                if constexpr (kQHalves) {
+                    if (!mbar_wait(bar(wQFullHi), ph, abort_flag)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 4 * kQLo; ks < DK / 16; ++ks) {  // the high half
+                        const uint32_t off = (ks >> 2) * kBlk + (ks & 3) * 32;
+                        mma_ss(tR, sdesc(sQ + off, 16, 1024), sdesc(sK + off, 16, 1024), id_qk, 1);
+                    }
                 }
                 mma_commit(bar(wAFull));
                 // S^T += (zeta V / kappa)^T K while the epilogue reads A: A operand = the
@@ -256,14 +283,20 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
                 if (!mbar_wait(bar(wARead), ph, abort_flag)) break;
                 tc_fence_after();
 #pragma unroll
-                for (int ks = 0; ks < DK / 16; ++ks) {
+                for (int ks = 0; ks < 4 * kQLo; ++ks) {
                     const uint32_t off = (ks >> 2) * kBlk + (ks & 3) * 32;
                     mma_ts(tR, tSop + ks * 8, sdesc(sQ + off, 16, 1024), id_oi, ks > 0);
                 }
+                mma_commit(bar(wQEmpty));  // the low part of Q may reload
+#pragma unroll
+                for (int ks = 4 * kQLo; ks < DK / 16; ++ks) {
+                    const uint32_t off = (ks >> 2) * kBlk + (ks & 3) * 32;
+                    mma_ts(tR, tSop + ks * 8, sdesc(sQ + off, 16, 1024), id_oi, 1);
+                }
                 // the update and the cross term are done: the state epilogue may read S and
-                // overwrite its bf16 copy; the Q tile may reload
+                // overwrite its bf16 copy; the high half of Q may reload
                 mma_commit(bar(wSFull));
-                mma_commit(bar(wQEmpty));
+                if constexpr (kQHalves) mma_commit(bar(wQEmptyHi));
                 // Z^T += (zeta V / kappa)^T P^T (B = P K-major, m blocks 16 KB apart)
                 if (!mbar_wait(bar(wPReady), ph, abort_flag)) break;
                 tc_fence_after();
