@@ -371,17 +371,16 @@ __device__ __forceinline__ const float* segment_start_state(const Params& p, int
     return p.state_in ? p.state_in + ((size_t)bh * dk) * p.dv + col : nullptr;
 }
 
-// Whether an instantiation may run the 128-token body: dk of 128 or 256, not the state-only
-// pass, and for the gated form only the forward direction.
-constexpr bool wide_capable(int dk, bool gated, bool state_only, bool rev = false) {
-    return !state_only && dk >= 128 && !(gated && rev);
+// Whether an instantiation may run the 128-token body: dk of 128 or 256, not the state-only pass.
+constexpr bool wide_capable(int dk, bool gated, bool state_only) {
+    return !state_only && dk >= 128;
 }
 
 // Gated: whether every gate of this CTA's segment lies in [kWideMinLog2 / log2(e), 0], the
 // per-token analogue of gamma >= 2^-0.75, so that the 128-token body's tile factors stay in
 // range. Read by all threads of the CTA; the answer is uniform.
-__device__ __forceinline__ bool gated_wide_ok(const Params& p, int bh, int seg) {
-    const int tbeg = seg * p.seg_chunks * kC;
+__device__ __forceinline__ bool gated_wide_ok(const Params& p, int bh, int tseg) {
+    const int tbeg = tseg * p.seg_chunks * kC;
     const int tend = min(tbeg + p.seg_chunks * kC, p.N);
     const float* G = p.decay_in + (size_t)bh * p.N;
     int ok = 1;
@@ -418,9 +417,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     asm volatile("griddepcontrol.wait;" ::: "memory");
     // Heads with gamma close to 1, and gated segments whose every gate is that mild, take the
     // 128-token body (tc_wide.cuh); the choice is per CTA, so one launch serves a mix.
-    if constexpr (wide_capable(DK, GATED, STATE_ONLY, REV)) {
+    if constexpr (wide_capable(DK, GATED, STATE_ONLY)) {
         if constexpr (GATED) {
-            if (gated_wide_ok(p, blockIdx.y, blockIdx.z)) {
+            // the segment's place in time (the time-reversed form chains segments from the last)
+            if (gated_wide_ok(p, blockIdx.y, REV ? p.units - 1 - (int)blockIdx.z : (int)blockIdx.z)) {
                 wide_body<DK, REV, true>(tm_q, tm_k, tm_v, tm_o, p, 0.f);
                 return;
             }

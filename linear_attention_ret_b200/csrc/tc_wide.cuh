@@ -126,7 +126,6 @@ __device__ __forceinline__ float tile_scan128(const float (&g)[4], float (&c)[4]
 template <int DK, bool REV, bool GATED = false>
 __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                                           const CUtensorMap& tm_o, const Params& p, float lg) {
-    static_assert(!(GATED && REV), "the time-reversed gated form takes the 64-token body");
     using Lay = WideLayout<DK>;
     // dk = 256: Q in two dk halves with their own barriers (each reloads once the cross term
     // has read it); at dk = 128 one Q barrier measured faster
@@ -154,7 +153,7 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
     auto tile_len = [&](int c) { return min(kW, tend - tile_t0(c)); };
     // gated: this head's gates g [N] (log-decay per token); the tile factors below replace
     // gamma^L by the tile decay exp2(c_last) and gamma^(L-1-m) by zeta_m = exp2(c_last - c_m),
-    // with c the tile's inclusive cumulative log2-decay
+    // with c the tile's inclusive cumulative log2-decay (REV: gamma^(i+1) by zeta_i = exp2(c_i))
     const float* G = GATED ? p.decay_in + (size_t)bh * p.N : nullptr;
 
     if (threadIdx.x == 0) {
@@ -388,7 +387,8 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const int tok = 4 * lane + i;
-                        rowf[tok] = tok < L ? kappa * exp2f(gc[i] - gl) : 0.f;  // kappa / zeta_j
+                        // kappa / zeta_j: zeta_j = exp2(c_last - c_j), REV exp2(c_j)
+                        rowf[tok] = tok < L ? kappa * exp2f(REV ? -gc[i] : gc[i] - gl) : 0.f;
                     }
                 }
             } else {
@@ -476,7 +476,7 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& tm_q, const CUtenso
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const int tok = 4 * lane + i;
-                        zk[tok] = tok < L ? exp2f(sgl - sgc[i]) * (1.f / kappa) : 0.f;
+                        zk[tok] = tok < L ? exp2f(REV ? sgc[i] : sgl - sgc[i]) * (1.f / kappa) : 0.f;
                     }
                 }
             } else {

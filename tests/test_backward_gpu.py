@@ -182,17 +182,21 @@ def test_backward_without_decay_gradient(cuda_lib, gated):
 # The dK and dV sums run over later tokens; on the tensor-core path they are computed by the
 # time-reversed forward kernels (chunks visited from the last back, upper-triangular mask,
 # mirrored decay factors). These cases reach each body of that kernel: the 128-token body
-# (gamma >= 0.595 with widths 128 or 256), the 64-token body with the merged output
-# accumulator (gamma in [0.5, 0.595)) and with split accumulators (gamma < 0.5, gated), on
-# sequences long enough for few heads to be cut into segments chained from the end, with
-# ragged last chunks.
+# (gamma >= 0.595, or gates in [-0.52, 0], with widths 128 or 256), the 64-token body with the
+# merged output accumulator (gamma in [0.5, 0.595)) and with split accumulators (gamma < 0.5,
+# steeper gates), on sequences long enough for few heads to be cut into segments chained from
+# the end, with ragged last chunks.
 REV_CASES = [
-    # B, H, N, dk, dv, gammas (None: gated)
+    # B, H, N, dk, dv, gammas (None: gated, gates x4; "mild": gated, gates as drawn)
     (1, 4, 450, 128, 128, [0.3, 0.55, 0.9, 0.999]),
     (1, 2, 300, 256, 256, [0.2, 0.45]),
     (2, 2, 700, 256, 512, [0.5, 0.7]),
     (1, 2, 1333, 128, 128, None),
     (1, 1, 2049, 256, 256, None),
+    # gates in [-0.52, 0] ("mild"): the gated passes take the 128-token body too
+    (1, 2, 700, 128, 128, "mild"),
+    (1, 1, 2049, 256, 256, "mild"),
+    (1, 2, 300, 256, 512, "mild"),
 ]
 
 
@@ -200,18 +204,19 @@ REV_CASES = [
 def test_backward_reversed_kernels_match_oracle(cuda_lib, B, H, N, dk, dv, gams):
     dtype = torch.bfloat16
     q, k, v, do, gen = _case(B, H, N, dk, dv, dtype, seed=5 * N + dk)
-    if gams is None:
-        decay = I.gate(B, H, N, gen) * 4.0
+    gated = gams is None or gams == "mild"
+    if gated:
+        decay = I.gate(B, H, N, gen) * (1.0 if gams == "mild" else 4.0)
         want = O.gated_backward(q, k, v, decay, do)
     else:
         decay = torch.tensor(gams, dtype=torch.float32)
         want = O.ret_backward(q, k, v, decay, do)
-    got = cuda_lib.chunkwise_backward(*(t.to(DEV) for t in (q, k, v, decay, do)), 64, gated=gams is None)
+    got = cuda_lib.chunkwise_backward(*(t.to(DEV) for t in (q, k, v, decay, do)), 64, gated=gated)
     assert cuda_lib.last_device_error() == 0
     for g, w, what in zip(got[:3], want[:3], ("dq", "dk", "dv")):
         _check(g, w, dtype, what)
-    _check_decay_grad(got[3], q, k, decay, got[0], got[1], want[3], want[0], want[1], dtype, gams is None,
-                      "dgamma" if gams else "dg")
+    _check_decay_grad(got[3], q, k, decay, got[0], got[1], want[3], want[0], want[1], dtype, gated,
+                      "dg" if gated else "dgamma")
 
 
 def test_backward_launches_on_tensor_cores(cuda_lib):
