@@ -17,6 +17,8 @@ batch of seeded synthetic input already resident in HBM:
                     segment end states, one all-gather, start states, ret_chunkwise per segment
   backward_1p3b     ret_chunkwise_backward on the retnet_1p3b shapes: dq, dk, dv and dgamma
                     from q, k, v, gamma and an output gradient dO
+  backward_gated    gated_ret_chunkwise_backward on the gated workload's shapes: dq, dk, dv and
+                    dg from q, k, v, g and dO
   msr_norm_1p3b     ret_msr_norm_gate on the retnet_1p3b output: per-head RMSNorm and swish gate
   retention_msr_1p3b  ret_chunkwise then ret_msr_norm_gate on its output (retnet_1p3b shapes)
 For N > 1 (torchrun, one rank per GPU) every rank runs its own batch of the
@@ -44,6 +46,7 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 L2_BYTES = 126 * 1024 * 1024
 NORM_EPS = 1e-5  # the norm epsilon the pages give as the module default
+GATED_BWD_SAMPLE_TOKENS = 2048  # tokens per head in the gated backward's CPU sample
 
 
 # ----------------------------------------------------------------------------- workload arithmetic
@@ -57,17 +60,21 @@ def workload(name: str):
         spec = workload("retnet_6p7b_long")
         spec.update(kind="seqpar", metric="retention tokens/s (sequence-parallel chunkwise fwd)")
         return spec
-    if name == "backward_1p3b":
-        cfg = I.CONFIGS["retnet_1p3b"]
+    if name in ("backward_1p3b", "backward_gated"):
+        gated = name == "backward_gated"
+        cfg = I.CONFIGS["gated" if gated else "retnet_1p3b"]
         B, H, N, dk, dv, C = cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk
         elt = 2
-        # reads q, k, v, dO; writes dq, dk, dv (dgamma is H floats)
-        io = B * H * N * (4 * dk + 3 * dv) * elt
+        # reads q, k, v, dO; writes dq, dk, dv (dgamma is H floats; gated: g read, dg written, fp32)
+        gb = 4 * B * H * N if gated else 0
+        io = B * H * N * (4 * dk + 3 * dv) * elt + 2 * gb
         # three contractions of the forward's shape: dQ (scores dO.v), dK (dO.v), dV (q.k)
         flops = 3 * B * H * N * (2 * C * (dk + dv) + 4 * dk * dv)
-        return dict(cfg=cfg, kind="backward", units=B * N, unit="tokens/s",
-                    metric="retention tokens/s (chunkwise backward)", tokens=B * N, bytes=io, flops=flops,
-                    h2d=B * H * N * (2 * dk + 2 * dv) * elt, d2h=B * H * N * (2 * dk + dv) * elt + H * 4)
+        return dict(cfg=cfg, kind="backward", gated=gated, units=B * N, unit="tokens/s",
+                    metric="retention tokens/s (gated chunkwise backward)" if gated
+                    else "retention tokens/s (chunkwise backward)", tokens=B * N, bytes=io, flops=flops,
+                    h2d=B * H * N * (2 * dk + 2 * dv) * elt + gb,
+                    d2h=B * H * N * (2 * dk + dv) * elt + (gb if gated else H * 4))
     if name in ("msr_norm_1p3b", "retention_msr_1p3b"):
         cfg = I.CONFIGS["retnet_1p3b"]
         B, H, N, dk, dv, C = cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk
@@ -122,7 +129,7 @@ KERNEL_SOURCES = {
     "backward": ("common.cuh", "tc_chunk.cuh", "tc_wide.cuh", "tc_state.cuh", "backward.cuh", "ret_api.cu"),
 }
 WORKLOAD_KERNELS = {"retnet_1p3b": "chunk", "retnet_6p7b_long": "chunk", "gated": "chunk", "seqpar_6p7b": "chunk",
-                    "decode": "decode", "gated_decode": "decode", "backward_1p3b": "backward",
+                    "decode": "decode", "gated_decode": "decode", "backward_1p3b": "backward", "backward_gated": "backward",
                     "msr_norm_1p3b": "norm", "retention_msr_1p3b": "chunk"}
 
 
@@ -304,8 +311,11 @@ def make_step(spec, dev, seed):
     if spec["kind"] == "backward":
         x["do"] = I.output_grad(cfg.B, cfg.H, cfg.N, cfg.dv, cfg.dtype, seed=seed).to(dev)
 
+        gated = spec["gated"]
+
         def step():
-            ret.chunkwise_backward(x["q"], x["k"], x["v"], x["gamma"], x["do"], cfg.chunk)
+            ret.chunkwise_backward(x["q"], x["k"], x["v"], x["g"] if gated else x["gamma"], x["do"], cfg.chunk,
+                                   gated=gated)
         return step, x, None, launches_per_call(spec)
     o = torch.empty(cfg.B, cfg.H, cfg.N, cfg.dv, dtype=cfg.dtype, device=dev)
     if spec["kind"] == "gated":
@@ -336,7 +346,8 @@ def launches_per_call(spec) -> int:
     if spec["kind"] == "ret_norm":
         return ret.chunkwise_launches(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk, cfg.dtype) + 1
     if spec["kind"] == "backward":
-        return ret.chunkwise_backward_launches(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk, cfg.dtype)
+        return ret.chunkwise_backward_launches(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk, cfg.dtype,
+                                               gated=spec["gated"])
     if spec["kind"] == "seqpar":
         _, world, _ = dist_env()
         n = cfg.N // world + (1 if cfg.N % world else 0)
@@ -422,8 +433,8 @@ def measure(args, name, spec, dev, stream, world, steps, cpu_budget):
                 "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs, copy)" if peak_src == "measured"
                 else "fallback 6.65 TB/s",
                 "kernel_ms": round(kern_ms, 5),
-                "scope": ("the whole step: " + str(launches) + " launches (the dQ and dK pieces, dV, the piece "
-                          "sums, the decay gradient)") if spec["kind"] == "backward"
+                "scope": ("the whole step: " + str(launches) + " launches (the dQ and dK passes, dV, the decay "
+                          "gradient)") if spec["kind"] == "backward"
                 else "the step's launches",
                 "tensor_tflops": round(spec["flops"] / (kern_ms / 1e3) / 1e12, 2),
                 "tensor_frac_of_bf16_burst": round(spec["flops"] / (kern_ms / 1e3) / 1e12 / tf_burst, 4),
@@ -547,12 +558,14 @@ def run_e2e(args, spec, dev, stream, world):
         xh["do"] = I.output_grad(cfg.B, cfg.H, cfg.N, cfg.dv, cfg.dtype, seed=rank_seed(rank)).pin_memory()
         xd = {k: torch.empty_like(t, device=dev) for k, t in xh.items()}
         outs_h = [torch.empty(xh[n].shape, dtype=cfg.dtype).pin_memory() for n in ("q", "k", "v")]
-        dgam_h = torch.empty(cfg.H, dtype=torch.float32).pin_memory()
+        gated = spec["gated"]
+        dgam_h = torch.empty(xh["g"].shape if gated else (cfg.H,), dtype=torch.float32).pin_memory()
 
         def step():
             for key in xh:
                 xd[key].copy_(xh[key], non_blocking=True)
-            grads = ret.chunkwise_backward(xd["q"], xd["k"], xd["v"], xd["gamma"], xd["do"], cfg.chunk)
+            grads = ret.chunkwise_backward(xd["q"], xd["k"], xd["v"], xd["g"] if gated else xd["gamma"], xd["do"],
+                                           cfg.chunk, gated=gated)
             for h, d in zip(outs_h + [dgam_h], grads):
                 h.copy_(d, non_blocking=True)
     else:
@@ -634,6 +647,15 @@ def _oracle_sample_step(spec, heads, seed=0):
         x["do"] = I.output_grad(x["q"].shape[0], cfg.H, cfg.N, cfg.dv, cfg.dtype, seed=seed)
     sl = {k: t.reshape(-1, *t.shape[2:])[:heads].unsqueeze(0) for k, t in x.items() if k != "gamma"}
     if spec["kind"] == "backward":
+        if spec["gated"]:
+            # the oracle's cost grows faster than N^2, so the sample is the first
+            # GATED_BWD_SAMPLE_TOKENS tokens of each head (a full head of 16384 takes ~17 min)
+            n = min(cfg.N, GATED_BWD_SAMPLE_TOKENS)
+            gs = {key: (t[:, :, :n] if key == "g" else t[:, :, :n, :]) for key, t in sl.items()}
+
+            def run():
+                O.gated_backward(gs["q"], gs["k"], gs["v"], gs["g"], gs["do"])
+            return run, heads * n / cfg.H
         gam = x["gamma"][torch.arange(heads) % cfg.H]
 
         def run():
@@ -675,7 +697,9 @@ def cpu_baseline(spec, budget_s: float = 12.0, single_budget_s: float = 4.0):
     run, units = _oracle_sample_step(spec, heads)
     reps, el = _time_oracle(run, budget_s)
     value = units * reps / el
-    what = "decode steps" if spec["kind"] == "decode" else f"{cfg.N} tokens"
+    what = ("decode steps" if spec["kind"] == "decode"
+            else f"the first {min(cfg.N, GATED_BWD_SAMPLE_TOKENS)} of {cfg.N} tokens"
+            if spec["kind"] == "backward" and spec.get("gated") else f"{cfg.N} tokens")
     covered = lambda n: (total_heads if spec["kind"] == "norm"  # the epilogue sample is the whole workload
                          else max(1, -(-n // cfg.H)) * cfg.H if spec["kind"] == "decode"  # whole batch rows
                          else n)
@@ -723,7 +747,9 @@ def run_reference(args, spec):
         run()
     el = time.perf_counter() - t0
     value = units * args.steps / el
-    what = "decode steps" if spec["kind"] == "decode" else f"{cfg.N} tokens"
+    what = ("decode steps" if spec["kind"] == "decode"
+            else f"the first {min(cfg.N, GATED_BWD_SAMPLE_TOKENS)} of {cfg.N} tokens"
+            if spec["kind"] == "backward" and spec.get("gated") else f"{cfg.N} tokens")
     if spec["kind"] == "norm":
         heads = cfg.B * cfg.H  # the epilogue sample is the whole workload
     sample = (f"each step: fp64 oracle on {heads} of {cfg.B * cfg.H} (b,h) heads x {what}, "

@@ -197,32 +197,46 @@ decay_grad_kernel(const T* __restrict__ q, const T* __restrict__ dq, const T* __
 }
 
 // In place: dg[bh, t] = sum_{u >= t} a[bh, u] (a suffix sum, since G_u includes g_t for
-// every u >= t). One block per (b, h), tiles of kBwdThreads tokens from the end of the
-// sequence with a running carry.
-__global__ void __launch_bounds__(kBwdThreads) gate_grad_scan_kernel(float* __restrict__ dg, int N) {
-    __shared__ float warp_s[kBwdWarps];
+// every u >= t). One block of kScanThreads per (b, h): each thread owns kScanPer consecutive
+// tokens of a span of kScanThreads * kScanPer (the whole row for N <= 16384), sums them from
+// its last token back, and adds the totals of the later threads (a warp scan, then the warps'
+// totals) and of the later spans (a running carry). All of a span's loads are in flight at once.
+constexpr int kScanThreads = 1024, kScanPer = 16;
+__global__ void __launch_bounds__(kScanThreads) gate_grad_scan_kernel(float* __restrict__ dg, int N) {
+    __shared__ float warp_s[kScanThreads / 32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     float* a = dg + (size_t)blockIdx.x * N;
     float carry = 0.f;
-    for (int tile_end = N; tile_end > 0; tile_end -= kBwdThreads) {
-        const int tile0 = max(0, tile_end - kBwdThreads);
-        const int len = tile_end - tile0;
-        const int j = threadIdx.x;
-        float x = j < len ? a[tile0 + j] : 0.f;
-        // inclusive suffix sum inside the warp
+    for (int end = N; end > 0; end -= kScanThreads * kScanPer) {
+        const int beg = max(0, end - kScanThreads * kScanPer);
+        const int t0 = beg + threadIdx.x * kScanPer;
+        float x[kScanPer];
+#pragma unroll
+        for (int i = 0; i < kScanPer; ++i) x[i] = t0 + i < end ? a[t0 + i] : 0.f;
+        float run = 0.f;  // suffix sums inside the thread's tokens
+#pragma unroll
+        for (int i = kScanPer - 1; i >= 0; --i) {
+            run += x[i];
+            x[i] = run;
+        }
+        // inclusive suffix sum of the threads' totals inside the warp
+        float incl = run;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const float y = __shfl_down_sync(0xffffffffu, x, o);
-            if (lane + o < 32) x += y;
+            const float y = __shfl_down_sync(0xffffffffu, incl, o);
+            if (lane + o < 32) incl += y;
         }
-        if (lane == 0) warp_s[warp] = x;  // the warp's total
+        if (lane == 0) warp_s[warp] = incl;  // the warp's total
         __syncthreads();
         float later = 0.f, total = 0.f;
-        for (int w2 = 0; w2 < kBwdWarps; ++w2) {
+        for (int w2 = 0; w2 < kScanThreads / 32; ++w2) {
             if (w2 > warp) later += warp_s[w2];
             total += warp_s[w2];
         }
-        if (j < len) a[tile0 + j] = x + later + carry;
+        const float after = incl - run + later + carry;  // every token after this thread's own
+#pragma unroll
+        for (int i = 0; i < kScanPer; ++i)
+            if (t0 + i < end) a[t0 + i] = x[i] + after;
         carry += total;
         __syncthreads();
     }

@@ -162,7 +162,7 @@ ret_status decay_grad(const T* q, const T* dq, const T* k, const T* dk, const fl
         decay_grad_kernel<T, false, GATED><<<grid, kBwdThreads, 0, st>>>(q, dq, k, dk, decay, out, H, N, dk_dim);
     ret_status r = launch_status();
     if (GATED && r == RET_OK) {
-        gate_grad_scan_kernel<<<(unsigned)BH, kBwdThreads, 0, st>>>(out, N);
+        gate_grad_scan_kernel<<<(unsigned)BH, kScanThreads, 0, st>>>(out, N);
         r = launch_status();
     }
     return r;
@@ -233,6 +233,7 @@ inline int backward_tc_launches(int B, int H, int N, int dk, int dv, bool gated,
 //   st: zero dq, dk | dQ piece 0 (adds onto dq) | wait s1, s2 -> dgamma/dg
 //   s1: dQ piece 1 (adds onto dq) | dK piece 1 (reversed, adds onto dk)
 //   s2: dK piece 0 (reversed, adds onto dk) | dV (reversed) | wait s1
+// (with one piece: dQ on st, dK on s1, dV on s2, all three side by side)
 // (more pieces alternate between the streams of their row; with one piece the dQ and dK
 // calls store dq and dk directly, with no zeroing). dQ = forward(dO, V, K); dK = reversed
 // forward(V, dO, Q); dV = reversed forward(K, Q, dO), each with the caller's gamma or gates
@@ -276,7 +277,8 @@ ret_status backward_tc(const void* q, const void* k, const void* v, const float*
     // dQ pieces on st and s1, then dK pieces on s2 and s1, dV on s2
     for (int p = 0; p < P && r == RET_OK; ++p) piece(false, dout, v, k, dq, p, p % 2 ? s1 : st);
     if (r == RET_OK) cu(cudaEventRecord(ev_q1, s1));  // s1's dQ pieces
-    for (int p = 0; p < P && r == RET_OK; ++p) piece(true, v, dout, q, dk_out, p, p % 2 ? s1 : s2);
+    // (with one piece s1 holds no dQ piece: dK goes there, so that dQ, dK and dV run side by side)
+    for (int p = 0; p < P && r == RET_OK; ++p) piece(true, v, dout, q, dk_out, p, (P == 1 || p % 2) ? s1 : s2);
     if (r == RET_OK) cu(cudaEventRecord(ev_k1, s1));  // s1's dK pieces
     if (r == RET_OK)
         ok(tc_chunk_launch<GATED, true>(k, q, dout, decay, dv_out, nullptr, nullptr, B, H, N, dk, dv, s2, 0, 0, conc));

@@ -11,7 +11,7 @@ sys.path.insert(0, ROOT)
 import bench  # noqa: E402
 
 WORKLOADS = ["retnet_1p3b", "retnet_6p7b_long", "gated", "decode", "gated_decode", "seqpar_6p7b", "backward_1p3b",
-             "msr_norm_1p3b", "retention_msr_1p3b"]
+             "backward_gated", "msr_norm_1p3b", "retention_msr_1p3b"]
 
 
 def test_backward_and_epilogue_arithmetic():
@@ -21,6 +21,10 @@ def test_backward_and_epilogue_arithmetic():
     assert bw["bytes"] == B * H * N * (dk + dk + dv + dv + dk + dk + dv) * 2
     assert bw["flops"] == 3 * B * H * N * (2 * C * (dk + dv) + 4 * dk * dv)
     assert bw["units"] == B * N and bw["kind"] == "backward"
+    # gated backward (B2 H8 N16384 dk = dv = 128): the same tensors, plus g read and dg written in fp32
+    gb = bench.workload("backward_gated")
+    Bg, Hg, Ng, d = 2, 8, 16384, 128
+    assert gb["bytes"] == Bg * Hg * Ng * 7 * d * 2 + 2 * Bg * Hg * Ng * 4 and gb["gated"] and not bw["gated"]
     nm = bench.workload("msr_norm_1p3b")
     assert nm["bytes"] == 3 * B * H * N * dv * 2  # o and gate in, y out
     rm = bench.workload("retention_msr_1p3b")
