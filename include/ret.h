@@ -164,10 +164,11 @@ RET_API ret_status ret_last_device_error(void* stream);
  * than 256 contracted in pieces) and small kernels of this library; takes
  * stream-ordered scratch (freed on the same stream). On the tensor-core path the
  * pieces are read in place, and the steps that do not depend on each other run
- * side by side on two library-owned streams of the current device, forked from and
- * joined back to `stream` with events: all work stays ordered on `stream` (and can
- * be captured in a graph). Concurrent calls from several host threads serialise
- * while they enqueue.
+ * side by side on five library-owned streams of the current device (four of the
+ * device's greatest priority for the dq and dk pieces, one of its least for dv),
+ * forked from and joined back to `stream` with events: all work stays ordered on
+ * `stream` (and can be captured in a graph). Concurrent calls from several host
+ * threads serialise while they enqueue.
  * bf16 needs 16-byte aligned tensors. Requires dk <= 256.
  */
 RET_API ret_status ret_chunkwise_backward(const void* q, const void* k, const void* v, const float* gamma,

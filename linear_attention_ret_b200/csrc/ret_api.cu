@@ -170,12 +170,14 @@ ret_status decay_grad(const T* q, const T* dq, const T* k, const T* dk, const fl
 
 inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
-// Two library streams per device, with events, for the steps of the backward that run side
-// by side. Held under the mutex from the first fork to the last join, so calls from several
-// host threads do not interleave their events.
-constexpr int kAuxEvents = 7;
+// Library streams per device, with events, for the steps of the backward that run side by
+// side: kAuxHi streams of the device's greatest priority for the passes that the decay
+// gradient waits for, and one of the least priority for the pass that it does not wait for.
+// Held under the mutex from the first fork to the last join, so calls from several host
+// threads do not interleave their events.
+constexpr int kAuxHi = 4, kAuxStreams = kAuxHi + 1, kAuxEvents = kAuxStreams + 1;
 struct AuxStreams {
-    cudaStream_t s[2] = {nullptr, nullptr};
+    cudaStream_t s[kAuxStreams] = {};
     cudaEvent_t ev[kAuxEvents] = {};
 };
 constexpr int kMaxDevices = 64;
@@ -197,7 +199,11 @@ inline AuxStreams* aux_streams() {
     if (!a.s[0]) {  // publish only once every stream and event exists
         AuxStreams n;
         bool ok = true;
-        for (cudaStream_t& x : n.s) ok = ok && cudaStreamCreateWithFlags(&x, cudaStreamNonBlocking) == cudaSuccess;
+        int least = 0, greatest = 0;
+        ok = cudaDeviceGetStreamPriorityRange(&least, &greatest) == cudaSuccess;
+        for (int i = 0; i < kAuxStreams; ++i)
+            ok = ok && cudaStreamCreateWithPriority(&n.s[i], cudaStreamNonBlocking, i < kAuxHi ? greatest : least) ==
+                           cudaSuccess;
         for (cudaEvent_t& e : n.ev) ok = ok && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
         if (!ok) {
             destroy_aux(n);
@@ -228,16 +234,18 @@ inline int backward_tc_launches(int B, int H, int N, int dk, int dv, bool gated,
     return n;
 }
 
-// The backward on the tensor-core path as a small graph of steps on the caller's stream st
-// and two library streams s1, s2:
-//   st: zero dq, dk | dQ piece 0 (adds onto dq) | wait s1, s2 -> dgamma/dg
-//   s1: dQ piece 1 (adds onto dq) | dK piece 1 (reversed, adds onto dk)
-//   s2: dK piece 0 (reversed, adds onto dk) | dV (reversed) | wait s1
-// (with one piece: dQ on st, dK on s1, dV on s2, all three side by side)
-// (more pieces alternate between the streams of their row; with one piece the dQ and dK
-// calls store dq and dk directly, with no zeroing). dQ = forward(dO, V, K); dK = reversed
-// forward(V, dO, Q); dV = reversed forward(K, Q, dO), each with the caller's gamma or gates
-// as they are.
+// The backward on the tensor-core path as a small graph of steps. Library streams h0..h3 (the
+// greatest priority) take the passes that the decay gradient needs, the low-priority stream
+// lo takes dV, which nothing in the call waits for:
+//   st: zero dq, dk | fork | wait h0..h3 -> dgamma/dg | wait lo
+//   h0, h1: dQ pieces 0, 1 (adding onto dq; more pieces alternate between the two)
+//   h2, h3: dK pieces 0, 1 (reversed, adding onto dk)
+//   lo:     dV (reversed)
+// All passes start together and the block scheduler serves the high-priority passes first, so
+// dV fills the SMs that they leave free and the decay gradient runs beside the end of dV. With
+// one piece the dQ and dK calls store dq and dk directly, with no zeroing. dQ = forward(dO, V,
+// K); dK = reversed forward(V, dO, Q); dV = reversed forward(K, Q, dO), each with the caller's
+// gamma or gates as they are.
 template <typename T, bool GATED>
 ret_status backward_tc(const void* q, const void* k, const void* v, const float* decay, const void* dout,
                        void* dq, void* dk_out, void* dv_out, float* ddecay, int B, int H, int N, int dk, int dv,
@@ -250,9 +258,10 @@ ret_status backward_tc(const void* q, const void* k, const void* v, const float*
     std::lock_guard<std::mutex> lock(aux_mutex());
     AuxStreams* a = aux_streams();
     if (!a) return RET_ERR_CUDA;
-    cudaStream_t s1 = a->s[0], s2 = a->s[1];
-    cudaEvent_t ev_fork = a->ev[0], ev_q1 = a->ev[1], ev_k1 = a->ev[2], ev_k = a->ev[3], ev_j1 = a->ev[4],
-                ev_j2 = a->ev[5];
+    cudaStream_t* hi = a->s;
+    cudaStream_t lo = a->s[kAuxHi];
+    cudaEvent_t ev_fork = a->ev[0];
+    cudaEvent_t* ev_done = a->ev + 1;  // one per library stream, after its last step
     // With several pieces, dq and dk start at zero and every piece adds its output tiles onto
     // them (in L2, in bf16, rounded once per addition): with two pieces each element is
     // round(a + b), whatever order the pieces' additions take.
@@ -270,31 +279,25 @@ ret_status backward_tc(const void* q, const void* k, const void* v, const float*
                       : tc_chunk_launch<GATED, false>(xp, yp, z, decay, out, nullptr, nullptr, B, H, N, w, dk, s, dv,
                                                       dv, conc, P > 1));
     };
-    if (r == RET_OK && cu(cudaEventRecord(ev_fork, st))) {
-        cu(cudaStreamWaitEvent(s1, ev_fork, 0));
-        cu(cudaStreamWaitEvent(s2, ev_fork, 0));
-    }
-    // dQ pieces on st and s1, then dK pieces on s2 and s1, dV on s2
-    for (int p = 0; p < P && r == RET_OK; ++p) piece(false, dout, v, k, dq, p, p % 2 ? s1 : st);
-    if (r == RET_OK) cu(cudaEventRecord(ev_q1, s1));  // s1's dQ pieces
-    // (with one piece s1 holds no dQ piece: dK goes there, so that dQ, dK and dV run side by side)
-    for (int p = 0; p < P && r == RET_OK; ++p) piece(true, v, dout, q, dk_out, p, (P == 1 || p % 2) ? s1 : s2);
-    if (r == RET_OK) cu(cudaEventRecord(ev_k1, s1));  // s1's dK pieces
+    if (r == RET_OK && cu(cudaEventRecord(ev_fork, st)))
+        for (int i = 0; i < kAuxStreams && r == RET_OK; ++i) cu(cudaStreamWaitEvent(a->s[i], ev_fork, 0));
+    // issue order: dQ pieces, dK pieces, then dV
+    for (int p = 0; p < P && r == RET_OK; ++p) piece(false, dout, v, k, dq, p, hi[p % 2]);
+    for (int p = 0; p < P && r == RET_OK; ++p) piece(true, v, dout, q, dk_out, p, hi[2 + p % 2]);
     if (r == RET_OK)
-        ok(tc_chunk_launch<GATED, true>(k, q, dout, decay, dv_out, nullptr, nullptr, B, H, N, dk, dv, s2, 0, 0, conc));
-    // decay gradient on st once dq (st, s1) and dk (s2, s1) are complete
-    if (r == RET_OK && ddecay && cu(cudaStreamWaitEvent(s2, ev_k1, 0)) && cu(cudaEventRecord(ev_k, s2)) &&
-        cu(cudaStreamWaitEvent(st, ev_q1, 0)) && cu(cudaStreamWaitEvent(st, ev_k, 0)))
+        ok(tc_chunk_launch<GATED, true>(k, q, dout, decay, dv_out, nullptr, nullptr, B, H, N, dk, dv, lo, 0, 0, conc));
+    // join every library stream back into st whatever happened: the high-priority ones before
+    // the decay gradient (it reads dq and dk), lo after it
+    bool joined = true;
+    for (int i = 0; i < kAuxStreams; ++i) joined = joined && cudaEventRecord(ev_done[i], a->s[i]) == cudaSuccess;
+    for (int i = 0; i < kAuxHi; ++i) joined = joined && cudaStreamWaitEvent(st, ev_done[i], 0) == cudaSuccess;
+    if (r == RET_OK && joined && ddecay)
         ok(decay_grad<T, GATED>(static_cast<const T*>(q), static_cast<const T*>(dq), static_cast<const T*>(k),
                                 static_cast<const T*>(dk_out), decay, ddecay, B * H, H, N, dk, st));
-    // join both library streams back into st whatever happened
-    const bool joined = cudaEventRecord(ev_j1, s1) == cudaSuccess && cudaEventRecord(ev_j2, s2) == cudaSuccess &&
-                        cudaStreamWaitEvent(st, ev_j1, 0) == cudaSuccess &&
-                        cudaStreamWaitEvent(st, ev_j2, 0) == cudaSuccess;
+    joined = joined && cudaStreamWaitEvent(st, ev_done[kAuxHi], 0) == cudaSuccess;
     if (!joined) {
         // the library streams could not be ordered before st: wait for them
-        cudaStreamSynchronize(s1);
-        cudaStreamSynchronize(s2);
+        for (int i = 0; i < kAuxStreams; ++i) cudaStreamSynchronize(a->s[i]);
         ok(RET_ERR_CUDA);
     }
     return r;

@@ -615,7 +615,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (!STATE_ONLY) {
         const int te = threadIdx.x - 64;          // 0..127
         const int quarter = warp & 3;             // TMEM lane quarter this warp may access
-        const int d = quarter * 32 + lane;        // dv column of the slice = TMEM lane
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         float* cum = reinterpret_cast<float*>(sm + Lay::kAgTab);  // gated: in-chunk cumsum (log2 units), per buffer
         float* rr = cum + 2 * kC;  // row factor of the drain, per buffer: r_j (split), 1 / zeta'_j (merged)
