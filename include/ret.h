@@ -19,8 +19,9 @@
  *        RMSNorm over the head dimension; g_proj feeding a swish gate).
  *
  * Conventions shared by every entry point
- *   - Pointers are DEVICE pointers owned by the caller. The library never frees
- *     caller memory and keeps no pointer after the call returns.
+ *   - Pointers are DEVICE pointers owned by the caller, except in the *_host
+ *     calls, whose tensors are in host memory. The library never frees caller
+ *     memory and keeps no pointer after the call returns.
  *   - Tensors are contiguous row-major, heads leading:
  *       q, k [B, H, N, dk]   v, o [B, H, N, dv]   state [B, H, dk, dv] (fp32)
  *       gamma [H] (fp32)     g [B, H, N] (fp32, natural-log decay, normally <= 0)
@@ -35,8 +36,9 @@
  *     outputs are then undefined.
  *   - Errors are returned, never raised: no exit(), no device trap.
  *   - Calls keep no per-call state (the library holds only per-device helpers
- *     it creates once: the no-allocation scratch buffer, and two streams with
- *     their events for the backward) and are safe from several host threads,
+ *     it creates once: the no-allocation scratch buffer, and five streams with
+ *     their events for the backward and the *_host calls) and are safe from
+ *     several host threads,
  *     except ret_chunkwise_noalloc, whose calls all share one scratch buffer:
  *     calls of it that overlap on the GPU race (see its declaration).
  *   - N == 0 is a valid empty problem: nothing is launched, state_out (if
@@ -138,6 +140,31 @@ RET_API ret_status gated_ret_chunkwise(const void* q, const void* k, const void*
                                void* o, const float* state_in, float* state_out,
                                int B, int H, int N, int dk, int dv, int chunk,
                                ret_dtype dt, void* stream);
+
+/*
+ * ret_chunkwise / gated_ret_chunkwise from HOST memory: q, k, v, gamma (or g) and
+ * o are host pointers with the layouts above; no initial or final state. The
+ * call copies the inputs to stream-ordered device buffers, computes and copies o
+ * back, pipelined over groups of heads (at most 8: whole batches when B >= 8,
+ * else runs of heads inside one batch): the copies in of later groups overlap
+ * the forward and the copy out of earlier ones, on `stream` and two library
+ * streams forked from it and joined back. It returns once everything is
+ * enqueued: o is complete when `stream` is. Host buffers should be page-locked
+ * (cudaHostAlloc, cudaHostRegister); pageable buffers still give the right
+ * result, but the driver then stages each copy and nothing overlaps. Each
+ * group's result is that of ret_chunkwise on the group alone: heads are
+ * independent, but the group's plan (the sequence segments that fill the SMs)
+ * can differ from the whole batch's, and with it the rounding. Limits and paths as
+ * ret_chunkwise; the device buffers are freed on `stream` before the call
+ * returns. Not in the pages: the host side of serving a layer whose activations
+ * live in host memory.
+ */
+RET_API ret_status ret_chunkwise_host(const void* q, const void* k, const void* v, const float* gamma,
+                              void* o, int B, int H, int N, int dk, int dv, int chunk,
+                              ret_dtype dt, void* stream);
+RET_API ret_status gated_ret_chunkwise_host(const void* q, const void* k, const void* v, const float* g,
+                                    void* o, int B, int H, int N, int dk, int dv, int chunk,
+                                    ret_dtype dt, void* stream);
 
 /* Static description of a status code. Never NULL. */
 RET_API const char* ret_status_str(ret_status s);

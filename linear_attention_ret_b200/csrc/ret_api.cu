@@ -155,8 +155,32 @@ template <typename T, bool GATED>
 ret_status decay_grad(const T* q, const T* dq, const T* k, const T* dk, const float* decay, float* out, int BH, int H,
                       int N, int dk_dim, cudaStream_t st) {
     if (!GATED && cudaMemsetAsync(out, 0, sizeof(float) * (size_t)H, st) != cudaSuccess) return RET_ERR_CUDA;
-    const dim3 grid((unsigned)((N + kGradTokens - 1) / kGradTokens), (unsigned)BH);
-    if (whole_chunks(dk_dim, sizeof(T)) && aligned16(q) && aligned16(dq) && aligned16(k) && aligned16(dk))
+    const int ntiles = (N + kGradTokens - 1) / kGradTokens;
+    const dim3 grid((unsigned)ntiles, (unsigned)BH);
+    const bool vec = whole_chunks(dk_dim, sizeof(T)) && aligned16(q) && aligned16(dq) && aligned16(k) && aligned16(dk);
+    const int C = vec ? dk_dim / RowIo<T, true>::kE : 0;  // 16-byte chunks per row
+    int lc = 0;
+    while ((1 << lc) < C) ++lc;
+    if (vec && C == (1 << lc) && C <= 32) {
+        // all of a tile's loads in flight; gated: in-tile suffix sums and tile totals, then
+        // the later tiles' totals added by a second, fully parallel kernel
+        float* tot = nullptr;
+        if (GATED && cudaMallocAsync(reinterpret_cast<void**>(&tot), sizeof(float) * (size_t)BH * ntiles, st) !=
+                         cudaSuccess)
+            return RET_ERR_CUDA;
+        decay_grad_flat_kernel<T, GATED><<<grid, kBwdThreads, 0, st>>>(q, dq, k, dk, decay, out, tot, H, N, lc);
+        ret_status r = launch_status();
+        if (GATED) {
+            if (r == RET_OK) {
+                const dim3 g2((unsigned)((ntiles + kCarryTiles - 1) / kCarryTiles), (unsigned)BH);
+                gate_grad_carry_kernel<<<g2, kBwdThreads, 0, st>>>(out, tot, N, ntiles);
+                r = launch_status();
+            }
+            if (cudaFreeAsync(tot, st) != cudaSuccess && r == RET_OK) r = RET_ERR_CUDA;
+        }
+        return r;
+    }
+    if (vec)
         decay_grad_kernel<T, true, GATED><<<grid, kBwdThreads, 0, st>>>(q, dq, k, dk, decay, out, H, N, dk_dim);
     else
         decay_grad_kernel<T, false, GATED><<<grid, kBwdThreads, 0, st>>>(q, dq, k, dk, decay, out, H, N, dk_dim);
@@ -175,7 +199,10 @@ inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 // gradient waits for, and one of the least priority for the pass that it does not wait for.
 // Held under the mutex from the first fork to the last join, so calls from several host
 // threads do not interleave their events.
-constexpr int kAuxHi = 4, kAuxStreams = kAuxHi + 1, kAuxEvents = kAuxStreams + 1;
+// The host-buffer forward (chunkwise_host_entry) uses the first two streams and events for
+// its fork, its groups and its joins.
+constexpr int kAuxHi = 4, kAuxStreams = kAuxHi + 1, kPipeGroups = 8;
+constexpr int kAuxEvents = std::max(kAuxStreams + 1, 3 + 2 * kPipeGroups);
 struct AuxStreams {
     cudaStream_t s[kAuxStreams] = {};
     cudaEvent_t ev[kAuxEvents] = {};
@@ -486,6 +513,108 @@ ret_status launch_step(const void* q, const void* k, const void* v, const float*
     return launch_status();
 }
 
+// The chunkwise forward from host buffers: q, k, v, the decay and o live in host memory.
+// The heads are cut into at most kPipeGroups groups (whole batches when B >= kPipeGroups,
+// else runs of heads inside one batch, so each group is one (B', H') problem with its own
+// slice of the decay) and pipelined over three streams:
+//   st:  fork | H2D of group 0 | H2D of group 1 | ...            | wait cs, os | free
+//   cs:        wait H2D g -> chunkwise forward of group g -> ...
+//   os:                      wait forward g -> D2H of group g's o -> ...
+// so the copies in (the larger part) run back to back while earlier groups compute and copy
+// out in the other direction. Device buffers come from the stream-ordered pool.
+template <bool GATED>
+ret_status chunkwise_host_entry(const void* q, const void* k, const void* v, const float* decay, void* o, int B,
+                                int H, int N, int dk, int dv, int chunk, ret_dtype dt, void* stream) {
+    ret_status s = check_common(B, H, N, dk, dv, dt);
+    if (s != RET_OK) return s;
+    if (chunk <= 0) return RET_ERR_SHAPE;
+    if (dk > 256) return RET_ERR_UNSUPPORTED;
+    if (N == 0) return RET_OK;
+    if (!q || !k || !v || !decay || !o) return RET_ERR_NULL;
+    cudaStream_t st = as_stream(stream);
+    const size_t es = dt == RET_F32 ? 4 : 2;
+    const size_t head_q = (size_t)N * dk * es, head_v = (size_t)N * dv * es, head_g = (size_t)N * sizeof(float);
+    const size_t BH = (size_t)B * H;
+    const size_t sz[5] = {BH * head_q, BH * head_q, BH * head_v, BH * head_v,
+                          GATED ? BH * head_g : (size_t)H * sizeof(float)};
+    size_t off[5], bytes = 0;
+    for (int i = 0; i < 5; ++i) {
+        off[i] = bytes;
+        bytes += align256(sz[i]);
+    }
+    // groups: (first batch, batches, first head, heads)
+    struct Group { int b0, nb, h0, nh; };
+    Group grp[kPipeGroups];
+    int G = 0;
+    if (B >= kPipeGroups) {
+        const int bpg = (B + kPipeGroups - 1) / kPipeGroups;
+        for (int b0 = 0; b0 < B; b0 += bpg) grp[G++] = {b0, std::min(bpg, B - b0), 0, H};
+    } else {
+        const int per_batch = kPipeGroups / B, hpg = (H + per_batch - 1) / per_batch;
+        for (int b = 0; b < B; ++b)
+            for (int h0 = 0; h0 < H; h0 += hpg) grp[G++] = {b, 1, h0, std::min(hpg, H - h0)};
+    }
+    std::lock_guard<std::mutex> lock(aux_mutex());
+    AuxStreams* a = aux_streams();
+    if (!a) return RET_ERR_CUDA;
+    cudaStream_t cs = a->s[0], os = a->s[1];
+    cudaEvent_t ev_fork = a->ev[0], ev_cs = a->ev[1], ev_os = a->ev[2];
+    cudaEvent_t* ev_in = a->ev + 3;                 // [kPipeGroups]: group g's inputs are on the device
+    cudaEvent_t* ev_out = a->ev + 3 + kPipeGroups;  // [kPipeGroups]: group g's o is computed
+    tc::keep_pool_memory();
+    uint8_t* buf = nullptr;
+    if (cudaMallocAsync(reinterpret_cast<void**>(&buf), bytes, st) != cudaSuccess) return RET_ERR_CUDA;
+    uint8_t* dq = buf + off[0];
+    uint8_t* dk_ = buf + off[1];
+    uint8_t* dv_ = buf + off[2];
+    uint8_t* do_ = buf + off[3];
+    float* ddec = reinterpret_cast<float*>(buf + off[4]);
+    const uint8_t* hq = static_cast<const uint8_t*>(q);
+    const uint8_t* hk = static_cast<const uint8_t*>(k);
+    const uint8_t* hv = static_cast<const uint8_t*>(v);
+    uint8_t* ho = static_cast<uint8_t*>(o);
+    ret_status r = RET_OK;
+    auto cu = [&](cudaError_t e) {
+        if (r == RET_OK && e != cudaSuccess) r = RET_ERR_CUDA;
+        return r == RET_OK;
+    };
+    auto h2d = [&](void* d, const void* h, size_t n) { return cu(cudaMemcpyAsync(d, h, n, cudaMemcpyHostToDevice, st)); };
+    if (!GATED) h2d(ddec, decay, sz[4]);
+    if (cu(cudaEventRecord(ev_fork, st))) {
+        cu(cudaStreamWaitEvent(cs, ev_fork, 0));
+        cu(cudaStreamWaitEvent(os, ev_fork, 0));
+    }
+    for (int gi = 0; gi < G && r == RET_OK; ++gi) {
+        const Group& g = grp[gi];
+        const size_t first = (size_t)g.b0 * H + g.h0, heads = (size_t)g.nb * g.nh;
+        h2d(dq + first * head_q, hq + first * head_q, heads * head_q);
+        h2d(dk_ + first * head_q, hk + first * head_q, heads * head_q);
+        h2d(dv_ + first * head_v, hv + first * head_v, heads * head_v);
+        if (GATED)
+            h2d(reinterpret_cast<uint8_t*>(ddec) + first * head_g, reinterpret_cast<const uint8_t*>(decay) +
+                first * head_g, heads * head_g);
+        if (!cu(cudaEventRecord(ev_in[gi], st)) || !cu(cudaStreamWaitEvent(cs, ev_in[gi], 0))) break;
+        const float* gdec = GATED ? ddec + first * N : ddec + g.h0;
+        const ret_status rc = chunkwise_entry<GATED>(dq + first * head_q, dk_ + first * head_q, dv_ + first * head_v,
+                                                     gdec, do_ + first * head_v, nullptr, nullptr, g.nb, g.nh, N, dk,
+                                                     dv, chunk, dt, cs);
+        if (rc != RET_OK && r == RET_OK) r = rc;
+        if (!cu(cudaEventRecord(ev_out[gi], cs)) || !cu(cudaStreamWaitEvent(os, ev_out[gi], 0))) break;
+        cu(cudaMemcpyAsync(ho + first * head_v, do_ + first * head_v, heads * head_v, cudaMemcpyDeviceToHost, os));
+    }
+    // join both library streams back into st whatever happened, then release the buffers
+    const bool joined = cudaEventRecord(ev_cs, cs) == cudaSuccess && cudaEventRecord(ev_os, os) == cudaSuccess &&
+                        cudaStreamWaitEvent(st, ev_cs, 0) == cudaSuccess &&
+                        cudaStreamWaitEvent(st, ev_os, 0) == cudaSuccess;
+    if (!joined) {
+        cudaStreamSynchronize(cs);
+        cudaStreamSynchronize(os);
+        if (r == RET_OK) r = RET_ERR_CUDA;
+    }
+    if (cudaFreeAsync(buf, st) != cudaSuccess && r == RET_OK) r = RET_ERR_CUDA;
+    return r;
+}
+
 }  // namespace
 
 extern "C" {
@@ -512,6 +641,16 @@ ret_status gated_ret_chunkwise(const void* q, const void* k, const void* v, cons
                                const float* state_in, float* state_out, int B, int H, int N, int dk, int dv,
                                int chunk, ret_dtype dt, void* stream) {
     return chunkwise_entry<true>(q, k, v, g, o, state_in, state_out, B, H, N, dk, dv, chunk, dt, stream);
+}
+
+ret_status ret_chunkwise_host(const void* q, const void* k, const void* v, const float* gamma, void* o, int B, int H,
+                              int N, int dk, int dv, int chunk, ret_dtype dt, void* stream) {
+    return chunkwise_host_entry<false>(q, k, v, gamma, o, B, H, N, dk, dv, chunk, dt, stream);
+}
+
+ret_status gated_ret_chunkwise_host(const void* q, const void* k, const void* v, const float* g, void* o, int B,
+                                    int H, int N, int dk, int dv, int chunk, ret_dtype dt, void* stream) {
+    return chunkwise_host_entry<true>(q, k, v, g, o, B, H, N, dk, dv, chunk, dt, stream);
 }
 
 ret_status ret_recurrent_step(const void* q, const void* k, const void* v, const float* gamma, float* state,

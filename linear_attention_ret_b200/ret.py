@@ -30,7 +30,8 @@ SYMBOLS = ("ret_parallel", "ret_chunkwise", "ret_recurrent_step", "gated_ret_chu
            "ret_chunkwise_noalloc", "ret_selftest_wait_timeout", "gated_ret_recurrent_step",
            "ret_chunkwise_state", "gated_ret_chunkwise_state", "ret_state_prefix", "ret_chunkwise_state_launches",
            "ret_chunkwise_backward", "gated_ret_chunkwise_backward", "ret_chunkwise_backward_launches",
-           "ret_msr_norm_gate", "ret_chunkwise_noalloc_scratch_bytes")
+           "ret_msr_norm_gate", "ret_chunkwise_noalloc_scratch_bytes", "ret_chunkwise_host",
+           "gated_ret_chunkwise_host")
 
 _lock = threading.Lock()
 _lib = None
@@ -67,6 +68,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
         lib.ret_state_prefix.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
         lib.ret_chunkwise_state_launches.argtypes = [_i, _i, _i, _i, _i, _i, _i]
         lib.ret_chunkwise_backward_launches.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i, _i]
+        for fn in ("ret_chunkwise_host", "gated_ret_chunkwise_host"):
+            getattr(lib, fn).argtypes = [_vp] * 5 + [_i] * 7 + [_vp]
+            getattr(lib, fn).restype = _i
         lib.ret_msr_norm_gate.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, ctypes.c_float, _i, _vp]
         lib.ret_msr_norm_gate.restype = _i
         for fn in ("ret_chunkwise_backward", "gated_ret_chunkwise_backward"):
@@ -128,6 +132,12 @@ def _cuda(*ts):
             dev = t.device
         elif t.device != dev:
             raise ValueError(f"tensors must be on one device, got {dev} and {t.device}")
+
+
+def _host(*ts):
+    for t in ts:
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous host (CPU) tensors")
 
 
 def _expect(name, t, shape, dtype=None):
@@ -218,6 +228,31 @@ def gated_ret_chunkwise(q, k, v, g, chunk, state_in=None, state_out=None, o=None
                                                              _ptr(state_in), _ptr(state_out), B, H, N, dk, dv,
                                                              int(chunk), _dt(q), _stream(stream)))
     return o
+
+
+def _chunkwise_host(name, q, k, v, decay, chunk, o, gated, stream, sync):
+    B, H, N, dk, dv = _seq_args(q, k, v, decay, gated, o)
+    if o is None:
+        o = torch.empty(B, H, N, dv, dtype=q.dtype, pin_memory=q.is_pinned())
+    _host(q, k, v, decay, o)
+    s = torch.cuda.current_stream() if stream is None else stream
+    _check(name, getattr(load(), name)(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(o), B, H, N, dk, dv,
+                                       int(chunk), _dt(q), ctypes.c_void_p(s.cuda_stream)))
+    if sync:
+        s.synchronize()
+    return o
+
+
+def ret_chunkwise_host(q, k, v, gamma, chunk, o=None, stream=None, sync=True):
+    """ret_chunkwise on host (CPU) tensors, pinned for copy/compute overlap: the library copies
+    the inputs in, computes and copies o back, pipelined over groups of heads, on the current
+    CUDA device. Returns o once the stream has completed (sync=False: once enqueued)."""
+    return _chunkwise_host("ret_chunkwise_host", q, k, v, gamma, chunk, o, False, stream, sync)
+
+
+def gated_ret_chunkwise_host(q, k, v, g, chunk, o=None, stream=None, sync=True):
+    """gated_ret_chunkwise on host (CPU) tensors; as ret_chunkwise_host."""
+    return _chunkwise_host("gated_ret_chunkwise_host", q, k, v, g, chunk, o, True, stream, sync)
 
 
 def ret_recurrent_step(q, k, v, gamma, state, o=None, stream=None):

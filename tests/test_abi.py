@@ -67,6 +67,19 @@ def test_chunkwise_validation(lib, fn):
     assert _call_chunkwise(lib, fn) == 1  # NULL q, k, v
 
 
+@pytest.mark.parametrize("fn", ["ret_chunkwise_host", "gated_ret_chunkwise_host"])
+def test_host_chunkwise_validation(lib, fn):
+    def call(B=1, H=1, N=8, dk=64, dv=64, chunk=64, dt=1):
+        return getattr(lib, fn)(*([None] * 5), B, H, N, dk, dv, chunk, dt, None)
+    assert call(B=0) == 2
+    assert call(N=-1) == 2
+    assert call(chunk=0) == 2
+    assert call(dt=5) == 3
+    assert call(dk=300) == 4
+    assert call(N=0) == 0   # empty: nothing copied, nothing launched
+    assert call() == 1      # NULL tensors
+
+
 def test_parallel_and_step_validation(lib):
     assert lib.ret_parallel(None, None, None, None, None, 1, 1, 4, 2000, 8, 0, None) == 4
     assert lib.ret_parallel(None, None, None, None, None, 1, 1, 4, 8, 8, 0, None) == 1
@@ -128,6 +141,19 @@ def test_bindings_refuse_host_tensors(lib):
         ret.msr_norm_gate(q, torch.zeros(1, 4, 1, 8))
     with pytest.raises(ValueError):
         ret.ret_chunkwise(q, q, q, torch.ones(1), 64)
+
+
+def test_host_bindings_check_shapes_before_the_library(lib):
+    """The host-buffer calls check shapes and dtypes before any pointer reaches the library."""
+    import torch
+    from linear_attention_ret_b200 import ret
+    q = torch.zeros(1, 2, 4, 8, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        ret.ret_chunkwise_host(q, q, q, torch.ones(3), 64)               # gamma [H] with H = 2
+    with pytest.raises(ValueError):
+        ret.gated_ret_chunkwise_host(q, q, q, torch.ones(1, 2, 5), 64)   # g [B, H, N]
+    with pytest.raises(ValueError):
+        ret.ret_chunkwise_host(q, q.float(), q, torch.ones(2), 64)       # k's dtype
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):

@@ -22,6 +22,7 @@ BWD_CASES = [
     (2, 1, 64, 64, 128, torch.bfloat16),
     (1, 2, 130, 64, 512, torch.bfloat16),   # dv pieces copied out (value width 64 is off the tensor-core path)
     (1, 1, 70, 32, 300, torch.float32),     # fp32 pieces of 256 and a ragged 44
+    (1, 2, 90, 48, 40, torch.float32),      # rows of 12 16-byte chunks: the decay gradient's per-warp form
 ]
 
 

@@ -1,0 +1,79 @@
+"""The host-buffer forward (ret_chunkwise_host, gated_ret_chunkwise_host): inputs and output in
+host memory, copies pipelined with the forward over groups of heads. Each group is computed as
+a problem of its own, whose plan (sequence segments to fill the SMs) may differ from the whole
+batch's, so the result is checked against the fp64 oracle, like every forward, and against the
+device-buffer call to the same tolerance; repeated calls agree bit for bit."""
+import pytest
+import torch
+
+from linear_attention_ret_b200 import inputs as I
+from linear_attention_ret_b200 import ret
+from oracle import oracle as O
+from tests.parity import TOL_BF16, TOL_F32, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+CASES = [
+    # B, H, N, dk, dv, chunk, dtype
+    (4, 8, 512, 256, 512, 64, torch.bfloat16),   # 8 groups of 4 heads inside one batch each
+    (1, 3, 300, 64, 128, 64, torch.bfloat16),    # 3 heads, one group each, ragged tail
+    (3, 5, 200, 128, 256, 64, torch.bfloat16),   # 2 groups per batch, of 3 and 2 heads
+    (9, 2, 130, 64, 128, 64, torch.bfloat16),    # B >= 8: groups of whole batches (2, 2, 2, 2, 1)
+    (2, 2, 100, 32, 48, 32, torch.float32),      # CUDA-core path
+]
+
+
+def _device_reference(q, k, v, decay, chunk, gated):
+    qd, kd, vd, dd = (t.to(DEV) for t in (q, k, v, decay))
+    o = ret.gated_ret_chunkwise(qd, kd, vd, dd, chunk) if gated else ret.ret_chunkwise(qd, kd, vd, dd, chunk)
+    return o.cpu()
+
+
+@pytest.mark.parametrize("gated", [False, True])
+@pytest.mark.parametrize("B,H,N,dk,dv,chunk,dtype", CASES)
+def test_host_call_matches_oracle(cuda_lib, B, H, N, dk, dv, chunk, dtype, gated):
+    gen = torch.Generator().manual_seed(B * 100 + H * 10 + N)
+    q, k, v = (t.pin_memory() for t in I.qkv(B, H, N, dk, dv, dtype, gen=gen))
+    decay = (I.gate(B, H, N, gen) if gated else I.gammas(H)).pin_memory()
+    f = ret.gated_ret_chunkwise_host if gated else ret.ret_chunkwise_host
+    o = f(q, k, v, decay, chunk)
+    assert ret.last_device_error() == 0
+    assert not o.is_cuda and o.shape == (B, H, N, dv)
+    tol = TOL_F32 if dtype == torch.float32 else TOL_BF16
+    want = (O.gated_chunkwise if gated else O.ret_chunkwise)(q, k, v, decay, chunk)[0]
+    err = rel_l2(o, want)
+    assert err <= tol, f"against the oracle: rel-L2 {err:.3e} > {tol:.0e}"
+    err = rel_l2(o, _device_reference(q, k, v, decay, chunk, gated).double())
+    assert err <= tol, f"against the device-buffer call: rel-L2 {err:.3e} > {tol:.0e}"
+    assert torch.equal(f(q, k, v, decay, chunk), o)   # the same plan every call
+
+
+def test_host_call_with_pageable_buffers_and_preallocated_output(cuda_lib):
+    B, H, N, dk, dv = 2, 8, 640, 128, 128
+    gen = torch.Generator().manual_seed(12)
+    q, k, v = I.qkv(B, H, N, dk, dv, torch.bfloat16, gen=gen)     # not page-locked
+    g = I.gate(B, H, N, gen)
+    o = torch.full((B, H, N, dv), float("nan"), dtype=torch.bfloat16)
+    out = ret.gated_ret_chunkwise_host(q, k, v, g, 64, o=o)
+    assert out is o
+    assert torch.equal(o, ret.gated_ret_chunkwise_host(q.pin_memory(), k.pin_memory(), v.pin_memory(),
+                                                       g.pin_memory(), 64))
+    err = rel_l2(o, O.gated_chunkwise(q, k, v, g, 64)[0])
+    assert err <= TOL_BF16, f"rel-L2 {err:.3e}"
+
+
+def test_host_call_back_to_back_on_a_side_stream(cuda_lib):
+    """Calls enqueued without waiting, on a stream other than the default: each result is
+    complete once the stream is."""
+    B, H, N, dk, dv = 4, 8, 512, 256, 512
+    gam = I.gammas(H)
+    ins = [tuple(t.pin_memory() for t in I.qkv(B, H, N, dk, dv, torch.bfloat16, seed=20 + i)) for i in range(3)]
+    outs = [torch.empty(B, H, N, dv, dtype=torch.bfloat16).pin_memory() for _ in ins]
+    s = torch.cuda.Stream()
+    for (q, k, v), o in zip(ins, outs):
+        ret.ret_chunkwise_host(q, k, v, gam, 64, o=o, stream=s, sync=False)
+    s.synchronize()
+    for (q, k, v), o in zip(ins, outs):
+        assert torch.equal(o, ret.ret_chunkwise_host(q, k, v, gam, 64))
