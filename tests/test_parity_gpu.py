@@ -375,6 +375,9 @@ SPLIT_CASES = [
     (1, 2, 1000, 64, 128),
     (1, 1, 2053, 128, 128),
     (2, 1, 777, 256, 256),
+    # dv of several 128-column slices, dk 64 and 128
+    (1, 1, 1500, 64, 256),
+    (1, 2, 1100, 128, 512),
 ]
 
 
