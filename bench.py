@@ -554,20 +554,16 @@ def run_e2e(args, spec, dev, stream, world):
                 ret.msr_norm_gate(o, xd["gate"], NORM_EPS, y=y)
             y_host.copy_(y, non_blocking=True)
     elif spec["kind"] == "backward":
+        # the host-buffer backward: inputs in and gradients out, pipelined over groups of heads
         xh = {k: t.pin_memory() for k, t in I.config_inputs(cfg, seed=rank_seed(rank)).items()}
         xh["do"] = I.output_grad(cfg.B, cfg.H, cfg.N, cfg.dv, cfg.dtype, seed=rank_seed(rank)).pin_memory()
-        xd = {k: torch.empty_like(t, device=dev) for k, t in xh.items()}
-        outs_h = [torch.empty(xh[n].shape, dtype=cfg.dtype).pin_memory() for n in ("q", "k", "v")]
         gated = spec["gated"]
-        dgam_h = torch.empty(xh["g"].shape if gated else (cfg.H,), dtype=torch.float32).pin_memory()
+        outs_h = tuple(torch.empty(xh[n].shape, dtype=cfg.dtype).pin_memory() for n in ("q", "k", "v")) + (
+            torch.empty(xh["g"].shape if gated else (cfg.H,), dtype=torch.float32).pin_memory(),)
 
         def step():
-            for key in xh:
-                xd[key].copy_(xh[key], non_blocking=True)
-            grads = ret.chunkwise_backward(xd["q"], xd["k"], xd["v"], xd["g"] if gated else xd["gamma"], xd["do"],
-                                           cfg.chunk, gated=gated)
-            for h, d in zip(outs_h + [dgam_h], grads):
-                h.copy_(d, non_blocking=True)
+            ret.chunkwise_backward_host(xh["q"], xh["k"], xh["v"], xh["g"] if gated else xh["gamma"], xh["do"],
+                                        cfg.chunk, gated=gated, out=outs_h, stream=stream)
     else:
         # the host-buffer entry point: the library copies the inputs in and o out itself,
         # pipelined with the forward over groups of heads; each call returns with o on the host

@@ -36,8 +36,8 @@
  *     outputs are then undefined.
  *   - Errors are returned, never raised: no exit(), no device trap.
  *   - Calls keep no per-call state (the library holds only per-device helpers
- *     it creates once: the no-allocation scratch buffer, and five streams with
- *     their events for the backward and the *_host calls) and are safe from
+ *     it creates once: the no-allocation scratch buffer, five streams with their
+ *     events for the backward and two for the *_host calls) and are safe from
  *     several host threads,
  *     except ret_chunkwise_noalloc, whose calls all share one scratch buffer:
  *     calls of it that overlap on the GPU race (see its declaration).
@@ -148,7 +148,7 @@ RET_API ret_status gated_ret_chunkwise(const void* q, const void* k, const void*
  * back, pipelined over groups of heads (at most 8: whole batches when B >= 8,
  * else runs of heads inside one batch): the copies in of later groups overlap
  * the forward and the copy out of earlier ones, on `stream` and two library
- * streams forked from it and joined back. It returns once everything is
+ * streams of the *_host calls, forked from it and joined back. It returns once everything is
  * enqueued: o is complete when `stream` is. Host buffers should be page-locked
  * (cudaHostAlloc, cudaHostRegister); pageable buffers still give the right
  * result, but the driver then stages each copy and nothing overlaps. Each
@@ -206,6 +206,28 @@ RET_API ret_status gated_ret_chunkwise_backward(const void* q, const void* k, co
                                         const void* dout, void* dq, void* dk, void* dv, float* dg,
                                         int B, int H, int N, int dk_dim, int dv_dim, int chunk,
                                         ret_dtype dt, void* stream);
+
+/*
+ * ret_chunkwise_backward / gated_ret_chunkwise_backward from HOST memory: every
+ * tensor (q, k, v, gamma or g, dout, dq, dk, dv, dgamma or dg) is a host pointer
+ * with the layouts above; dgamma / dg may be NULL. The heads are cut into the
+ * groups of ret_chunkwise_host and pipelined the same way: the copies in of later
+ * groups overlap the backward and the copies out of earlier ones. Each group runs
+ * the device-buffer backward on its heads; dgamma, which sums over batches, is
+ * gathered per group on the device and added there once every group is done.
+ * Returns once everything is enqueued: the outputs are complete when `stream` is.
+ * Host buffers should be page-locked for the copies to overlap. Device buffers
+ * come from the stream-ordered pool and are freed on `stream` before the call
+ * returns. Limits as ret_chunkwise_backward. Not in the pages.
+ */
+RET_API ret_status ret_chunkwise_backward_host(const void* q, const void* k, const void* v, const float* gamma,
+                                       const void* dout, void* dq, void* dk, void* dv, float* dgamma,
+                                       int B, int H, int N, int dk_dim, int dv_dim, int chunk,
+                                       ret_dtype dt, void* stream);
+RET_API ret_status gated_ret_chunkwise_backward_host(const void* q, const void* k, const void* v, const float* g,
+                                             const void* dout, void* dq, void* dk, void* dv, float* dg,
+                                             int B, int H, int N, int dk_dim, int dv_dim, int chunk,
+                                             ret_dtype dt, void* stream);
 
 /*
  * Sequence split into consecutive segments computed separately (for example

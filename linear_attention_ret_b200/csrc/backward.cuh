@@ -328,6 +328,16 @@ gate_grad_carry_kernel(float* __restrict__ dg, const float* __restrict__ tile_to
     }
 }
 
+// out[h] = sum_g rows[g, h]: the per-group dgamma rows of a host-buffer backward.
+__global__ void __launch_bounds__(kBwdThreads)
+sum_rows_kernel(const float* __restrict__ rows, int G, int H, float* __restrict__ out) {
+    const int h = blockIdx.x * blockDim.x + threadIdx.x;
+    if (h >= H) return;
+    float s = 0.f;
+    for (int g = 0; g < G; ++g) s += rows[(size_t)g * H + h];
+    out[h] = s;
+}
+
 // In place: dg[bh, t] = sum_{u >= t} a[bh, u] (a suffix sum, since G_u includes g_t for
 // every u >= t). One block of kScanThreads per (b, h): each thread owns kScanPer consecutive
 // tokens of a span of kScanThreads * kScanPer (the whole row for N <= 16384), sums them from

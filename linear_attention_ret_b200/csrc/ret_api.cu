@@ -199,10 +199,7 @@ inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 // gradient waits for, and one of the least priority for the pass that it does not wait for.
 // Held under the mutex from the first fork to the last join, so calls from several host
 // threads do not interleave their events.
-// The host-buffer forward (chunkwise_host_entry) uses the first two streams and events for
-// its fork, its groups and its joins.
-constexpr int kAuxHi = 4, kAuxStreams = kAuxHi + 1, kPipeGroups = 8;
-constexpr int kAuxEvents = std::max(kAuxStreams + 1, 3 + 2 * kPipeGroups);
+constexpr int kAuxHi = 4, kAuxStreams = kAuxHi + 1, kAuxEvents = kAuxStreams + 1;
 struct AuxStreams {
     cudaStream_t s[kAuxStreams] = {};
     cudaEvent_t ev[kAuxEvents] = {};
@@ -513,15 +510,68 @@ ret_status launch_step(const void* q, const void* k, const void* v, const float*
     return launch_status();
 }
 
+// Streams of the host-buffer calls, one set per device with its own mutex (held while a call
+// enqueues): cs runs the groups' device work, os their copies out, and the events order them.
+// They are separate from the backward's streams, which a host-buffer backward uses inside
+// each group.
+constexpr int kPipeGroups = 8;
+struct HostPipe {
+    cudaStream_t cs = nullptr, os = nullptr;
+    cudaEvent_t ev[4 + 2 * kPipeGroups] = {};
+};
+inline std::mutex& pipe_mutex() {
+    static std::mutex m;
+    return m;
+}
+inline HostPipe* host_pipe() {
+    static HostPipe pipes[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    HostPipe& hp = pipes[dev];
+    if (!hp.cs) {  // publish only once every stream and event exists
+        HostPipe n;
+        bool ok = cudaStreamCreateWithFlags(&n.cs, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&n.os, cudaStreamNonBlocking) == cudaSuccess;
+        for (cudaEvent_t& e : n.ev) ok = ok && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
+        if (!ok) {
+            for (cudaEvent_t e : n.ev)
+                if (e) cudaEventDestroy(e);
+            if (n.cs) cudaStreamDestroy(n.cs);
+            if (n.os) cudaStreamDestroy(n.os);
+            return nullptr;
+        }
+        hp = n;
+    }
+    return &hp;
+}
+
+// The heads of a host-buffer call cut into at most kPipeGroups groups: whole batches when
+// B >= kPipeGroups, else runs of heads inside one batch, so that each group is one (B', H')
+// problem with its own slice of gamma (heads h0 .. h0 + nh) or of g.
+struct HeadGroup {
+    int b0, nb, h0, nh;
+};
+inline int head_groups(int B, int H, HeadGroup (&grp)[kPipeGroups]) {
+    int G = 0;
+    if (B >= kPipeGroups) {
+        const int bpg = (B + kPipeGroups - 1) / kPipeGroups;
+        for (int b0 = 0; b0 < B; b0 += bpg) grp[G++] = {b0, std::min(bpg, B - b0), 0, H};
+    } else {
+        const int per_batch = kPipeGroups / B, hpg = (H + per_batch - 1) / per_batch;
+        for (int b = 0; b < B; ++b)
+            for (int h0 = 0; h0 < H; h0 += hpg) grp[G++] = {b, 1, h0, std::min(hpg, H - h0)};
+    }
+    return G;
+}
+
 // The chunkwise forward from host buffers: q, k, v, the decay and o live in host memory.
-// The heads are cut into at most kPipeGroups groups (whole batches when B >= kPipeGroups,
-// else runs of heads inside one batch, so each group is one (B', H') problem with its own
-// slice of the decay) and pipelined over three streams:
+// The heads are cut into head_groups() and pipelined over three streams:
 //   st:  fork | H2D of group 0 | H2D of group 1 | ...            | wait cs, os | free
 //   cs:        wait H2D g -> chunkwise forward of group g -> ...
 //   os:                      wait forward g -> D2H of group g's o -> ...
 // so the copies in (the larger part) run back to back while earlier groups compute and copy
-// out in the other direction. Device buffers come from the stream-ordered pool.
+// out in the other direction. Device buffers come from the stream-ordered pool. The backward
+// from host buffers below follows the same plan.
 template <bool GATED>
 ret_status chunkwise_host_entry(const void* q, const void* k, const void* v, const float* decay, void* o, int B,
                                 int H, int N, int dk, int dv, int chunk, ret_dtype dt, void* stream) {
@@ -542,25 +592,15 @@ ret_status chunkwise_host_entry(const void* q, const void* k, const void* v, con
         off[i] = bytes;
         bytes += align256(sz[i]);
     }
-    // groups: (first batch, batches, first head, heads)
-    struct Group { int b0, nb, h0, nh; };
-    Group grp[kPipeGroups];
-    int G = 0;
-    if (B >= kPipeGroups) {
-        const int bpg = (B + kPipeGroups - 1) / kPipeGroups;
-        for (int b0 = 0; b0 < B; b0 += bpg) grp[G++] = {b0, std::min(bpg, B - b0), 0, H};
-    } else {
-        const int per_batch = kPipeGroups / B, hpg = (H + per_batch - 1) / per_batch;
-        for (int b = 0; b < B; ++b)
-            for (int h0 = 0; h0 < H; h0 += hpg) grp[G++] = {b, 1, h0, std::min(hpg, H - h0)};
-    }
-    std::lock_guard<std::mutex> lock(aux_mutex());
-    AuxStreams* a = aux_streams();
-    if (!a) return RET_ERR_CUDA;
-    cudaStream_t cs = a->s[0], os = a->s[1];
-    cudaEvent_t ev_fork = a->ev[0], ev_cs = a->ev[1], ev_os = a->ev[2];
-    cudaEvent_t* ev_in = a->ev + 3;                 // [kPipeGroups]: group g's inputs are on the device
-    cudaEvent_t* ev_out = a->ev + 3 + kPipeGroups;  // [kPipeGroups]: group g's o is computed
+    HeadGroup grp[kPipeGroups];
+    const int G = head_groups(B, H, grp);
+    std::lock_guard<std::mutex> lock(pipe_mutex());
+    HostPipe* hp = host_pipe();
+    if (!hp) return RET_ERR_CUDA;
+    cudaStream_t cs = hp->cs, os = hp->os;
+    cudaEvent_t ev_fork = hp->ev[0], ev_cs = hp->ev[1], ev_os = hp->ev[2];
+    cudaEvent_t* ev_in = hp->ev + 4;                 // [kPipeGroups]: group g's inputs are on the device
+    cudaEvent_t* ev_out = hp->ev + 4 + kPipeGroups;  // [kPipeGroups]: group g's results are computed
     tc::keep_pool_memory();
     uint8_t* buf = nullptr;
     if (cudaMallocAsync(reinterpret_cast<void**>(&buf), bytes, st) != cudaSuccess) return RET_ERR_CUDA;
@@ -585,7 +625,7 @@ ret_status chunkwise_host_entry(const void* q, const void* k, const void* v, con
         cu(cudaStreamWaitEvent(os, ev_fork, 0));
     }
     for (int gi = 0; gi < G && r == RET_OK; ++gi) {
-        const Group& g = grp[gi];
+        const HeadGroup& g = grp[gi];
         const size_t first = (size_t)g.b0 * H + g.h0, heads = (size_t)g.nb * g.nh;
         h2d(dq + first * head_q, hq + first * head_q, heads * head_q);
         h2d(dk_ + first * head_q, hk + first * head_q, heads * head_q);
@@ -603,6 +643,118 @@ ret_status chunkwise_host_entry(const void* q, const void* k, const void* v, con
         cu(cudaMemcpyAsync(ho + first * head_v, do_ + first * head_v, heads * head_v, cudaMemcpyDeviceToHost, os));
     }
     // join both library streams back into st whatever happened, then release the buffers
+    const bool joined = cudaEventRecord(ev_cs, cs) == cudaSuccess && cudaEventRecord(ev_os, os) == cudaSuccess &&
+                        cudaStreamWaitEvent(st, ev_cs, 0) == cudaSuccess &&
+                        cudaStreamWaitEvent(st, ev_os, 0) == cudaSuccess;
+    if (!joined) {
+        cudaStreamSynchronize(cs);
+        cudaStreamSynchronize(os);
+        if (r == RET_OK) r = RET_ERR_CUDA;
+    }
+    if (cudaFreeAsync(buf, st) != cudaSuccess && r == RET_OK) r = RET_ERR_CUDA;
+    return r;
+}
+
+// The backward from host buffers: q, k, v, the decay and dO in host memory, dq, dk, dv and
+// the decay gradient written back to host memory. Same plan as chunkwise_host_entry: the
+// copies in run back to back on st; cs runs each group's backward (the device-buffer call,
+// with its own library streams) once its inputs have landed; os copies its gradients out.
+// Each group's arrays start on 256-byte boundaries of the device buffers. dgamma sums over
+// batches and tokens, so each group writes its heads' share into a row of its own
+// (zeroed first, [G, H]) and one small kernel adds the rows once every group is done.
+template <bool GATED>
+ret_status backward_host_entry(const void* q, const void* k, const void* v, const float* decay, const void* dout,
+                               void* dq, void* dk_out, void* dv_out, float* ddecay, int B, int H, int N, int dk,
+                               int dv, int chunk, ret_dtype dt, void* stream) {
+    ret_status s = check_common(B, H, N, dk, dv, dt);
+    if (s != RET_OK) return s;
+    if (chunk <= 0) return RET_ERR_SHAPE;
+    if (dk > 256) return RET_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !decay || !dout || !dq || !dk_out || !dv_out) return RET_ERR_NULL;
+    if (N == 0) {
+        if (!GATED && ddecay) std::memset(ddecay, 0, sizeof(float) * (size_t)H);
+        return RET_OK;
+    }
+    cudaStream_t st = as_stream(stream);
+    const size_t es = dt == RET_F32 ? 4 : 2;
+    const size_t head_q = (size_t)N * dk * es, head_v = (size_t)N * dv * es, head_g = (size_t)N * sizeof(float);
+    HeadGroup grp[kPipeGroups];
+    const int G = head_groups(B, H, grp);
+    // per array, each group's region from a 256-byte boundary
+    size_t goff[kPipeGroups + 1][3] = {};  // [group][q-like, v-like, per-token fp32]
+    for (int gi = 0; gi < G; ++gi) {
+        const size_t heads = (size_t)grp[gi].nb * grp[gi].nh;
+        goff[gi + 1][0] = goff[gi][0] + align256(heads * head_q);
+        goff[gi + 1][1] = goff[gi][1] + align256(heads * head_v);
+        goff[gi + 1][2] = goff[gi][2] + align256(heads * head_g);
+    }
+    const size_t QB = goff[G][0], VB = goff[G][1], GB = goff[G][2];
+    // q, k, dq, dk | v, dO, dv | g, dg (gated) or gamma, dgamma rows and sum (fixed)
+    const size_t fixed_bytes = align256(sizeof(float) * H) * 2 + align256(sizeof(float) * (size_t)G * H);
+    const size_t bytes = 4 * QB + 3 * VB + (GATED ? 2 * GB : fixed_bytes);
+    std::lock_guard<std::mutex> lock(pipe_mutex());
+    HostPipe* hp = host_pipe();
+    if (!hp) return RET_ERR_CUDA;
+    cudaStream_t cs = hp->cs, os = hp->os;
+    cudaEvent_t ev_fork = hp->ev[0], ev_cs = hp->ev[1], ev_os = hp->ev[2], ev_sum = hp->ev[3];
+    cudaEvent_t* ev_in = hp->ev + 4;
+    cudaEvent_t* ev_out = hp->ev + 4 + kPipeGroups;
+    tc::keep_pool_memory();
+    uint8_t* buf = nullptr;
+    if (cudaMallocAsync(reinterpret_cast<void**>(&buf), bytes, st) != cudaSuccess) return RET_ERR_CUDA;
+    uint8_t* d_q = buf;
+    uint8_t* d_k = d_q + QB;
+    uint8_t* d_dq = d_k + QB;
+    uint8_t* d_dk = d_dq + QB;
+    uint8_t* d_v = d_dk + QB;
+    uint8_t* d_do = d_v + VB;
+    uint8_t* d_dv = d_do + VB;
+    uint8_t* d_g = d_dv + VB;                       // gated: g, then dg
+    uint8_t* d_dg = d_g + GB;
+    float* d_gamma = reinterpret_cast<float*>(d_g);  // fixed: gamma [H], dgamma rows [G, H], dgamma [H]
+    float* d_rows = reinterpret_cast<float*>(d_g + align256(sizeof(float) * H));
+    float* d_dgamma = reinterpret_cast<float*>(d_g + align256(sizeof(float) * H) + align256(sizeof(float) * (size_t)G * H));
+    ret_status r = RET_OK;
+    auto cu = [&](cudaError_t e) {
+        if (r == RET_OK && e != cudaSuccess) r = RET_ERR_CUDA;
+        return r == RET_OK;
+    };
+    auto h2d = [&](void* d, const void* h, size_t n) { return cu(cudaMemcpyAsync(d, h, n, cudaMemcpyHostToDevice, st)); };
+    auto d2h = [&](void* h, const void* d, size_t n) { return cu(cudaMemcpyAsync(h, d, n, cudaMemcpyDeviceToHost, os)); };
+    const bool want_dgamma = !GATED && ddecay;
+    if (!GATED) h2d(d_gamma, decay, sizeof(float) * H);
+    if (want_dgamma) cu(cudaMemsetAsync(d_rows, 0, sizeof(float) * (size_t)G * H, st));
+    if (cu(cudaEventRecord(ev_fork, st))) {
+        cu(cudaStreamWaitEvent(cs, ev_fork, 0));
+        cu(cudaStreamWaitEvent(os, ev_fork, 0));
+    }
+    for (int gi = 0; gi < G && r == RET_OK; ++gi) {
+        const HeadGroup& g = grp[gi];
+        const size_t first = (size_t)g.b0 * H + g.h0, heads = (size_t)g.nb * g.nh;
+        const size_t oq = goff[gi][0], ov = goff[gi][1], og = goff[gi][2];
+        h2d(d_q + oq, static_cast<const uint8_t*>(q) + first * head_q, heads * head_q);
+        h2d(d_k + oq, static_cast<const uint8_t*>(k) + first * head_q, heads * head_q);
+        h2d(d_v + ov, static_cast<const uint8_t*>(v) + first * head_v, heads * head_v);
+        h2d(d_do + ov, static_cast<const uint8_t*>(dout) + first * head_v, heads * head_v);
+        if (GATED) h2d(d_g + og, reinterpret_cast<const uint8_t*>(decay) + first * head_g, heads * head_g);
+        if (!cu(cudaEventRecord(ev_in[gi], st)) || !cu(cudaStreamWaitEvent(cs, ev_in[gi], 0))) break;
+        const float* gdec = GATED ? reinterpret_cast<const float*>(d_g + og) : d_gamma + g.h0;
+        float* gdd = GATED ? (ddecay ? reinterpret_cast<float*>(d_dg + og) : nullptr)
+                           : (want_dgamma ? d_rows + (size_t)gi * H + g.h0 : nullptr);
+        const ret_status rc = backward_entry<GATED>(d_q + oq, d_k + oq, d_v + ov, gdec, d_do + ov, d_dq + oq, d_dk + oq,
+                                                    d_dv + ov, gdd, g.nb, g.nh, N, dk, dv, chunk, dt, cs);
+        if (rc != RET_OK && r == RET_OK) r = rc;
+        if (!cu(cudaEventRecord(ev_out[gi], cs)) || !cu(cudaStreamWaitEvent(os, ev_out[gi], 0))) break;
+        d2h(static_cast<uint8_t*>(dq) + first * head_q, d_dq + oq, heads * head_q);
+        d2h(static_cast<uint8_t*>(dk_out) + first * head_q, d_dk + oq, heads * head_q);
+        d2h(static_cast<uint8_t*>(dv_out) + first * head_v, d_dv + ov, heads * head_v);
+        if (GATED && ddecay) d2h(reinterpret_cast<uint8_t*>(ddecay) + first * head_g, d_dg + og, heads * head_g);
+    }
+    if (want_dgamma && r == RET_OK) {
+        sum_rows_kernel<<<(H + kBwdThreads - 1) / kBwdThreads, kBwdThreads, 0, cs>>>(d_rows, G, H, d_dgamma);
+        if (cu(cudaGetLastError()) && cu(cudaEventRecord(ev_sum, cs)) && cu(cudaStreamWaitEvent(os, ev_sum, 0)))
+            d2h(ddecay, d_dgamma, sizeof(float) * H);
+    }
     const bool joined = cudaEventRecord(ev_cs, cs) == cudaSuccess && cudaEventRecord(ev_os, os) == cudaSuccess &&
                         cudaStreamWaitEvent(st, ev_cs, 0) == cudaSuccess &&
                         cudaStreamWaitEvent(st, ev_os, 0) == cudaSuccess;
@@ -750,6 +902,19 @@ ret_status gated_ret_chunkwise_backward(const void* q, const void* k, const void
                                         void* dq, void* dk, void* dv, float* dg, int B, int H, int N, int dk_dim,
                                         int dv_dim, int chunk, ret_dtype dt, void* stream) {
     return backward_entry<true>(q, k, v, g, dout, dq, dk, dv, dg, B, H, N, dk_dim, dv_dim, chunk, dt, stream);
+}
+
+ret_status ret_chunkwise_backward_host(const void* q, const void* k, const void* v, const float* gamma,
+                                       const void* dout, void* dq, void* dk, void* dv, float* dgamma, int B, int H,
+                                       int N, int dk_dim, int dv_dim, int chunk, ret_dtype dt, void* stream) {
+    return backward_host_entry<false>(q, k, v, gamma, dout, dq, dk, dv, dgamma, B, H, N, dk_dim, dv_dim, chunk, dt,
+                                      stream);
+}
+
+ret_status gated_ret_chunkwise_backward_host(const void* q, const void* k, const void* v, const float* g,
+                                             const void* dout, void* dq, void* dk, void* dv, float* dg, int B, int H,
+                                             int N, int dk_dim, int dv_dim, int chunk, ret_dtype dt, void* stream) {
+    return backward_host_entry<true>(q, k, v, g, dout, dq, dk, dv, dg, B, H, N, dk_dim, dv_dim, chunk, dt, stream);
 }
 
 int ret_chunkwise_state_launches(int B, int H, int N, int dk, int dv, int chunk, ret_dtype dt) {

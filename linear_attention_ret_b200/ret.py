@@ -31,7 +31,7 @@ SYMBOLS = ("ret_parallel", "ret_chunkwise", "ret_recurrent_step", "gated_ret_chu
            "ret_chunkwise_state", "gated_ret_chunkwise_state", "ret_state_prefix", "ret_chunkwise_state_launches",
            "ret_chunkwise_backward", "gated_ret_chunkwise_backward", "ret_chunkwise_backward_launches",
            "ret_msr_norm_gate", "ret_chunkwise_noalloc_scratch_bytes", "ret_chunkwise_host",
-           "gated_ret_chunkwise_host")
+           "gated_ret_chunkwise_host", "ret_chunkwise_backward_host", "gated_ret_chunkwise_backward_host")
 
 _lock = threading.Lock()
 _lib = None
@@ -73,7 +73,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
             getattr(lib, fn).restype = _i
         lib.ret_msr_norm_gate.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, ctypes.c_float, _i, _vp]
         lib.ret_msr_norm_gate.restype = _i
-        for fn in ("ret_chunkwise_backward", "gated_ret_chunkwise_backward"):
+        for fn in ("ret_chunkwise_backward", "gated_ret_chunkwise_backward", "ret_chunkwise_backward_host",
+                   "gated_ret_chunkwise_backward_host"):
             getattr(lib, fn).argtypes = [_vp] * 9 + [_i] * 7 + [_vp]
             getattr(lib, fn).restype = _i
         lib.ret_chunkwise_state_launches.restype = _i
@@ -321,6 +322,37 @@ def chunkwise_backward(q, k, v, decay, dout, chunk, gated=False, ddecay=True, st
     name = "gated_ret_chunkwise_backward" if gated else "ret_chunkwise_backward"
     _check(name, getattr(load(), name)(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(dout), _ptr(dq), _ptr(dkk),
                                        _ptr(dvv), _ptr(dd), B, H, N, dk, dv, int(chunk), _dt(q), _stream(stream)))
+    return dq, dkk, dvv, dd
+
+
+def chunkwise_backward_host(q, k, v, decay, dout, chunk, gated=False, ddecay=True, out=None, stream=None, sync=True):
+    """chunkwise_backward on host (CPU) tensors, pinned for copy/compute overlap: the library
+    copies the inputs in and the gradients out, pipelined over groups of heads, on the current
+    CUDA device. out: optional (dq, dk, dv, ddecay) host tensors to write. Returns them once the
+    stream has completed (sync=False: once enqueued)."""
+    B, H, N, dk, dv = _seq_args(q, k, v, decay, gated)
+    _expect("dout", dout, (B, H, N, dv), q.dtype)
+    pin = q.is_pinned()
+    if out is None:
+        dd = None
+        if ddecay:
+            dd = torch.empty((B, H, N) if gated else (H,), dtype=torch.float32, pin_memory=pin)
+        out = (torch.empty(B, H, N, dk, dtype=q.dtype, pin_memory=pin),
+               torch.empty(B, H, N, dk, dtype=q.dtype, pin_memory=pin),
+               torch.empty(B, H, N, dv, dtype=q.dtype, pin_memory=pin), dd)
+    dq, dkk, dvv, dd = out
+    _expect("dq", dq, (B, H, N, dk), q.dtype)
+    _expect("dk", dkk, (B, H, N, dk), q.dtype)
+    _expect("dv", dvv, (B, H, N, dv), q.dtype)
+    _expect("ddecay", dd, (B, H, N) if gated else (H,), torch.float32)
+    _host(*(t for t in (q, k, v, decay, dout, dq, dkk, dvv, dd) if t is not None))
+    s = torch.cuda.current_stream() if stream is None else stream
+    name = "gated_ret_chunkwise_backward_host" if gated else "ret_chunkwise_backward_host"
+    _check(name, getattr(load(), name)(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(dout), _ptr(dq), _ptr(dkk),
+                                       _ptr(dvv), _ptr(dd), B, H, N, dk, dv, int(chunk), _dt(q),
+                                       ctypes.c_void_p(s.cuda_stream)))
+    if sync:
+        s.synchronize()
     return dq, dkk, dvv, dd
 
 

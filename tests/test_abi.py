@@ -89,7 +89,8 @@ def test_parallel_and_step_validation(lib):
     assert lib.ret_recurrent_step(None, None, None, None, None, None, 1, 1, 8, 8, 2, None) == 3
 
 
-@pytest.mark.parametrize("fn", ["ret_chunkwise_backward", "gated_ret_chunkwise_backward"])
+@pytest.mark.parametrize("fn", ["ret_chunkwise_backward", "gated_ret_chunkwise_backward",
+                                "ret_chunkwise_backward_host", "gated_ret_chunkwise_backward_host"])
 def test_backward_validation(lib, fn):
     def call(B=1, H=1, N=8, dk=64, dv=64, chunk=64, dt=1):
         return getattr(lib, fn)(*([None] * 9), B, H, N, dk, dv, chunk, dt, None)

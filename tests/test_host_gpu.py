@@ -77,3 +77,55 @@ def test_host_call_back_to_back_on_a_side_stream(cuda_lib):
     s.synchronize()
     for (q, k, v), o in zip(ins, outs):
         assert torch.equal(o, ret.ret_chunkwise_host(q, k, v, gam, 64))
+
+
+BWD_CASES = [
+    # B, H, N, dk, dv, dtype
+    (4, 8, 256, 256, 512, torch.bfloat16),   # 8 groups; two dv pieces per group
+    (2, 3, 200, 128, 128, torch.bfloat16),   # groups of 2 and 1 heads
+    (9, 2, 100, 64, 128, torch.bfloat16),    # groups of whole batches
+    (1, 2, 90, 48, 40, torch.float32),       # CUDA-core path, rows of 12 chunks
+]
+
+
+@pytest.mark.parametrize("gated", [False, True])
+@pytest.mark.parametrize("B,H,N,dk,dv,dtype", BWD_CASES)
+def test_host_backward_matches_oracle(cuda_lib, B, H, N, dk, dv, dtype, gated):
+    gen = torch.Generator().manual_seed(7 * B + 3 * H + N)
+    q, k, v = I.qkv(B, H, N, dk, dv, dtype, gen=gen)
+    do = (torch.randn(B, H, N, dv, generator=gen) / dv ** 0.5).to(dtype)
+    decay = I.gate(B, H, N, gen) * 4.0 if gated else torch.tensor([0.96875, 0.999, 0.9, 0.75, 0.5][:H] + [0.99] * max(0, H - 5))
+    host = [t.pin_memory() for t in (q, k, v, decay, do)]
+    got = ret.chunkwise_backward_host(*host, 64, gated=gated)
+    assert ret.last_device_error() == 0
+    assert all(not t.is_cuda for t in got)
+    dev = ret.chunkwise_backward(*(t.to(DEV) for t in (q, k, v, decay, do)), 64, gated=gated)
+    want = (O.gated_backward if gated else O.ret_backward)(q, k, v, decay, do)
+    tol = TOL_F32 if dtype == torch.float32 else TOL_BF16
+    for name, g, d, w in zip(("dq", "dk", "dv"), got[:3], dev[:3], want[:3]):
+        assert rel_l2(g, w) <= tol, f"{name} against the oracle"
+        assert rel_l2(g, d.double().cpu()) <= tol, f"{name} against the device-buffer call"
+    # the decay gradient against the device-buffer call (which is checked against the oracle and
+    # its formula elsewhere): it sums a_t = q_t.dQ_t - k_t.dK_t with cancellation, and a group's
+    # dq, dk may round differently from the whole batch's, so the bound scales with the summed
+    # magnitudes |q_t.dQ_t| + |k_t.dK_t| (suffix sums for dg; sum_t t(..)/gamma for dgamma)
+    qd, kd, dqd, dkd = (t.double().cpu() for t in (q, k, dev[0], dev[1]))
+    mag = (qd * dqd).abs().sum(-1) + (kd * dkd).abs().sum(-1)
+    if gated:
+        scale = mag.flip(-1).cumsum(-1).flip(-1)
+    else:
+        scale = (torch.arange(N, dtype=torch.float64) * mag).sum((0, 2)) / decay.double()
+    rel = 1e-5 if dtype == torch.float32 else 1e-2
+    assert torch.all((got[3].double() - dev[3].double().cpu()).abs() <= rel * scale + 1e-12)
+
+
+def test_host_backward_without_decay_gradient(cuda_lib):
+    B, H, N, dk, dv = 2, 4, 300, 128, 256
+    q, k, v = (t.pin_memory() for t in I.qkv(B, H, N, dk, dv, torch.bfloat16, seed=9))
+    do = I.output_grad(B, H, N, dv, torch.bfloat16, seed=9).pin_memory()
+    gam = I.gammas(H).pin_memory()
+    with_dd = ret.chunkwise_backward_host(q, k, v, gam, do, 64)
+    without = ret.chunkwise_backward_host(q, k, v, gam, do, 64, ddecay=False)
+    assert without[3] is None
+    for a, b in zip(with_dd[:3], without[:3]):
+        assert torch.equal(a, b)
