@@ -14,8 +14,8 @@
 // zeta V / kappa in place and finally write kappa T. Tiles are 64 tokens for a fixed decay
 // (four stages at dk = 256: more copies in flight) and 128 tokens for the gated form, whose
 // per-tile work (a scan of the gates, exponentials, more frequent rescaling) is better
-// amortised over longer tiles; its gates are read 256 tokens ahead, since their latency
-// exceeds a tile's work. REV visits the tiles from the last back with the reversed
+// amortised over longer tiles; its gates are copied asynchronously into a shared-memory ring
+// kGateTiles tiles ahead, since their latency exceeds a tile's work. REV visits the tiles from the last back with the reversed
 // direction's key weights (see chunk_tc_kernel). All waits are bounded like the other
 // bodies'.
 #pragma once
@@ -25,6 +25,17 @@ namespace tc {
 
 constexpr int kSThreads = 192;
 constexpr int kMaxSStages = 8;
+constexpr int kGateTiles = 4;  // gated: tiles of gates in flight ahead of the scan
+
+// 4-byte asynchronous copy global -> shared (zero-filled when bytes == 0), its group commit
+// and the wait for all but the newest n groups.
+__device__ __forceinline__ void cp_async4(float* dst, const float* src, int bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // tokens per tile of the state-only pass
 __host__ __device__ constexpr int state_tile(bool gated) { return gated ? 128 : 64; }
@@ -39,7 +50,8 @@ struct StateLayout {
     static constexpr int kBar = kStages * kStageBytes;
     static constexpr int kNumBars = 4 * kStages + 1;            // full, empty, zv, upd per stage; drain
     static constexpr int kTab = kBar + kNumBars * 8;            // zeta / kappa [TT], gated cumsum [TT]
-    static constexpr int kTmemSlot = kTab + 2 * TT * 4;
+    static constexpr int kGRing = kTab + 2 * TT * 4;            // gated: raw gates of kGateTiles tiles
+    static constexpr int kTmemSlot = kGRing + kGateTiles * TT * 4;
     static constexpr int kAbort = kTmemSlot + 4;
     static constexpr int kBytes = kAbort + 4;
     static constexpr int kSmemAlloc = kBytes + 1024;            // slack to align the base to 1024 B
@@ -192,24 +204,26 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         };
         const float lg = GATED ? 0.f : log2f(p.decay_in[bh % p.H]);
         const float* G = GATED ? p.decay_in + (size_t)bh * p.N : nullptr;
-        // gated: lane l of warp 2 holds gates GPL l .. GPL l + GPL - 1 of tiles c .. c + PF - 1
-        // (read 256 tokens ahead, kept as they are in memory and scaled to log2 units where the
-        // tile's scan reads them, so that no instruction waits for a load before it is needed)
-        constexpr int GPL = kST / 32, PF = 256 / kST;
-        float gq[PF][GPL];
-        auto load_tile_gates = [&](int c, float (&x)[GPL]) {
+        // gated: warp 2 copies the raw gates of tile c into ring slot c % kGateTiles with
+        // asynchronous 4-byte copies (lane l: tokens GPL l .. GPL l + GPL - 1, zeros past the
+        // tile), kGateTiles tiles ahead of the scan, one commit group per tile, so the scan of a
+        // tile waits only for copies issued several tiles before; registers never wait on the
+        // newest loads.
+        constexpr int GPL = kST / 32;
+        float* gring = reinterpret_cast<float*>(sm + Lay::kGRing);
+        auto issue_gates = [&](int c) {
+            float* dst = gring + (c % kGateTiles) * kST + GPL * ts;
+            const int t0 = c < ntiles ? tile_t0(c) : 0, L = c < ntiles ? tile_len(c) : 0;
 #pragma unroll
-            for (int i = 0; i < GPL; ++i) x[i] = 0.f;
-            if (c < ntiles) {
-                const int t0 = tile_t0(c), L = tile_len(c);
-#pragma unroll
-                for (int i = 0; i < GPL; ++i)
-                    if (GPL * ts + i < L) x[i] = G[t0 + GPL * ts + i];
+            for (int i = 0; i < GPL; ++i) {
+                const bool in = GPL * ts + i < L;
+                cp_async4(dst + i, in ? G + t0 + GPL * ts + i : G, in ? 4 : 0);
             }
+            cp_async_commit();
         };
         if (GATED && ts < 32) {
 #pragma unroll
-            for (int f = 0; f < PF; ++f) load_tile_gates(f, gq[f]);
+            for (int f = 0; f < kGateTiles; ++f) issue_gates(f);
         }
         float kappa = 1.f, ldec_sum = 0.f;
         bool ok = true;
@@ -219,16 +233,14 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             float ldec;
             if (GATED) {
                 if (ts < 32) {
+                    cp_async_wait<kGateTiles - 1>();  // tile c's group (the oldest in flight) landed
+                    const float* gs = gring + (c % kGateTiles) * kST + GPL * ts;
                     float y[GPL];
 #pragma unroll
-                    for (int i = 0; i < GPL; ++i) y[i] = gq[0][i] * kLog2e;
+                    for (int i = 0; i < GPL; ++i) y[i] = gs[i] * kLog2e;
                     if constexpr (kST == 64) warp_cumsum64(y[0], y[1], lane, cum);
                     else warp_cumsum128(y, lane, cum);
-#pragma unroll
-                    for (int f = 0; f + 1 < PF; ++f)
-#pragma unroll
-                        for (int i = 0; i < GPL; ++i) gq[f][i] = gq[f + 1][i];
-                    load_tile_gates(c + PF, gq[PF - 1]);
+                    issue_gates(c + kGateTiles);  // into the slot just read (each lane its own words)
                 }
                 asm volatile("bar.sync 1, 128;" ::: "memory");
                 ldec = cum[L - 1];
@@ -301,6 +313,7 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             asm volatile("bar.sync 1, 128;" ::: "memory");
             if (ts == 0) mbar_arrive(bar(sbar(sZV, s, NS)));
         }
+        if (GATED && ts < 32) asm volatile("cp.async.wait_all;" ::: "memory");  // no copy outlives the CTA
         // the end state S = kappa T, rows dk of column dv0 + d, and the total decay
         if (ok && wait_all(sbar(sUpd, (ntiles - 1) % NS, NS), ((ntiles - 1) / NS) & 1)) {
             tc_fence_after();
