@@ -20,5 +20,9 @@ v and o [B, H, N, dv], states [B, H, dk, dv] fp32, bf16 or fp32 inputs):
 * ``ret.chunkwise_state`` and ``ret.state_prefix``: segment end states and start
   states for a sequence split across calls or GPUs; ``seqpar.sequence_parallel_chunkwise``
   runs the whole split over a torch.distributed group.
+* ``ret.ret_chunkwise_host`` / ``ret.gated_ret_chunkwise_host`` and
+  ``ret.chunkwise_backward_host``: the forward and the backward on host (CPU) tensors,
+  page-locked for overlap; the library copies them in and the results out, pipelined
+  with the compute over groups of heads.
 """
 __all__ = ["ret", "inputs", "build", "seqpar", "autograd"]
