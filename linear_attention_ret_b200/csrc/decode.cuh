@@ -8,7 +8,7 @@
 // adjacent dv columns of one head and walks all dk rows: rows are 16-byte
 // vectors, a warp touches 512 contiguous bytes per row, and the q.S reduction
 // over dk stays inside the thread (no shuffles, no shared-memory reduction).
-// Eight rows are in flight per thread to cover HBM latency; loads and stores
+// Sixteen rows are in flight per thread to cover HBM latency; loads and stores
 // use the streaming (evict-first) cache hint because the state is touched once.
 #pragma once
 
@@ -17,7 +17,7 @@
 namespace ret {
 
 constexpr int kDecThreads = 128;
-constexpr int kDecUnroll = 8;
+constexpr int kDecUnroll = 16;
 
 // decay: gamma [H] (fixed), or g [B, H] natural-log step decays (GATED)
 template <typename T, bool GATED>
