@@ -129,3 +129,46 @@ def test_host_backward_without_decay_gradient(cuda_lib):
     assert without[3] is None
     for a, b in zip(with_dd[:3], without[:3]):
         assert torch.equal(a, b)
+
+
+def _head(t, b, h):
+    return t[b:b + 1, h:h + 1].contiguous()
+
+
+@pytest.mark.parametrize("name", ["retnet_1p3b", "retnet_6p7b_long", "gated"])
+def test_full_size_host_call_sampled_heads(cuda_lib, name):
+    """The host-buffer forward at the workloads' full sizes, as the bench's e2e part calls it,
+    against the oracle on sampled heads (one of them in the last head group)."""
+    cfg = I.CONFIGS[name]
+    x = {key: t.pin_memory() for key, t in I.config_inputs(cfg).items()}
+    gated = "g" in x
+    if gated:
+        o = ret.gated_ret_chunkwise_host(x["q"], x["k"], x["v"], x["g"], cfg.chunk)
+    else:
+        o = ret.ret_chunkwise_host(x["q"], x["k"], x["v"], x["gamma"], cfg.chunk)
+    assert ret.last_device_error() == 0
+    for b, h in [(0, 0), (cfg.B - 1, cfg.H - 1)]:
+        q, k, v = (_head(x[n], b, h) for n in ("q", "k", "v"))
+        if gated:
+            want = O.gated_chunkwise(q, k, v, _head(x["g"], b, h), cfg.chunk)[0]
+        else:
+            want = O.ret_chunkwise(q, k, v, x["gamma"][h:h + 1], cfg.chunk)[0]
+        err = rel_l2(o[b:b + 1, h:h + 1], want)
+        assert err <= TOL_BF16, f"{name} head ({b},{h}): rel-L2 {err:.3e}"
+
+
+@pytest.mark.parametrize("gated", [False, True])
+def test_full_size_host_backward_matches_device_call(cuda_lib, gated):
+    """The host-buffer backward at the backward workloads' full sizes against the device-buffer
+    call (itself checked against the oracle on sampled heads at full size)."""
+    cfg = I.CONFIGS["gated" if gated else "retnet_1p3b"]
+    x = I.config_inputs(cfg)
+    do = I.output_grad(cfg.B, cfg.H, cfg.N, cfg.dv, cfg.dtype, seed=0)
+    decay = x["g"] if gated else x["gamma"]
+    got = ret.chunkwise_backward_host(*(t.pin_memory() for t in (x["q"], x["k"], x["v"], decay, do)), cfg.chunk,
+                                      gated=gated)
+    dev = ret.chunkwise_backward(*(t.to(DEV) for t in (x["q"], x["k"], x["v"], decay, do)), cfg.chunk, gated=gated)
+    assert ret.last_device_error() == 0
+    for name, g, d in zip(("dq", "dk", "dv"), got[:3], dev[:3]):
+        err = rel_l2(g, d.double().cpu())
+        assert err <= TOL_BF16, f"{name}: rel-L2 {err:.3e}"
